@@ -1,0 +1,124 @@
+/*
+ * fp64 CPU oracle for multi-head ReLU linear self-attention (forward).
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the bench's CPU
+ * baseline leg load this file's library. It shares no code, header, table or
+ * helper with the CUDA library and never runs on the product path.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - Feature map phi = ReLU, phi(x) = max(x, 0).
+ *      "08_sana高效高分辨率生成" (papers-3lj.pages.dev), section
+ *      "Linear Attention 的原理": phi = ReLU; KV = phi(K)^T V is d x d and does
+ *      not depend on n; A = phi(Q) KV.
+ *  - Normalised form  phi(Q)(phi(K)^T V) / (phi(Q) phi(K)^T 1).
+ *      "linear-diffusion-transformer-4k-efficient-generation"
+ *      (blog.hotdry.top), section "核心架构：Linear Attention 与 DC-AE 的协同设计".
+ *  - The two shared terms sum_n phi(K_n)^T V_n and sum_n phi(K_n)^T are formed
+ *    once and reused by every query (O(N) work).
+ *      "SANA: Efficient High-Resolution Image Synthesis with Linear Diffusion
+ *      Transformers" (phd-frog.tistory.com/40), section 2.2, "선형 어텐션 블럭"
+ *      (the prose around Eq. 1; the equation itself is lost from the page).
+ *  - Both shared terms as one d x (d+1) product phi(K)^T [V | 1]: the "padding"
+ *    that the same walk-through's section "Triton을 통한 학습/추론 가속화" lists
+ *    among the element-wise steps fused into the matmul, read here as a ones
+ *    column appended to V.
+ *
+ * Readings where the pages are silent (each one is also listed in the design
+ * notes): eps is added to the normaliser only, O = num / (den + eps); heads are
+ * independent with head size d; no 1/sqrt(d) or 1/N scale; a row whose
+ * normaliser is 0 gives 0 / eps = 0.
+ *
+ * Layout (the same one the library documents): Q, K, V, O are (B, N, H, d)
+ * row-major, element (b, n, h, i) at ((b*N + n)*H + h)*d + i. The state S is
+ * (B, H, d, d+1) row-major, entry (b, h, i, j) at ((b*H + h)*d + i)*(d+1) + j,
+ * with column j = d holding the normaliser sum_n phi(K_{n,i}).
+ *
+ * All arithmetic is IEEE double. Sums run in token order n = 0 .. N-1 and
+ * feature order i = 0 .. d-1, nothing is blocked or reordered. OpenMP only
+ * spreads independent (b, h) pairs or independent query rows over threads, which
+ * does not change any sum.
+ */
+#include <stddef.h>
+#include <omp.h>
+
+static double relu(double x) { return x > 0.0 ? x : 0.0; }
+
+/* offset of element (b, n, h, i) in a (B, N, H, d) row-major tensor */
+static size_t at_bnhd(long b, long n, long h, long i, long N, long H, long d)
+{
+    return (((size_t)b * N + n) * H + h) * d + i;
+}
+
+/* offset of entry (b, h, i, j) in a (B, H, d, d+1) row-major state */
+static size_t at_state(long b, long h, long i, long j, long H, long d)
+{
+    return (((size_t)b * H + h) * d + i) * (d + 1) + j;
+}
+
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+
+/*
+ * S[b,h] = sum over n of phi(K[b,n,h,:])^T [V[b,n,h,:] | 1].
+ * S[b,h,i,j] = sum_n relu(K[b,n,h,i]) * V[b,n,h,j]   for j < d
+ * S[b,h,i,d] = sum_n relu(K[b,n,h,i]) * 1
+ */
+void oracle_state(const double* K, const double* V, long B, long N, long H, long d,
+                  double* S)
+{
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b) {
+        for (long h = 0; h < H; ++h) {
+            for (long i = 0; i < d; ++i)
+                for (long j = 0; j <= d; ++j)
+                    S[at_state(b, h, i, j, H, d)] = 0.0;
+            for (long n = 0; n < N; ++n) {
+                for (long i = 0; i < d; ++i) {
+                    double k = relu(K[at_bnhd(b, n, h, i, N, H, d)]);
+                    for (long j = 0; j < d; ++j)
+                        S[at_state(b, h, i, j, H, d)] += k * V[at_bnhd(b, n, h, j, N, H, d)];
+                    S[at_state(b, h, i, d, H, d)] += k * 1.0;
+                }
+            }
+        }
+    }
+}
+
+/*
+ * For each query row (b, n, h):
+ *   num_j = sum_i relu(Q[b,n,h,i]) * S[b,h,i,j]   (j < d)
+ *   den   = sum_i relu(Q[b,n,h,i]) * S[b,h,i,d]
+ *   O[b,n,h,j] = num_j / (den + eps)
+ * If den_out is not NULL it receives den for every (b, n, h).
+ */
+void oracle_apply(const double* Q, const double* S, long B, long N, long H, long d,
+                  double eps, double* O, double* den_out)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (long b = 0; b < B; ++b) {
+        for (long n = 0; n < N; ++n) {
+            for (long h = 0; h < H; ++h) {
+                double den = 0.0;
+                for (long i = 0; i < d; ++i)
+                    den += relu(Q[at_bnhd(b, n, h, i, N, H, d)]) * S[at_state(b, h, i, d, H, d)];
+                for (long j = 0; j < d; ++j) {
+                    double num = 0.0;
+                    for (long i = 0; i < d; ++i)
+                        num += relu(Q[at_bnhd(b, n, h, i, N, H, d)]) * S[at_state(b, h, i, j, H, d)];
+                    O[at_bnhd(b, n, h, j, N, H, d)] = num / (den + eps);
+                }
+                if (den_out)
+                    den_out[((size_t)b * N + n) * H + h] = den;
+            }
+        }
+    }
+}
+
+/* forward = state, then apply (the scratch state is caller-provided) */
+void oracle_forward(const double* Q, const double* K, const double* V,
+                    long B, long N, long H, long d, double eps,
+                    double* S, double* O)
+{
+    oracle_state(K, V, B, N, H, d, S);
+    oracle_apply(Q, S, B, N, H, d, eps, O, NULL);
+}

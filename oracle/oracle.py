@@ -1,0 +1,107 @@
+"""ctypes wrapper around the fp64 C oracle for ReLU linear attention.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this module. It shares no code with the
+CUDA library. What the oracle computes, with the passages it follows, is written
+at the top of ``linattn_oracle.c``.
+
+Inputs are numpy arrays of shape (B, N, H, d); they are converted to float64
+(lossless for the bf16 and fp32 values the workloads use). Outputs are float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(HERE, "linattn_oracle.c")
+LIBRARY = os.path.join(HERE, "liboracle.so")
+
+_c_long = ctypes.c_long
+_c_double = ctypes.c_double
+_ptr = ctypes.c_void_p
+
+
+def compile_library(source: str = SOURCE, out: str = LIBRARY, extra_flags=()) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math) into ``out``."""
+    cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+           *extra_flags, source, "-o", out]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return out
+
+
+def _stale(lib: str, src: str) -> bool:
+    return (not os.path.exists(lib)) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+class Oracle:
+    """Loaded oracle library. ``path`` may point at another build of the same
+    source (the mutation tests load deliberately broken copies this way)."""
+
+    def __init__(self, path: str | None = None):
+        if path is None:
+            path = LIBRARY
+            if _stale(path, SOURCE):
+                compile_library()
+        self.path = path
+        lib = ctypes.CDLL(path)
+        lib.oracle_state.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long, _ptr]
+        lib.oracle_state.restype = None
+        lib.oracle_apply.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long,
+                                     _c_double, _ptr, _ptr]
+        lib.oracle_apply.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        self._lib = lib
+
+    @staticmethod
+    def _f64(x) -> np.ndarray:
+        a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+        if a.ndim != 4:
+            raise ValueError(f"expected a (B, N, H, d) array, got shape {a.shape}")
+        return a
+
+    def num_threads(self) -> int:
+        return int(self._lib.oracle_num_threads())
+
+    def state(self, K, V) -> np.ndarray:
+        """S = phi(K)^T [V | 1] per (b, h): shape (B, H, d, d+1), float64."""
+        K = self._f64(K)
+        V = self._f64(V)
+        if K.shape != V.shape:
+            raise ValueError("K and V must have the same shape")
+        B, N, H, d = K.shape
+        S = np.empty((B, H, d, d + 1), dtype=np.float64)
+        self._lib.oracle_state(K.ctypes.data, V.ctypes.data, B, N, H, d, S.ctypes.data)
+        return S
+
+    def apply(self, Q, S, eps: float, return_den: bool = False):
+        """O = (phi(Q) S[:, :d]) / (phi(Q) S[:, d] + eps): shape (B, N, H, d)."""
+        Q = self._f64(Q)
+        S = np.ascontiguousarray(np.asarray(S, dtype=np.float64))
+        B, N, H, d = Q.shape
+        if S.shape != (B, H, d, d + 1):
+            raise ValueError(f"state shape {S.shape} does not match Q {Q.shape}")
+        O = np.empty((B, N, H, d), dtype=np.float64)
+        den = np.empty((B, N, H), dtype=np.float64) if return_den else None
+        self._lib.oracle_apply(Q.ctypes.data, S.ctypes.data, B, N, H, d, float(eps),
+                               O.ctypes.data, den.ctypes.data if return_den else None)
+        return (O, den) if return_den else O
+
+    def forward(self, Q, K, V, eps: float, return_den: bool = False):
+        S = self.state(K, V)
+        return self.apply(Q, S, eps, return_den=return_den)
+
+
+_DEFAULT: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``linattn_oracle.c`` (compiled on first use)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT

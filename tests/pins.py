@@ -1,0 +1,277 @@
+"""Pins for the fp64 oracle: checks against what the pages and the mathematics
+fix, none of which reuses the oracle's own code.
+
+Each ``pin_*`` function takes an oracle object (anything with ``state``,
+``apply`` and ``forward`` like ``oracle.Oracle``) and raises AssertionError if
+the oracle disagrees with the pin. ``tests/test_oracle_pins.py`` runs them on
+the real oracle; ``tests/test_oracle_mutants.py`` runs them on copies of the
+oracle with a planted mistake and requires each copy to fail at least one.
+
+Passages:
+  * normalised form phi(Q)(phi(K)^T V) / (phi(Q) phi(K)^T 1):
+    "linear-diffusion-transformer-4k-efficient-generation" (blog.hotdry.top),
+    section "核心架构：Linear Attention 与 DC-AE 的协同设计";
+  * phi = ReLU and the d x d intermediate KV = phi(K)^T V, A = phi(Q) KV:
+    "08_sana高效高分辨率生成" (papers-3lj.pages.dev), "Linear Attention 的原理";
+  * the shared terms are computed once for all queries, which equals the
+    per-query n x n form: "SANA: Efficient High-Resolution Image Synthesis with
+    Linear Diffusion Transformers" (phd-frog.tistory.com/40), section 2.2,
+    "선형 어텐션 블럭" (Eq. 1 prose).
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+
+
+def bruteforce(Q, K, V, eps):
+    """The quadratic definition: W = phi(Q) phi(K)^T (N x N per (b, h)),
+    O = (W V) / (W 1 + eps). numpy fp64, per (b, h) slice of (B, N, H, d)."""
+    Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
+    B, N, H, d = Q.shape
+    O = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            q = np.maximum(Q[b, :, h, :], 0.0)
+            k = np.maximum(K[b, :, h, :], 0.0)
+            W = q @ k.T
+            O[b, :, h, :] = (W @ V[b, :, h, :]) / (W.sum(axis=1, keepdims=True) + eps)
+    return O
+
+
+def row_relerr(O, R):
+    """normwise relative error per (b, n, h) row of length d; rows with a zero
+    reference norm report the plain norm of O (so they must be exactly 0)."""
+    num = np.linalg.norm(O - R, axis=-1)
+    den = np.linalg.norm(R, axis=-1)
+    return np.where(den > 0, num / np.where(den > 0, den, 1.0), num)
+
+
+def _rng_inputs(seed, B=2, N=33, H=3, d=8, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return tuple(scale * rng.standard_normal((B, N, H, d)) for _ in range(3))
+
+
+# --------------------------------------------------------------------- pins --
+
+def pin_bruteforce(orc, Q, K, V, eps, tol=1e-12):
+    """Reassociated oracle == explicit n x n form to tol (normwise per row);
+    rows whose reference is exactly 0 must be exactly 0."""
+    O = orc.forward(Q, K, V, eps)
+    R = bruteforce(Q, K, V, eps)
+    err = row_relerr(O, R)
+    assert np.all(np.isfinite(O)), "oracle produced non-finite values"
+    assert err.max() <= tol, f"max row rel err vs brute force {err.max():.3e} > {tol}"
+    zero = np.linalg.norm(R, axis=-1) == 0
+    assert np.all(O[zero] == 0.0), "rows with phi(Q)=0 must be exactly 0"
+
+
+def exact_rational(Q, K, V, eps: Fraction):
+    """The quadratic definition in exact rational arithmetic (small inputs)."""
+    B, N, H, d = Q.shape
+    out = np.empty((B, N, H, d), dtype=object)
+    relu = (lambda x: x if x > 0 else Fraction(0))
+    for b in range(B):
+        for h in range(H):
+            for n in range(N):
+                w = [sum((relu(Fraction(Q[b, n, h, i])) * relu(Fraction(K[b, m, h, i]))
+                          for i in range(d)), Fraction(0)) for m in range(N)]
+                den = sum(w, Fraction(0)) + eps
+                for j in range(d):
+                    num = sum((w[m] * Fraction(V[b, m, h, j]) for m in range(N)), Fraction(0))
+                    out[b, n, h, j] = num / den
+    return out
+
+
+def pin_exact_integers(orc, seed=11):
+    """Small-integer inputs with eps = 1/4: every product and sum the oracle
+    forms is exact in fp64, so its result must equal the correctly rounded
+    exact rational value, bit for bit."""
+    rng = np.random.default_rng(seed)
+    B, N, H, d = 2, 5, 2, 3
+    Q, K, V = (rng.integers(-3, 4, size=(B, N, H, d)).astype(np.float64) for _ in range(3))
+    Q[0, 1, 0, :] = -np.abs(Q[0, 1, 0, :]) - 1  # one all-negative query row
+    eps = Fraction(1, 4)
+    ref = exact_rational(Q, K, V, eps)
+    O = orc.forward(Q, K, V, float(eps))
+    want = np.vectorize(float)(ref).astype(np.float64)
+    assert np.array_equal(O, want), f"oracle != exact rational result:\n{O}\n{want}"
+
+
+def pin_hand_example(orc):
+    """A hand-worked case (d = 2, N = 2, one head).
+    phi(Q_0) = [1, 0]; phi(K) = [[1, 2], [3, 0]] -> weights w = [1, 3], sum 4.
+    num = 1*[1, 2] + 3*[3, 4] = [10, 14].  eps = 0 -> [2.5, 3.5];
+    eps = 1 -> [2, 2.8].  Query 1 = [-1, 2] -> phi = [0, 2]: w = [4, 0],
+    num = 4*[1, 2] = [4, 8], den 4 -> [1, 2] (eps 0) or [0.8, 1.6] (eps 1)."""
+    Q = np.array([[1.0, -1.0], [-1.0, 2.0]]).reshape(1, 2, 1, 2)
+    K = np.array([[1.0, 2.0], [3.0, -1.0]]).reshape(1, 2, 1, 2)
+    V = np.array([[1.0, 2.0], [3.0, 4.0]]).reshape(1, 2, 1, 2)
+    O0 = orc.forward(Q, K, V, 0.0).reshape(2, 2)
+    O1 = orc.forward(Q, K, V, 1.0).reshape(2, 2)
+    assert np.array_equal(O0, np.array([[2.5, 3.5], [1.0, 2.0]])), O0
+    assert np.allclose(O1, np.array([[2.0, 2.8], [0.8, 1.6]]), rtol=1e-15, atol=0), O1
+
+
+def pin_single_token(orc, seed=3):
+    """N = 1: O_n = V_0 * s / (s + eps) with s = phi(Q_n) . phi(K_0)."""
+    Q, K, V = _rng_inputs(seed, B=2, N=1, H=3, d=8)
+    Qm, _, _ = _rng_inputs(seed + 1, B=2, N=7, H=3, d=8)
+    eps = 0.25
+    O = orc.apply(Qm, orc.state(K, V), eps)
+    s = np.einsum("bnhi,bhi->bnh", np.maximum(Qm, 0), np.maximum(K[:, 0], 0))
+    want = V[:, 0][:, None, :, :] * (s / (s + eps))[..., None]
+    assert np.allclose(O, want, rtol=1e-13, atol=1e-300), np.abs(O - want).max()
+
+
+def pin_equal_keys(orc, seed=4):
+    """All keys equal to one positive vector c: every query with phi(Q) != 0
+    weights all tokens equally, so O_n = mean_m V_m (up to eps / den)."""
+    Q, _, V = _rng_inputs(seed, B=2, N=40, H=2, d=8)
+    c = np.abs(np.random.default_rng(seed + 9).standard_normal((2, 1, 2, 8))) + 0.5
+    K = np.broadcast_to(c, Q.shape).copy()
+    O, den = orc.forward(Q, K, V, 1e-15, return_den=True)
+    mean = V.mean(axis=1, keepdims=True)
+    live = den > 0
+    err = np.abs(O - mean)[live]
+    assert err.max() <= 1e-12 * max(1.0, np.abs(mean).max()), err.max()
+
+
+def pin_one_hot(orc):
+    """phi(Q_n) = e_{i_n} and one-hot keys K_m = e_{m mod d}: w_nm = [m mod d ==
+    i_n], so O_n is the mean of the V rows whose key is hot at i_n."""
+    B, N, H, d = 1, 23, 2, 4
+    rng = np.random.default_rng(5)
+    V = rng.standard_normal((B, N, H, d))
+    K = np.full((B, N, H, d), -1.0)
+    for m in range(N):
+        K[0, m, :, m % d] = 2.0
+    Q = np.full((B, N, H, d), -0.5)
+    hot = rng.integers(0, d, size=N)
+    for n in range(N):
+        Q[0, n, :, hot[n]] = 1.5
+    O = orc.forward(Q, K, V, 0.0)
+    for n in range(N):
+        sel = [m for m in range(N) if m % d == hot[n]]
+        want = V[0, sel].mean(axis=0)
+        assert np.allclose(O[0, n], want, rtol=1e-13, atol=1e-15), (n, O[0, n], want)
+
+
+def pin_constant_column(orc, seed=6):
+    """A constant V column c comes back as c * den / (den + eps): exactly c up to
+    eps / den on rows with den > 0, and 0 on rows with den = 0."""
+    Q, K, V = _rng_inputs(seed, B=2, N=50, H=3, d=8)
+    Q[1, 3, 2, :] = -1.0  # a zero-weight row
+    V[..., 5] = 0.375
+    O, den = orc.forward(Q, K, V, 1e-15, return_den=True)
+    live = den > 0
+    assert np.allclose(O[..., 5][live], 0.375, rtol=1e-13, atol=0)
+    assert np.all(O[..., 5][~live] == 0.0)
+
+
+def pin_key_permutation(orc, seed=7):
+    """Permuting the token order of (K, V) jointly leaves O unchanged."""
+    Q, K, V = _rng_inputs(seed, B=2, N=41, H=3, d=8)
+    perm = np.random.default_rng(seed).permutation(41)
+    O1 = orc.forward(Q, K, V, 1e-15)
+    O2 = orc.forward(Q, K[:, perm], V[:, perm], 1e-15)
+    assert row_relerr(O2, O1).max() <= 1e-13
+
+
+def pin_query_permutation_and_independence(orc, seed=8):
+    """Permuting queries permutes output rows bit for bit; changing another
+    (b, h) slice, or K/V of another head, leaves a head's output unchanged."""
+    Q, K, V = _rng_inputs(seed, B=2, N=29, H=3, d=8)
+    O = orc.forward(Q, K, V, 1e-15)
+    perm = np.random.default_rng(seed).permutation(29)
+    Op = orc.forward(Q[:, perm], K, V, 1e-15)
+    assert np.array_equal(Op, O[:, perm])
+    Q2, K2, V2 = Q.copy(), K.copy(), V.copy()
+    Q2[:, :, 1] += 3.0
+    K2[:, :, 1] *= -2.0
+    V2[1] = 7.0
+    O2 = orc.forward(Q2, K2, V2, 1e-15)
+    assert np.array_equal(O2[0][:, [0, 2]], O[0][:, [0, 2]])
+
+
+def pin_convex_hull(orc, seed=9):
+    """Weights phi(Q_n).phi(K_m) >= 0, so each O_{n,i} is den/(den+eps) times a
+    convex combination of column i of V: it stays in the hull of V[:, i] and 0."""
+    Q, K, V = _rng_inputs(seed, B=2, N=64, H=3, d=8)
+    O = orc.forward(Q, K, V, 1e-15)
+    lo = np.minimum(V.min(axis=1, keepdims=True), 0.0)
+    hi = np.maximum(V.max(axis=1, keepdims=True), 0.0)
+    tol = 1e-12
+    assert np.all(O >= lo - tol) and np.all(O <= hi + tol)
+
+
+def pin_zero_query(orc, seed=10):
+    """A query with phi(Q) = 0 gives num = den = 0 and O = 0 / eps = 0 exactly."""
+    Q, K, V = _rng_inputs(seed, B=1, N=16, H=2, d=8)
+    Q[..., 0] = np.abs(Q[..., 0]) + 0.1   # every other row keeps a live feature
+    K[..., 0] = np.abs(K[..., 0]) + 0.1
+    Q[0, [2, 9], :, :] = -np.abs(Q[0, [2, 9], :, :]) - 0.1
+    O = orc.forward(Q, K, V, 1e-15)
+    assert np.all(O[0, [2, 9]] == 0.0)
+    assert np.all(np.linalg.norm(np.delete(O[0], [2, 9], axis=0), axis=-1) > 0)
+
+
+def pin_scale_invariance(orc, seed=12):
+    """With eps = 0, scaling Q or K by a power of two changes nothing, bit for bit
+    (every product scales exactly and the ratio cancels)."""
+    Q, K, V = _rng_inputs(seed, B=2, N=30, H=2, d=8)
+    Q = np.abs(Q) + 0.01  # no zero rows, so no 0/0 with eps = 0
+    O = orc.forward(Q, K, V, 0.0)
+    assert np.array_equal(orc.forward(4.0 * Q, 0.5 * K, V, 0.0), O)
+
+
+def pin_linearity_in_v(orc, seed=13):
+    """O is linear in V: O(aV + bV') = a O(V) + b O(V')."""
+    Q, K, V = _rng_inputs(seed, B=2, N=30, H=2, d=8)
+    _, _, V2 = _rng_inputs(seed + 1, B=2, N=30, H=2, d=8)
+    a, b = -1.5, 0.75
+    lhs = orc.forward(Q, K, a * V + b * V2, 1e-15)
+    rhs = a * orc.forward(Q, K, V, 1e-15) + b * orc.forward(Q, K, V2, 1e-15)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-13)
+
+
+def pin_state_definition(orc, seed=14):
+    """The state alone: column d is the per-feature sum of phi(K); the d x d
+    block is phi(K)^T V, checked by an explicit outer-product sum per token."""
+    Q, K, V = _rng_inputs(seed, B=2, N=17, H=3, d=5)
+    S = orc.state(K, V)
+    for b in range(2):
+        for h in range(3):
+            acc = np.zeros((5, 6))
+            for n in range(17):
+                k = np.maximum(K[b, n, h], 0.0)
+                acc += np.outer(k, np.append(V[b, n, h], 1.0))
+            assert np.allclose(S[b, h], acc, rtol=1e-13, atol=1e-13)
+
+
+def tiny_inputs():
+    """The 16x16-latent oracle check: B=1, N=256, H=4, d=32 from seed 0 (fp32)."""
+    import torch  # noqa: F401  (the generator lives in the product package)
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS["tiny"]
+    (_, src) = make_inputs(w, keep_source=True)
+    return tuple(t.double().numpy() for t in src), w.eps
+
+
+def pin_bruteforce_tiny(orc):
+    (Q, K, V), eps = tiny_inputs()
+    pin_bruteforce(orc, Q, K, V, eps)
+
+
+def pin_bruteforce_random(orc, seed=15):
+    Q, K, V = _rng_inputs(seed, B=2, N=37, H=3, d=6)
+    pin_bruteforce(orc, Q, K, V, 1e-15)
+
+
+ALL_PINS = [
+    pin_bruteforce_tiny, pin_bruteforce_random, pin_exact_integers, pin_hand_example,
+    pin_single_token, pin_equal_keys, pin_one_hot, pin_constant_column,
+    pin_key_permutation, pin_query_permutation_and_independence, pin_convex_hull,
+    pin_zero_query, pin_scale_invariance, pin_linearity_in_v, pin_state_definition,
+]
