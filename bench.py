@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Bench of the ReLU linear-attention forward at the 4096px Sana shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = the whole forward (state phi(K)^T[V|1] over all tokens, fixed-order
+chunk reduction, apply phi(Q)S and normalise) over one synthetic batch of the
+4096px workload: B=2 (CFG pair), N=16384 tokens (128x128 latent), H=70, d=32,
+bf16 Q/K/V, bf16 output. Inputs are 440 MB and the output 147 MB per step, more
+than the 126 MB L2, so no explicit L2 flush is done between steps.
+
+Prints one JSON line (rank 0). `value` is GB/s of algorithmic traffic (Q, K, V
+read once, O written once) over the device-timed steps, summed over ranks and
+divided by the slowest rank's time. Multi-GPU runs give every rank its own
+4096px problem (independent batches: weak scaling, no data-path collective).
+
+`--impl reference` times the fp64 CPU oracle (the only reference there is) on
+bounded samples of the same workload, on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ReLU linear-attn GB/s (% of B200 HBM peak) and Mtokens/s at 4096px shape"
+UNIT = "GB/s"
+WORKLOAD = "4096px"
+FALLBACK_HBM_GBS = 6650.0
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--workload", default=WORKLOAD,
+                   help="named workload (profiling runs use smaller ones; the bench line is 4096px)")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle baseline sample")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if args.steps < 1:
+        p.error("--steps must be >= 1")
+    return args
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, 1965.0, "fallback"
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(bytes_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's time."""
+    return bytes_per_rank * world / max_seconds / 1e9
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        busy = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle --
+
+def oracle_sample(w, seconds: float, max_heads: int | None = None):
+    """Time the fp64 oracle (as it stands) on whole heads of workload w, all N
+    tokens each, adding heads until about `seconds` of CPU work is done.
+    Returns (GB/s, Mtokens/s, threads, sample description, seconds)."""
+    import numpy as np
+    import torch
+    from oracle import default
+    from linear_attention_diffusion_relu_b200.workloads import make_inputs
+    orc = default()
+    Q, K, V = make_inputs(w)      # host tensors, bf16
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if max_heads is not None:
+        pairs = pairs[:max_heads]
+    done, elapsed = [], 0.0
+    step = 2
+    while done != pairs and elapsed < seconds:
+        batch = pairs[len(done):len(done) + step]
+        sl = [(torch.stack([t[b, :, h, :] for b, h in batch], dim=1)[None]
+               .to(torch.float64).numpy()) for t in (Q, K, V)]
+        t0 = time.perf_counter()
+        S = orc.state(sl[1], sl[2])
+        O = orc.apply(sl[0], S, w.eps)
+        elapsed += time.perf_counter() - t0
+        assert np.isfinite(O).all()
+        done += batch
+        step = min(step * 2, 16)
+    token_heads = len(done) * w.N
+    nbytes = token_heads * w.d * (3 * 2 + 2)
+    desc = (f"{w.name}: {len(done)} of {w.B * w.H} (b,h) pairs, all {w.N} tokens each "
+            f"({token_heads} token-heads), fp64 oracle state+apply")
+    return nbytes / elapsed / 1e9, token_heads / w.H / elapsed / 1e6, orc.num_threads(), desc, elapsed
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS
+    w = WORKLOADS[WORKLOAD]
+    per_step = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step / 4, max_heads=2)
+    vals, mts, secs = [], [], []
+    desc, cores = "", 0
+    for _ in range(args.steps):
+        gbs, mtok, cores, desc, s = oracle_sample(w, per_step)
+        vals.append(gbs)
+        mts.append(mtok)
+        secs.append(s)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "mtokens_per_s": statistics.median(mts),
+        "config": {"workload": WORKLOAD, "B": w.B, "N": w.N, "H": w.H, "d": w.d,
+                   "sample_per_step": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from linear_attention_diffusion_relu_b200 import ops
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    ops.load_library()
+
+    w = WORKLOADS[args.workload]
+    B, N, H, d = w.B, w.N, w.H, w.d
+    Q, K, V = make_inputs(w, device=dev)
+    if rank > 0:   # every rank its own independent batch of the same shape
+        Q, K, V = (t.roll(shifts=rank, dims=1).contiguous() for t in (Q, K, V))
+    out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=dev)
+    ws = ops.make_workspace(B, N, H, d, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ops.kv_state(K, V, state=state, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        ops.apply(Q, state, out_dtype=torch.bfloat16, eps=w.eps, out=out)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+
+    ms = start.elapsed_time(end) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+    bytes_per_step = w.algorithmic_bytes(2)
+    value = aggregate_gbs(bytes_per_step, world, ms_max / 1e3)
+    mtok = B * N * world / (ms_max / 1e3) / 1e6
+
+    ks_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
+    ka_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
+    hbm_peak, sm_max_mhz, peak_src = measured_peaks()
+    # both halves move 128 B per token-head (K+V read; Q read + bf16 O write)
+    half_bytes = w.token_heads * d * 4
+    kernels = {"kv_state(KS+KR)": (ks_ms, half_bytes), "apply(KA)": (ka_ms, half_bytes)}
+    dom = max(kernels, key=lambda k: kernels[k][0])
+    dom_ms, dom_bytes = kernels[dom]
+    impl = ops.implementation()
+    if impl["bound"] == "alu":
+        flops = w.token_heads * 2 * d * (d + 1)
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        peak = SMS * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dom,
+                "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                "hbm_gbs_of_measured": dom_bytes / (dom_ms / 1e3) / 1e9 / hbm_peak}
+    else:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": impl.get("traffic", {}).get(dom),
+                "kernel": dom, "peak_source": f"{peak_src} copy bandwidth (burst)"}
+    roof["ms_per_launch"] = dom_ms
+    roof["kernels_ms"] = {k: v[0] for k, v in kernels.items()}
+
+    e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, mt, cores, desc, _ = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": gbs, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+               "mtokens_per_s": mt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "mtokens_per_s": mtok, "pct_of_hbm_peak": 100.0 * value / (hbm_peak * world),
+            "config": {"workload": w.name, "B": B, "N": N, "H": H, "d": d,
+                       "io": "bf16 Q/K/V in, bf16 O out, fp32 state and accumulation",
+                       "eps": w.eps, "per_rank": "one independent 4096px batch",
+                       "parallelism": f"dp{world}",
+                       "l2": (f"inputs {w.token_heads * d * 6 / 1e6:.0f} MB + output "
+                              f"{w.token_heads * d * 2 / 1e6:.0f} MB per step vs the 126 MB L2; no flush"),
+                       "kernel_impl": impl["name"]},
+            "roofline": roof, "e2e": e2e, "clocks": clk,
+            "gpu_launches": ops.forward_launches(B, N, H, d) * args.steps,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, w, dev, stream, world):
+    """Same metric through the public call with host buffers: every step copies
+    Q, K, V from pinned host memory, runs forward, and copies O back."""
+    import torch
+    from linear_attention_diffusion_relu_b200 import ops
+    from linear_attention_diffusion_relu_b200.workloads import make_inputs
+    hQ, hK, hV = (t.pin_memory() for t in make_inputs(w))
+    hO = torch.empty(hQ.shape, dtype=torch.bfloat16).pin_memory()
+    dQ, dK, dV = (torch.empty_like(t, device=dev) for t in (hQ, hK, hV))
+    dO = torch.empty(hQ.shape, dtype=torch.bfloat16, device=dev)
+    ws = ops.make_workspace(w.B, w.N, w.H, w.d, dev)
+
+    def one():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        ops.forward(dQ, dK, dV, out_dtype=torch.bfloat16, eps=w.eps, out=dO, workspace=ws)
+        hO.copy_(dO, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, dev)
+    h2d = 3 * hQ.numel() * hQ.element_size()
+    d2h = hO.numel() * hO.element_size()
+    return {"value": aggregate_gbs(w.algorithmic_bytes(2), world, ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,158 @@
+/*
+ * sana_linattn.h - C ABI of the B200 (sm_100a) multi-head ReLU linear
+ * self-attention forward used by Sana's Linear DiT.
+ *
+ * The operation, per batch b and head h, with phi = ReLU:
+ *
+ *     S     = phi(K)^T [V | 1]                       d x (d+1), fp32
+ *     O_n   = (phi(Q_n) S[:, 0:d]) / (phi(Q_n) S[:, d] + eps)
+ *
+ * Sources (page title, section):
+ *   - "08_sana高效高分辨率生成" (papers-3lj.pages.dev), "Linear Attention 的原理":
+ *     phi = ReLU, KV = phi(K)^T V is d x d whatever the token count, and
+ *     A = phi(Q) KV.
+ *   - "linear-diffusion-transformer-4k-efficient-generation" (blog.hotdry.top),
+ *     "核心架构：Linear Attention 与 DC-AE 的协同设计": the normalised form
+ *     phi(Q)(phi(K)^T V) / (phi(Q) phi(K)^T 1).
+ *   - "SANA: Efficient High-Resolution Image Synthesis with Linear Diffusion
+ *     Transformers" (phd-frog.tistory.com/40), section 2.2 "선형 어텐션 블럭":
+ *     the two shared terms (phi(K)^T V and phi(K)^T 1) are computed once and
+ *     reused by every query; section "Triton을 통한 학습/추론 가속화": the
+ *     activation, precision conversion, padding and division are fused into the
+ *     matrix products (here: the ones column of [V | 1] is that padding, and the
+ *     division happens in the apply kernel's epilogue).
+ *   eps is added to the normaliser only; the pages write the formula without it.
+ *
+ * Layout
+ *   Q, K, V, O : (B, N, H, d) row-major. Element (b, n, h, i) is at
+ *                ((b*N + n)*H + h)*d + i. Q, K, V are bfloat16.
+ *                O is float32 or bfloat16 (round to nearest even).
+ *   state      : (B, H, d, d+1) row-major float32. Entry (b, h, i, j) is at
+ *                ((b*H + h)*d + i)*(d+1) + j. Column j = d is the normaliser
+ *                sum_n phi(K[b,n,h,i]).
+ *
+ * Ownership and execution
+ *   Every pointer is a DEVICE pointer owned by the caller; the library never
+ *   allocates, frees or synchronises. All work is enqueued on `stream`
+ *   (NULL = the legacy default stream) and the calls return as soon as it is
+ *   enqueued. Inputs must not alias outputs. The result is deterministic: the
+ *   same inputs and sizes give bit-identical outputs on every run, and
+ *   sana_linattn_forward gives exactly the bits of sana_linattn_kv_state
+ *   followed by sana_linattn_apply.
+ *
+ * Errors
+ *   Arguments are checked on the host before anything is launched; on any
+ *   error nothing is enqueued and the status says why:
+ *     SANA_LA_ERR_INVALID_ARG  null pointer, B, N or H < 1, a pointer not 16-byte
+ *                              aligned, eps negative or not finite, an unknown
+ *                              output dtype, or sizes whose element count
+ *                              overflows 63 bits;
+ *     SANA_LA_ERR_UNSUPPORTED  d not 32 or 64;
+ *     SANA_LA_ERR_WORKSPACE    workspace smaller than sana_linattn_workspace_bytes;
+ *     SANA_LA_ERR_CUDA         a CUDA call or launch failed (details from
+ *                              sana_linattn_last_error()).
+ *   Faults inside a kernel surface at the caller's next synchronisation, as
+ *   with any CUDA library. NaN or Inf inputs are outside the contract.
+ *   The functions are thread-safe; sana_linattn_last_error is per thread.
+ */
+#ifndef SANA_LINATTN_H
+#define SANA_LINATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same handle type as cudaStream_t, declared here without CUDA headers. */
+typedef struct CUstream_st* sana_la_stream_t;
+
+typedef enum {
+    SANA_LA_OK = 0,
+    SANA_LA_ERR_INVALID_ARG = 1,
+    SANA_LA_ERR_UNSUPPORTED = 2,
+    SANA_LA_ERR_WORKSPACE = 3,
+    SANA_LA_ERR_CUDA = 4
+} sana_la_status;
+
+typedef enum {
+    SANA_LA_OUT_F32 = 0,
+    SANA_LA_OUT_BF16 = 1
+} sana_la_out_dtype;
+
+/*
+ * Bytes of device workspace that sana_linattn_kv_state and
+ * sana_linattn_forward need for these sizes (a pure function of the sizes).
+ * The workspace holds the fp32 partial states of the token chunks, and for
+ * sana_linattn_forward also the reduced state. Returns 0 for invalid or
+ * unsupported sizes. Any content is acceptable on entry; it is scratch.
+ */
+size_t sana_linattn_workspace_bytes(int B, int N, int H, int d);
+
+/*
+ * The shared terms: state = phi(K)^T [V | 1] for every (b, h)
+ * ("08_sana高效高分辨率生成", "Linear Attention 的原理"; the Sana walk-through,
+ * section 2.2, Eq. 1 prose; the ones column is the "padding" of its Triton
+ * section).
+ *   K, V      bf16 (B, N, H, d), device.
+ *   state     fp32 (B, H, d, d+1), device, written in full.
+ *   workspace device scratch of at least sana_linattn_workspace_bytes(B,N,H,d).
+ * The token range is split into fixed chunks whose partial states are summed in
+ * ascending chunk order, so the result does not depend on scheduling.
+ */
+sana_la_status sana_linattn_kv_state(const void* K, const void* V,
+                                     int B, int N, int H, int d,
+                                     float* state,
+                                     void* workspace, size_t workspace_bytes,
+                                     sana_la_stream_t stream);
+
+/*
+ * The per-query product and normalisation:
+ *   O[b,n,h,:] = (phi(Q[b,n,h,:]) state[b,h,:,0:d]) / (phi(Q[b,n,h,:]) state[b,h,:,d] + eps)
+ * ("linear-diffusion-transformer-4k-efficient-generation", normalised form;
+ * "08_sana高效高分辨率生成", A = phi(Q) KV).
+ *   Q         bf16 (B, N, H, d), device.
+ *   state     fp32 (B, H, d, d+1), device (e.g. from sana_linattn_kv_state).
+ *   O         (B, N, H, d) device, fp32 or bf16 per out_dtype, written in full.
+ *   eps       finite, >= 0; a row with phi(Q) = 0 gives exactly 0.
+ */
+sana_la_status sana_linattn_apply(const void* Q, const float* state,
+                                  int B, int N, int H, int d,
+                                  void* O, sana_la_out_dtype out_dtype, float eps,
+                                  sana_la_stream_t stream);
+
+/*
+ * The whole forward: sana_linattn_kv_state into the workspace, then
+ * sana_linattn_apply. Same arguments and rules as the two calls above; the
+ * result is bit-identical to calling them in sequence.
+ */
+sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
+                                    int B, int N, int H, int d,
+                                    void* O, sana_la_out_dtype out_dtype, float eps,
+                                    void* workspace, size_t workspace_bytes,
+                                    sana_la_stream_t stream);
+
+/*
+ * Number of kernel launches one sana_linattn_forward call enqueues for these
+ * sizes (0 for invalid or unsupported sizes). Useful for graph capture and for
+ * counting launches in a profile.
+ */
+int sana_linattn_forward_launches(int B, int N, int H, int d);
+
+/*
+ * Static text naming the kernel set compiled into this library and the
+ * resource that bounds its dominant kernel, as "impl=<name>;bound=<hbm|alu>".
+ */
+const char* sana_linattn_build_info(void);
+
+/* Static English text for a status code. */
+const char* sana_linattn_status_string(sana_la_status status);
+
+/* Text of the last CUDA error seen by a call on this thread ("" if none). */
+const char* sana_linattn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SANA_LINATTN_H */

@@ -1,0 +1,204 @@
+"""Python binding of ``libsana_linattn.so`` (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this module
+checks torch tensors (dtype, shape, contiguity, device), passes raw device
+pointers and the current CUDA stream, and raises on any non-OK status. There is
+no CPU path: CPU tensors are rejected and a missing library raises.
+
+The functions mirror the C ABI in ``include/sana_linattn.h``:
+
+    workspace_bytes(B, N, H, d)
+    kv_state(K, V, state=None, workspace=None)             -> state (B, H, d, d+1) fp32
+    apply(Q, state, out_dtype=torch.bfloat16, eps=1e-15, out=None) -> O (B, N, H, d)
+    forward(Q, K, V, out_dtype=torch.bfloat16, eps=1e-15, out=None, workspace=None) -> O
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libsana_linattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = range(5)
+OUT_F32, OUT_BF16 = 0, 1
+
+SYMBOLS = (
+    "sana_linattn_workspace_bytes",
+    "sana_linattn_kv_state",
+    "sana_linattn_apply",
+    "sana_linattn_forward",
+    "sana_linattn_forward_launches",
+    "sana_linattn_build_info",
+    "sana_linattn_status_string",
+    "sana_linattn_last_error",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LinAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def load_library(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load the C-ABI library and declare its signatures. Raises if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None and path == LIBRARY:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build it with "
+                "`python -m linear_attention_diffusion_relu_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(path)
+        vp, i, sz, f, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+        lib.sana_linattn_workspace_bytes.argtypes = [i, i, i, i]
+        lib.sana_linattn_workspace_bytes.restype = sz
+        lib.sana_linattn_kv_state.argtypes = [vp, vp, i, i, i, i, vp, vp, sz, vp]
+        lib.sana_linattn_kv_state.restype = st
+        lib.sana_linattn_apply.argtypes = [vp, vp, i, i, i, i, vp, i, f, vp]
+        lib.sana_linattn_apply.restype = st
+        lib.sana_linattn_forward.argtypes = [vp, vp, vp, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_forward.restype = st
+        lib.sana_linattn_status_string.argtypes = [st]
+        lib.sana_linattn_status_string.restype = ctypes.c_char_p
+        lib.sana_linattn_forward_launches.argtypes = [i, i, i, i]
+        lib.sana_linattn_forward_launches.restype = ctypes.c_int
+        lib.sana_linattn_build_info.argtypes = []
+        lib.sana_linattn_build_info.restype = ctypes.c_char_p
+        lib.sana_linattn_last_error.argtypes = []
+        lib.sana_linattn_last_error.restype = ctypes.c_char_p
+        if path == LIBRARY:
+            _lib = lib
+        return lib
+
+
+def _check(lib, status: int, what: str):
+    if status != OK:
+        msg = lib.sana_linattn_status_string(status).decode()
+        extra = lib.sana_linattn_last_error().decode()
+        raise LinAttnError(status, f"{what}: {msg}" + (f" [{extra}]" if extra else ""))
+
+
+def _out_code(dtype) -> int:
+    if dtype == torch.float32:
+        return OUT_F32
+    if dtype == torch.bfloat16:
+        return OUT_BF16
+    raise ValueError(f"output dtype must be float32 or bfloat16, got {dtype}")
+
+
+def _check_bnhd(name, t, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must have shape (B, N, H, d), got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (B, N, H, d) row-major")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} shape {tuple(t.shape)} != {tuple(shape)}")
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def workspace_bytes(B: int, N: int, H: int, d: int) -> int:
+    return int(load_library().sana_linattn_workspace_bytes(B, N, H, d))
+
+
+def forward_launches(B: int, N: int, H: int, d: int) -> int:
+    """Kernel launches one forward call enqueues for these sizes."""
+    return int(load_library().sana_linattn_forward_launches(B, N, H, d))
+
+
+def implementation() -> dict:
+    """Kernel set compiled into the loaded library, e.g. {"name": ..., "bound": ...}."""
+    info = load_library().sana_linattn_build_info().decode()
+    kv = dict(part.split("=", 1) for part in info.split(";") if "=" in part)
+    return {"name": kv.get("impl", "?"), "bound": kv.get("bound", "hbm"), "raw": info}
+
+
+def make_workspace(B: int, N: int, H: int, d: int, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(B, N, H, d)
+    if n == 0:
+        raise ValueError(f"unsupported sizes B={B} N={N} H={H} d={d}")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kv_state(K: torch.Tensor, V: torch.Tensor, state: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """state = phi(K)^T [V | 1] per (b, h), fp32 (B, H, d, d+1)."""
+    _check_bnhd("K", K)
+    _check_bnhd("V", V, K.shape)
+    B, N, H, d = K.shape
+    if state is None:
+        state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=K.device)
+    elif (state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d + 1)
+          or not state.is_contiguous() or state.device != K.device):
+        raise ValueError("state must be contiguous float32 (B, H, d, d+1) on K's device")
+    if workspace is None:
+        workspace = make_workspace(B, N, H, d, K.device)
+    lib = load_library()
+    st = lib.sana_linattn_kv_state(K.data_ptr(), V.data_ptr(), B, N, H, d, state.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   _stream(K.device))
+    _check(lib, st, "sana_linattn_kv_state")
+    return state
+
+
+def _prep_out(out, shape, dtype, device):
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype or not out.is_contiguous() \
+            or out.device != device:
+        raise ValueError(f"out must be contiguous {dtype} {tuple(shape)} on {device}")
+    return out
+
+
+def apply(Q: torch.Tensor, state: torch.Tensor, out_dtype=torch.bfloat16, eps: float = 1e-15,
+          out: torch.Tensor | None = None) -> torch.Tensor:
+    """O = (phi(Q) state[..., :d]) / (phi(Q) state[..., d] + eps)."""
+    _check_bnhd("Q", Q)
+    B, N, H, d = Q.shape
+    if (state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d + 1)
+            or not state.is_contiguous() or state.device != Q.device):
+        raise ValueError("state must be contiguous float32 (B, H, d, d+1) on Q's device")
+    code = _out_code(out_dtype)
+    out = _prep_out(out, Q.shape, out_dtype, Q.device)
+    lib = load_library()
+    st = lib.sana_linattn_apply(Q.data_ptr(), state.data_ptr(), B, N, H, d, out.data_ptr(), code,
+                                float(eps), _stream(Q.device))
+    _check(lib, st, "sana_linattn_apply")
+    return out
+
+
+def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.bfloat16,
+            eps: float = 1e-15, out: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Whole ReLU linear-attention forward; bit-identical to kv_state + apply."""
+    _check_bnhd("Q", Q)
+    _check_bnhd("K", K, Q.shape)
+    _check_bnhd("V", V, Q.shape)
+    B, N, H, d = Q.shape
+    code = _out_code(out_dtype)
+    out = _prep_out(out, Q.shape, out_dtype, Q.device)
+    if workspace is None:
+        workspace = make_workspace(B, N, H, d, Q.device)
+    lib = load_library()
+    st = lib.sana_linattn_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d,
+                                  out.data_ptr(), code, float(eps), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream(Q.device))
+    _check(lib, st, "sana_linattn_forward")
+    return out

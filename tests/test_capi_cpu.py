@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every function the header declares, and
+rejects bad arguments on the host before launching anything. No GPU needed:
+every call here returns before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_diffusion_relu_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(sana_linattn_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sana_linattn_kv_state", "sana_linattn_apply", "sana_linattn_forward",
+                     "sana_linattn_workspace_bytes"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(ops.SYMBOLS) <= set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        s = lib.sana_linattn_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.sana_linattn_status_string(99).decode() == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    ws = lib.sana_linattn_workspace_bytes
+    assert ws(2, 16384, 70, 32) > 0
+    assert ws(2, 16384, 70, 32) % 256 == 0
+    assert ws(1, 1, 1, 32) > 0
+    assert ws(1, 1, 1, 48) == 0          # unsupported head size
+    assert ws(0, 16, 1, 32) == 0
+    assert ws(1, 0, 1, 32) == 0
+    assert ws(1, 16, -1, 64) == 0
+    # at least the reduced state plus one partial per (b, h)
+    assert ws(2, 16384, 70, 32) >= 2 * 70 * 32 * 33 * 4 * 2
+    # does not grow without bound with N (chunk count is capped)
+    assert ws(1, 1 << 20, 36, 32) < 64 << 20
+
+
+FAKE = 1 << 20   # aligned, never dereferenced: every call below fails its host checks
+
+
+def test_null_and_size_errors(lib):
+    f = lib.sana_linattn_forward
+    wsb = lib.sana_linattn_workspace_bytes(1, 64, 2, 32)
+    assert f(None, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 0, 64, 2, 32, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 0, 2, 32, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 48, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE, 7, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, -1.0, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, float("nan"), FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, float("inf"), FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE + 2, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE + 8, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, FAKE, 1, 1e-15, FAKE, wsb - 1, None) == ops.ERR_WORKSPACE
+    # element count overflow
+    assert f(FAKE, FAKE, FAKE, 1 << 30, 1 << 30, 1 << 10, 32, FAKE, 1, 0.0, FAKE, wsb, None) \
+        == ops.ERR_INVALID_ARG
+
+
+def test_kv_state_and_apply_errors(lib):
+    ks, ap = lib.sana_linattn_kv_state, lib.sana_linattn_apply
+    wsb = lib.sana_linattn_workspace_bytes(2, 100, 3, 64)
+    assert ks(FAKE, None, 2, 100, 3, 64, FAKE, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert ks(FAKE, FAKE, 2, 100, 3, 16, FAKE, FAKE, wsb, None) == ops.ERR_UNSUPPORTED
+    assert ks(FAKE, FAKE, 2, 100, 3, 64, FAKE + 4, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+    assert ks(FAKE, FAKE, 2, 100, 3, 64, FAKE, FAKE, 0, None) == ops.ERR_WORKSPACE
+    assert ap(None, FAKE, 2, 100, 3, 64, FAKE, 0, 0.0, None) == ops.ERR_INVALID_ARG
+    assert ap(FAKE, FAKE, 2, 100, 3, 64, FAKE, 2, 0.0, None) == ops.ERR_INVALID_ARG
+    assert ap(FAKE, FAKE, 2, 100, 3, 64, FAKE, 0, -1e-3, None) == ops.ERR_INVALID_ARG
+    assert ap(FAKE, FAKE, 2, -100, 3, 64, FAKE, 0, 0.0, None) == ops.ERR_INVALID_ARG
+    assert lib.sana_linattn_last_error().decode() == ""
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    x = torch.zeros((1, 8, 1, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.forward(x, x, x)
+
+
+def test_library_is_sm100a_only():
+    """The build targets sm_100a and nothing else (no PTX for other archs)."""
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+    assert not any("compute_90" in f or "sm_90" in f for f in build.NVCC_FLAGS)

@@ -1,0 +1,195 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small and mid-size shapes compare every output element; the full-size Sana
+shapes compare every row of sampled heads (the oracle rebuilds those heads'
+states from all N tokens). Also: determinism, forward == kv_state + apply bit
+for bit, guard bands around outputs and workspace, streams, error paths."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_diffusion_relu_b200 import ops
+from linear_attention_diffusion_relu_b200.workloads import WORKLOADS, Workload, make_inputs
+from tests.parity import check_output, head_slice, to_f64
+
+pytestmark = pytest.mark.gpu
+
+OUT_DTYPES = [torch.float32, torch.bfloat16]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from linear_attention_diffusion_relu_b200 import build
+    build.build()
+    ops.load_library()
+
+
+def _dt(dtype):
+    return "f32" if dtype == torch.float32 else "bf16"
+
+
+def _full_check(oracle, Q, K, V, eps, dtype, what):
+    O = ops.forward(Q, K, V, out_dtype=dtype, eps=eps)
+    torch.cuda.synchronize()
+    ref = oracle.forward(to_f64(Q), to_f64(K), to_f64(V), eps)
+    check_output(O, ref, what)
+    return O, ref
+
+
+SMALL = [(1, 1, 1, 32), (1, 7, 3, 32), (2, 31, 2, 64), (1, 129, 5, 32), (2, 1000, 3, 32),
+         (1, 4097, 2, 64), (3, 513, 7, 32), (1, 2048, 70, 32), (2, 300, 18, 64)]
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B{}N{}H{}d{}".format(*s))
+def test_small_shapes(oracle, shape, dtype):
+    B, N, H, d = shape
+    w = Workload("adhoc", B, N, H, d, seed=100 + N + H)
+    Q, K, V = make_inputs(w, device="cuda")
+    _full_check(oracle, Q, K, V, 1e-15, dtype, f"{shape}")
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+@pytest.mark.parametrize("name", ["tiny", "1024px", "2048px"])
+def test_named_configs_every_element(oracle, name, dtype):
+    w = WORKLOADS[name]
+    Q, K, V = make_inputs(w, device="cuda")
+    O, ref = _full_check(oracle, Q, K, V, w.eps, dtype, name)
+    if name == "tiny":
+        rows = list(w.neg_rows)
+        assert torch.all(O[0, rows] == 0)
+
+
+def _sampled_heads_check(oracle, w, Q, K, V, dtype, heads, rows=None):
+    O = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps)
+    torch.cuda.synchronize()
+    Qh, Kh, Vh = (head_slice(t, heads) for t in (Q, K, V))
+    S = oracle.state(Kh, Vh)
+    if rows is not None:
+        Qh = Qh[:, rows]
+    ref = oracle.apply(Qh, S, w.eps)
+    got = O[:, :, list(heads), :]
+    if rows is not None:
+        got = got[:, torch.as_tensor(rows, device=O.device)]
+    check_output(got, ref, f"{w.name} heads {heads}")
+
+
+FULL = ["4096px", "ragged_N16381", "d64", "sweep_N1024", "sweep_N16384", "sweep_N65536"]
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_heads(oracle, name, dtype):
+    w = WORKLOADS[name]
+    Q, K, V = make_inputs(w, device="cuda")
+    heads = sorted({0, w.H // 2, w.H - 1})
+    _sampled_heads_check(oracle, w, Q, K, V, dtype, heads)
+
+
+@pytest.mark.parametrize("name", ["sweep_N262144", "sweep_N1048576"])
+def test_longest_sweep_sampled_rows(oracle, name):
+    """Largest token counts: inputs drawn with the seeded CUDA generator; the
+    oracle rebuilds two heads' states from all N tokens and checks 4096 rows."""
+    w = WORKLOADS[name]
+    Q, K, V = make_inputs(w, device="cuda", generator_device="cuda")
+    rows = np.sort(np.random.default_rng(0).choice(w.N, size=4096, replace=False))
+    rows[0], rows[-1] = 0, w.N - 1
+    for dtype in OUT_DTYPES:
+        _sampled_heads_check(oracle, w, Q, K, V, dtype, [1, w.H - 2], rows=rows)
+
+
+def test_state_matches_oracle(oracle):
+    """kv_state alone: each entry within 1e-5 of the sum of |terms| it adds up
+    (an fp32 accumulation bound with ample margin), at a multi-chunk size."""
+    w = replace(WORKLOADS["sweep_N16384"], H=5)
+    Q, K, V = make_inputs(w, device="cuda")
+    S = ops.kv_state(K, V)
+    torch.cuda.synchronize()
+    Kd, Vd = to_f64(K), to_f64(V)
+    ref = oracle.state(Kd, Vd)
+    mag = oracle.state(Kd, np.abs(Vd))
+    err = np.abs(to_f64(S) - ref)
+    assert np.all(err <= 1e-5 * mag + 1e-30), (err / (mag + 1e-30)).max()
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+def test_deterministic_and_split_equals_forward(dtype):
+    w = WORKLOADS["2048px"]
+    Q, K, V = make_inputs(w, device="cuda")
+    O1 = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps)
+    O2 = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps)
+    S = ops.kv_state(K, V)
+    O3 = ops.apply(Q, S, out_dtype=dtype, eps=w.eps)
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(O1.view(bits), O2.view(bits))
+    assert torch.equal(O1.view(bits), O3.view(bits))
+    S2 = ops.kv_state(K, V)
+    assert torch.equal(S.view(torch.int32), S2.view(torch.int32))
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+def test_guard_bands(dtype):
+    """Outputs and workspace are written only inside their extents."""
+    B, N, H, d = 2, 1531, 6, 32
+    w = Workload("guard", B, N, H, d, seed=7)
+    Q, K, V = make_inputs(w, device="cuda")
+    pad = 4096
+    n_out = B * N * H * d
+    big = torch.full((pad + n_out + pad,), 12345.0 if dtype == torch.float32 else 77.0,
+                     dtype=dtype, device="cuda")
+    O = big[pad:pad + n_out].view(B, N, H, d)
+    wsb = ops.workspace_bytes(B, N, H, d)
+    wsbig = torch.full((256 + wsb + 4096,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = wsbig[256:256 + wsb]
+    ops.forward(Q, K, V, out_dtype=dtype, out=O, workspace=ws)
+    torch.cuda.synchronize()
+    sentinel = big[0].item()
+    assert torch.all(big[:pad] == sentinel) and torch.all(big[pad + n_out:] == sentinel)
+    assert torch.all(wsbig[:256] == 0xA5) and torch.all(wsbig[256 + wsb:] == 0xA5)
+
+
+def test_runs_on_caller_stream(oracle):
+    w = Workload("stream", 1, 777, 3, 64, seed=9)
+    Q, K, V = make_inputs(w, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        O = ops.forward(Q, K, V, out_dtype=torch.float32)
+    s.synchronize()
+    check_output(O, oracle.forward(to_f64(Q), to_f64(K), to_f64(V), 1e-15), "side stream")
+
+
+def test_key_permutation_and_constant_column(oracle):
+    w = Workload("inv", 1, 3000, 4, 32, seed=11)
+    Q, K, V = make_inputs(w, device="cuda")
+    V[..., 7] = 0.375
+    O = ops.forward(Q, K, V, out_dtype=torch.float32)
+    perm = torch.randperm(w.N, generator=torch.Generator().manual_seed(1)).cuda()
+    Op = ops.forward(Q, K[:, perm].contiguous(), V[:, perm].contiguous(), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.forward(to_f64(Q), to_f64(K), to_f64(V), 1e-15)
+    check_output(Op, ref, "permuted keys")
+    live = np.linalg.norm(ref, axis=-1) > 0
+    col = to_f64(O)[..., 7][live]
+    assert np.allclose(col, 0.375, rtol=1e-5, atol=0)
+
+
+def test_error_paths_on_device():
+    Q = torch.zeros((1, 64, 2, 32), dtype=torch.bfloat16, device="cuda")
+    flat = torch.zeros(1 + Q.numel(), dtype=torch.bfloat16, device="cuda")
+    mis = flat[1:].view(1, 64, 2, 32)          # 2-byte offset: misaligned
+    with pytest.raises(ops.LinAttnError) as e:
+        ops.forward(mis, Q, Q)
+    assert e.value.status == ops.ERR_INVALID_ARG
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ops.LinAttnError) as e:
+        ops.forward(Q, Q, Q, workspace=ws)
+    assert e.value.status == ops.ERR_WORKSPACE
+    x = torch.zeros((1, 64, 2, 48), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ops.LinAttnError) as e:
+        ops.forward(x, x, x, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == ops.ERR_UNSUPPORTED
