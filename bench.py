@@ -328,7 +328,7 @@ def run_ours(args):
             "mtokens_per_s": mtok, "pct_of_hbm_peak": 100.0 * value / (hbm_peak * world),
             "config": {"workload": w.name, "B": B, "N": N, "H": H, "d": d,
                        "io": "bf16 Q/K/V in, bf16 O out, fp32 state and accumulation",
-                       "eps": w.eps, "per_rank": "one independent 4096px batch",
+                       "eps": w.eps, "per_rank": f"one independent {w.name} batch",
                        "parallelism": f"dp{world}",
                        "l2": (f"inputs {w.token_heads * d * 6 / 1e6:.0f} MB + output "
                               f"{w.token_heads * d * 2 / 1e6:.0f} MB per step vs the 126 MB L2; no flush"),
