@@ -1,0 +1,61 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2): the time used
+for the job is the slowest rank's, and the value counts every rank's bytes."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        w, r, local = bench.dist_env()
+        ms = 1.0 + rank                      # rank 1 is slower
+        ms_max = bench.max_over_ranks(ms)
+        value = bench.aggregate_gbs(1_000_000_000, w, ms_max / 1e3)
+        q.put((r, w, local, ms_max, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_aggregate_two_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, (r, w, local, ms_max, value) in enumerate(res):
+        assert (r, w, local) == (rank, 2, rank)
+        assert ms_max == pytest.approx(2.0)              # slowest rank
+        assert value == pytest.approx(2 * 1e9 / 2e-3 / 1e9)  # both ranks' bytes / slowest time
+
+
+def test_single_process_identity():
+    import bench
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.aggregate_gbs(10**9, 1, 1.0) == pytest.approx(1.0)
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]) == 0
+    assert capsys.readouterr().out == ""
