@@ -133,6 +133,34 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     sana_la_stream_t stream);
 
 /*
+ * sana_linattn_forward without a workspace argument, for callers that cannot
+ * allocate device memory: code that runs under an allocator it does not own
+ * (a host application or framework that hands out all device memory itself),
+ * serving loops that must not allocate once started, and callers bound to an
+ * interface that passes only inputs and outputs (no scratch buffer).
+ * The paper has no counterpart to this call; it exists for those callers.
+ *
+ * The scratch sits in a fixed 16 MiB device array inside this library, which
+ * every GPU that loads the library keeps until the process exits. Sizes whose
+ * sana_linattn_workspace_bytes exceeds 16 MiB are rejected with
+ * SANA_LA_ERR_WORKSPACE (sana_linattn_last_error says how much they need); the
+ * 4096px shape (B=2, N=16384, H=70, d=32) fits. The call allocates nothing.
+ *
+ * Its first call on a device looks up the array's device address (with the
+ * calling thread's current device, which must be the device of Q, K, V, O and
+ * `stream`); make that first call before any stream capture. All calls on a
+ * device share the array: calls whose work can overlap on the GPU (e.g. on
+ * unordered streams) race and give wrong results; order them on one stream.
+ * The array needs no clearing between calls. Results are bit-identical to
+ * sana_linattn_forward with a caller workspace. Arguments and other errors are
+ * as for sana_linattn_forward.
+ */
+sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const void* V,
+                                            int B, int N, int H, int d,
+                                            void* O, sana_la_out_dtype out_dtype, float eps,
+                                            sana_la_stream_t stream);
+
+/*
  * Number of kernel launches one sana_linattn_forward call enqueues for these
  * sizes (0 for invalid or unsupported sizes). Useful for graph capture and for
  * counting launches in a profile.

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/sana_linattn.h"
 #include "common.cuh"
@@ -206,5 +207,76 @@ const char* sana_linattn_status_string(sana_la_status status) {
 }
 
 const char* sana_linattn_last_error(void) { return g_last_error; }
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Forward without caller-provided scratch.
+//
+// The scratch that sana_linattn_forward takes as `workspace` lives here in a
+// fixed device array instead. Loading this library reserves it on every GPU
+// that uses the library, until the process exits. Every call on a device
+// shares the one array: calls whose kernels overlap on that device (different
+// streams, no ordering between them) race on it. Nothing in it has to start at
+// zero: each call writes every byte it later reads.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_scratch_mutex;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device. The host-side
+// name is only a stand-in; the address comes from cudaGetSymbolAddress, asked
+// once per device (with that device current) and cached.
+sana_la_status static_scratch_address(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_last_error("cudaGetDevice", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return SANA_LA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (g_static_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            set_last_error("cudaGetSymbolAddress(g_static_scratch)", e);
+            return SANA_LA_ERR_CUDA;
+        }
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return SANA_LA_OK;
+}
+
+}  // namespace
+
+extern "C" sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const void* V,
+                                                       int B, int N, int H, int d,
+                                                       void* O, sana_la_out_dtype out_dtype,
+                                                       float eps, sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!Q || !K || !V || !O) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    const size_t need = sana_linattn_workspace_bytes(B, N, H, d);
+    if (need > kStaticScratchBytes) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "these sizes need %zu bytes of scratch; the static scratch holds %zu",
+                      need, kStaticScratchBytes);
+        return SANA_LA_ERR_WORKSPACE;
+    }
+    void* scratch = nullptr;
+    if ((st = static_scratch_address(&scratch)) != SANA_LA_OK) return st;
+    return sana_linattn_forward(Q, K, V, B, N, H, d, O, out_dtype, eps, scratch,
+                                kStaticScratchBytes, stream);
+}
+
+extern "C" {
 
 }  // extern "C"
