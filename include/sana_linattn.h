@@ -173,6 +173,16 @@ int sana_linattn_forward_launches(int B, int N, int H, int d);
  */
 const char* sana_linattn_build_info(void);
 
+/*
+ * Diagnostic: the first error code a kernel of this library recorded on the
+ * current device (0 = none; 1 = a pipeline wait inside a kernel ran past its
+ * ~2 s limit, after which that kernel stopped early and its outputs are not
+ * valid). With clear != 0 the code is reset to 0. This call synchronises with
+ * the device; call it after the work it should cover has completed (e.g.
+ * after cudaDeviceSynchronize), not in a hot loop.
+ */
+sana_la_status sana_linattn_device_error(unsigned int* code, int clear);
+
 /* Static English text for a status code. */
 const char* sana_linattn_status_string(sana_la_status status);
 

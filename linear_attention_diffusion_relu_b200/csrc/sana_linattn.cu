@@ -1,15 +1,18 @@
-// C ABI of the ReLU linear-attention forward: argument checks, the split-N
-// plan, and kernel launches on the caller's stream. See include/sana_linattn.h
-// for the contract.
+// C ABI of the ReLU linear-attention forward: argument checks, the work
+// plans, TMA tensor maps, and kernel launches on the caller's stream. See
+// include/sana_linattn.h for the contract.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/sana_linattn.h"
 #include "common.cuh"
-#include "simt_kernels.cuh"
+#include "tc_kernels.cuh"
 
 namespace {
 
@@ -20,38 +23,44 @@ void set_last_error(const char* where, cudaError_t e) {
                   cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-constexpr int kSMs = 148;             // B200
-constexpr int kTargetUnits = 4 * kSMs;
-constexpr int kMinChunk = 256;        // fewest tokens a chunk may hold
-constexpr int kChunkAlign = 64;
+constexpr int kSMs = 148;             // B200: one persistent CTA per SM
 constexpr long long kMaxElems = 1LL << 62;
+constexpr long long kMaxGrid = 0x7fffffffLL;
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Split of the token range into C chunks of `chunk` tokens (the last may be
-// short). A pure function of the sizes, so workspace size and reduction order
-// never depend on the device or on timing.
+// Work plans of the three kernels. A pure function of the sizes: the
+// workspace size and the order in which partial states are summed never
+// depend on the device or on timing.
 struct Plan {
-    int C;
-    int chunk;
-    size_t partial_bytes;   // fp32 (B, H, C, d, d+1)
+    sana::tc::KsParams ks;
+    sana::tc::KaParams ka;
+    size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
     size_t state_bytes;     // fp32 (B, H, d, d+1)
 };
 
 Plan make_plan(int B, int N, int H, int d) {
-    const int heads_per_group = (d == 32) ? 4 : 2;   // 128 state rows per group
-    const long long groups = cdiv(H, heads_per_group);
-    const long long per_chunk_units = (long long)B * groups;
-    long long C = cdiv(kTargetUnits, per_chunk_units);
-    C = std::max(1LL, std::min(C, cdiv(N, kMinChunk)));
-    long long chunk = cdiv(cdiv(N, C), kChunkAlign) * kChunkAlign;
-    C = cdiv(N, chunk);
-    Plan p;
-    p.C = (int)C;
-    p.chunk = (int)chunk;
+    const int G = 128 / d;                        // heads per 128-row group
+    const long long groups = cdiv(H, G);
+    Plan p{};
+    p.ks.N = N;
+    p.ks.H = H;
+    p.ks.groups = (int)groups;
+    p.ks.tiles_per_bg = (int)cdiv(N, sana::tc::KS_TILE);
+    p.ks.total_tiles = (long long)B * groups * p.ks.tiles_per_bg;
+    p.ks.grid = (int)std::min<long long>(kSMs, p.ks.total_tiles);
+    const long long longest = cdiv(p.ks.total_tiles, p.ks.grid);
+    p.ks.max_seg = (int)((longest - 1) / p.ks.tiles_per_bg + 2);
+    p.ka.N = N;
+    p.ka.H = H;
+    p.ka.groups = (int)groups;
+    p.ka.tiles_per_bg = (int)cdiv(N, sana::tc::KA_TILE);
+    p.ka.total_units = (long long)B * groups * p.ka.tiles_per_bg;
+    p.ka.grid = (int)std::min<long long>(kSMs, p.ka.total_units);
+    p.ka.eps = 0.0f;
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
-    p.partial_bytes = align256((size_t)B * H * C * dd);
+    p.partial_bytes = align256((size_t)p.ks.grid * p.ks.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * dd);
     return p;
 }
@@ -63,6 +72,9 @@ sana_la_status check_sizes(int B, int N, int H, int d) {
     if (d != 32 && d != 64) return SANA_LA_ERR_UNSUPPORTED;
     const long long elems = (long long)B * N;
     if (elems > kMaxElems / ((long long)H * d)) return SANA_LA_ERR_INVALID_ARG;
+    // one batch of one tensor must stay under the 2^40-byte TMA stride limit
+    if ((long long)N * H * d * 2 >= (1LL << 40)) return SANA_LA_ERR_UNSUPPORTED;
+    if ((long long)B * H > kMaxGrid) return SANA_LA_ERR_UNSUPPORTED;
     return SANA_LA_OK;
 }
 
@@ -79,34 +91,101 @@ sana_la_status launch_status(const char* where) {
     return SANA_LA_OK;
 }
 
-constexpr long long kMaxGrid = 0x7fffffffLL;
+// ------------------------------------------------------------- TMA maps ----
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
 
+// (B, N, H*d) bf16 tensor viewed as 3-D {H*d, N, B}; boxes of 64 elements
+// (128 bytes, one swizzle span) by `rows` tokens, 128-byte swizzle, zero fill
+// outside the tensor (tokens >= N and heads >= H read as 0).
+sana_la_status make_tmap(CUtensorMap* m, const void* base, int B, int N, int H, int d, int rows) {
+    auto encode = tensor_map_encoder();
+    if (encode == nullptr) {
+        std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+        return SANA_LA_ERR_CUDA;
+    }
+    const cuuint64_t row_elems = (cuuint64_t)H * d;
+    cuuint64_t dims[3] = {row_elems, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {row_elems * 2, row_elems * 2 * (cuuint64_t)N};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return SANA_LA_ERR_CUDA;
+    }
+    return SANA_LA_OK;
+}
+
+// Opt a kernel into its dynamic shared memory size, once per device.
+template <typename Kernel>
+sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_last_error("cudaGetDevice", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return SANA_LA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) {
+        set_last_error("cudaFuncSetAttribute", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return SANA_LA_OK;
+}
+
+// ------------------------------------------------------------- launches ----
 template <int D>
-sana_la_status run_kv_state(const __nv_bfloat16* K, const __nv_bfloat16* V, int B, int N, int H,
-                            const Plan& p, float* partial, float* state, cudaStream_t s) {
-    const long long units = (long long)B * H * p.C;
-    if (units > kMaxGrid) return SANA_LA_ERR_UNSUPPORTED;
-    sana::simt::ks_partial<D><<<(unsigned)units, sana::simt::kThreads, 0, s>>>(
-        K, V, N, H, p.C, p.chunk, partial);
-    sana_la_status st = launch_status("ks_partial");
-    if (st != SANA_LA_OK) return st;
-    sana::simt::kr_reduce<D><<<(unsigned)((long long)B * H), 256, 0, s>>>(partial, p.C, state);
-    return launch_status("kr_reduce");
+sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, const Plan& p,
+                            float* partial, float* state, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmK, tmV;
+    sana_la_status st;
+    if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
+    if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KS_SMEM_BYTES, smem_set)) != SANA_LA_OK)
+        return st;
+    sana::tc::ks_state_tc<D><<<p.ks.grid, sana::tc::kThreads, sana::tc::KS_SMEM_BYTES, s>>>(
+        tmK, tmV, p.ks, partial);
+    if ((st = launch_status("ks_state_tc")) != SANA_LA_OK) return st;
+    sana::tc::kr_reduce_tc<D><<<(unsigned)((long long)B * H), 256, 0, s>>>(partial, p.ks, state);
+    return launch_status("kr_reduce_tc");
 }
 
 template <int D>
-sana_la_status run_apply(const __nv_bfloat16* Q, const float* state, int B, int N, int H,
-                         void* O, sana_la_out_dtype od, float eps, cudaStream_t s) {
-    const long long tiles = cdiv(N, sana::simt::kApplyTokens);
-    const long long units = (long long)B * H * tiles;
-    if (units > kMaxGrid) return SANA_LA_ERR_UNSUPPORTED;
-    if (od == SANA_LA_OUT_BF16)
-        sana::simt::ka_apply<D, true><<<(unsigned)units, sana::simt::kThreads, 0, s>>>(
-            Q, state, N, H, (int)tiles, eps, O);
-    else
-        sana::simt::ka_apply<D, false><<<(unsigned)units, sana::simt::kThreads, 0, s>>>(
-            Q, state, N, H, (int)tiles, eps, O);
-    return launch_status("ka_apply");
+sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, void* O,
+                         sana_la_out_dtype od, float eps, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set_bf16{0}, smem_set_f32{0};
+    Plan p = make_plan(B, N, H, D);
+    p.ka.eps = eps;
+    CUtensorMap tmQ;
+    sana_la_status st;
+    if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
+    constexpr int smem = sana::tc::KaLayout<D>::SMEM_BYTES;
+    if (od == SANA_LA_OUT_BF16) {
+        if ((st = ensure_smem(sana::tc::ka_apply_tc<D, true>, smem, smem_set_bf16)) != SANA_LA_OK) return st;
+        sana::tc::ka_apply_tc<D, true><<<p.ka.grid, sana::tc::kThreads, smem, s>>>(tmQ, p.ka, state, O);
+    } else {
+        if ((st = ensure_smem(sana::tc::ka_apply_tc<D, false>, smem, smem_set_f32)) != SANA_LA_OK) return st;
+        sana::tc::ka_apply_tc<D, false><<<p.ka.grid, sana::tc::kThreads, smem, s>>>(tmQ, p.ka, state, O);
+    }
+    return launch_status("ka_apply_tc");
 }
 
 sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d,
@@ -116,17 +195,14 @@ sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, 
     const size_t need = p.partial_bytes + (need_state_area ? p.state_bytes : 0);
     if (ws_bytes < need) return SANA_LA_ERR_WORKSPACE;
     float* partial = static_cast<float*>(ws);
-    auto k = static_cast<const __nv_bfloat16*>(K);
-    auto v = static_cast<const __nv_bfloat16*>(V);
-    return d == 32 ? run_kv_state<32>(k, v, B, N, H, p, partial, state, s)
-                   : run_kv_state<64>(k, v, B, N, H, p, partial, state, s);
+    return d == 32 ? run_kv_state<32>(K, V, B, N, H, p, partial, state, s)
+                   : run_kv_state<64>(K, V, B, N, H, p, partial, state, s);
 }
 
 sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d,
                           void* O, sana_la_out_dtype od, float eps, cudaStream_t s) {
-    auto q = static_cast<const __nv_bfloat16*>(Q);
-    return d == 32 ? run_apply<32>(q, state, B, N, H, O, od, eps, s)
-                   : run_apply<64>(q, state, B, N, H, O, od, eps, s);
+    return d == 32 ? run_apply<32>(Q, state, B, N, H, O, od, eps, s)
+                   : run_apply<64>(Q, state, B, N, H, O, od, eps, s);
 }
 
 }  // namespace
@@ -193,7 +269,28 @@ int sana_linattn_forward_launches(int B, int N, int H, int d) {
     return 3;   // KS, KR, KA
 }
 
-const char* sana_linattn_build_info(void) { return "impl=simt-ffma;bound=alu"; }
+const char* sana_linattn_build_info(void) { return "impl=tcgen05-tma;bound=hbm"; }
+
+sana_la_status sana_linattn_device_error(unsigned int* code, int clear) {
+    g_last_error[0] = '\0';
+    if (!code) return SANA_LA_ERR_INVALID_ARG;
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, sana::tc::g_device_error, sizeof(v));
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemcpyFromSymbol", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    if (clear && v != 0) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(sana::tc::g_device_error, &zero, sizeof(zero));
+        if (e != cudaSuccess) {
+            set_last_error("cudaMemcpyToSymbol", e);
+            return SANA_LA_ERR_CUDA;
+        }
+    }
+    *code = v;
+    return SANA_LA_OK;
+}
 
 const char* sana_linattn_status_string(sana_la_status status) {
     switch (status) {

@@ -33,6 +33,7 @@ SYMBOLS = (
     "sana_linattn_forward",
     "sana_linattn_forward_launches",
     "sana_linattn_build_info",
+    "sana_linattn_device_error",
     "sana_linattn_status_string",
     "sana_linattn_last_error",
 )
@@ -73,6 +74,8 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_forward_launches.restype = ctypes.c_int
         lib.sana_linattn_build_info.argtypes = []
         lib.sana_linattn_build_info.restype = ctypes.c_char_p
+        lib.sana_linattn_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+        lib.sana_linattn_device_error.restype = st
         lib.sana_linattn_last_error.argtypes = []
         lib.sana_linattn_last_error.restype = ctypes.c_char_p
         if path == LIBRARY:
@@ -128,6 +131,16 @@ def implementation() -> dict:
     info = load_library().sana_linattn_build_info().decode()
     kv = dict(part.split("=", 1) for part in info.split(";") if "=" in part)
     return {"name": kv.get("impl", "?"), "bound": kv.get("bound", "hbm"), "raw": info}
+
+
+def device_error(clear: bool = False) -> int:
+    """First error code a kernel recorded on the current device (0 = none).
+    Synchronising diagnostic: call after the covered work has completed."""
+    lib = load_library()
+    code = ctypes.c_uint(0)
+    _check(lib, lib.sana_linattn_device_error(ctypes.byref(code), int(clear)),
+           "sana_linattn_device_error")
+    return int(code.value)
 
 
 def make_workspace(B: int, N: int, H: int, d: int, device="cuda") -> torch.Tensor:
