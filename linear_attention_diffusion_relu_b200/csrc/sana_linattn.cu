@@ -40,6 +40,23 @@ struct Plan {
     size_t state_bytes;     // fp32 (B, H, d, d+1)
 };
 
+// Lockstep schedule of S slabs of T tiles over at most kSMs CTAs (see the
+// comment at the top of tc_kernels.cuh).
+sana::tc::Sched make_sched(long long S, long long T) {
+    sana::tc::Sched q{};
+    q.S = (int)S;
+    q.T = (int)T;
+    if (S <= kSMs) {
+        q.R = (int)std::min<long long>(kSMs / S, T);
+        q.grid = (int)(S * q.R);
+    } else {
+        q.R = 1;
+        q.grid = kSMs;
+    }
+    q.max_seg = (int)cdiv(S, q.grid);
+    return q;
+}
+
 Plan make_plan(int B, int N, int H, int d) {
     const int G = 128 / d;                        // heads per 128-row group
     const long long groups = cdiv(H, G);
@@ -47,20 +64,14 @@ Plan make_plan(int B, int N, int H, int d) {
     p.ks.N = N;
     p.ks.H = H;
     p.ks.groups = (int)groups;
-    p.ks.tiles_per_bg = (int)cdiv(N, sana::tc::KS_TILE);
-    p.ks.total_tiles = (long long)B * groups * p.ks.tiles_per_bg;
-    p.ks.grid = (int)std::min<long long>(kSMs, p.ks.total_tiles);
-    const long long longest = cdiv(p.ks.total_tiles, p.ks.grid);
-    p.ks.max_seg = (int)((longest - 1) / p.ks.tiles_per_bg + 2);
+    p.ks.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KS_TILE));
     p.ka.N = N;
     p.ka.H = H;
     p.ka.groups = (int)groups;
-    p.ka.tiles_per_bg = (int)cdiv(N, sana::tc::KA_TILE);
-    p.ka.total_units = (long long)B * groups * p.ka.tiles_per_bg;
-    p.ka.grid = (int)std::min<long long>(kSMs, p.ka.total_units);
+    p.ka.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KA_TILE));
     p.ka.eps = 0.0f;
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
-    p.partial_bytes = align256((size_t)p.ks.grid * p.ks.max_seg * G * dd);
+    p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * dd);
     return p;
 }
@@ -106,22 +117,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// (B, N, H*d) bf16 tensor viewed as 3-D {H*d, N, B}; boxes of 64 elements
-// (128 bytes, one swizzle span) by `rows` tokens, 128-byte swizzle, zero fill
-// outside the tensor (tokens >= N and heads >= H read as 0).
-sana_la_status make_tmap(CUtensorMap* m, const void* base, int B, int N, int H, int d, int rows) {
+// (B, N, H*d) tensor viewed as 3-D {H*d, N, B}; boxes of 128 bytes (one
+// swizzle span: 64 bf16 or 32 fp32 elements) by `rows` tokens, 128-byte
+// swizzle. Loads read zeros outside the tensor (tokens >= N, heads >= H);
+// stores skip those parts.
+sana_la_status make_tmap(CUtensorMap* m, const void* base, int B, int N, int H, int d, int rows,
+                         bool fp32 = false) {
     auto encode = tensor_map_encoder();
     if (encode == nullptr) {
         std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
         return SANA_LA_ERR_CUDA;
     }
+    const cuuint64_t esize = fp32 ? 4 : 2;
     const cuuint64_t row_elems = (cuuint64_t)H * d;
     cuuint64_t dims[3] = {row_elems, (cuuint64_t)N, (cuuint64_t)B};
-    cuuint64_t strides[2] = {row_elems * 2, row_elems * 2 * (cuuint64_t)N};
-    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint64_t strides[2] = {row_elems * esize, row_elems * esize * (cuuint64_t)N};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / esize), (cuuint32_t)rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = encode(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -161,31 +176,37 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KS_SMEM_BYTES, smem_set)) != SANA_LA_OK)
         return st;
-    sana::tc::ks_state_tc<D><<<p.ks.grid, sana::tc::kThreads, sana::tc::KS_SMEM_BYTES, s>>>(
+    sana::tc::ks_state_tc<D><<<p.ks.q.grid, sana::tc::kThreads, sana::tc::KS_SMEM_BYTES, s>>>(
         tmK, tmV, p.ks, partial);
     if ((st = launch_status("ks_state_tc")) != SANA_LA_OK) return st;
-    sana::tc::kr_reduce_tc<D><<<(unsigned)((long long)B * H), 256, 0, s>>>(partial, p.ks, state);
+    const dim3 kr_grid((unsigned)((long long)B * H), (D * (D + 1) + sana::tc::KR_THREADS - 1) / sana::tc::KR_THREADS);
+    sana::tc::kr_reduce_tc<D><<<kr_grid, sana::tc::KR_THREADS, 0, s>>>(partial, p.ks, state);
     return launch_status("kr_reduce_tc");
+}
+
+template <int D, bool OUT_BF16>
+sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N, int H,
+                            const Plan& p, const float* state, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmO;
+    sana_la_status st;
+    if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
+    constexpr int smem = sana::tc::KaLayout<D, OUT_BF16>::SMEM_BYTES;
+    if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16>, smem, smem_set)) != SANA_LA_OK) return st;
+    sana::tc::ka_apply_tc<D, OUT_BF16><<<p.ka.q.grid, sana::tc::kThreads, smem, s>>>(tmQ, tmO, p.ka, state);
+    return launch_status("ka_apply_tc");
 }
 
 template <int D>
 sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, void* O,
                          sana_la_out_dtype od, float eps, cudaStream_t s) {
-    static std::atomic<uint64_t> smem_set_bf16{0}, smem_set_f32{0};
     Plan p = make_plan(B, N, H, D);
     p.ka.eps = eps;
     CUtensorMap tmQ;
     sana_la_status st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::KaLayout<D>::SMEM_BYTES;
-    if (od == SANA_LA_OUT_BF16) {
-        if ((st = ensure_smem(sana::tc::ka_apply_tc<D, true>, smem, smem_set_bf16)) != SANA_LA_OK) return st;
-        sana::tc::ka_apply_tc<D, true><<<p.ka.grid, sana::tc::kThreads, smem, s>>>(tmQ, p.ka, state, O);
-    } else {
-        if ((st = ensure_smem(sana::tc::ka_apply_tc<D, false>, smem, smem_set_f32)) != SANA_LA_OK) return st;
-        sana::tc::ka_apply_tc<D, false><<<p.ka.grid, sana::tc::kThreads, smem, s>>>(tmQ, p.ka, state, O);
-    }
-    return launch_status("ka_apply_tc");
+    return od == SANA_LA_OUT_BF16 ? launch_apply<D, true>(tmQ, O, B, N, H, p, state, s)
+                                  : launch_apply<D, false>(tmQ, O, B, N, H, p, state, s);
 }
 
 sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d,

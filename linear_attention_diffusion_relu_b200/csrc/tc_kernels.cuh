@@ -3,7 +3,7 @@
 // KS  ks_state_tc   partial states  phi(K)^T [V | 1]  on UMMA, fp32 in TMEM
 // KR  kr_reduce_tc  fixed-order sum of the partials of each (b, h)
 // KA  ka_apply_tc   phi(Q) S on UMMA (S split into bf16 hi + lo), then
-//                   O = num / (den + eps) in the epilogue
+//                   O = num / (den + eps) in the epilogue, stored by TMA
 //
 // The two contractions ("08_sana高效高分辨率生成", "Linear Attention 的原理":
 // KV = phi(K)^T V, A = phi(Q) KV; the normaliser of the normalised form in
@@ -18,10 +18,22 @@
 // of a token row. TMA moves one group row of a tile as two 128-byte-wide boxes
 // with the 128-byte swizzle.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warps 0-3  workers: phi on the staged tile, state staging (KA), epilogue
-//   warp  4    TMA producer (one lane)
-//   warp  5    UMMA issuer (one lane)
+// Warp roles (320 threads, one CTA per SM):
+//   warps 0-7  workers: phi on the staged tile, state staging (KA), epilogue;
+//              warps w and w+4 share TMEM lanes 32*(w%4).. and split the heads
+//   warp  8    TMA producer (one lane)
+//   warp  9    UMMA issuer (one lane)
+//
+// Schedule ("lockstep"): the B*groups (b, group) slabs are dealt out so that
+// the CTAs running at the same time read the same token rows of every group,
+// i.e. whole contiguous rows of Q, K and V, instead of 256-byte pieces of
+// unrelated rows; on B200 that raised the HBM throughput of both kernels by
+// 25-50 %. With S slabs and at most 148 CTAs:
+//   S <= 148: R = min(148 / S, tiles) CTAs share a slab; CTA c takes slab
+//             c % S and its tiles r, r + R, r + 2R, ... with r = c / S.
+//   S >  148: CTA c takes slabs c, c + 148, ... with all their tiles.
+// Each (CTA, slab) pair is one "segment"; KS writes one partial state per
+// segment and KR adds a slab's segments in ascending CTA order.
 // Every mbarrier wait is bounded; a wait that runs out sets an error code and
 // the whole CTA winds down (drains its TMA loads and UMMAs, frees TMEM).
 #pragma once
@@ -34,12 +46,14 @@
 namespace sana {
 namespace tc {
 
-constexpr int kWorkerThreads = 128;
+constexpr int kWorkerThreads = 256;
+constexpr int kWorkerWarps = kWorkerThreads / 32;
 constexpr int kThreads = kWorkerThreads + 64;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kProducerWarp = kWorkerWarps;
+constexpr int kMmaWarp = kWorkerWarps + 1;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytesRow = 128;            // one swizzled row of a box
+constexpr int kSmemLimit = 232448;           // dynamic shared memory per CTA on sm_100
 
 __device__ uint32_t g_device_error;          // first error code seen by any kernel
 
@@ -52,42 +66,76 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// phi on n16 16-byte chunks starting at base; thread t takes chunks t, t+128, ...
-__device__ __forceinline__ void relu_smem(uint8_t* base, int n16, int tid) {
-    for (int c = tid; c < n16; c += kWorkerThreads) {
-        uint4* p = reinterpret_cast<uint4*>(base + (size_t)c * 16);
-        uint4 v = *p;
-        v.x = relu_bf16x2(v.x);
-        v.y = relu_bf16x2(v.y);
-        v.z = relu_bf16x2(v.z);
-        v.w = relu_bf16x2(v.w);
-        *p = v;
+// phi on N16 16-byte chunks at base; worker t takes chunks t, t+128, ...
+// All loads are issued before the stores so they overlap.
+template <int N16>
+__device__ __forceinline__ void relu_smem(uint8_t* base, int tid) {
+    constexpr int PER = N16 / kWorkerThreads;
+    static_assert(N16 % kWorkerThreads == 0, "whole chunks per worker");
+    uint4 v[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) v[j] = *reinterpret_cast<const uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        v[j].x = relu_bf16x2(v[j].x);
+        v[j].y = relu_bf16x2(v[j].y);
+        v[j].z = relu_bf16x2(v[j].z);
+        v[j].w = relu_bf16x2(v[j].w);
+        *reinterpret_cast<uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16) = v[j];
     }
 }
 
-// ===================================================================== KS ===
-//
-// Work split: the (b, group) slabs are cut into 64-token tiles, numbered
-// t = bg * tiles_per_bg + tile. CTA c takes tiles [c*T/grid, (c+1)*T/grid);
-// each run of its tiles that belongs to one bg is a "segment" and yields one
-// partial state per head, at slot (c * max_seg + k) with k = bg - first bg of c.
-// The reduction kernel sums a bg's segments in ascending c, i.e. token order.
-struct KsParams {
-    int N, H, groups, tiles_per_bg, grid, max_seg;
-    long long total_tiles;
+// Bounded wait whose outcome is the same for every lane of the warp: if any
+// lane gives up, all do. Worker code paths stay warp-uniform this way, so a
+// wind-down never leaves part of a warp at a warp-synchronous instruction.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* err) {
+    const bool ok = ptx::mbar_wait(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// One arrival per worker warp (barriers are initialised with kWorkerWarps).
+// Each lane has already fenced its own writes; __syncwarp orders them before
+// lane 0's arrive, which releases them to the waiting thread.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
+}
+
+// =============================================================== schedule ===
+struct Sched {
+    int S;          // (b, group) slabs = B * groups
+    int T;          // tiles per slab
+    int R;          // CTAs sharing one slab (1 when S > grid)
+    int grid;       // CTAs
+    int max_seg;    // most slabs one CTA visits
 };
 
-__host__ __device__ __forceinline__ long long ks_tile_begin(long long c, const KsParams& p) {
-    return c * p.total_tiles / p.grid;
+// tiles per segment of CTA c
+__host__ __device__ __forceinline__ int sched_tps(int c, const Sched& q) {
+    const int r = c / q.S;
+    return (q.T - r + q.R - 1) / q.R;
+}
+// segments (slabs) of CTA c
+__host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
+    return (q.S - c % q.S + q.grid - 1) / q.grid;
+}
+// i-th tile of CTA c -> (slab, tile, segment index)
+__host__ __device__ __forceinline__ void sched_item(int c, int i, int tps, const Sched& q,
+                                                    int& slab, int& tile, int& seg) {
+    seg = i / tps;
+    slab = c % q.S + seg * q.grid;
+    tile = c / q.S + (i % tps) * q.R;
 }
 
-// the CTA whose range holds tile t
-__host__ __device__ __forceinline__ long long ks_cta_of(long long t, const KsParams& p) {
-    return ((t + 1) * p.grid - 1) / p.total_tiles;
-}
+// ===================================================================== KS ===
+struct KsParams {
+    int N, H, groups;
+    Sched q;
+};
 
 constexpr int KS_TILE = 64;                                // tokens per stage
-constexpr int KS_STAGES = 5;
+constexpr int KS_STAGES = 6;
 constexpr int KS_BOX_BYTES = KS_TILE * kBoxBytesRow;       // 8 KB
 constexpr int KS_STAGE_BYTES = 4 * KS_BOX_BYTES;           // K0 K1 V0 V1
 constexpr int KS_ONES_OFF = KS_STAGES * KS_STAGE_BYTES;
@@ -95,6 +143,7 @@ constexpr int KS_BAR_OFF = KS_ONES_OFF + 1024;
 constexpr int KS_NUM_BARS = 3 * KS_STAGES + 5;
 constexpr int KS_CTL_OFF = KS_BAR_OFF + KS_NUM_BARS * 8;
 constexpr int KS_SMEM_BYTES = KS_CTL_OFF + 64 + 1024;      // + alignment slack
+static_assert(KS_SMEM_BYTES <= kSmemLimit, "KS shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -119,19 +168,18 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const long long t_begin = ks_tile_begin(blockIdx.x, p);
-    const int ntiles = (int)(ks_tile_begin(blockIdx.x + 1, p) - t_begin);
-    const long long bg_first = t_begin / p.tiles_per_bg;
+    const int tps = sched_tps(blockIdx.x, p.q);
+    const int ntiles = tps * sched_nseg(blockIdx.x, p.q);
 
     if (tid == 0) {
         for (int s = 0; s < KS_STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
-            ptx::mbar_init(&relu_done[s], kWorkerThreads);
+            ptx::mbar_init(&relu_done[s], kWorkerWarps);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], kWorkerThreads);
+            ptx::mbar_init(&acc_empty[a], 4);           // the epilogue warps 0-3
         }
         ptx::mbar_init(mma_done, 1);
         ctl->abort = 0;
@@ -165,12 +213,10 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i % KS_STAGES;
                 if (!ptx::mbar_wait(&empty[s], ((i / KS_STAGES) & 1) ^ 1, abort, err)) break;
-                const long long t = t_begin + i;
-                const long long bg = t / p.tiles_per_bg;
-                const int tile = (int)(t % p.tiles_per_bg);
-                const int b = (int)(bg / p.groups);
-                const int g = (int)(bg % p.groups);
-                const int x0 = g * 128;
+                int slab, tile, seg;
+                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+                const int b = slab / p.groups;
+                const int x0 = (slab % p.groups) * 128;
                 const int y = tile * KS_TILE;
                 uint8_t* st = stage_ptr(s);
                 ptx::mbar_arrive_expect_tx(&full[s], KS_STAGE_BYTES);
@@ -193,12 +239,9 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 ptx::smem_desc(ptx::smem_u32(smem + KS_ONES_OFF), 256, 128, ptx::kLayoutNone);
             int seg = -1;
             bool first = true;
-            bool ok = true;
-            for (int i = 0; i < ntiles && ok; ++i) {
-                const long long t = t_begin + i;
-                const long long bg = t / p.tiles_per_bg;
-                const bool seg_start = (i == 0) || ((t - 1) / p.tiles_per_bg != bg);
-                const bool seg_end = (i == ntiles - 1) || ((t + 1) / p.tiles_per_bg != bg);
+            for (int i = 0; i < ntiles; ++i) {
+                const bool seg_start = (i % tps) == 0;
+                const bool seg_end = (i % tps) == tps - 1;
                 if (seg_start) {
                     ++seg;
                     if (!ptx::mbar_wait(&acc_empty[seg & 1], ((seg >> 1) & 1) ^ 1, abort, err)) break;
@@ -231,21 +274,19 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         }
     } else {
         // --------------------------------------------------------- workers ----
-        int seg = -1;
         for (int i = 0; i < ntiles; ++i) {
-            const long long t = t_begin + i;
-            const long long bg = t / p.tiles_per_bg;
-            const bool seg_end = (i == ntiles - 1) || ((t + 1) / p.tiles_per_bg != bg);
-            if (i == 0 || (t - 1) / p.tiles_per_bg != bg) ++seg;
+            const bool seg_end = (i % tps) == tps - 1;
+            const int seg = i / tps;
             const int s = i % KS_STAGES;
-            if (!ptx::mbar_wait(&full[s], (i / KS_STAGES) & 1, abort, err)) break;
-            relu_smem(stage_ptr(s), 2 * KS_BOX_BYTES / 16, tid);      // phi on the K boxes only
+            if (!warp_wait(&full[s], (i / KS_STAGES) & 1, abort, err)) break;
+            relu_smem<2 * KS_BOX_BYTES / 16>(stage_ptr(s), tid);     // phi on the K boxes only
             ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&relu_done[s]);
-            if (seg_end) {
-                // epilogue: this segment's partial states, TMEM -> workspace
+            warp_arrive(&relu_done[s]);
+            if (seg_end && warp < 4) {
+                // epilogue (warps 0-3, one per TMEM lane quarter): this segment's
+                // partial states, TMEM -> workspace
                 const int buf = seg & 1;
-                if (!ptx::mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort, err)) break;
+                if (!warp_wait(&acc_full[buf], (seg >> 1) & 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const int hh = warp / (D / 32);                  // head within the group
                 const int row = (warp % (D / 32)) * 32 + lane;   // state row i of that head
@@ -254,11 +295,12 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 __syncwarp();
                 ptx::tmem_ld_row<D>(lane_addr + hh * D, lane_addr + 128, v, &nrm);
                 ptx::tc_fence_before_sync();
-                ptx::mbar_arrive(&acc_empty[buf]);
-                const int g = (int)(bg % p.groups);
-                const int h = g * G + hh;
+                warp_arrive(&acc_empty[buf]);
+                int slab, tile, sg;
+                sched_item(blockIdx.x, i, tps, p.q, slab, tile, sg);
+                const int h = (slab % p.groups) * G + hh;
                 if (h < p.H) {
-                    const long long slot = ((long long)blockIdx.x * p.max_seg + (bg - bg_first)) * G + hh;
+                    const long long slot = ((long long)blockIdx.x * p.q.max_seg + seg) * G + hh;
                     float* P = partial + slot * DD + (long long)row * (D + 1);
 #pragma unroll
                     for (int j = 0; j < D; ++j) P[j] = v[j];
@@ -278,103 +320,123 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
 }
 
 // ===================================================================== KR ===
+// One thread per state entry (grid: (b, h) x entry blocks), so every load is
+// independent and the kernel costs about one L2 round trip. The segments of a
+// slab are added in ascending CTA order: the partial of CTA c = (slab % grid)
+// + r * S, segment slab / grid, for r = 0 .. R-1.
+constexpr int KR_THREADS = 128;
+
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(KR_THREADS)
 kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restrict__ state)
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
+    const int e = blockIdx.y * KR_THREADS + threadIdx.x;
+    if (e >= DD) return;
     const long long bh = blockIdx.x;
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
-    const int hh = h % G;
-    const long long bg = (long long)b * p.groups + h / G;
-    const long long c_lo = ks_cta_of(bg * p.tiles_per_bg, p);
-    const long long c_hi = ks_cta_of(bg * p.tiles_per_bg + p.tiles_per_bg - 1, p);
-    for (int e = threadIdx.x; e < DD; e += blockDim.x) {
-        float s = 0.0f;
-        for (long long c = c_lo; c <= c_hi; ++c) {
-            const long long k = bg - ks_tile_begin(c, p) / p.tiles_per_bg;
-            s += partial[((c * p.max_seg + k) * G + hh) * DD + e];
-        }
-        state[bh * DD + e] = s;
-    }
+    const int slab = b * p.groups + h / G;
+    const int seg = slab / p.q.grid;
+    const int c0 = slab % p.q.grid;
+    const float* src = partial + (((long long)c0 * p.q.max_seg + seg) * G + h % G) * DD + e;
+    const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
+    float s = 0.0f;
+    for (int r = 0; r < p.q.R; ++r) s += src[r * step];
+    state[bh * DD + e] = s;
 }
 
 // ===================================================================== KA ===
 //
-// Unit = (b, group, 128-token tile), numbered u = bg * tiles_per_bg + tile;
-// CTA c takes units [c*U/grid, (c+1)*U/grid).
+// Unit = one 128-token tile of a (b, group) slab, dealt out by the lockstep
+// schedule above.
 struct KaParams {
-    int N, H, groups, tiles_per_bg, grid;
-    long long total_units;
+    int N, H, groups;
+    Sched q;
     float eps;
 };
 
 constexpr int KA_TILE = 128;                               // tokens = UMMA M
-constexpr int KA_STAGES = 4;
 constexpr int KA_BOX_BYTES = KA_TILE * kBoxBytesRow;       // 16 KB
 constexpr int KA_STAGE_BYTES = 2 * KA_BOX_BYTES;           // one group row of 128 tokens
 
-template <int D>
+template <int D, bool OUT_BF16>
 struct KaLayout {
     static constexpr int G = 128 / D;
     static constexpr int NA = D + 16;                      // UMMA N: d numerator cols + normaliser + pad
     static constexpr int SBO = (D / 8) * 128;              // 8-row group stride of the K-major state
     static constexpr int MAT_BYTES = (NA / 8) * SBO;       // one bf16 NA x D matrix
     static constexpr int STATE_BUF_BYTES = G * 2 * MAT_BYTES;   // hi and lo for every head
-    static constexpr int STATE_OFF = KA_STAGES * KA_STAGE_BYTES;
-    static constexpr int BAR_OFF = STATE_OFF + 2 * STATE_BUF_BYTES;
-    static constexpr int NUM_BARS = 3 * KA_STAGES + 5;
+    static constexpr int OUT_BYTES = OUT_BF16 ? 2 : 4;
+    static constexpr int OUT_BOXES = 128 * OUT_BYTES / kBoxBytesRow;   // boxes per output group row
+    static constexpr int OUT_BOX_ELEMS = kBoxBytesRow / OUT_BYTES;
+    static constexpr int STAGING_BYTES = OUT_BOXES * KA_BOX_BYTES;
+    // One state buffer (a CTA keeps its group unless there are more slabs
+    // than CTAs) and as many Q stages as fit next to it and the staging tile.
+    static constexpr int STATE_BUFS = 1;
+    static constexpr int STAGES = (kSmemLimit - 4096 - STATE_BUF_BYTES - STAGING_BYTES) / KA_STAGE_BYTES > 6
+                                      ? 6 : (kSmemLimit - 4096 - STATE_BUF_BYTES - STAGING_BYTES) / KA_STAGE_BYTES;
+    static constexpr int STATE_OFF = STAGES * KA_STAGE_BYTES;
+    static constexpr int STAGING_OFF = STATE_OFF + STATE_BUFS * STATE_BUF_BYTES;
+    static constexpr int BAR_OFF = STAGING_OFF + STAGING_BYTES;
+    static constexpr int NUM_BARS = 3 * STAGES + 7;
     static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = CTL_OFF + 64 + 1024;
     static constexpr int ACC_COLS = 256 / G;               // TMEM columns per head
+    static_assert(SMEM_BYTES <= kSmemLimit, "KA shared memory");
 };
 
 // element (n, k) of a K-major, unswizzled bf16 matrix made of 8x8 core matrices
-template <int D>
+template <int SBO>
 __device__ __forceinline__ int state_off(int n, int k) {
-    return (n >> 3) * KaLayout<D>::SBO + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+    return (n >> 3) * SBO + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
 }
 
 template <int D, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const KaParams p,
-            const float* __restrict__ state, void* __restrict__ O)
+ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+            const KaParams p, const float* __restrict__ state)
 {
-    using L = KaLayout<D>;
+    using L = KaLayout<D, OUT_BF16>;
     constexpr int G = L::G;
     constexpr int DD = D * (D + 1);
+    constexpr int S = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* full = bars;
-    uint64_t* empty = bars + KA_STAGES;
-    uint64_t* relu_done = bars + 2 * KA_STAGES;
-    uint64_t* acc_full = bars + 3 * KA_STAGES;
+    uint64_t* empty = bars + S;
+    uint64_t* relu_done = bars + 2 * S;
+    uint64_t* acc_full = bars + 3 * S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* mma_done = acc_full + 4;
+    uint64_t* stg_free = acc_full + 5;      // staging tile may be rewritten
+    uint64_t* stg_full = acc_full + 6;      // staging tile written by every worker warp
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + L::CTL_OFF);
     volatile int* abort = &ctl->abort;
     uint32_t* err = &g_device_error;
+    uint8_t* staging = smem + L::STAGING_OFF;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const long long u_begin = (long long)blockIdx.x * p.total_units / p.grid;
-    const int nunits = (int)((long long)(blockIdx.x + 1) * p.total_units / p.grid - u_begin);
+    const int tps = sched_tps(blockIdx.x, p.q);
+    const int nunits = tps * sched_nseg(blockIdx.x, p.q);
 
     if (tid == 0) {
-        for (int s = 0; s < KA_STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
-            ptx::mbar_init(&relu_done[s], kWorkerThreads);
+            ptx::mbar_init(&relu_done[s], kWorkerWarps);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], kWorkerThreads);
+            ptx::mbar_init(&acc_empty[a], kWorkerWarps);
         }
         ptx::mbar_init(mma_done, 1);
+        ptx::mbar_init(stg_free, 1);
+        ptx::mbar_init(stg_full, kWorkerWarps);
         ctl->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -382,15 +444,19 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const KaParams p,
         ptx::tmem_alloc(&ctl->tmem_base, kTmemCols);
         ptx::tmem_relinquish();
     }
-    if (warp == kProducerWarp && lane == 0) ptx::prefetch_tmap(&tmQ);
-    // padding columns n in (d, NA) of both state buffers are zero for good
+    if (warp == kProducerWarp && lane == 0) {
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmO);
+    }
+    // padding columns n in (d, NA) of every state buffer are zero for good
     if (tid < kWorkerThreads) {
-        for (int e = tid; e < 2 * G * 2 * (L::NA - D - 1) * D; e += kWorkerThreads) {
+        constexpr int PAD = L::NA - D - 1;
+        for (int e = tid; e < L::STATE_BUFS * G * 2 * PAD * D; e += kWorkerThreads) {
             const int k = e % D;
-            const int n = D + 1 + (e / D) % (L::NA - D - 1);
-            const int mat = e / (D * (L::NA - D - 1));
+            const int n = D + 1 + (e / D) % PAD;
+            const int mat = e / (D * PAD);
             *reinterpret_cast<__nv_bfloat16*>(smem + L::STATE_OFF + mat * L::MAT_BYTES +
-                                              state_off<D>(n, k)) = __float2bfloat16_rn(0.0f);
+                                              state_off<L::SBO>(n, k)) = __float2bfloat16_rn(0.0f);
         }
     }
     ptx::tc_fence_before_sync();
@@ -399,44 +465,40 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const KaParams p,
     const uint32_t tmem = ctl->tmem_base;
 
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KA_STAGE_BYTES; };
-    auto state_buf = [&](int sb) { return smem + L::STATE_OFF + sb * L::STATE_BUF_BYTES; };
+    auto state_buf = [&](int sb) { return smem + L::STATE_OFF + (sb % L::STATE_BUFS) * L::STATE_BUF_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int issued = 0;
             for (int i = 0; i < nunits; ++i) {
-                const int s = i % KA_STAGES;
-                if (!ptx::mbar_wait(&empty[s], ((i / KA_STAGES) & 1) ^ 1, abort, err)) break;
-                const long long u = u_begin + i;
-                const long long bg = u / p.tiles_per_bg;
-                const int tile = (int)(u % p.tiles_per_bg);
-                const int b = (int)(bg / p.groups);
-                const int x0 = (int)(bg % p.groups) * 128;
+                const int s = i % S;
+                if (!ptx::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, abort, err)) break;
+                int slab, tile, seg;
+                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+                const int b = slab / p.groups;
+                const int x0 = (slab % p.groups) * 128;
                 ptx::mbar_arrive_expect_tx(&full[s], KA_STAGE_BYTES);
                 ptx::tma_load_3d(stage_ptr(s), &tmQ, &full[s], x0, tile * KA_TILE, b);
                 ptx::tma_load_3d(stage_ptr(s) + KA_BOX_BYTES, &tmQ, &full[s], x0 + 64, tile * KA_TILE, b);
                 issued = i + 1;
             }
-            for (int i = (issued > KA_STAGES ? issued - KA_STAGES : 0); i < issued; ++i)
-                ptx::mbar_wait(&full[i % KA_STAGES], (i / KA_STAGES) & 1, nullptr, err);
+            for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+                ptx::mbar_wait(&full[i % S], (i / S) & 1, nullptr, err);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- UMMA issuer ----
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, L::NA, 0, 0);
-            int sb = -1;
             for (int i = 0; i < nunits; ++i) {
-                const long long u = u_begin + i;
-                const long long bg = u / p.tiles_per_bg;
-                if (i == 0 || (u - 1) / p.tiles_per_bg != bg) ++sb;
-                const int s = i % KA_STAGES;
+                const int sb = i / tps;                  // state buffer use count = segment
+                const int s = i % S;
                 const int buf = i & 1;
-                if (!ptx::mbar_wait(&relu_done[s], (i / KA_STAGES) & 1, abort, err)) break;
+                if (!ptx::mbar_wait(&relu_done[s], (i / S) & 1, abort, err)) break;
                 if (!ptx::mbar_wait(&acc_empty[buf], ((i >> 1) & 1) ^ 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const uint32_t a_base = ptx::smem_u32(stage_ptr(s));
-                const uint32_t s_base = ptx::smem_u32(state_buf(sb & 1));
+                const uint32_t s_base = ptx::smem_u32(state_buf(sb));
 #pragma unroll
                 for (int hh = 0; hh < G; ++hh) {
                     const uint32_t d_tmem = tmem + (uint32_t)buf * 256u + (uint32_t)(hh * L::ACC_COLS);
@@ -461,16 +523,19 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const KaParams p,
         }
     } else {
         // --------------------------------------------------------- workers ----
-        int sb = -1;
-        // stage unit i: (new state group ->) state hi/lo staging, then phi on the Q tile
+        // stage unit i: (new segment ->) state hi/lo staging, then phi on the Q tile
         auto prep = [&](int i) -> bool {
-            const long long u = u_begin + i;
-            const long long bg = u / p.tiles_per_bg;
-            if (i == 0 || (u - 1) / p.tiles_per_bg != bg) {
-                ++sb;
-                uint8_t* dst = state_buf(sb & 1);
-                const int b = (int)(bg / p.groups);
-                const int g = (int)(bg % p.groups);
+            if (i % tps == 0) {
+                const int sb = i / tps;
+                if (L::STATE_BUFS == 1 && i > 0) {
+                    // one buffer: the previous unit's UMMAs must be done reading it
+                    if (!warp_wait(&acc_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, err)) return false;
+                }
+                uint8_t* dst = state_buf(sb);
+                int slab, tile, seg;
+                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+                const int b = slab / p.groups;
+                const int g = slab % p.groups;
                 for (int hh = 0; hh < G; ++hh) {
                     const int h = g * G + hh;
                     const float* src = state + ((long long)b * p.H + h) * DD;
@@ -482,70 +547,87 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const KaParams p,
                         const float v = (h < p.H) ? src[e] : 0.0f;
                         const __nv_bfloat16 vh = __float2bfloat16_rn(v);
                         const __nv_bfloat16 vl = __float2bfloat16_rn(v - __bfloat162float(vh));
-                        *reinterpret_cast<__nv_bfloat16*>(mhi + state_off<D>(n, k)) = vh;
-                        *reinterpret_cast<__nv_bfloat16*>(mlo + state_off<D>(n, k)) = vl;
+                        *reinterpret_cast<__nv_bfloat16*>(mhi + state_off<L::SBO>(n, k)) = vh;
+                        *reinterpret_cast<__nv_bfloat16*>(mlo + state_off<L::SBO>(n, k)) = vl;
                     }
                 }
             }
-            const int s = i % KA_STAGES;
-            if (!ptx::mbar_wait(&full[s], (i / KA_STAGES) & 1, abort, err)) return false;
-            relu_smem(stage_ptr(s), KA_STAGE_BYTES / 16, tid);
+            const int s = i % S;
+            if (!warp_wait(&full[s], (i / S) & 1, abort, err)) return false;
+            relu_smem<KA_STAGE_BYTES / 16>(stage_ptr(s), tid);
             ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&relu_done[s]);
+            warp_arrive(&relu_done[s]);
             return true;
         };
+        const int m = (warp & 3) * 32 + lane;                // token row of the tile = TMEM lane
+        constexpr int HPW = G / 2;                           // heads per worker warp
+        const int hh0 = (warp >> 2) * HPW;
         bool ok = nunits > 0 ? prep(0) : true;
         for (int i = 0; i < nunits && ok; ++i) {
             if (i + 1 < nunits && !prep(i + 1)) break;
             // epilogue of unit i
             const int buf = i & 1;
-            if (!ptx::mbar_wait(&acc_full[buf], (i >> 1) & 1, abort, err)) break;
+            if (!warp_wait(&acc_full[buf], (i >> 1) & 1, abort, err)) break;
             ptx::tc_fence_after_sync();
-            const long long u = u_begin + i;
-            const long long bg = u / p.tiles_per_bg;
-            const int tile = (int)(u % p.tiles_per_bg);
-            const int b = (int)(bg / p.groups);
-            const int g = (int)(bg % p.groups);
-            const long long n = (long long)tile * KA_TILE + warp * 32 + lane;
-            const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)buf * 256u;
+            int slab, tile, seg;
+            sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+            const int b = slab / p.groups;
+            const int g = slab % p.groups;
+            // the previous unit's TMA store must have finished reading the staging tile
+            if (tid == 0) {
+                ptx::bulk_wait_group_read<0>();
+                ptx::mbar_arrive(stg_free);
+            }
+            if (!warp_wait(stg_free, i & 1, abort, err)) break;
+            const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)buf * 256u;
 #pragma unroll 1
-            for (int hh = 0; hh < G; ++hh) {
+            for (int hh = hh0; hh < hh0 + HPW; ++hh) {
                 float num[D], den;
                 __syncwarp();
                 ptx::tmem_ld_row<D>(lane_addr + hh * L::ACC_COLS, lane_addr + hh * L::ACC_COLS + D,
                                     num, &den);
-                const int h = g * G + hh;
-                if (n < p.N && h < p.H) {
-                    const float r = 1.0f / (den + p.eps);
-                    const long long off = (((long long)b * p.N + n) * p.H + h) * D;
+                const float r = 1.0f / (den + p.eps);
+                // row m of the staging tile, 128-byte swizzle: chunk q lands at q ^ (m % 8)
+#pragma unroll
+                for (int j = 0; j < D; j += 16 / L::OUT_BYTES) {
+                    const int f = (hh * D + j) * L::OUT_BYTES;        // byte offset in the group row
+                    uint4 w;
                     if (OUT_BF16) {
-                        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(O) + off;
-#pragma unroll
-                        for (int j = 0; j < D; j += 8) {
-                            uint4 w;
-                            w.x = float2_to_bf16x2(num[j + 0] * r, num[j + 1] * r);
-                            w.y = float2_to_bf16x2(num[j + 2] * r, num[j + 3] * r);
-                            w.z = float2_to_bf16x2(num[j + 4] * r, num[j + 5] * r);
-                            w.w = float2_to_bf16x2(num[j + 6] * r, num[j + 7] * r);
-                            stg_stream(o + j, w);
-                        }
+                        w.x = float2_to_bf16x2(num[j + 0] * r, num[j + 1] * r);
+                        w.y = float2_to_bf16x2(num[j + 2] * r, num[j + 3] * r);
+                        w.z = float2_to_bf16x2(num[j + 4] * r, num[j + 5] * r);
+                        w.w = float2_to_bf16x2(num[j + 6] * r, num[j + 7] * r);
                     } else {
-                        float* o = reinterpret_cast<float*>(O) + off;
-#pragma unroll
-                        for (int j = 0; j < D; j += 4) {
-                            uint4 w;
-                            w.x = __float_as_uint(num[j + 0] * r);
-                            w.y = __float_as_uint(num[j + 1] * r);
-                            w.z = __float_as_uint(num[j + 2] * r);
-                            w.w = __float_as_uint(num[j + 3] * r);
-                            stg_stream(o + j, w);
-                        }
+                        w.x = __float_as_uint(num[j + 0] * r);
+                        w.y = __float_as_uint(num[j + 1] * r);
+                        w.z = __float_as_uint(num[j + 2] * r);
+                        w.w = __float_as_uint(num[j + 3] * r);
                     }
+                    const int box = f / kBoxBytesRow;
+                    const int q = (f % kBoxBytesRow) / 16;
+                    *reinterpret_cast<uint4*>(staging + box * KA_BOX_BYTES + m * kBoxBytesRow +
+                                              ((q ^ (m & 7)) * 16)) = w;
                 }
             }
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(&acc_empty[buf]);
+            warp_arrive(&acc_empty[buf]);
+            ptx::fence_proxy_async_smem();
+            warp_arrive(stg_full);
+            if (warp == 0) {
+                if (!warp_wait(stg_full, i & 1, abort, err)) break;
+                if (lane == 0) {
+                    const int x0 = g * 128;
+                    const int y = tile * KA_TILE;
+#pragma unroll
+                    for (int bx = 0; bx < L::OUT_BOXES; ++bx) {
+                        const int x = x0 + bx * L::OUT_BOX_ELEMS;
+                        if (x < p.H * D) ptx::tma_store_3d(&tmO, staging + bx * KA_BOX_BYTES, x, y, b);
+                    }
+                    ptx::bulk_commit_group();
+                }
+            }
         }
+        if (tid == 0) ptx::bulk_wait_group<0>();
     }
 
     ptx::tc_fence_before_sync();
