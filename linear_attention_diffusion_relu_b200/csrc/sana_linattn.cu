@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include <cudaTypedefs.h>
 
@@ -145,6 +146,31 @@ sana_la_status make_tmap(CUtensorMap* m, const void* base, int B, int N, int H, 
     return SANA_LA_OK;
 }
 
+// Launch on `s`; with `overlap` the kernel may start before the preceding
+// kernel of the stream has finished (programmatic stream serialization). Only
+// kernels that wait with griddepcontrol.wait before reading that kernel's
+// results, and whose other inputs were ready before it started, use it.
+template <typename... KArgs, typename... Args>
+sana_la_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      bool overlap, const char* name, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e != cudaSuccess) {
+        set_last_error(name, e);
+        return SANA_LA_ERR_CUDA;
+    }
+    return launch_status(name);
+}
+
 // Opt a kernel into its dynamic shared memory size, once per device.
 template <typename Kernel>
 sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
@@ -176,37 +202,41 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KS_SMEM_BYTES, smem_set)) != SANA_LA_OK)
         return st;
-    sana::tc::ks_state_tc<D><<<p.ks.q.grid, sana::tc::kThreads, sana::tc::KS_SMEM_BYTES, s>>>(
-        tmK, tmV, p.ks, partial);
-    if ((st = launch_status("ks_state_tc")) != SANA_LA_OK) return st;
+    if ((st = launch(sana::tc::ks_state_tc<D>, dim3(p.ks.q.grid), dim3(sana::tc::kThreads),
+                     sana::tc::KS_SMEM_BYTES, s, false, "ks_state_tc", tmK, tmV, p.ks, partial)) != SANA_LA_OK)
+        return st;
+    // the reduction overlaps the state kernel's tail; it waits for its results
     const dim3 kr_grid((unsigned)((long long)B * H), (D * (D + 1) + sana::tc::KR_THREADS - 1) / sana::tc::KR_THREADS);
-    sana::tc::kr_reduce_tc<D><<<kr_grid, sana::tc::KR_THREADS, 0, s>>>(partial, p.ks, state);
-    return launch_status("kr_reduce_tc");
+    return launch(sana::tc::kr_reduce_tc<D>, kr_grid, dim3(sana::tc::KR_THREADS), 0, s, true, "kr_reduce_tc",
+                  (const float*)partial, p.ks, state);
 }
 
 template <int D, bool OUT_BF16>
 sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N, int H,
-                            const Plan& p, const float* state, cudaStream_t s) {
+                            const Plan& p, const float* state, cudaStream_t s, bool overlap) {
     static std::atomic<uint64_t> smem_set{0};
     CUtensorMap tmO;
     sana_la_status st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
     constexpr int smem = sana::tc::KaLayout<D, OUT_BF16>::SMEM_BYTES;
     if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16>, smem, smem_set)) != SANA_LA_OK) return st;
-    sana::tc::ka_apply_tc<D, OUT_BF16><<<p.ka.q.grid, sana::tc::kThreads, smem, s>>>(tmQ, tmO, p.ka, state);
-    return launch_status("ka_apply_tc");
+    return launch(sana::tc::ka_apply_tc<D, OUT_BF16>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
+                  overlap, "ka_apply_tc", tmQ, tmO, p.ka, state);
 }
 
+// `overlap`: called right after this library's own state kernels on the same
+// stream (forward), so Q was ready before they started and the apply kernel
+// may start early; a standalone apply waits for everything before it.
 template <int D>
 sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, void* O,
-                         sana_la_out_dtype od, float eps, cudaStream_t s) {
+                         sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
     Plan p = make_plan(B, N, H, D);
     p.ka.eps = eps;
     CUtensorMap tmQ;
     sana_la_status st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
-    return od == SANA_LA_OUT_BF16 ? launch_apply<D, true>(tmQ, O, B, N, H, p, state, s)
-                                  : launch_apply<D, false>(tmQ, O, B, N, H, p, state, s);
+    return od == SANA_LA_OUT_BF16 ? launch_apply<D, true>(tmQ, O, B, N, H, p, state, s, overlap)
+                                  : launch_apply<D, false>(tmQ, O, B, N, H, p, state, s, overlap);
 }
 
 sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d,
@@ -221,9 +251,9 @@ sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, 
 }
 
 sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d,
-                          void* O, sana_la_out_dtype od, float eps, cudaStream_t s) {
-    return d == 32 ? run_apply<32>(Q, state, B, N, H, O, od, eps, s)
-                   : run_apply<64>(Q, state, B, N, H, O, od, eps, s);
+                          void* O, sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
+    return d == 32 ? run_apply<32>(Q, state, B, N, H, O, od, eps, s, overlap)
+                   : run_apply<64>(Q, state, B, N, H, O, od, eps, s, overlap);
 }
 
 }  // namespace
@@ -260,7 +290,7 @@ sana_la_status sana_linattn_apply(const void* Q, const float* state, int B, int 
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(Q) || !aligned16(state) || !aligned16(O)) return SANA_LA_ERR_INVALID_ARG;
     return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps,
-                      reinterpret_cast<cudaStream_t>(stream));
+                      reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
@@ -282,7 +312,7 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = kv_state_impl(K, V, B, N, H, d, state, workspace, workspace_bytes, s, true);
     if (st != SANA_LA_OK) return st;
-    return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps, s);
+    return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps, s, true);
 }
 
 int sana_linattn_forward_launches(int B, int N, int H, int d) {

@@ -203,6 +203,8 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
+    // the reduction kernel may be scheduled now; it waits for this grid's results
+    if (tid == 0) ptx::launch_dependents();
 
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KS_STAGE_BYTES; };
 
@@ -332,6 +334,11 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
+    // The apply kernel of a forward pass may be scheduled now: its Q loads only
+    // need ks_state_tc to have started, and it waits for this grid before
+    // reading the state.
+    ptx::launch_dependents();
+    ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
     const int e = blockIdx.y * KR_THREADS + threadIdx.x;
     if (e >= DD) return;
     const long long bh = blockIdx.x;
@@ -350,7 +357,17 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 // ===================================================================== KA ===
 //
 // Unit = one 128-token tile of a (b, group) slab, dealt out by the lockstep
-// schedule above.
+// schedule above. Per unit:
+//   producer  TMA: the Q tile (128 tokens x one group row) into a stage
+//   workers   read their token row from the stage, apply phi in registers and
+//             store it into TMEM as the UMMA A operand (the stage is free
+//             again as soon as it is read)
+//   UMMA      per head: D = phi(Q) S_hi + phi(Q) S_lo (A from TMEM, the
+//             state in shared memory as bf16 hi and lo parts)
+//   workers   D -> registers, O = num / (den + eps), into a swizzled staging
+//             tile, written to global memory by a TMA store
+// TMEM: the accumulator at columns [0, 256) (head h at h * 256/G) and two A
+// buffers of 64 columns at 256 and 320.
 struct KaParams {
     int N, H, groups;
     Sched q;
@@ -360,6 +377,7 @@ struct KaParams {
 constexpr int KA_TILE = 128;                               // tokens = UMMA M
 constexpr int KA_BOX_BYTES = KA_TILE * kBoxBytesRow;       // 16 KB
 constexpr int KA_STAGE_BYTES = 2 * KA_BOX_BYTES;           // one group row of 128 tokens
+constexpr uint32_t KA_A_COL = 256;                         // first A buffer column
 
 template <int D, bool OUT_BF16>
 struct KaLayout {
@@ -367,23 +385,24 @@ struct KaLayout {
     static constexpr int NA = D + 16;                      // UMMA N: d numerator cols + normaliser + pad
     static constexpr int SBO = (D / 8) * 128;              // 8-row group stride of the K-major state
     static constexpr int MAT_BYTES = (NA / 8) * SBO;       // one bf16 NA x D matrix
-    static constexpr int STATE_BUF_BYTES = G * 2 * MAT_BYTES;   // hi and lo for every head
+    static constexpr int STATE_BYTES = G * 2 * MAT_BYTES;  // hi and lo for every head
     static constexpr int OUT_BYTES = OUT_BF16 ? 2 : 4;
     static constexpr int OUT_BOXES = 128 * OUT_BYTES / kBoxBytesRow;   // boxes per output group row
     static constexpr int OUT_BOX_ELEMS = kBoxBytesRow / OUT_BYTES;
-    static constexpr int STAGING_BYTES = OUT_BOXES * KA_BOX_BYTES;
-    // One state buffer (a CTA keeps its group unless there are more slabs
-    // than CTAs) and as many Q stages as fit next to it and the staging tile.
-    static constexpr int STATE_BUFS = 1;
-    static constexpr int STAGES = (kSmemLimit - 4096 - STATE_BUF_BYTES - STAGING_BYTES) / KA_STAGE_BYTES > 6
-                                      ? 6 : (kSmemLimit - 4096 - STATE_BUF_BYTES - STAGING_BYTES) / KA_STAGE_BYTES;
+    static constexpr int STG_BYTES = OUT_BOXES * KA_BOX_BYTES;
+    static constexpr int AVAIL = kSmemLimit - 4096 - STATE_BYTES;
+    // two staging tiles if that still leaves four Q stages, else one
+    static constexpr int STG_BUFS = (AVAIL - 2 * STG_BYTES) / KA_STAGE_BYTES >= 4 ? 2 : 1;
+    static constexpr int STAGES_FIT = (AVAIL - STG_BUFS * STG_BYTES) / KA_STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
     static constexpr int STATE_OFF = STAGES * KA_STAGE_BYTES;
-    static constexpr int STAGING_OFF = STATE_OFF + STATE_BUFS * STATE_BUF_BYTES;
-    static constexpr int BAR_OFF = STAGING_OFF + STAGING_BYTES;
-    static constexpr int NUM_BARS = 3 * STAGES + 7;
+    static constexpr int STG_OFF = STATE_OFF + STATE_BYTES;
+    static constexpr int BAR_OFF = STG_OFF + STG_BUFS * STG_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 9;
     static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = CTL_OFF + 64 + 1024;
     static constexpr int ACC_COLS = 256 / G;               // TMEM columns per head
+    static_assert(STAGES >= 3, "KA needs at least three Q stages");
     static_assert(SMEM_BYTES <= kSmemLimit, "KA shared memory");
 };
 
@@ -405,18 +424,18 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + S;
-    uint64_t* relu_done = bars + 2 * S;
-    uint64_t* acc_full = bars + 3 * S;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* mma_done = acc_full + 4;
-    uint64_t* stg_free = acc_full + 5;      // staging tile may be rewritten
-    uint64_t* stg_full = acc_full + 6;      // staging tile written by every worker warp
+    uint64_t* full = bars;                  // [S] Q tile landed
+    uint64_t* empty = bars + S;             // [S] Q tile read by every worker warp
+    uint64_t* a_full = bars + 2 * S;        // [2] A operand in TMEM
+    uint64_t* acc_full = a_full + 2;        // UMMAs of a unit done
+    uint64_t* acc_empty = a_full + 3;       // accumulator read by every worker warp
+    uint64_t* stg_free = a_full + 4;        // staging tile of this unit may be written
+    uint64_t* stg_full = a_full + 5;        // [2] staging tile written by every worker warp
+    uint64_t* mma_done = a_full + 7;
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + L::CTL_OFF);
     volatile int* abort = &ctl->abort;
     uint32_t* err = &g_device_error;
-    uint8_t* staging = smem + L::STAGING_OFF;
+    uint8_t* sstate = smem + L::STATE_OFF;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -427,16 +446,16 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 1);
-            ptx::mbar_init(&relu_done[s], kWorkerWarps);
+            ptx::mbar_init(&empty[s], kWorkerWarps);
         }
-        for (int a = 0; a < 2; ++a) {
-            ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], kWorkerWarps);
-        }
-        ptx::mbar_init(mma_done, 1);
+        ptx::mbar_init(&a_full[0], kWorkerWarps);
+        ptx::mbar_init(&a_full[1], kWorkerWarps);
+        ptx::mbar_init(acc_full, 1);
+        ptx::mbar_init(acc_empty, kWorkerWarps);
         ptx::mbar_init(stg_free, 1);
-        ptx::mbar_init(stg_full, kWorkerWarps);
+        ptx::mbar_init(&stg_full[0], kWorkerWarps);
+        ptx::mbar_init(&stg_full[1], kWorkerWarps);
+        ptx::mbar_init(mma_done, 1);
         ctl->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -448,15 +467,15 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         ptx::prefetch_tmap(&tmQ);
         ptx::prefetch_tmap(&tmO);
     }
-    // padding columns n in (d, NA) of every state buffer are zero for good
+    // padding columns n in (d, NA) of the state are zero for good
     if (tid < kWorkerThreads) {
         constexpr int PAD = L::NA - D - 1;
-        for (int e = tid; e < L::STATE_BUFS * G * 2 * PAD * D; e += kWorkerThreads) {
+        for (int e = tid; e < G * 2 * PAD * D; e += kWorkerThreads) {
             const int k = e % D;
             const int n = D + 1 + (e / D) % PAD;
             const int mat = e / (D * PAD);
-            *reinterpret_cast<__nv_bfloat16*>(smem + L::STATE_OFF + mat * L::MAT_BYTES +
-                                              state_off<L::SBO>(n, k)) = __float2bfloat16_rn(0.0f);
+            *reinterpret_cast<__nv_bfloat16*>(sstate + mat * L::MAT_BYTES + state_off<L::SBO>(n, k)) =
+                __float2bfloat16_rn(0.0f);
         }
     }
     ptx::tc_fence_before_sync();
@@ -465,7 +484,6 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const uint32_t tmem = ctl->tmem_base;
 
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KA_STAGE_BYTES; };
-    auto state_buf = [&](int sb) { return smem + L::STATE_OFF + (sb % L::STATE_BUFS) * L::STATE_BUF_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
@@ -490,48 +508,53 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         // ---------------------------------------------------- UMMA issuer ----
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, L::NA, 0, 0);
+            const uint32_t s_base = ptx::smem_u32(sstate);
             for (int i = 0; i < nunits; ++i) {
-                const int sb = i / tps;                  // state buffer use count = segment
-                const int s = i % S;
-                const int buf = i & 1;
-                if (!ptx::mbar_wait(&relu_done[s], (i / S) & 1, abort, err)) break;
-                if (!ptx::mbar_wait(&acc_empty[buf], ((i >> 1) & 1) ^ 1, abort, err)) break;
+                if (!ptx::mbar_wait(&a_full[i & 1], (i >> 1) & 1, abort, err)) break;
+                if (!ptx::mbar_wait(acc_empty, (i & 1) ^ 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
-                const uint32_t a_base = ptx::smem_u32(stage_ptr(s));
-                const uint32_t s_base = ptx::smem_u32(state_buf(sb));
+                const uint32_t a_base = tmem + KA_A_COL + (uint32_t)(i & 1) * 64u;
 #pragma unroll
                 for (int hh = 0; hh < G; ++hh) {
-                    const uint32_t d_tmem = tmem + (uint32_t)buf * 256u + (uint32_t)(hh * L::ACC_COLS);
+                    const uint32_t d_tmem = tmem + (uint32_t)(hh * L::ACC_COLS);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
-                        const int f = hh * D * 2 + ks * 32;       // byte offset in the group row
-                        const uint64_t a = ptx::smem_desc(a_base + (f / 128) * KA_BOX_BYTES + (f % 128),
-                                                          16, 1024, ptx::kLayoutSW128);
+                        const uint32_t a = a_base + (uint32_t)(hh * D / 2 + ks * 8);
                         const uint32_t hi = s_base + (hh * 2 + 0) * L::MAT_BYTES + ks * 256;
                         const uint32_t lo = s_base + (hh * 2 + 1) * L::MAT_BYTES + ks * 256;
-                        ptx::umma_f16_ss(d_tmem, a, ptx::smem_desc(hi, 128, L::SBO, ptx::kLayoutNone),
+                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(hi, 128, L::SBO, ptx::kLayoutNone),
                                          idesc, ks > 0);
-                        ptx::umma_f16_ss(d_tmem, a, ptx::smem_desc(lo, 128, L::SBO, ptx::kLayoutNone),
+                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(lo, 128, L::SBO, ptx::kLayoutNone),
                                          idesc, true);
                     }
                 }
-                ptx::umma_commit(&empty[s]);
-                ptx::umma_commit(&acc_full[buf]);
+                ptx::umma_commit(acc_full);
             }
             ptx::umma_commit(mma_done);
             ptx::mbar_wait(mma_done, 0, nullptr, err);
         }
     } else {
         // --------------------------------------------------------- workers ----
-        // stage unit i: (new segment ->) state hi/lo staging, then phi on the Q tile
+        // Warps w and w+4 own token rows m = 32*(w%4) + lane (their TMEM lanes);
+        // warp w < 4 takes box 0 of the group row and heads [0, G/2), warp w >= 4
+        // box 1 and heads [G/2, G).
+        const int m = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        constexpr int HPW = G / 2;
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+
+        // A operand of unit i: (new segment ->) the state as bf16 hi + lo in
+        // shared memory; phi(Q) row m, this warp's half, into A buffer i & 1.
+        // In a forward pass this kernel may start while the reduction of the
+        // state is still running (programmatic launch): the Q loads above do not
+        // depend on it, the state does.
+        ptx::wait_prerequisite_grid();
         auto prep = [&](int i) -> bool {
             if (i % tps == 0) {
-                const int sb = i / tps;
-                if (L::STATE_BUFS == 1 && i > 0) {
-                    // one buffer: the previous unit's UMMAs must be done reading it
-                    if (!warp_wait(&acc_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, err)) return false;
+                if (i > 0) {
+                    // the previous unit's UMMAs must be done reading the state
+                    if (!warp_wait(acc_full, (i - 1) & 1, abort, err)) return false;
                 }
-                uint8_t* dst = state_buf(sb);
                 int slab, tile, seg;
                 sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
                 const int b = slab / p.groups;
@@ -539,8 +562,8 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 for (int hh = 0; hh < G; ++hh) {
                     const int h = g * G + hh;
                     const float* src = state + ((long long)b * p.H + h) * DD;
-                    uint8_t* mhi = dst + (hh * 2 + 0) * L::MAT_BYTES;
-                    uint8_t* mlo = dst + (hh * 2 + 1) * L::MAT_BYTES;
+                    uint8_t* mhi = sstate + (hh * 2 + 0) * L::MAT_BYTES;
+                    uint8_t* mlo = sstate + (hh * 2 + 1) * L::MAT_BYTES;
                     for (int e = tid; e < DD; e += kWorkerThreads) {
                         const int k = e / (D + 1);       // state row i = UMMA K index
                         const int n = e % (D + 1);       // state column j = UMMA N index
@@ -551,57 +574,75 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         *reinterpret_cast<__nv_bfloat16*>(mlo + state_off<L::SBO>(n, k)) = vl;
                     }
                 }
+                ptx::fence_proxy_async_smem();
             }
             const int s = i % S;
             if (!warp_wait(&full[s], (i / S) & 1, abort, err)) return false;
-            relu_smem<KA_STAGE_BYTES / 16>(stage_ptr(s), tid);
-            ptx::fence_proxy_async_smem();
-            warp_arrive(&relu_done[s]);
+            // row m of box `half`: logical 16-byte chunk q sits at q ^ (m % 8)
+            const uint8_t* row = stage_ptr(s) + half * KA_BOX_BYTES + m * kBoxBytesRow;
+            uint32_t r[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row + ((q ^ (m & 7)) * 16));
+                r[4 * q + 0] = relu_bf16x2(v.x);
+                r[4 * q + 1] = relu_bf16x2(v.y);
+                r[4 * q + 2] = relu_bf16x2(v.z);
+                r[4 * q + 3] = relu_bf16x2(v.w);
+            }
+            warp_arrive(&empty[s]);
+            __syncwarp();
+            ptx::tmem_st32_wait(lane_base + KA_A_COL + (uint32_t)(i & 1) * 64u + (uint32_t)half * 32u, r);
+            ptx::tc_fence_before_sync();
+            warp_arrive(&a_full[i & 1]);
             return true;
         };
-        const int m = (warp & 3) * 32 + lane;                // token row of the tile = TMEM lane
-        constexpr int HPW = G / 2;                           // heads per worker warp
-        const int hh0 = (warp >> 2) * HPW;
+
         bool ok = nunits > 0 ? prep(0) : true;
         for (int i = 0; i < nunits && ok; ++i) {
             if (i + 1 < nunits && !prep(i + 1)) break;
-            // epilogue of unit i
-            const int buf = i & 1;
-            if (!warp_wait(&acc_full[buf], (i >> 1) & 1, abort, err)) break;
+            // ---- epilogue of unit i
+            if (!warp_wait(acc_full, i & 1, abort, err)) break;
             ptx::tc_fence_after_sync();
+            float num[HPW][D], den[HPW];
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < HPW; ++j) {
+                const uint32_t col = (uint32_t)((half * HPW + j) * L::ACC_COLS);
+                ptx::tmem_ld_row<D>(lane_base + col, lane_base + col + D, num[j], &den[j]);
+            }
+            ptx::tc_fence_before_sync();
+            warp_arrive(acc_empty);
             int slab, tile, seg;
             sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
             const int b = slab / p.groups;
             const int g = slab % p.groups;
-            // the previous unit's TMA store must have finished reading the staging tile
+            uint8_t* staging = smem + L::STG_OFF + (i % L::STG_BUFS) * L::STG_BYTES;
+            // the TMA store that last read this staging tile must be done reading it
             if (tid == 0) {
-                ptx::bulk_wait_group_read<0>();
+                if (L::STG_BUFS == 2) ptx::bulk_wait_group_read<1>();
+                else ptx::bulk_wait_group_read<0>();
                 ptx::mbar_arrive(stg_free);
             }
             if (!warp_wait(stg_free, i & 1, abort, err)) break;
-            const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)buf * 256u;
-#pragma unroll 1
-            for (int hh = hh0; hh < hh0 + HPW; ++hh) {
-                float num[D], den;
-                __syncwarp();
-                ptx::tmem_ld_row<D>(lane_addr + hh * L::ACC_COLS, lane_addr + hh * L::ACC_COLS + D,
-                                    num, &den);
-                const float r = 1.0f / (den + p.eps);
+#pragma unroll
+            for (int j = 0; j < HPW; ++j) {
+                const int hh = half * HPW + j;
+                const float rcp = 1.0f / (den[j] + p.eps);
                 // row m of the staging tile, 128-byte swizzle: chunk q lands at q ^ (m % 8)
 #pragma unroll
-                for (int j = 0; j < D; j += 16 / L::OUT_BYTES) {
-                    const int f = (hh * D + j) * L::OUT_BYTES;        // byte offset in the group row
+                for (int e = 0; e < D; e += 16 / L::OUT_BYTES) {
+                    const int f = (hh * D + e) * L::OUT_BYTES;        // byte offset in the group row
                     uint4 w;
                     if (OUT_BF16) {
-                        w.x = float2_to_bf16x2(num[j + 0] * r, num[j + 1] * r);
-                        w.y = float2_to_bf16x2(num[j + 2] * r, num[j + 3] * r);
-                        w.z = float2_to_bf16x2(num[j + 4] * r, num[j + 5] * r);
-                        w.w = float2_to_bf16x2(num[j + 6] * r, num[j + 7] * r);
+                        w.x = float2_to_bf16x2(num[j][e + 0] * rcp, num[j][e + 1] * rcp);
+                        w.y = float2_to_bf16x2(num[j][e + 2] * rcp, num[j][e + 3] * rcp);
+                        w.z = float2_to_bf16x2(num[j][e + 4] * rcp, num[j][e + 5] * rcp);
+                        w.w = float2_to_bf16x2(num[j][e + 6] * rcp, num[j][e + 7] * rcp);
                     } else {
-                        w.x = __float_as_uint(num[j + 0] * r);
-                        w.y = __float_as_uint(num[j + 1] * r);
-                        w.z = __float_as_uint(num[j + 2] * r);
-                        w.w = __float_as_uint(num[j + 3] * r);
+                        w.x = __float_as_uint(num[j][e + 0] * rcp);
+                        w.y = __float_as_uint(num[j][e + 1] * rcp);
+                        w.z = __float_as_uint(num[j][e + 2] * rcp);
+                        w.w = __float_as_uint(num[j][e + 3] * rcp);
                     }
                     const int box = f / kBoxBytesRow;
                     const int q = (f % kBoxBytesRow) / 16;
@@ -609,12 +650,10 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                               ((q ^ (m & 7)) * 16)) = w;
                 }
             }
-            ptx::tc_fence_before_sync();
-            warp_arrive(&acc_empty[buf]);
             ptx::fence_proxy_async_smem();
-            warp_arrive(stg_full);
+            warp_arrive(&stg_full[i & 1]);
             if (warp == 0) {
-                if (!warp_wait(stg_full, i & 1, abort, err)) break;
+                if (!warp_wait(&stg_full[i & 1], (i >> 1) & 1, abort, err)) break;
                 if (lane == 0) {
                     const int x0 = g * 128;
                     const int y = tile * KA_TILE;
