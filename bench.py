@@ -38,7 +38,11 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
 # the same build (profiles/), keyed by (kernel set, workload, kernel); None when
 # the kernels changed since the counters were taken
-TRAFFIC_PER_LAUNCH = {}
+TRAFFIC_PER_LAUNCH = {
+    # profiles/tc_kernels_sweep_N65536.md, scaled by token-heads (x 0.9722)
+    ("tcgen05-tma", "4096px", "kv_state(KS+KR)"): 297.8e6 + 2.4e6,
+    ("tcgen05-tma", "4096px", "apply(KA)"): 240.4e6,
+}
 SMS = 148
 FP32_LANES_PER_SM = 128
 
