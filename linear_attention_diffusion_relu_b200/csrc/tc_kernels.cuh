@@ -398,7 +398,7 @@ struct KaLayout {
     static constexpr int STATE_OFF = STAGES * KA_STAGE_BYTES;
     static constexpr int STG_OFF = STATE_OFF + STATE_BYTES;
     static constexpr int BAR_OFF = STG_OFF + STG_BUFS * STG_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 9;
+    static constexpr int NUM_BARS = 2 * STAGES + 12;
     static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = CTL_OFF + 64 + 1024;
     static constexpr int ACC_COLS = 256 / G;               // TMEM columns per head
@@ -429,9 +429,9 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* a_full = bars + 2 * S;        // [2] A operand in TMEM
     uint64_t* acc_full = a_full + 2;        // UMMAs of a unit done
     uint64_t* acc_empty = a_full + 3;       // accumulator read by every worker warp
-    uint64_t* stg_free = a_full + 4;        // staging tile of this unit may be written
-    uint64_t* stg_full = a_full + 5;        // [2] staging tile written by every worker warp
-    uint64_t* mma_done = a_full + 7;
+    uint64_t* stg_free = a_full + 4;        // [2 halves] this half's staging boxes may be written
+    uint64_t* stg_full = a_full + 6;        // [2 halves][2] this half's staging boxes written
+    uint64_t* mma_done = a_full + 10;
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + L::CTL_OFF);
     volatile int* abort = &ctl->abort;
     uint32_t* err = &g_device_error;
@@ -452,9 +452,11 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         ptx::mbar_init(&a_full[1], kWorkerWarps);
         ptx::mbar_init(acc_full, 1);
         ptx::mbar_init(acc_empty, kWorkerWarps);
-        ptx::mbar_init(stg_free, 1);
-        ptx::mbar_init(&stg_full[0], kWorkerWarps);
-        ptx::mbar_init(&stg_full[1], kWorkerWarps);
+        for (int h = 0; h < 2; ++h) {
+            ptx::mbar_init(&stg_free[h], 1);
+            ptx::mbar_init(&stg_full[2 * h + 0], kWorkerWarps / 2);
+            ptx::mbar_init(&stg_full[2 * h + 1], kWorkerWarps / 2);
+        }
         ptx::mbar_init(mma_done, 1);
         ctl->abort = 0;
         ptx::fence_mbar_init();
@@ -542,6 +544,11 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int half = warp >> 2;
         constexpr int HPW = G / 2;
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        // Each half stores its own output boxes (its heads' bytes of the row):
+        // the leader (lane 0 of warp 0 / warp 4) issues and tracks those stores.
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        constexpr int HALF_BOXES = L::OUT_BOXES / 2;
+        if (leader) ptx::mbar_arrive(&stg_free[half]);      // staging is free for unit 0
 
         // A operand of unit i: (new segment ->) the state as bf16 hi + lo in
         // shared memory; phi(Q) row m, this warp's half, into A buffer i & 1.
@@ -617,13 +624,9 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int b = slab / p.groups;
             const int g = slab % p.groups;
             uint8_t* staging = smem + L::STG_OFF + (i % L::STG_BUFS) * L::STG_BYTES;
-            // the TMA store that last read this staging tile must be done reading it
-            if (tid == 0) {
-                if (L::STG_BUFS == 2) ptx::bulk_wait_group_read<1>();
-                else ptx::bulk_wait_group_read<0>();
-                ptx::mbar_arrive(stg_free);
-            }
-            if (!warp_wait(stg_free, i & 1, abort, err)) break;
+            // this half's boxes of the staging tile must be free (the leader
+            // released them after the store that last read them)
+            if (!warp_wait(&stg_free[half], i & 1, abort, err)) break;
 #pragma unroll
             for (int j = 0; j < HPW; ++j) {
                 const int hh = half * HPW + j;
@@ -651,22 +654,28 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
             }
             ptx::fence_proxy_async_smem();
-            warp_arrive(&stg_full[i & 1]);
-            if (warp == 0) {
-                if (!warp_wait(&stg_full[i & 1], (i >> 1) & 1, abort, err)) break;
+            warp_arrive(&stg_full[2 * half + (i & 1)]);
+            if ((warp & 3) == 0) {
+                if (!warp_wait(&stg_full[2 * half + (i & 1)], (i >> 1) & 1, abort, err)) break;
                 if (lane == 0) {
                     const int x0 = g * 128;
                     const int y = tile * KA_TILE;
 #pragma unroll
-                    for (int bx = 0; bx < L::OUT_BOXES; ++bx) {
+                    for (int k = 0; k < HALF_BOXES; ++k) {
+                        const int bx = half * HALF_BOXES + k;
                         const int x = x0 + bx * L::OUT_BOX_ELEMS;
                         if (x < p.H * D) ptx::tma_store_3d(&tmO, staging + bx * KA_BOX_BYTES, x, y, b);
                     }
                     ptx::bulk_commit_group();
+                    // release the staging boxes for unit i + 1: the store that last
+                    // used them (unit i + 1 - STG_BUFS) must be done reading
+                    if (L::STG_BUFS == 2) ptx::bulk_wait_group_read<1>();
+                    else ptx::bulk_wait_group_read<0>();
+                    ptx::mbar_arrive(&stg_free[half]);
                 }
             }
         }
-        if (tid == 0) ptx::bulk_wait_group<0>();
+        if (leader) ptx::bulk_wait_group<0>();
     }
 
     ptx::tc_fence_before_sync();
