@@ -39,6 +39,7 @@ struct Plan {
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
     size_t state_bytes;     // fp32 (B, H, d, d+1)
+    size_t gbar_bytes;      // grid-barrier word of the single-launch forward
 };
 
 // Lockstep schedule of S slabs of T tiles over at most kSMs CTAs (see the
@@ -74,6 +75,7 @@ Plan make_plan(int B, int N, int H, int d) {
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * dd);
+    p.gbar_bytes = 256;
     return p;
 }
 
@@ -200,10 +202,10 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
     sana_la_status st;
     if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
-    if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KS_SMEM_BYTES, smem_set)) != SANA_LA_OK)
+    if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KsMap::BYTES, smem_set)) != SANA_LA_OK)
         return st;
     if ((st = launch(sana::tc::ks_state_tc<D>, dim3(p.ks.q.grid), dim3(sana::tc::kThreads),
-                     sana::tc::KS_SMEM_BYTES, s, false, "ks_state_tc", tmK, tmV, p.ks, partial)) != SANA_LA_OK)
+                     sana::tc::KsMap::BYTES, s, false, "ks_state_tc", tmK, tmV, p.ks, partial)) != SANA_LA_OK)
         return st;
     // the reduction overlaps the state kernel's tail; it waits for its results
     const dim3 kr_grid((unsigned)((long long)B * H), (D * (D + 1) + sana::tc::KR_THREADS - 1) / sana::tc::KR_THREADS);
@@ -218,7 +220,7 @@ sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N,
     CUtensorMap tmO;
     sana_la_status st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::KaLayout<D, OUT_BF16>::SMEM_BYTES;
+    constexpr int smem = sana::tc::KaMap<D, OUT_BF16>::BYTES;
     if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16>, smem, smem_set)) != SANA_LA_OK) return st;
     return launch(sana::tc::ka_apply_tc<D, OUT_BF16>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
                   overlap, "ka_apply_tc", tmQ, tmO, p.ka, state);
@@ -237,6 +239,54 @@ sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H,
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
     return od == SANA_LA_OUT_BF16 ? launch_apply<D, true>(tmQ, O, B, N, H, p, state, s, overlap)
                                   : launch_apply<D, false>(tmQ, O, B, N, H, p, state, s, overlap);
+}
+
+// The whole forward as one cooperative launch (fwd_fused_tc). Returns
+// SANA_LA_ERR_UNSUPPORTED, with nothing enqueued, when the device refuses a
+// cooperative launch of this size, so the caller can use the three kernels.
+template <int D, bool OUT_BF16>
+sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
+                                    int H, const Plan& p, float* partial, unsigned* gbar, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmK, tmV, tmQ, tmO;
+    sana_la_status st;
+    if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
+    constexpr int smem = sana::tc::FwdMap<D, OUT_BF16>::BYTES;
+    auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16>;
+    if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
+    const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, sana::tc::kThreads, smem) != cudaSuccess ||
+        (long long)sms * per_sm < grid) {
+        cudaGetLastError();
+        return SANA_LA_ERR_UNSUPPORTED;
+    }
+    cudaError_t e = cudaMemsetAsync(gbar, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemsetAsync(grid barrier)", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(sana::tc::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, gbar);
+    if (e != cudaSuccess) {
+        set_last_error("fwd_fused_tc", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    return launch_status("fwd_fused_tc");
 }
 
 sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d,
@@ -263,7 +313,7 @@ extern "C" {
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
     const Plan p = make_plan(B, N, H, d);
-    return p.partial_bytes + p.state_bytes;
+    return p.partial_bytes + p.state_bytes + p.gbar_bytes;
 }
 
 sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,
@@ -306,10 +356,23 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
-    const Plan p = make_plan(B, N, H, d);
-    if (workspace_bytes < p.partial_bytes + p.state_bytes) return SANA_LA_ERR_WORKSPACE;
-    float* state = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.partial_bytes);
+    Plan p = make_plan(B, N, H, d);
+    if (workspace_bytes < p.partial_bytes + p.state_bytes + p.gbar_bytes) return SANA_LA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    float* partial = reinterpret_cast<float*>(ws);
+    float* state = reinterpret_cast<float*>(ws + p.partial_bytes);
+    unsigned* gbar = reinterpret_cast<unsigned*>(ws + p.partial_bytes + p.state_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // one cooperative launch: state phase, grid barrier, apply phase
+    p.ka.eps = eps;
+    const bool bf16 = out_dtype == SANA_LA_OUT_BF16;
+    st = d == 32 ? (bf16 ? launch_forward_fused<32, true>(Q, K, V, O, B, N, H, p, partial, gbar, s)
+                         : launch_forward_fused<32, false>(Q, K, V, O, B, N, H, p, partial, gbar, s))
+                 : (bf16 ? launch_forward_fused<64, true>(Q, K, V, O, B, N, H, p, partial, gbar, s)
+                         : launch_forward_fused<64, false>(Q, K, V, O, B, N, H, p, partial, gbar, s));
+    if (st != SANA_LA_ERR_UNSUPPORTED) return st;
+    // the device cannot hold the whole grid at once: the same kernels as
+    // kv_state + apply, overlapped by programmatic launch
     st = kv_state_impl(K, V, B, N, H, d, state, workspace, workspace_bytes, s, true);
     if (st != SANA_LA_OK) return st;
     return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps, s, true);
@@ -317,7 +380,7 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
 
 int sana_linattn_forward_launches(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
-    return 3;   // KS, KR, KA
+    return 1;   // fwd_fused_tc (after a 4-byte memset of its barrier word)
 }
 
 const char* sana_linattn_build_info(void) { return "impl=tcgen05-tma;bound=hbm"; }

@@ -139,39 +139,17 @@ constexpr int KS_STAGES = 6;
 constexpr int KS_BOX_BYTES = KS_TILE * kBoxBytesRow;       // 8 KB
 constexpr int KS_STAGE_BYTES = 4 * KS_BOX_BYTES;           // K0 K1 V0 V1
 constexpr int KS_ONES_OFF = KS_STAGES * KS_STAGE_BYTES;
-constexpr int KS_BAR_OFF = KS_ONES_OFF + 1024;
+constexpr int KS_DATA_BYTES = KS_ONES_OFF + 1024;          // stages + the ones tile
 constexpr int KS_NUM_BARS = 3 * KS_STAGES + 5;
-constexpr int KS_CTL_OFF = KS_BAR_OFF + KS_NUM_BARS * 8;
-constexpr int KS_SMEM_BYTES = KS_CTL_OFF + 64 + 1024;      // + alignment slack
-static_assert(KS_SMEM_BYTES <= kSmemLimit, "KS shared memory");
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-            const KsParams p, float* __restrict__ partial)
-{
-    constexpr int G = 128 / D;
-    constexpr int DD = D * (D + 1);
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KS_BAR_OFF);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + KS_STAGES;
-    uint64_t* relu_done = bars + 2 * KS_STAGES;
-    uint64_t* acc_full = bars + 3 * KS_STAGES;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* mma_done = acc_full + 4;
-    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + KS_CTL_OFF);
-    volatile int* abort = &ctl->abort;
-    uint32_t* err = &g_device_error;
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    const int tps = sched_tps(blockIdx.x, p.q);
-    const int ntiles = tps * sched_nseg(blockIdx.x, p.q);
-
-    if (tid == 0) {
+struct KsBars {
+    uint64_t* full;        // [KS_STAGES] K and V tiles landed
+    uint64_t* empty;       // [KS_STAGES] tiles read by the UMMAs
+    uint64_t* relu_done;   // [KS_STAGES] phi applied to the K tile
+    uint64_t* acc_full;    // [2] a segment's accumulator complete
+    uint64_t* acc_empty;   // [2] accumulator read by the epilogue warps 0-3
+    uint64_t* mma_done;
+    __device__ void init() const {
         for (int s = 0; s < KS_STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
@@ -179,33 +157,45 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], 4);           // the epilogue warps 0-3
+            ptx::mbar_init(&acc_empty[a], 4);
         }
         ptx::mbar_init(mma_done, 1);
-        ctl->abort = 0;
-        ptx::fence_mbar_init();
     }
-    if (warp == 0) {
-        ptx::tmem_alloc(&ctl->tmem_base, kTmemCols);
-        ptx::tmem_relinquish();
-    }
-    if (warp == kProducerWarp && lane == 0) {
-        ptx::prefetch_tmap(&tmK);
-        ptx::prefetch_tmap(&tmV);
-    }
+};
+
+__device__ __forceinline__ KsBars ks_bars(uint64_t* b) {
+    return KsBars{b, b + KS_STAGES, b + 2 * KS_STAGES, b + 3 * KS_STAGES, b + 3 * KS_STAGES + 2,
+                  b + 3 * KS_STAGES + 4};
+}
+
+__device__ __forceinline__ void ks_fill_ones(uint8_t* smem, int tid) {
     // constant all-ones bf16 operand (16 tokens x 16 columns) for the normaliser column
     if (tid < 32) {
         uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
         reinterpret_cast<uint4*>(smem + KS_ONES_OFF)[tid] = ones;
         ptx::fence_proxy_async_smem();
     }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
-    // the reduction kernel may be scheduled now; it waits for this grid's results
-    if (tid == 0) ptx::launch_dependents();
+}
 
+// The state phase for CTA `cta`: partial states phi(K)^T [V | 1] of its
+// segments into `partial`. Every role returns once its part is done. Stage s
+// of this phase is free again once bar.empty[s] has completed the phase of the
+// last tile that used it (the single-launch kernel's apply phase waits for
+// that before it loads into the same bytes).
+template <int D>
+__device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
+                                         int cta, float* __restrict__ partial, uint8_t* smem,
+                                         const KsBars& bar, uint32_t tmem, volatile int* abort,
+                                         uint32_t* err)
+{
+    constexpr int G = 128 / D;
+    constexpr int DD = D * (D + 1);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    if (cta >= p.q.grid) return;
+    const int tps = sched_tps(cta, p.q);
+    const int ntiles = tps * sched_nseg(cta, p.q);
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KS_STAGE_BYTES; };
 
     if (warp == kProducerWarp) {
@@ -214,23 +204,23 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             int issued = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i % KS_STAGES;
-                if (!ptx::mbar_wait(&empty[s], ((i / KS_STAGES) & 1) ^ 1, abort, err)) break;
+                if (!ptx::mbar_wait(&bar.empty[s], ((i / KS_STAGES) & 1) ^ 1, abort, err)) break;
                 int slab, tile, seg;
-                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+                sched_item(cta, i, tps, p.q, slab, tile, seg);
                 const int b = slab / p.groups;
                 const int x0 = (slab % p.groups) * 128;
                 const int y = tile * KS_TILE;
                 uint8_t* st = stage_ptr(s);
-                ptx::mbar_arrive_expect_tx(&full[s], KS_STAGE_BYTES);
-                ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, &tmK, &full[s], x0, y, b);
-                ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, &tmK, &full[s], x0 + 64, y, b);
-                ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, &tmV, &full[s], x0, y, b);
-                ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, &tmV, &full[s], x0 + 64, y, b);
+                ptx::mbar_arrive_expect_tx(&bar.full[s], KS_STAGE_BYTES);
+                ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b);
+                ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b);
+                ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b);
+                ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b);
                 issued = i + 1;
             }
             // drain: every issued load must land before the CTA may exit
             for (int i = (issued > KS_STAGES ? issued - KS_STAGES : 0); i < issued; ++i)
-                ptx::mbar_wait(&full[i % KS_STAGES], (i / KS_STAGES) & 1, nullptr, err);
+                ptx::mbar_wait(&bar.full[i % KS_STAGES], (i / KS_STAGES) & 1, nullptr, err);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- UMMA issuer ----
@@ -246,12 +236,12 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 const bool seg_end = (i % tps) == tps - 1;
                 if (seg_start) {
                     ++seg;
-                    if (!ptx::mbar_wait(&acc_empty[seg & 1], ((seg >> 1) & 1) ^ 1, abort, err)) break;
+                    if (!ptx::mbar_wait(&bar.acc_empty[seg & 1], ((seg >> 1) & 1) ^ 1, abort, err)) break;
                     ptx::tc_fence_after_sync();
                     first = true;
                 }
                 const int s = i % KS_STAGES;
-                if (!ptx::mbar_wait(&relu_done[s], (i / KS_STAGES) & 1, abort, err)) break;
+                if (!ptx::mbar_wait(&bar.relu_done[s], (i / KS_STAGES) & 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const uint32_t d_tmem = tmem + (uint32_t)(seg & 1) * 256u;
                 const uint32_t k_addr = ptx::smem_u32(stage_ptr(s));
@@ -268,11 +258,11 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                     ptx::umma_f16_ss(d_tmem + 128, a, ones_desc, idesc_1, acc);
                 }
                 first = false;
-                ptx::umma_commit(&empty[s]);
-                if (seg_end) ptx::umma_commit(&acc_full[seg & 1]);
+                ptx::umma_commit(&bar.empty[s]);
+                if (seg_end) ptx::umma_commit(&bar.acc_full[seg & 1]);
             }
-            ptx::umma_commit(mma_done);
-            ptx::mbar_wait(mma_done, 0, nullptr, err);
+            ptx::umma_commit(bar.mma_done);
+            ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
         }
     } else {
         // --------------------------------------------------------- workers ----
@@ -280,15 +270,15 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             const bool seg_end = (i % tps) == tps - 1;
             const int seg = i / tps;
             const int s = i % KS_STAGES;
-            if (!warp_wait(&full[s], (i / KS_STAGES) & 1, abort, err)) break;
+            if (!warp_wait(&bar.full[s], (i / KS_STAGES) & 1, abort, err)) break;
             relu_smem<2 * KS_BOX_BYTES / 16>(stage_ptr(s), tid);     // phi on the K boxes only
             ptx::fence_proxy_async_smem();
-            warp_arrive(&relu_done[s]);
+            warp_arrive(&bar.relu_done[s]);
             if (seg_end && warp < 4) {
                 // epilogue (warps 0-3, one per TMEM lane quarter): this segment's
                 // partial states, TMEM -> workspace
                 const int buf = seg & 1;
-                if (!warp_wait(&acc_full[buf], (seg >> 1) & 1, abort, err)) break;
+                if (!warp_wait(&bar.acc_full[buf], (seg >> 1) & 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const int hh = warp / (D / 32);                  // head within the group
                 const int row = (warp % (D / 32)) * 32 + lane;   // state row i of that head
@@ -297,12 +287,12 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 __syncwarp();
                 ptx::tmem_ld_row<D>(lane_addr + hh * D, lane_addr + 128, v, &nrm);
                 ptx::tc_fence_before_sync();
-                warp_arrive(&acc_empty[buf]);
+                warp_arrive(&bar.acc_empty[buf]);
                 int slab, tile, sg;
-                sched_item(blockIdx.x, i, tps, p.q, slab, tile, sg);
+                sched_item(cta, i, tps, p.q, slab, tile, sg);
                 const int h = (slab % p.groups) * G + hh;
                 if (h < p.H) {
-                    const long long slot = ((long long)blockIdx.x * p.q.max_seg + seg) * G + hh;
+                    const long long slot = ((long long)cta * p.q.max_seg + seg) * G + hh;
                     float* P = partial + slot * DD + (long long)row * (D + 1);
 #pragma unroll
                     for (int j = 0; j < D; ++j) P[j] = v[j];
@@ -311,21 +301,18 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             }
         }
     }
+}
 
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        __syncwarp();
-        ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, kTmemCols);
-    }
+// Partial-state slot of segment `seg` of CTA `c` for head hh of the group.
+// A slab's R partials are those of CTAs (slab % grid) + r * S, r = 0 .. R-1,
+// segment slab / grid; they are always added in ascending r.
+__device__ __forceinline__ long long ks_slot(long long c, int seg, int hh, int G, const KsParams& p) {
+    return (c * p.q.max_seg + seg) * G + hh;
 }
 
 // ===================================================================== KR ===
 // One thread per state entry (grid: (b, h) x entry blocks), so every load is
-// independent and the kernel costs about one L2 round trip. The segments of a
-// slab are added in ascending CTA order: the partial of CTA c = (slab % grid)
-// + r * S, segment slab / grid, for r = 0 .. R-1.
+// independent and the kernel costs about one L2 round trip.
 constexpr int KR_THREADS = 128;
 
 template <int D>
@@ -334,8 +321,8 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
-    // The apply kernel of a forward pass may be scheduled now: its Q loads only
-    // need ks_state_tc to have started, and it waits for this grid before
+    // The apply kernel of a two-call forward may be scheduled now: its Q loads
+    // only need ks_state_tc to have started, and it waits for this grid before
     // reading the state.
     ptx::launch_dependents();
     ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
@@ -345,9 +332,7 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
     const int slab = b * p.groups + h / G;
-    const int seg = slab / p.q.grid;
-    const int c0 = slab % p.q.grid;
-    const float* src = partial + (((long long)c0 * p.q.max_seg + seg) * G + h % G) * DD + e;
+    const float* src = partial + ks_slot(slab % p.q.grid, slab / p.q.grid, h % G, G, p) * DD + e;
     const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
     float s = 0.0f;
     for (int r = 0; r < p.q.R; ++r) s += src[r * step];
@@ -365,7 +350,8 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 //   UMMA      per head: D = phi(Q) S_hi + phi(Q) S_lo (A from TMEM, the
 //             state in shared memory as bf16 hi and lo parts)
 //   workers   D -> registers, O = num / (den + eps), into a swizzled staging
-//             tile, written to global memory by a TMA store
+//             tile, written to global memory by a TMA store (each half of the
+//             worker warps stores its own heads' boxes)
 // TMEM: the accumulator at columns [0, 256) (head h at h * 256/G) and two A
 // buffers of 64 columns at 256 and 320.
 struct KaParams {
@@ -378,6 +364,7 @@ constexpr int KA_TILE = 128;                               // tokens = UMMA M
 constexpr int KA_BOX_BYTES = KA_TILE * kBoxBytesRow;       // 16 KB
 constexpr int KA_STAGE_BYTES = 2 * KA_BOX_BYTES;           // one group row of 128 tokens
 constexpr uint32_t KA_A_COL = 256;                         // first A buffer column
+constexpr int kBarRegion = 4096;                           // barriers + control block + slack
 
 template <int D, bool OUT_BF16>
 struct KaLayout {
@@ -390,20 +377,17 @@ struct KaLayout {
     static constexpr int OUT_BOXES = 128 * OUT_BYTES / kBoxBytesRow;   // boxes per output group row
     static constexpr int OUT_BOX_ELEMS = kBoxBytesRow / OUT_BYTES;
     static constexpr int STG_BYTES = OUT_BOXES * KA_BOX_BYTES;
-    static constexpr int AVAIL = kSmemLimit - 4096 - STATE_BYTES;
+    static constexpr int AVAIL = kSmemLimit - 1024 - kBarRegion - STATE_BYTES;
     // two staging tiles if that still leaves four Q stages, else one
     static constexpr int STG_BUFS = (AVAIL - 2 * STG_BYTES) / KA_STAGE_BYTES >= 4 ? 2 : 1;
     static constexpr int STAGES_FIT = (AVAIL - STG_BUFS * STG_BYTES) / KA_STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
     static constexpr int STATE_OFF = STAGES * KA_STAGE_BYTES;
     static constexpr int STG_OFF = STATE_OFF + STATE_BYTES;
-    static constexpr int BAR_OFF = STG_OFF + STG_BUFS * STG_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 12;
-    static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = CTL_OFF + 64 + 1024;
+    static constexpr int DATA_BYTES = STG_OFF + STG_BUFS * STG_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 14;
     static constexpr int ACC_COLS = 256 / G;               // TMEM columns per head
     static_assert(STAGES >= 3, "KA needs at least three Q stages");
-    static_assert(SMEM_BYTES <= kSmemLimit, "KA shared memory");
 };
 
 // element (n, k) of a K-major, unswizzled bf16 matrix made of 8x8 core matrices
@@ -413,38 +397,20 @@ __device__ __forceinline__ int state_off(int n, int k) {
 }
 
 template <int D, bool OUT_BF16>
-__global__ void __launch_bounds__(kThreads, 1)
-ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-            const KaParams p, const float* __restrict__ state)
-{
+struct KaBars {
     using L = KaLayout<D, OUT_BF16>;
-    constexpr int G = L::G;
-    constexpr int DD = D * (D + 1);
-    constexpr int S = L::STAGES;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-    uint64_t* full = bars;                  // [S] Q tile landed
-    uint64_t* empty = bars + S;             // [S] Q tile read by every worker warp
-    uint64_t* a_full = bars + 2 * S;        // [2] A operand in TMEM
-    uint64_t* acc_full = a_full + 2;        // UMMAs of a unit done
-    uint64_t* acc_empty = a_full + 3;       // accumulator read by every worker warp
-    uint64_t* stg_free = a_full + 4;        // [2 halves] this half's staging boxes may be written
-    uint64_t* stg_full = a_full + 6;        // [2 halves][2] this half's staging boxes written
-    uint64_t* mma_done = a_full + 10;
-    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + L::CTL_OFF);
-    volatile int* abort = &ctl->abort;
-    uint32_t* err = &g_device_error;
-    uint8_t* sstate = smem + L::STATE_OFF;
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    const int tps = sched_tps(blockIdx.x, p.q);
-    const int nunits = tps * sched_nseg(blockIdx.x, p.q);
-
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
+    uint64_t* full;        // [STAGES] Q tile landed
+    uint64_t* empty;       // [STAGES] Q tile read by every worker warp
+    uint64_t* a_full;      // [2] A operand in TMEM (and the state staged)
+    uint64_t* acc_full;    // UMMAs of a unit done
+    uint64_t* acc_empty;   // accumulator read by every worker warp
+    uint64_t* stg_free;    // [2 halves] this half's staging boxes may be written
+    uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
+    uint64_t* mma_done;
+    uint64_t* grid_ready;  // (single launch) every CTA's partial states are in memory
+    uint64_t* p1_written;  // (single launch) this CTA's partial states are written
+    __device__ void init() const {
+        for (int s = 0; s < L::STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], kWorkerWarps);
         }
@@ -458,53 +424,113 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             ptx::mbar_init(&stg_full[2 * h + 1], kWorkerWarps / 2);
         }
         ptx::mbar_init(mma_done, 1);
-        ctl->abort = 0;
-        ptx::fence_mbar_init();
+        ptx::mbar_init(grid_ready, 1);
+        ptx::mbar_init(p1_written, 4);
     }
-    if (warp == 0) {
-        ptx::tmem_alloc(&ctl->tmem_base, kTmemCols);
-        ptx::tmem_relinquish();
-    }
-    if (warp == kProducerWarp && lane == 0) {
-        ptx::prefetch_tmap(&tmQ);
-        ptx::prefetch_tmap(&tmO);
-    }
-    // padding columns n in (d, NA) of the state are zero for good
+};
+
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ KaBars<D, OUT_BF16> ka_bars(uint64_t* b) {
+    constexpr int S = KaLayout<D, OUT_BF16>::STAGES;
+    uint64_t* a = b + 2 * S;
+    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 12};
+}
+
+// zero the padding columns n in (d, NA) of the staged state
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid) {
+    using L = KaLayout<D, OUT_BF16>;
     if (tid < kWorkerThreads) {
         constexpr int PAD = L::NA - D - 1;
-        for (int e = tid; e < G * 2 * PAD * D; e += kWorkerThreads) {
+        for (int e = tid; e < L::G * 2 * PAD * D; e += kWorkerThreads) {
             const int k = e % D;
             const int n = D + 1 + (e / D) % PAD;
             const int mat = e / (D * PAD);
-            *reinterpret_cast<__nv_bfloat16*>(sstate + mat * L::MAT_BYTES + state_off<L::SBO>(n, k)) =
-                __float2bfloat16_rn(0.0f);
+            *reinterpret_cast<__nv_bfloat16*>(smem + L::STATE_OFF + mat * L::MAT_BYTES +
+                                              state_off<L::SBO>(n, k)) = __float2bfloat16_rn(0.0f);
         }
     }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
+}
 
+// Where the apply phase gets the state of a slab from:
+//   state != nullptr   the reduced fp32 state (B, H, d, d+1) of the reduction kernel
+//   otherwise          the partial states of the state phase (same launch), summed
+//                      here in the reduction kernel's order, once `gbar` shows
+//                      every CTA has written them
+struct KaStateSrc {
+    const float* state;
+    const float* partial;
+    KsParams ks;
+    unsigned* gbar;
+    unsigned gbar_target;
+};
+
+// Bounded spin until every CTA of the grid has arrived at the barrier word.
+__device__ __forceinline__ bool grid_wait(unsigned* gbar, unsigned target, volatile int* abort,
+                                          uint32_t* err) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (;;) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
+        if (v >= target) return true;
+        if (*abort) return false;
+        if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
+            atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(256);
+    }
+}
+
+// The apply phase for CTA `cta`.
+// `prev_empty`/`prev_tiles` (single launch): the state phase's stage barriers
+// and how many tiles it loaded; Q stage s (< 6) reuses its stage s, so the
+// first load into each waits until the state phase released that stage.
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorMap* tmO, const KaParams& p,
+                                         int cta, const KaStateSrc& src, uint8_t* smem,
+                                         const KaBars<D, OUT_BF16>& bar, uint32_t tmem,
+                                         volatile int* abort, uint32_t* err,
+                                         uint64_t* prev_empty = nullptr, int prev_tiles = 0)
+{
+    using L = KaLayout<D, OUT_BF16>;
+    constexpr int G = L::G;
+    constexpr int DD = D * (D + 1);
+    constexpr int S = L::STAGES;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    if (cta >= p.q.grid) return;
+    uint8_t* sstate = smem + L::STATE_OFF;
+    const int tps = sched_tps(cta, p.q);
+    const int nunits = tps * sched_nseg(cta, p.q);
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KA_STAGE_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int issued = 0;
+            static_assert(L::STAGES <= KS_STAGES && KA_STAGE_BYTES == KS_STAGE_BYTES, "stage reuse");
             for (int i = 0; i < nunits; ++i) {
                 const int s = i % S;
-                if (!ptx::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, abort, err)) break;
+                if (!ptx::mbar_wait(&bar.empty[s], ((i / S) & 1) ^ 1, abort, err)) break;
+                if (prev_empty != nullptr && i < S) {
+                    // the state phase's next (never issued) use of stage s
+                    const int j = prev_tiles + ((s - prev_tiles) % KS_STAGES + KS_STAGES) % KS_STAGES;
+                    if (!ptx::mbar_wait(&prev_empty[s], ((j / KS_STAGES) & 1) ^ 1, abort, err)) break;
+                }
                 int slab, tile, seg;
-                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+                sched_item(cta, i, tps, p.q, slab, tile, seg);
                 const int b = slab / p.groups;
                 const int x0 = (slab % p.groups) * 128;
-                ptx::mbar_arrive_expect_tx(&full[s], KA_STAGE_BYTES);
-                ptx::tma_load_3d(stage_ptr(s), &tmQ, &full[s], x0, tile * KA_TILE, b);
-                ptx::tma_load_3d(stage_ptr(s) + KA_BOX_BYTES, &tmQ, &full[s], x0 + 64, tile * KA_TILE, b);
+                ptx::mbar_arrive_expect_tx(&bar.full[s], KA_STAGE_BYTES);
+                ptx::tma_load_3d(stage_ptr(s), tmQ, &bar.full[s], x0, tile * KA_TILE, b);
+                ptx::tma_load_3d(stage_ptr(s) + KA_BOX_BYTES, tmQ, &bar.full[s], x0 + 64, tile * KA_TILE, b);
                 issued = i + 1;
             }
             for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-                ptx::mbar_wait(&full[i % S], (i / S) & 1, nullptr, err);
+                ptx::mbar_wait(&bar.full[i % S], (i / S) & 1, nullptr, err);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- UMMA issuer ----
@@ -512,8 +538,8 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, L::NA, 0, 0);
             const uint32_t s_base = ptx::smem_u32(sstate);
             for (int i = 0; i < nunits; ++i) {
-                if (!ptx::mbar_wait(&a_full[i & 1], (i >> 1) & 1, abort, err)) break;
-                if (!ptx::mbar_wait(acc_empty, (i & 1) ^ 1, abort, err)) break;
+                if (!ptx::mbar_wait(&bar.a_full[i & 1], (i >> 1) & 1, abort, err)) break;
+                if (!ptx::mbar_wait(bar.acc_empty, (i & 1) ^ 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const uint32_t a_base = tmem + KA_A_COL + (uint32_t)(i & 1) * 64u;
 #pragma unroll
@@ -530,10 +556,10 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                          idesc, true);
                     }
                 }
-                ptx::umma_commit(acc_full);
+                ptx::umma_commit(bar.acc_full);
             }
-            ptx::umma_commit(mma_done);
-            ptx::mbar_wait(mma_done, 0, nullptr, err);
+            ptx::umma_commit(bar.mma_done);
+            ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
         }
     } else {
         // --------------------------------------------------------- workers ----
@@ -548,43 +574,88 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         // the leader (lane 0 of warp 0 / warp 4) issues and tracks those stores.
         const bool leader = (warp & 3) == 0 && lane == 0;
         constexpr int HALF_BOXES = L::OUT_BOXES / 2;
-        if (leader) ptx::mbar_arrive(&stg_free[half]);      // staging is free for unit 0
+        if (leader) ptx::mbar_arrive(&bar.stg_free[half]);      // staging is free for unit 0
+        // With the reduced state from a preceding kernel: this kernel may have
+        // started before that kernel finished (programmatic launch); the Q loads
+        // do not depend on it, the state does.
+        if (src.state != nullptr) ptx::wait_prerequisite_grid();
 
-        // A operand of unit i: (new segment ->) the state as bf16 hi + lo in
-        // shared memory; phi(Q) row m, this warp's half, into A buffer i & 1.
-        // In a forward pass this kernel may start while the reduction of the
-        // state is still running (programmatic launch): the Q loads above do not
-        // depend on it, the state does.
-        ptx::wait_prerequisite_grid();
+        // stage the state of `slab` in shared memory as bf16 hi + lo parts
+        bool grid_synced = false;
+        auto stage_state = [&](int slab) -> bool {
+            if (src.state == nullptr && !grid_synced) {
+                // the partial states of every CTA must be in memory (once)
+                if (tid == 0) {
+                    if (grid_wait(src.gbar, src.gbar_target, abort, err)) ptx::mbar_arrive(bar.grid_ready);
+                }
+                if (!warp_wait(bar.grid_ready, 0, abort, err)) return false;
+                grid_synced = true;
+            }
+            const int b = slab / p.groups;
+            const int g = slab % p.groups;
+            // entry x = hh * DD + e of the group; this thread takes x = tid + 256 j
+            constexpr int NE = (G * DD + kWorkerThreads - 1) / kWorkerThreads;
+            float v[NE];
+#pragma unroll
+            for (int j = 0; j < NE; ++j) v[j] = 0.0f;
+            if (src.state != nullptr) {
+#pragma unroll
+                for (int j = 0; j < NE; ++j) {
+                    const int x = tid + j * kWorkerThreads;
+                    const int h = g * G + x / DD;
+                    if (x < G * DD && h < p.H) v[j] = src.state[((long long)b * p.H + h) * DD + x % DD];
+                }
+            } else {
+                // the same additions, in the same order, as kr_reduce_tc: the R
+                // partials of the slab in ascending r, each round's loads in flight
+                // together
+                const long long kstep = (long long)src.ks.q.S * src.ks.q.max_seg * G * DD;
+                const float* base = src.partial +
+                    ks_slot(slab % src.ks.q.grid, slab / src.ks.q.grid, 0, G, src.ks) * DD;
+                for (int r = 0; r < src.ks.q.R; ++r) {
+                    float t[NE];
+#pragma unroll
+                    for (int j = 0; j < NE; ++j) {
+                        const int x = tid + j * kWorkerThreads;
+                        t[j] = x < G * DD ? __ldcg(base + r * kstep + x) : 0.0f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < NE; ++j) v[j] += t[j];
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < NE; ++j) {
+                const int x = tid + j * kWorkerThreads;
+                if (x < G * DD) {
+                    const int hh = x / DD;
+                    const int e = x % DD;
+                    const int k = e / (D + 1);       // state row i = UMMA K index
+                    const int n = e % (D + 1);       // state column j = UMMA N index
+                    const float vv = (g * G + hh < p.H) ? v[j] : 0.0f;
+                    const __nv_bfloat16 vh = __float2bfloat16_rn(vv);
+                    const __nv_bfloat16 vl = __float2bfloat16_rn(vv - __bfloat162float(vh));
+                    *reinterpret_cast<__nv_bfloat16*>(sstate + (hh * 2 + 0) * L::MAT_BYTES + state_off<L::SBO>(n, k)) = vh;
+                    *reinterpret_cast<__nv_bfloat16*>(sstate + (hh * 2 + 1) * L::MAT_BYTES + state_off<L::SBO>(n, k)) = vl;
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            return true;
+        };
+
+        // A operand of unit i: phi(Q) row m, this warp's half, into A buffer
+        // i & 1; at the first unit of a segment also the state of its slab.
         auto prep = [&](int i) -> bool {
             if (i % tps == 0) {
                 if (i > 0) {
                     // the previous unit's UMMAs must be done reading the state
-                    if (!warp_wait(acc_full, (i - 1) & 1, abort, err)) return false;
+                    if (!warp_wait(bar.acc_full, (i - 1) & 1, abort, err)) return false;
                 }
                 int slab, tile, seg;
-                sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
-                const int b = slab / p.groups;
-                const int g = slab % p.groups;
-                for (int hh = 0; hh < G; ++hh) {
-                    const int h = g * G + hh;
-                    const float* src = state + ((long long)b * p.H + h) * DD;
-                    uint8_t* mhi = sstate + (hh * 2 + 0) * L::MAT_BYTES;
-                    uint8_t* mlo = sstate + (hh * 2 + 1) * L::MAT_BYTES;
-                    for (int e = tid; e < DD; e += kWorkerThreads) {
-                        const int k = e / (D + 1);       // state row i = UMMA K index
-                        const int n = e % (D + 1);       // state column j = UMMA N index
-                        const float v = (h < p.H) ? src[e] : 0.0f;
-                        const __nv_bfloat16 vh = __float2bfloat16_rn(v);
-                        const __nv_bfloat16 vl = __float2bfloat16_rn(v - __bfloat162float(vh));
-                        *reinterpret_cast<__nv_bfloat16*>(mhi + state_off<L::SBO>(n, k)) = vh;
-                        *reinterpret_cast<__nv_bfloat16*>(mlo + state_off<L::SBO>(n, k)) = vl;
-                    }
-                }
-                ptx::fence_proxy_async_smem();
+                sched_item(cta, i, tps, p.q, slab, tile, seg);
+                if (!stage_state(slab)) return false;
             }
             const int s = i % S;
-            if (!warp_wait(&full[s], (i / S) & 1, abort, err)) return false;
+            if (!warp_wait(&bar.full[s], (i / S) & 1, abort, err)) return false;
             // row m of box `half`: logical 16-byte chunk q sits at q ^ (m % 8)
             const uint8_t* row = stage_ptr(s) + half * KA_BOX_BYTES + m * kBoxBytesRow;
             uint32_t r[32];
@@ -596,11 +667,11 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 r[4 * q + 2] = relu_bf16x2(v.z);
                 r[4 * q + 3] = relu_bf16x2(v.w);
             }
-            warp_arrive(&empty[s]);
+            warp_arrive(&bar.empty[s]);
             __syncwarp();
             ptx::tmem_st32_wait(lane_base + KA_A_COL + (uint32_t)(i & 1) * 64u + (uint32_t)half * 32u, r);
             ptx::tc_fence_before_sync();
-            warp_arrive(&a_full[i & 1]);
+            warp_arrive(&bar.a_full[i & 1]);
             return true;
         };
 
@@ -608,7 +679,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int i = 0; i < nunits && ok; ++i) {
             if (i + 1 < nunits && !prep(i + 1)) break;
             // ---- epilogue of unit i
-            if (!warp_wait(acc_full, i & 1, abort, err)) break;
+            if (!warp_wait(bar.acc_full, i & 1, abort, err)) break;
             ptx::tc_fence_after_sync();
             float num[HPW][D], den[HPW];
             __syncwarp();
@@ -618,15 +689,15 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 ptx::tmem_ld_row<D>(lane_base + col, lane_base + col + D, num[j], &den[j]);
             }
             ptx::tc_fence_before_sync();
-            warp_arrive(acc_empty);
+            warp_arrive(bar.acc_empty);
             int slab, tile, seg;
-            sched_item(blockIdx.x, i, tps, p.q, slab, tile, seg);
+            sched_item(cta, i, tps, p.q, slab, tile, seg);
             const int b = slab / p.groups;
             const int g = slab % p.groups;
             uint8_t* staging = smem + L::STG_OFF + (i % L::STG_BUFS) * L::STG_BYTES;
             // this half's boxes of the staging tile must be free (the leader
             // released them after the store that last read them)
-            if (!warp_wait(&stg_free[half], i & 1, abort, err)) break;
+            if (!warp_wait(&bar.stg_free[half], i & 1, abort, err)) break;
 #pragma unroll
             for (int j = 0; j < HPW; ++j) {
                 const int hh = half * HPW + j;
@@ -654,9 +725,9 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
             }
             ptx::fence_proxy_async_smem();
-            warp_arrive(&stg_full[2 * half + (i & 1)]);
+            warp_arrive(&bar.stg_full[2 * half + (i & 1)]);
             if ((warp & 3) == 0) {
-                if (!warp_wait(&stg_full[2 * half + (i & 1)], (i >> 1) & 1, abort, err)) break;
+                if (!warp_wait(&bar.stg_full[2 * half + (i & 1)], (i >> 1) & 1, abort, err)) break;
                 if (lane == 0) {
                     const int x0 = g * 128;
                     const int y = tile * KA_TILE;
@@ -664,27 +735,180 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     for (int k = 0; k < HALF_BOXES; ++k) {
                         const int bx = half * HALF_BOXES + k;
                         const int x = x0 + bx * L::OUT_BOX_ELEMS;
-                        if (x < p.H * D) ptx::tma_store_3d(&tmO, staging + bx * KA_BOX_BYTES, x, y, b);
+                        if (x < p.H * D) ptx::tma_store_3d(tmO, staging + bx * KA_BOX_BYTES, x, y, b);
                     }
                     ptx::bulk_commit_group();
                     // release the staging boxes for unit i + 1: the store that last
                     // used them (unit i + 1 - STG_BUFS) must be done reading
                     if (L::STG_BUFS == 2) ptx::bulk_wait_group_read<1>();
                     else ptx::bulk_wait_group_read<0>();
-                    ptx::mbar_arrive(&stg_free[half]);
+                    ptx::mbar_arrive(&bar.stg_free[half]);
                 }
             }
         }
         if (leader) ptx::bulk_wait_group<0>();
     }
+}
 
+// ============================================================ the kernels ===
+// Shared memory of every kernel: a data region (the largest phase it runs;
+// the phases of the single-launch kernel reuse it one after the other), then
+// the mbarriers of its phases, then the control block.
+template <int DATA>
+struct SmemMap {
+    static constexpr int BAR_OFF = DATA;
+    static constexpr int CTL_OFF = BAR_OFF + 2048;
+    static constexpr int BYTES = CTL_OFF + 64 + 1024;      // + 1 KB alignment slack
+    static_assert(BYTES <= kSmemLimit, "shared memory");
+};
+
+__device__ __forceinline__ void kernel_prologue(SharedCtl* ctl, int tid) {
+    if (tid == 0) ctl->abort = 0;
+    if ((tid >> 5) == 0) {
+        ptx::tmem_alloc(&ctl->tmem_base, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+}
+
+__device__ __forceinline__ void kernel_epilogue(SharedCtl* ctl, int tid) {
     ptx::tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if ((tid >> 5) == 0) {
         __syncwarp();
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, kTmemCols);
+        ptx::tmem_dealloc(ctl->tmem_base, kTmemCols);
     }
+}
+
+using KsMap = SmemMap<KS_DATA_BYTES>;
+template <int D, bool OUT_BF16>
+using KaMap = SmemMap<KaLayout<D, OUT_BF16>::DATA_BYTES>;
+template <int D, bool OUT_BF16>
+using FwdMap = SmemMap<(KaLayout<D, OUT_BF16>::DATA_BYTES > KS_DATA_BYTES ? KaLayout<D, OUT_BF16>::DATA_BYTES
+                                                                          : KS_DATA_BYTES)>;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+            const KsParams p, float* __restrict__ partial)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    const KsBars bar = ks_bars(reinterpret_cast<uint64_t*>(smem + KsMap::BAR_OFF));
+    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + KsMap::CTL_OFF);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        bar.init();
+        ptx::fence_mbar_init();
+    }
+    kernel_prologue(ctl, tid);
+    if (tid == kProducerWarp * 32) {
+        ptx::prefetch_tmap(&tmK);
+        ptx::prefetch_tmap(&tmV);
+    }
+    ks_fill_ones(smem, tid);
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    // the reduction kernel may be scheduled now; it waits for this grid's results
+    if (tid == 0) ptx::launch_dependents();
+    ks_phase<D>(&tmK, &tmV, p, blockIdx.x, partial, smem, bar, ctl->tmem_base, &ctl->abort, &g_device_error);
+    kernel_epilogue(ctl, tid);
+}
+
+template <int D, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+            const KaParams p, const float* __restrict__ state)
+{
+    using Map = KaMap<D, OUT_BF16>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    const auto bar = ka_bars<D, OUT_BF16>(reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF));
+    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Map::CTL_OFF);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        bar.init();
+        ptx::fence_mbar_init();
+    }
+    kernel_prologue(ctl, tid);
+    if (tid == kProducerWarp * 32) {
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmO);
+    }
+    ka_zero_state_padding<D, OUT_BF16>(smem, tid);
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0u};
+    ka_phase<D, OUT_BF16>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
+                          &g_device_error);
+    kernel_epilogue(ctl, tid);
+}
+
+// The whole forward in one cooperative launch: the state phase, a grid-wide
+// barrier (bounded), then the apply phase, which sums each slab's partial
+// states itself in the reduction kernel's order. The apply phase's Q loads
+// start as soon as the state phase has released its shared memory, so they
+// overlap the barrier. `gbar` must be zero at launch.
+template <int D, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+             const KsParams ks, const KaParams ka, float* __restrict__ partial, unsigned* gbar)
+{
+    using Map = FwdMap<D, OUT_BF16>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF);
+    const KsBars kbar = ks_bars(bars);
+    const auto abar = ka_bars<D, OUT_BF16>(bars + KS_NUM_BARS);
+    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Map::CTL_OFF);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    if (tid == 0) {
+        kbar.init();
+        abar.init();
+        ptx::fence_mbar_init();
+    }
+    kernel_prologue(ctl, tid);
+    if (tid == kProducerWarp * 32) {
+        ptx::prefetch_tmap(&tmK);
+        ptx::prefetch_tmap(&tmV);
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmO);
+    }
+    ks_fill_ones(smem, tid);
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    ks_phase<D>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error);
+
+    // Warps 0-3 have written this CTA's partial states (after the last
+    // accumulator was complete, i.e. after every state-phase UMMA): make them
+    // visible and arrive. Every worker waits for that before it touches the
+    // apply phase's shared memory or TMEM, which reuse the state phase's.
+    if (warp < 4) {
+        __threadfence();
+        warp_arrive(abar.p1_written);
+    }
+    if (warp < kWorkerWarps) {
+        warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
+        // every CTA arrives at the grid barrier, with or without apply work
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(gbar, 1u);
+        }
+        ka_zero_state_padding<D, OUT_BF16>(smem, tid);
+    }
+    KaStateSrc src{nullptr, partial, ks, gbar, gridDim.x};
+    const int ks_tiles = (int)blockIdx.x < ks.q.grid
+        ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
+    ka_phase<D, OUT_BF16>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
+                          kbar.empty, ks_tiles);
+    kernel_epilogue(ctl, tid);
 }
 
 }  // namespace tc

@@ -41,7 +41,9 @@ def _full_check(oracle, Q, K, V, eps, dtype, what):
 
 
 SMALL = [(1, 1, 1, 32), (1, 7, 3, 32), (2, 31, 2, 64), (1, 129, 5, 32), (2, 1000, 3, 32),
-         (1, 4097, 2, 64), (3, 513, 7, 32), (1, 2048, 70, 32), (2, 300, 18, 64)]
+         (1, 4097, 2, 64), (3, 513, 7, 32), (1, 2048, 70, 32), (2, 300, 18, 64),
+         # more (b, head-group) slabs than CTAs: several segments per CTA
+         (5, 100, 150, 32), (16, 200, 20, 64)]
 
 
 @pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
@@ -130,6 +132,25 @@ def test_deterministic_and_split_equals_forward(dtype):
     assert torch.equal(O1.view(bits), O3.view(bits))
     S2 = ops.kv_state(K, V)
     assert torch.equal(S.view(torch.int32), S2.view(torch.int32))
+
+
+BITWISE = [(1, 1, 1, 32), (2, 31, 2, 64), (2, 1531, 6, 32), (5, 100, 150, 32), (16, 200, 20, 64),
+           (1, 16381, 36, 32)]
+
+
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+@pytest.mark.parametrize("shape", BITWISE, ids=lambda s: "B{}N{}H{}d{}".format(*s))
+def test_single_launch_forward_equals_two_calls(shape, dtype):
+    """forward (one launch: state phase, grid barrier, apply phase) gives the
+    bits of kv_state followed by apply (three launches)."""
+    B, N, H, d = shape
+    w = Workload("bits", B, N, H, d, seed=31 + N)
+    Q, K, V = make_inputs(w, device="cuda")
+    O1 = ops.forward(Q, K, V, out_dtype=dtype)
+    O2 = ops.apply(Q, ops.kv_state(K, V), out_dtype=dtype)
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(O1.view(bits), O2.view(bits))
 
 
 @pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
