@@ -612,15 +612,25 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 const long long kstep = (long long)src.ks.q.S * src.ks.q.max_seg * G * DD;
                 const float* base = src.partial +
                     ks_slot(slab % src.ks.q.grid, slab / src.ks.q.grid, 0, G, src.ks) * DD;
-                for (int r = 0; r < src.ks.q.R; ++r) {
-                    float t[NE];
+                constexpr int RB = NE * 3 <= 64 ? 3 : (NE * 2 <= 64 ? 2 : 1);   // rounds per batch
+                for (int r0 = 0; r0 < src.ks.q.R; r0 += RB) {
+                    float t[RB][NE];
 #pragma unroll
-                    for (int j = 0; j < NE; ++j) {
-                        const int x = tid + j * kWorkerThreads;
-                        t[j] = x < G * DD ? __ldcg(base + r * kstep + x) : 0.0f;
+                    for (int rb = 0; rb < RB; ++rb) {
+#pragma unroll
+                        for (int j = 0; j < NE; ++j) {
+                            const int x = tid + j * kWorkerThreads;
+                            t[rb][j] = (x < G * DD && r0 + rb < src.ks.q.R)
+                                           ? __ldcg(base + (r0 + rb) * kstep + x) : 0.0f;
+                        }
                     }
 #pragma unroll
-                    for (int j = 0; j < NE; ++j) v[j] += t[j];
+                    for (int rb = 0; rb < RB; ++rb) {
+                        if (r0 + rb < src.ks.q.R) {
+#pragma unroll
+                            for (int j = 0; j < NE; ++j) v[j] += t[rb][j];
+                        }
+                    }
                 }
             }
 #pragma unroll
