@@ -183,6 +183,16 @@ const char* sana_linattn_build_info(void);
  */
 sana_la_status sana_linattn_device_error(unsigned int* code, int clear);
 
+/*
+ * Self-test of the failure detection (no counterpart in the paper): launches
+ * one small kernel that waits on an in-kernel barrier nothing ever arrives at,
+ * with a limit of `limit_us` microseconds (1 .. 10,000,000). The wait gives up,
+ * records error code 1 for sana_linattn_device_error and the kernel returns;
+ * the device stays usable. Returns SANA_LA_ERR_INVALID_ARG for a limit out of
+ * range. Asynchronous on `stream`.
+ */
+sana_la_status sana_linattn_selftest_wait_timeout(unsigned int limit_us, sana_la_stream_t stream);
+
 /* Static English text for a status code. */
 const char* sana_linattn_status_string(sana_la_status status);
 

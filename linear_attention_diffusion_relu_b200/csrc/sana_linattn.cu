@@ -406,6 +406,14 @@ sana_la_status sana_linattn_device_error(unsigned int* code, int clear) {
     return SANA_LA_OK;
 }
 
+sana_la_status sana_linattn_selftest_wait_timeout(unsigned int limit_us, sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (limit_us == 0 || limit_us > 10000000u) return SANA_LA_ERR_INVALID_ARG;
+    sana::tc::wait_timeout_selftest<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_us * 1000ull);
+    return launch_status("wait_timeout_selftest");
+}
+
 const char* sana_linattn_status_string(sana_la_status status) {
     switch (status) {
         case SANA_LA_OK: return "ok";

@@ -921,5 +921,19 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     kernel_epilogue(ctl, tid);
 }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives at, with the given limit; the wait gives up, records
+// kErrWaitTimeout in g_device_error and the kernel returns normally.
+__global__ void wait_timeout_selftest(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    if (threadIdx.x == 0) {
+        abort = 0;
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+        ptx::mbar_wait(&bar, 0, &abort, &g_device_error, limit_ns);
+    }
+}
+
 }  // namespace tc
 }  // namespace sana

@@ -34,6 +34,7 @@ SYMBOLS = (
     "sana_linattn_forward_launches",
     "sana_linattn_build_info",
     "sana_linattn_device_error",
+    "sana_linattn_selftest_wait_timeout",
     "sana_linattn_status_string",
     "sana_linattn_last_error",
 )
@@ -76,6 +77,8 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_build_info.restype = ctypes.c_char_p
         lib.sana_linattn_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
         lib.sana_linattn_device_error.restype = st
+        lib.sana_linattn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        lib.sana_linattn_selftest_wait_timeout.restype = st
         lib.sana_linattn_last_error.argtypes = []
         lib.sana_linattn_last_error.restype = ctypes.c_char_p
         if path == LIBRARY:
@@ -141,6 +144,13 @@ def device_error(clear: bool = False) -> int:
     _check(lib, lib.sana_linattn_device_error(ctypes.byref(code), int(clear)),
            "sana_linattn_device_error")
     return int(code.value)
+
+
+def selftest_wait_timeout(limit_us: int = 20000) -> None:
+    """Run the bounded-wait self-test kernel on the current stream (see the header)."""
+    lib = load_library()
+    _check(lib, lib.sana_linattn_selftest_wait_timeout(int(limit_us), _stream(torch.cuda.current_device())),
+           "sana_linattn_selftest_wait_timeout")
 
 
 def make_workspace(B: int, N: int, H: int, d: int, device="cuda") -> torch.Tensor:

@@ -98,6 +98,9 @@ def test_kv_state_and_apply_errors(lib):
     assert ap(FAKE, FAKE, 2, 100, 3, 64, FAKE, 0, -1e-3, None) == ops.ERR_INVALID_ARG
     assert ap(FAKE, FAKE, 2, -100, 3, 64, FAKE, 0, 0.0, None) == ops.ERR_INVALID_ARG
     assert lib.sana_linattn_last_error().decode() == ""
+    # self-test limits are checked before any launch
+    assert lib.sana_linattn_selftest_wait_timeout(0, None) == ops.ERR_INVALID_ARG
+    assert lib.sana_linattn_selftest_wait_timeout(20_000_000, None) == ops.ERR_INVALID_ARG
 
 
 def test_binding_rejects_cpu_tensors(lib):

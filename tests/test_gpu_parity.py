@@ -216,6 +216,22 @@ def test_error_paths_on_device():
     assert e.value.status == ops.ERR_UNSUPPORTED
 
 
+def test_bounded_wait_times_out_and_reports():
+    """A wait on a barrier nothing arrives at gives up after its limit, records
+    error code 1, and the context stays usable (a forward afterwards is correct)."""
+    torch.cuda.synchronize()
+    assert ops.device_error(clear=True) == 0
+    ops.selftest_wait_timeout(20000)          # 20 ms limit
+    torch.cuda.synchronize()
+    assert ops.device_error(clear=True) == 1
+    assert ops.device_error() == 0
+    w = Workload("after_timeout", 1, 100, 3, 32, seed=5)
+    Q, K, V = make_inputs(w, device="cuda")
+    from oracle import default
+    check_output(ops.forward(Q, K, V, out_dtype=torch.float32),
+                 default().forward(to_f64(Q), to_f64(K), to_f64(V), 1e-15), "after timeout")
+
+
 def test_no_kernel_recorded_an_error():
     """Every pipeline wait in the kernels is bounded; none ran out in this run."""
     torch.cuda.synchronize()
