@@ -39,9 +39,6 @@ FALLBACK_HBM_GBS = 6650.0
 # the same build (profiles/), keyed by (kernel set, workload, kernel); None when
 # the kernels changed since the counters were taken
 TRAFFIC_PER_LAUNCH = {
-    # profiles/tc_kernels_sweep_N65536.md, scaled by token-heads (x 0.9722)
-    ("tcgen05-tma", "4096px", "kv_state(KS+KR)"): 297.8e6 + 2.4e6,
-    ("tcgen05-tma", "4096px", "apply(KA)"): 240.4e6,
 }
 SMS = 148
 FP32_LANES_PER_SM = 128
@@ -295,8 +292,20 @@ def run_ours(args):
     value = aggregate_gbs(bytes_per_step, world, ms_max / 1e3)
     mtok = B * N * world / (ms_max / 1e3) / 1e6
 
-    # ---- kernel breakdown: the same kernels through the two-call API, with
-    # events between the state half and the apply half
+    # ---- the dominant (and only) kernel of a forward, fwd_fused_tc: events
+    # around every launch give its average launch duration
+    n_launch = min(args.steps, 2000)
+    lev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+    torch.cuda.synchronize(dev)
+    for i in range(n_launch):
+        lev[2 * i].record(stream)
+        step()
+        lev[2 * i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    fused_ms = statistics.mean(lev[2 * i].elapsed_time(lev[2 * i + 1]) for i in range(n_launch))
+
+    # ---- breakdown: the same phases as separate kernels through the two-call
+    # API, with events between the state half and the apply half
     n_split = min(args.steps, 2000)
     for _ in range(3):
         split_step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
@@ -308,12 +317,15 @@ def run_ours(args):
     ks_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
     ka_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
     hbm_peak, sm_max_mhz, peak_src = measured_peaks()
-    # both halves move 128 B per token-head (K+V read; Q read + bf16 O write)
-    half_bytes = w.token_heads * d * 4
-    kernels = {"kv_state(KS+KR)": (ks_ms, half_bytes), "apply(KA)": (ka_ms, half_bytes)}
-    dom = max(kernels, key=lambda k: kernels[k][0])
-    dom_ms, dom_bytes = kernels[dom]
     impl = ops.implementation()
+    launches = ops.forward_launches(B, N, H, d)
+    if launches == 1:
+        dom, dom_ms, dom_bytes = "fwd_fused_tc", fused_ms, bytes_per_step
+    else:   # three-kernel forward: the larger half (128 B per token-head each)
+        half_bytes = w.token_heads * d * 4
+        halves = {"kv_state(KS+KR)": ks_ms, "apply(KA)": ka_ms}
+        dom = max(halves, key=halves.get)
+        dom_ms, dom_bytes = halves[dom], half_bytes
     if impl["bound"] == "alu":
         flops = w.token_heads * 2 * d * (d + 1)
         achieved = flops / (dom_ms / 1e3) / 1e12
@@ -327,9 +339,11 @@ def run_ours(args):
                 "frac": achieved / hbm_peak, "traffic": TRAFFIC_PER_LAUNCH.get((impl["name"], w.name, dom)),
                 "kernel": dom, "peak_source": f"{peak_src} copy bandwidth (burst)"}
     roof["ms_per_launch"] = dom_ms
-    roof["kernels_ms"] = {k: v[0] for k, v in kernels.items()}
-    roof["timing"] = (f"per-kernel times: CUDA events around kv_state and apply in a {n_split}-step "
-                      "loop of the two-call API right after the timed forward loop")
+    roof["algorithmic_bytes_per_launch"] = dom_bytes
+    roof["split_api_ms"] = {"kv_state(KS+KR)": ks_ms, "apply(KA)": ka_ms}
+    roof["timing"] = (f"launch duration: CUDA events around each of {n_launch} forward launches right "
+                      f"after the timed loop; split_api_ms: events around kv_state and apply in a "
+                      f"{n_split}-step loop of the two-call API")
 
     e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, world)
 
@@ -354,7 +368,7 @@ def run_ours(args):
                               f"{w.token_heads * d * 2 / 1e6:.0f} MB per step vs the 126 MB L2; no flush"),
                        "kernel_impl": impl["name"]},
             "roofline": roof, "e2e": e2e, "clocks": clk,
-            "gpu_launches": ops.forward_launches(B, N, H, d) * args.steps,
+            "gpu_launches": launches * args.steps,
         }
         if cpu is not None:
             line["cpu_baseline"] = cpu

@@ -125,6 +125,13 @@ sana_la_status sana_linattn_apply(const void* Q, const float* state,
  * The whole forward: sana_linattn_kv_state into the workspace, then
  * sana_linattn_apply. Same arguments and rules as the two calls above; the
  * result is bit-identical to calling them in sequence.
+ * It runs as one cooperative kernel launch (state phase, grid-wide barrier,
+ * apply phase). The barrier uses per-CTA flags in the workspace tagged with a
+ * number unique to the call, so the workspace needs no initialisation. Under
+ * stream capture the call also records a memset of those flags before the
+ * kernel, because a replayed graph reuses the captured number. Where the
+ * device cannot hold the whole grid at once, the call falls back to the
+ * kernels of the two calls above.
  */
 sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     int B, int N, int H, int d,
@@ -162,8 +169,9 @@ sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const 
 
 /*
  * Number of kernel launches one sana_linattn_forward call enqueues for these
- * sizes (0 for invalid or unsupported sizes). Useful for graph capture and for
- * counting launches in a profile.
+ * sizes (0 for invalid or unsupported sizes): 1 (the single cooperative
+ * launch; a captured call adds one memset node). Useful for counting launches
+ * in a profile.
  */
 int sana_linattn_forward_launches(int B, int N, int H, int d);
 

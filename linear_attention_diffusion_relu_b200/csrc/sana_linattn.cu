@@ -3,10 +3,12 @@
 // include/sana_linattn.h for the contract.
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <utility>
 
 #include <cudaTypedefs.h>
@@ -25,6 +27,7 @@ void set_last_error(const char* where, cudaError_t e) {
 }
 
 constexpr int kSMs = 148;             // B200: one persistent CTA per SM
+constexpr int kMaxDevicesCached = 64; // per-device caches of launch properties
 constexpr long long kMaxElems = 1LL << 62;
 constexpr long long kMaxGrid = 0x7fffffffLL;
 
@@ -39,7 +42,7 @@ struct Plan {
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
     size_t state_bytes;     // fp32 (B, H, d, d+1)
-    size_t gbar_bytes;      // grid-barrier word of the single-launch forward
+    size_t flag_bytes;      // grid-barrier flags of the single-launch forward (one per CTA)
 };
 
 // Lockstep schedule of S slabs of T tiles over at most kSMs CTAs (see the
@@ -75,7 +78,7 @@ Plan make_plan(int B, int N, int H, int d) {
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * dd);
-    p.gbar_bytes = 256;
+    p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
     return p;
 }
 
@@ -244,10 +247,36 @@ sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H,
 // The whole forward as one cooperative launch (fwd_fused_tc). Returns
 // SANA_LA_ERR_UNSUPPORTED, with nothing enqueued, when the device refuses a
 // cooperative launch of this size, so the caller can use the three kernels.
+// Epochs of the single-launch forward's grid barrier: unique per launch within
+// the process, and started at a random point so that flags another process
+// left in reused memory do not match either.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{[] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32 ^ (unsigned long long)rd() ^
+                (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count()) | 1ull;
+    }()};
+    unsigned long long e = counter.fetch_add(1, std::memory_order_relaxed);
+    return e != 0 ? e : counter.fetch_add(1, std::memory_order_relaxed);
+}
+
+// Blocks of `kernel` one SM holds at once, asked once per device.
+template <typename Kernel>
+int blocks_per_sm(Kernel kernel, int threads, int smem, std::atomic<int> (&cache)[kMaxDevicesCached], int dev) {
+    if (dev < 0 || dev >= kMaxDevicesCached) return -1;
+    int v = cache[dev].load(std::memory_order_acquire);
+    if (v > 0) return v;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, threads, smem) != cudaSuccess) return -1;
+    cache[dev].store(v, std::memory_order_release);
+    return v;
+}
+
 template <int D, bool OUT_BF16>
 sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
-                                    int H, const Plan& p, float* partial, unsigned* gbar, cudaStream_t s) {
+                                    int H, const Plan& p, float* partial, unsigned long long* flags,
+                                    cudaStream_t s) {
     static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<int> per_sm_cache[kMaxDevicesCached];
     CUtensorMap tmK, tmV, tmQ, tmO;
     sana_la_status st;
     if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
@@ -258,18 +287,32 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16>;
     if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
     const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
-    int dev = 0, sms = 0, per_sm = 0;
+    int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, sana::tc::kThreads, smem) != cudaSuccess ||
-        (long long)sms * per_sm < grid) {
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
         return SANA_LA_ERR_UNSUPPORTED;
     }
-    cudaError_t e = cudaMemsetAsync(gbar, 0, sizeof(unsigned), s);
+    const int per_sm = blocks_per_sm(kernel, sana::tc::kThreads, smem, per_sm_cache, dev);
+    if (per_sm <= 0 || (long long)sms * per_sm < grid) {
+        cudaGetLastError();
+        return SANA_LA_ERR_UNSUPPORTED;
+    }
+    const unsigned long long epoch = next_epoch();
+    // A captured graph replays the same epoch: there the flags are cleared by
+    // a memset node before each launch instead.
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &capture);
     if (e != cudaSuccess) {
-        set_last_error("cudaMemsetAsync(grid barrier)", e);
+        set_last_error("cudaStreamIsCapturing", e);
         return SANA_LA_ERR_CUDA;
+    }
+    if (capture != cudaStreamCaptureStatusNone) {
+        e = cudaMemsetAsync(flags, 0, sizeof(unsigned long long) * (size_t)grid, s);
+        if (e != cudaSuccess) {
+            set_last_error("cudaMemsetAsync(grid barrier flags)", e);
+            return SANA_LA_ERR_CUDA;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -281,7 +324,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, gbar);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch);
     if (e != cudaSuccess) {
         set_last_error("fwd_fused_tc", e);
         return SANA_LA_ERR_CUDA;
@@ -313,7 +356,7 @@ extern "C" {
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
     const Plan p = make_plan(B, N, H, d);
-    return p.partial_bytes + p.state_bytes + p.gbar_bytes;
+    return p.partial_bytes + p.state_bytes + p.flag_bytes;
 }
 
 sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,
@@ -357,19 +400,19 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
     Plan p = make_plan(B, N, H, d);
-    if (workspace_bytes < p.partial_bytes + p.state_bytes + p.gbar_bytes) return SANA_LA_ERR_WORKSPACE;
+    if (workspace_bytes < p.partial_bytes + p.state_bytes + p.flag_bytes) return SANA_LA_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     float* partial = reinterpret_cast<float*>(ws);
     float* state = reinterpret_cast<float*>(ws + p.partial_bytes);
-    unsigned* gbar = reinterpret_cast<unsigned*>(ws + p.partial_bytes + p.state_bytes);
+    auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes + p.state_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // one cooperative launch: state phase, grid barrier, apply phase
     p.ka.eps = eps;
     const bool bf16 = out_dtype == SANA_LA_OUT_BF16;
-    st = d == 32 ? (bf16 ? launch_forward_fused<32, true>(Q, K, V, O, B, N, H, p, partial, gbar, s)
-                         : launch_forward_fused<32, false>(Q, K, V, O, B, N, H, p, partial, gbar, s))
-                 : (bf16 ? launch_forward_fused<64, true>(Q, K, V, O, B, N, H, p, partial, gbar, s)
-                         : launch_forward_fused<64, false>(Q, K, V, O, B, N, H, p, partial, gbar, s));
+    st = d == 32 ? (bf16 ? launch_forward_fused<32, true>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                         : launch_forward_fused<32, false>(Q, K, V, O, B, N, H, p, partial, flags, s))
+                 : (bf16 ? launch_forward_fused<64, true>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                         : launch_forward_fused<64, false>(Q, K, V, O, B, N, H, p, partial, flags, s));
     if (st != SANA_LA_ERR_UNSUPPORTED) return st;
     // the device cannot hold the whole grid at once: the same kernels as
     // kv_state + apply, overlapped by programmatic launch
@@ -380,7 +423,7 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
 
 int sana_linattn_forward_launches(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
-    return 1;   // fwd_fused_tc (after a 4-byte memset of its barrier word)
+    return 1;   // fwd_fused_tc (plus a memset of its barrier flags when captured in a graph)
 }
 
 const char* sana_linattn_build_info(void) { return "impl=tcgen05-tma;bound=hbm"; }

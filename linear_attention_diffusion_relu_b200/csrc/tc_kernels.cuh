@@ -455,31 +455,52 @@ __device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid) {
 // Where the apply phase gets the state of a slab from:
 //   state != nullptr   the reduced fp32 state (B, H, d, d+1) of the reduction kernel
 //   otherwise          the partial states of the state phase (same launch), summed
-//                      here in the reduction kernel's order, once `gbar` shows
-//                      every CTA has written them
+//                      here in the reduction kernel's order, once every CTA's
+//                      arrival flag holds this launch's epoch
 struct KaStateSrc {
     const float* state;
     const float* partial;
     KsParams ks;
-    unsigned* gbar;
-    unsigned gbar_target;
+    const unsigned long long* flags;   // one arrival flag per CTA of the grid
+    unsigned long long epoch;          // unique to this launch (set by the host)
+    int nflags;
 };
 
-// Bounded spin until every CTA of the grid has arrived at the barrier word.
-__device__ __forceinline__ bool grid_wait(unsigned* gbar, unsigned target, volatile int* abort,
-                                          uint32_t* err) {
+// Grid-wide barrier of the single-launch forward. CTA c announces that its
+// partial states are in memory by storing the launch's epoch into flags[c]
+// (after a fence); the barrier is passed when every flag holds the epoch.
+// The host draws a new 64-bit epoch for every launch, so flags left by earlier
+// launches (or any other bytes) never pass for this one and the flag array
+// needs no reset between launches.
+__device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned long long epoch) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
+}
+
+// Bounded spin of one whole warp until every flag holds `epoch` (warp-uniform
+// result). On a timeout it records the error code and sets *abort.
+__device__ __forceinline__ bool grid_wait(const unsigned long long* flags, int nflags,
+                                          unsigned long long epoch, volatile int* abort, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (;;) {
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
-        if (v >= target) return true;
-        if (*abort) return false;
-        if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
-            atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
-            *abort = 1;
-            return false;
+        bool mine = true;
+        for (int c = lane; c < nflags; c += 32) {
+            unsigned long long v;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + c) : "memory");
+            mine = mine && v == epoch;
         }
-        __nanosleep(256);
+        if (__all_sync(0xffffffffu, mine)) return true;
+        bool give_up = *abort != 0;
+        if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
+            if (lane == 0) {
+                atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
+                *abort = 1;
+            }
+            give_up = true;
+        }
+        if (__any_sync(0xffffffffu, give_up)) return false;
+        __nanosleep(200);
     }
 }
 
@@ -585,8 +606,9 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         auto stage_state = [&](int slab) -> bool {
             if (src.state == nullptr && !grid_synced) {
                 // the partial states of every CTA must be in memory (once)
-                if (tid == 0) {
-                    if (grid_wait(src.gbar, src.gbar_target, abort, err)) ptx::mbar_arrive(bar.grid_ready);
+                if (warp == 0) {
+                    if (grid_wait(src.flags, src.nflags, src.epoch, abort, err) && lane == 0)
+                        ptx::mbar_arrive(bar.grid_ready);
                 }
                 if (!warp_wait(bar.grid_ready, 0, abort, err)) return false;
                 grid_synced = true;
@@ -850,7 +872,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0u};
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, 0};
     ka_phase<D, OUT_BF16>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
                           &g_device_error);
     kernel_epilogue(ctl, tid);
@@ -860,12 +882,14 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 // barrier (bounded), then the apply phase, which sums each slab's partial
 // states itself in the reduction kernel's order. The apply phase's Q loads
 // start as soon as the state phase has released its shared memory, so they
-// overlap the barrier. `gbar` must be zero at launch.
+// overlap the barrier. `flags` has one slot per CTA; `epoch` is unique to the
+// launch.
 template <int D, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-             const KsParams ks, const KaParams ka, float* __restrict__ partial, unsigned* gbar)
+             const KsParams ks, const KaParams ka, float* __restrict__ partial,
+             unsigned long long* flags, const unsigned long long epoch)
 {
     using Map = FwdMap<D, OUT_BF16>;
     extern __shared__ uint8_t smem_raw[];
@@ -907,13 +931,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     if (warp < kWorkerWarps) {
         warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
         // every CTA arrives at the grid barrier, with or without apply work
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(gbar, 1u);
-        }
+        if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
         ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     }
-    KaStateSrc src{nullptr, partial, ks, gbar, gridDim.x};
+    KaStateSrc src{nullptr, partial, ks, flags, epoch, (int)gridDim.x};
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
     ka_phase<D, OUT_BF16>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,

@@ -174,6 +174,56 @@ def test_guard_bands(dtype):
     assert torch.all(wsbig[:256] == 0xA5) and torch.all(wsbig[256 + wsb:] == 0xA5)
 
 
+@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
+def test_forward_in_cuda_graph(dtype):
+    """A captured forward replays correctly with new inputs each time: the
+    grid barrier's flags are cleared by the captured memset, not by a fresh
+    epoch (which a replay cannot draw)."""
+    B, N, H, d = 2, 3001, 9, 32
+    w = Workload("graph", B, N, H, d, seed=41)
+    Q, K, V = make_inputs(w, device="cuda")
+    O = torch.empty((B, N, H, d), dtype=dtype, device="cuda")
+    ws = ops.make_workspace(B, N, H, d, "cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ops.forward(Q, K, V, out_dtype=dtype, out=O, workspace=ws)      # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        ops.forward(Q, K, V, out_dtype=dtype, out=O, workspace=ws)
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    for seed in (1, 2, 3):
+        Qn, Kn, Vn = make_inputs(Workload("graph", B, N, H, d, seed=seed), device="cuda")
+        Q.copy_(Qn), K.copy_(Kn), V.copy_(Vn)
+        O.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = ops.forward(Qn, Kn, Vn, out_dtype=dtype)
+        torch.cuda.synchronize()
+        assert torch.equal(O.view(bits), ref.view(bits)), seed
+    assert ops.device_error() == 0
+
+
+def test_workspace_shared_across_shapes_and_calls():
+    """One workspace, sized for the largest shape, serves forwards of several
+    shapes interleaved with kv_state calls; each result equals a forward with a
+    fresh workspace bit for bit (stale partial states or barrier flags of an
+    earlier call never leak into a later one)."""
+    shapes = [(2, 1531, 6, 32), (1, 16381, 36, 32), (3, 200, 5, 64), (2, 1531, 6, 32)]
+    wsb = max(ops.workspace_bytes(*sh) for sh in shapes)
+    ws = torch.randint(0, 256, (wsb,), dtype=torch.uint8, device="cuda",
+                       generator=torch.Generator("cuda").manual_seed(5))
+    for i, (B, N, H, d) in enumerate(shapes * 2):
+        Q, K, V = make_inputs(Workload("shared", B, N, H, d, seed=60 + i), device="cuda")
+        O = ops.forward(Q, K, V, out_dtype=torch.float32, workspace=ws[:ops.workspace_bytes(B, N, H, d)])
+        ops.kv_state(K, V, workspace=ws[:ops.workspace_bytes(B, N, H, d)])
+        ref = ops.forward(Q, K, V, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert torch.equal(O.view(torch.int32), ref.view(torch.int32)), (B, N, H, d)
+    assert ops.device_error() == 0
+
+
 def test_runs_on_caller_stream(oracle):
     w = Workload("stream", 1, 777, 3, 64, seed=9)
     Q, K, V = make_inputs(w, device="cuda")
