@@ -34,12 +34,24 @@
  * (B, H, d, d+1) row-major, entry (b, h, i, j) at ((b*H + h)*d + i)*(d+1) + j,
  * with column j = d holding the normaliser sum_n phi(K_{n,i}).
  *
+ * Block-causal form ("linear-diffusion-transformer-4k-efficient-generation",
+ * section "技术演进：从图像到视频与世界模型": SANA-Video turns the linear
+ * attention into block causal linear attention; the pages give no formula).
+ * Reading: the tokens form blocks of L consecutive tokens (block j holds tokens
+ * j*L .. min((j+1)*L, N) - 1, e.g. one latent video frame per block; the
+ * video row of the token table in "08_sana高效高分辨率生成", section
+ * "Linear Attention 的原理", has 16 frames of 65,536 tokens); a query of
+ * block j attends to every key of blocks 0 .. j, so it uses the prefix state
+ *   P[b,h,j] = sum over tokens n < min((j+1)*L, N) of phi(K_n)^T [V_n | 1]
+ * in place of S. The prefix states are (B, H, nblk, d, d+1), nblk = ceil(N/L).
+ *
  * All arithmetic is IEEE double. Sums run in token order n = 0 .. N-1 and
  * feature order i = 0 .. d-1, nothing is blocked or reordered. OpenMP only
  * spreads independent (b, h) pairs or independent query rows over threads, which
  * does not change any sum.
  */
 #include <stddef.h>
+#include <stdlib.h>
 #include <omp.h>
 
 static double relu(double x) { return x > 0.0 ? x : 0.0; }
@@ -121,4 +133,70 @@ void oracle_forward(const double* Q, const double* K, const double* V,
 {
     oracle_state(K, V, B, N, H, d, S);
     oracle_apply(Q, S, B, N, H, d, eps, O, NULL);
+}
+
+/* offset of entry (b, h, j, i, c) in (B, H, nblk, d, d+1) prefix states */
+static size_t at_prefix(long b, long h, long j, long i, long c, long H, long nblk, long d)
+{
+    return ((((size_t)b * H + h) * nblk + j) * d + i) * (d + 1) + c;
+}
+
+/*
+ * Block-causal prefix states: for every (b, h) a running sum over tokens in
+ * order; after the last token of block j the running sum is P[b,h,j].
+ */
+void oracle_block_causal_state(const double* K, const double* V, long B, long N, long H, long d,
+                               long L, double* P)
+{
+    const long nblk = (N + L - 1) / L;
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b) {
+        for (long h = 0; h < H; ++h) {
+            double* run = (double*)malloc(sizeof(double) * (size_t)d * (d + 1));
+            for (long e = 0; e < d * (d + 1); ++e)
+                run[e] = 0.0;
+            for (long j = 0; j < nblk; ++j) {
+                const long end = (j + 1) * L < N ? (j + 1) * L : N;
+                for (long n = j * L; n < end; ++n) {
+                    for (long i = 0; i < d; ++i) {
+                        double k = relu(K[at_bnhd(b, n, h, i, N, H, d)]);
+                        for (long c = 0; c < d; ++c)
+                            run[i * (d + 1) + c] += k * V[at_bnhd(b, n, h, c, N, H, d)];
+                        run[i * (d + 1) + d] += k * 1.0;
+                    }
+                }
+                for (long i = 0; i < d; ++i)
+                    for (long c = 0; c <= d; ++c)
+                        P[at_prefix(b, h, j, i, c, H, nblk, d)] = run[i * (d + 1) + c];
+            }
+            free(run);
+        }
+    }
+}
+
+/*
+ * Block-causal apply: query row (b, n, h) of block j = n / L uses P[b,h,j]:
+ *   O[b,n,h,c] = (sum_i relu(Q_i) P[b,h,j,i,c]) / (sum_i relu(Q_i) P[b,h,j,i,d] + eps)
+ */
+void oracle_block_causal_apply(const double* Q, const double* P, long B, long N, long H, long d,
+                               long L, double eps, double* O)
+{
+    const long nblk = (N + L - 1) / L;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (long b = 0; b < B; ++b) {
+        for (long n = 0; n < N; ++n) {
+            const long j = n / L;
+            for (long h = 0; h < H; ++h) {
+                double den = 0.0;
+                for (long i = 0; i < d; ++i)
+                    den += relu(Q[at_bnhd(b, n, h, i, N, H, d)]) * P[at_prefix(b, h, j, i, d, H, nblk, d)];
+                for (long c = 0; c < d; ++c) {
+                    double num = 0.0;
+                    for (long i = 0; i < d; ++i)
+                        num += relu(Q[at_bnhd(b, n, h, i, N, H, d)]) * P[at_prefix(b, h, j, i, c, H, nblk, d)];
+                    O[at_bnhd(b, n, h, c, N, H, d)] = num / (den + eps);
+                }
+            }
+        }
+    }
 }

@@ -53,6 +53,12 @@ class Oracle:
         lib.oracle_apply.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long,
                                      _c_double, _ptr, _ptr]
         lib.oracle_apply.restype = None
+        lib.oracle_block_causal_state.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long,
+                                                  _c_long, _ptr]
+        lib.oracle_block_causal_state.restype = None
+        lib.oracle_block_causal_apply.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long,
+                                                  _c_long, _c_double, _ptr]
+        lib.oracle_block_causal_apply.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         self._lib = lib
@@ -94,6 +100,37 @@ class Oracle:
     def forward(self, Q, K, V, eps: float, return_den: bool = False):
         S = self.state(K, V)
         return self.apply(Q, S, eps, return_den=return_den)
+
+
+    def block_causal_state(self, K, V, L: int) -> np.ndarray:
+        """Inclusive prefix states of blocks of L tokens: (B, H, nblk, d, d+1)."""
+        K = self._f64(K)
+        V = self._f64(V)
+        if K.shape != V.shape:
+            raise ValueError("K and V must have the same shape")
+        if L < 1:
+            raise ValueError("block length must be >= 1")
+        B, N, H, d = K.shape
+        nblk = -(-N // L)
+        P = np.empty((B, H, nblk, d, d + 1), dtype=np.float64)
+        self._lib.oracle_block_causal_state(K.ctypes.data, V.ctypes.data, B, N, H, d, int(L),
+                                            P.ctypes.data)
+        return P
+
+    def block_causal_apply(self, Q, P, L: int, eps: float) -> np.ndarray:
+        """O for block-causal attention from the prefix states P."""
+        Q = self._f64(Q)
+        P = np.ascontiguousarray(np.asarray(P, dtype=np.float64))
+        B, N, H, d = Q.shape
+        if L < 1 or P.shape != (B, H, -(-N // L), d, d + 1):
+            raise ValueError(f"prefix states {P.shape} do not match Q {Q.shape} and L={L}")
+        O = np.empty((B, N, H, d), dtype=np.float64)
+        self._lib.oracle_block_causal_apply(Q.ctypes.data, P.ctypes.data, B, N, H, d, int(L),
+                                            float(eps), O.ctypes.data)
+        return O
+
+    def block_causal_forward(self, Q, K, V, L: int, eps: float) -> np.ndarray:
+        return self.block_causal_apply(Q, self.block_causal_state(K, V, L), L, eps)
 
 
 _DEFAULT: Oracle | None = None

@@ -70,16 +70,17 @@ def pin_bruteforce(orc, Q, K, V, eps, tol=1e-12):
 def exact_rational(Q, K, V, eps: Fraction):
     """The quadratic definition in exact rational arithmetic (small inputs)."""
     B, N, H, d = Q.shape
+    M = K.shape[1]           # keys may be fewer than queries (a causal prefix)
     out = np.empty((B, N, H, d), dtype=object)
     relu = (lambda x: x if x > 0 else Fraction(0))
     for b in range(B):
         for h in range(H):
             for n in range(N):
                 w = [sum((relu(Fraction(Q[b, n, h, i])) * relu(Fraction(K[b, m, h, i]))
-                          for i in range(d)), Fraction(0)) for m in range(N)]
+                          for i in range(d)), Fraction(0)) for m in range(M)]
                 den = sum(w, Fraction(0)) + eps
                 for j in range(d):
-                    num = sum((w[m] * Fraction(V[b, m, h, j]) for m in range(N)), Fraction(0))
+                    num = sum((w[m] * Fraction(V[b, m, h, j]) for m in range(M)), Fraction(0))
                     out[b, n, h, j] = num / den
     return out
 
@@ -269,9 +270,91 @@ def pin_bruteforce_random(orc, seed=15):
     pin_bruteforce(orc, Q, K, V, 1e-15)
 
 
+# ------------------------------------------------------------ block-causal --
+# "linear-diffusion-transformer-4k-efficient-generation", section
+# "技术演进：从图像到视频与世界模型" (SANA-Video: block causal linear attention).
+# Reading: blocks of L consecutive tokens; a query of block j sees the keys of
+# blocks 0 .. j.
+
+def bruteforce_block_causal(Q, K, V, L, eps):
+    """The quadratic definition with a block mask: W[n, m] = phi(Q_n).phi(K_m)
+    where m // L <= n // L, else 0; O = (W V) / (W 1 + eps)."""
+    Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
+    B, N, H, d = Q.shape
+    blk = np.arange(N) // L
+    mask = (blk[None, :] <= blk[:, None]).astype(np.float64)
+    O = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            W = (np.maximum(Q[b, :, h, :], 0.0) @ np.maximum(K[b, :, h, :], 0.0).T) * mask
+            O[b, :, h, :] = (W @ V[b, :, h, :]) / (W.sum(axis=1, keepdims=True) + eps)
+    return O
+
+
+def pin_block_causal_bruteforce(orc, seed=21):
+    """Oracle == masked n x n form for several block lengths, including L = 1
+    (token-causal), a ragged last block, and L >= N (no mask)."""
+    Q, K, V = _rng_inputs(seed, B=2, N=37, H=3, d=8)
+    Q[1, 12, 1, :] = -np.abs(Q[1, 12, 1, :]) - 0.1   # a zero-weight row
+    for L in (1, 4, 10, 37, 64):
+        O = orc.block_causal_forward(Q, K, V, L, 1e-15)
+        R = bruteforce_block_causal(Q, K, V, L, 1e-15)
+        err = row_relerr(O, R)
+        assert err.max() <= 1e-12, (L, err.max())
+        zero = np.linalg.norm(R, axis=-1) == 0
+        assert np.all(O[zero] == 0.0)
+
+
+def pin_block_causal_exact_integers(orc, seed=22):
+    """Small integers, eps = 1/4, L = 2: equal to the correctly rounded exact
+    rational value of the masked definition, block by block."""
+    rng = np.random.default_rng(seed)
+    B, N, H, d, L = 1, 5, 2, 3, 2
+    Q, K, V = (rng.integers(-3, 4, size=(B, N, H, d)).astype(np.float64) for _ in range(3))
+    O = orc.block_causal_forward(Q, K, V, L, 0.25)
+    for n in range(N):
+        end = (n // L + 1) * L
+        want = exact_rational(Q[:, n:n + 1], K[:, :end], V[:, :end], Fraction(1, 4))
+        assert np.array_equal(O[:, n:n + 1], np.vectorize(float)(want).astype(np.float64)), n
+
+
+def pin_block_causal_reductions(orc, seed=23):
+    """L >= N is the plain forward, bit for bit; the last prefix state is the
+    full state; block 0 alone is the plain forward over block 0's tokens."""
+    Q, K, V = _rng_inputs(seed, B=2, N=30, H=2, d=8)
+    assert np.array_equal(orc.block_causal_forward(Q, K, V, 30, 1e-15), orc.forward(Q, K, V, 1e-15))
+    P = orc.block_causal_state(K, V, 7)
+    assert P.shape == (2, 2, 5, 8, 9)
+    assert np.array_equal(P[:, :, -1], orc.state(K, V))
+    assert np.array_equal(P[:, :, 0], orc.state(K[:, :7], V[:, :7]))
+    O = orc.block_causal_forward(Q, K, V, 7, 1e-15)
+    assert np.array_equal(O[:, :7], orc.forward(Q[:, :7], K[:, :7], V[:, :7], 1e-15))
+
+
+def pin_block_causal_no_future(orc, seed=24):
+    """Keys and values of later blocks never reach earlier blocks' outputs (bit
+    for bit); those of the query's own block do."""
+    Q, K, V = _rng_inputs(seed, B=1, N=40, H=2, d=8)
+    L = 8
+    O = orc.block_causal_forward(Q, K, V, L, 1e-15)
+    K2, V2 = K.copy(), V.copy()
+    K2[:, 24:] = 5.0 * np.abs(K2[:, 24:])
+    V2[:, 24:] += 3.0
+    O2 = orc.block_causal_forward(Q, K2, V2, L, 1e-15)
+    assert np.array_equal(O2[:, :24], O[:, :24])
+    assert np.all(np.abs(O2[:, 24:] - O[:, 24:]).max(axis=-1) > 0)
+    K3 = K.copy()
+    K3[:, 23] = 4.0 * np.abs(K3[:, 23])      # last token of block 2
+    O3 = orc.block_causal_forward(Q, K3, V, L, 1e-15)
+    assert np.array_equal(O3[:, :16], O[:, :16])
+    assert np.all(np.abs(O3[:, 16:24] - O[:, 16:24]).max(axis=-1) > 0)
+
+
 ALL_PINS = [
     pin_bruteforce_tiny, pin_bruteforce_random, pin_exact_integers, pin_hand_example,
     pin_single_token, pin_equal_keys, pin_one_hot, pin_constant_column,
     pin_key_permutation, pin_query_permutation_and_independence, pin_convex_hull,
     pin_zero_query, pin_scale_invariance, pin_linearity_in_v, pin_state_definition,
+    pin_block_causal_bruteforce, pin_block_causal_exact_integers, pin_block_causal_reductions,
+    pin_block_causal_no_future,
 ]

@@ -51,6 +51,27 @@ MUTANTS = [
     ("num_skips_first_feature",
      "for (long i = 0; i < d; ++i)\n                        num +=",
      "for (long i = 1; i < d; ++i)\n                        num +=", 0),
+    # block-causal form
+    ("bc_no_relu_on_K",
+     "double k = relu(K[at_bnhd(b, n, h, i, N, H, d)]);",
+     "double k = K[at_bnhd(b, n, h, i, N, H, d)];", 1),
+    ("bc_block_drops_last_token",
+     "const long end = (j + 1) * L < N ? (j + 1) * L : N;",
+     "const long end = (j + 1) * L - 1 < N ? (j + 1) * L - 1 : N;", 0),
+    ("bc_block_skips_first_token",
+     "for (long n = j * L; n < end; ++n) {",
+     "for (long n = j * L + 1; n < end; ++n) {", 0),
+    ("bc_query_uses_previous_block",
+     "const long j = n / L;",
+     "const long j = n / L > 0 ? n / L - 1 : 0;", 0),
+    ("bc_query_uses_next_block",
+     "const long j = n / L;",
+     "const long j = n / L < nblk - 1 ? n / L + 1 : n / L;", 0),
+    ("bc_den_from_column_0",
+     "* P[at_prefix(b, h, j, i, d, H, nblk, d)];",
+     "* P[at_prefix(b, h, j, i, 0, H, nblk, d)];", 0),
+    ("bc_no_eps",
+     "] = num / (den + eps);", "] = num / (den);", 1),
 ]
 
 
