@@ -160,6 +160,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------- CPU oracle --
 
+def input_generator(w) -> str:
+    """Where the workload's inputs are drawn: the seeded CUDA generator for the
+    largest shapes (a host draw of billions of values takes minutes), else the
+    host generator."""
+    import torch
+    big = w.token_heads * w.d * 3 > 2_000_000_000
+    return "cuda" if big and torch.cuda.is_available() else "cpu"
+
+
 def oracle_sample(w, seconds: float, max_heads: int | None = None):
     """Time the fp64 oracle (as it stands) on whole heads of workload w, all N
     tokens each, adding heads until about `seconds` of CPU work is done.
@@ -169,7 +178,7 @@ def oracle_sample(w, seconds: float, max_heads: int | None = None):
     from oracle import default
     from linear_attention_diffusion_relu_b200.workloads import make_inputs
     orc = default()
-    Q, K, V = make_inputs(w)      # host tensors, bf16
+    Q, K, V = (t.cpu() for t in make_inputs(w, generator_device=input_generator(w)))   # bf16
     pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
     if max_heads is not None:
         pairs = pairs[:max_heads]
@@ -180,8 +189,10 @@ def oracle_sample(w, seconds: float, max_heads: int | None = None):
         sl = [(torch.stack([t[b, :, h, :] for b, h in batch], dim=1)[None]
                .to(torch.float64).numpy()) for t in (Q, K, V)]
         t0 = time.perf_counter()
-        S = orc.state(sl[1], sl[2])
-        O = orc.apply(sl[0], S, w.eps)
+        if w.block:
+            O = orc.block_causal_apply(sl[0], orc.block_causal_state(sl[1], sl[2], w.block), w.block, w.eps)
+        else:
+            O = orc.apply(sl[0], orc.state(sl[1], sl[2]), w.eps)
         elapsed += time.perf_counter() - t0
         assert np.isfinite(O).all()
         done += batch
@@ -189,7 +200,8 @@ def oracle_sample(w, seconds: float, max_heads: int | None = None):
     token_heads = len(done) * w.N
     nbytes = token_heads * w.d * (3 * 2 + 2)
     desc = (f"{w.name}: {len(done)} of {w.B * w.H} (b,h) pairs, all {w.N} tokens each "
-            f"({token_heads} token-heads), fp64 oracle state+apply")
+            f"({token_heads} token-heads), fp64 oracle state+apply"
+            + (f", block-causal L={w.block}" if w.block else ""))
     return nbytes / elapsed / 1e9, token_heads / w.H / elapsed / 1e6, orc.num_threads(), desc, elapsed
 
 
@@ -198,7 +210,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     from linear_attention_diffusion_relu_b200.workloads import WORKLOADS
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     per_step = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, per_step / 4, max_heads=2)
@@ -216,7 +228,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "mtokens_per_s": statistics.median(mts),
-        "config": {"workload": WORKLOAD, "B": w.B, "N": w.N, "H": w.H, "d": w.d,
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d,
                    "sample_per_step": desc},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc},
@@ -245,23 +257,36 @@ def run_ours(args):
     ops.load_library()
 
     w = WORKLOADS[args.workload]
-    B, N, H, d = w.B, w.N, w.H, w.d
-    Q, K, V = make_inputs(w, device=dev)
+    B, N, H, d, L = w.B, w.N, w.H, w.d, w.block
+    Q, K, V = make_inputs(w, device=dev, generator_device=input_generator(w))
     if rank > 0:   # every rank its own independent batch of the same shape
         Q, K, V = (t.roll(shifts=rank, dims=1).contiguous() for t in (Q, K, V))
     out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
-    state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=dev)
-    ws = ops.make_workspace(B, N, H, d, dev)
     stream = torch.cuda.current_stream(dev)
+    if L:   # block-causal: prefix states of blocks of L tokens
+        state = torch.empty((B, H, ops.num_blocks(N, L), d, d + 1), dtype=torch.float32, device=dev)
+        ws = ops.make_block_causal_workspace(B, N, H, d, L, dev)
+    else:
+        state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=dev)
+        ws = ops.make_workspace(B, N, H, d, dev)
 
     def step():
-        ops.forward(Q, K, V, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws)
+        if L:
+            ops.block_causal_forward(Q, K, V, L, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws)
+        else:
+            ops.forward(Q, K, V, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws)
 
     def split_step(ev):
         ev[0].record(stream)
-        ops.kv_state(K, V, state=state, workspace=ws)
+        if L:
+            ops.block_causal_kv_state(K, V, L, states=state, workspace=ws)
+        else:
+            ops.kv_state(K, V, state=state, workspace=ws)
         ev[1].record(stream)
-        ops.apply(Q, state, out_dtype=torch.bfloat16, eps=w.eps, out=out)
+        if L:
+            ops.block_causal_apply(Q, state, L, out_dtype=torch.bfloat16, eps=w.eps, out=out)
+        else:
+            ops.apply(Q, state, out_dtype=torch.bfloat16, eps=w.eps, out=out)
         ev[2].record(stream)
 
     for _ in range(args.warmup):
@@ -318,7 +343,7 @@ def run_ours(args):
     ka_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
     hbm_peak, sm_max_mhz, peak_src = measured_peaks()
     impl = ops.implementation()
-    launches = ops.forward_launches(B, N, H, d)
+    launches = ops.block_causal_forward_launches(B, N, H, d, L) if L else ops.forward_launches(B, N, H, d)
     if launches == 1:
         dom, dom_ms, dom_bytes = "fwd_fused_tc", fused_ms, bytes_per_step
     else:   # three-kernel forward: the larger half (128 B per token-head each)
@@ -361,6 +386,7 @@ def run_ours(args):
             "dtype": "bf16", "data": "synthetic",
             "mtokens_per_s": mtok, "pct_of_hbm_peak": 100.0 * value / (hbm_peak * world),
             "config": {"workload": w.name, "B": B, "N": N, "H": H, "d": d,
+                       **({"form": "block-causal", "block": L} if L else {}),
                        "io": "bf16 Q/K/V in, bf16 O out, fp32 state and accumulation",
                        "eps": w.eps, "per_rank": f"one independent {w.name} batch",
                        "parallelism": f"dp{world}",
@@ -385,17 +411,23 @@ def run_e2e(args, w, dev, stream, world):
     import torch
     from linear_attention_diffusion_relu_b200 import ops
     from linear_attention_diffusion_relu_b200.workloads import make_inputs
-    hQ, hK, hV = (t.pin_memory() for t in make_inputs(w))
+    hQ, hK, hV = (t.cpu().pin_memory() for t in make_inputs(w, generator_device=input_generator(w)))
     hO = torch.empty(hQ.shape, dtype=torch.bfloat16).pin_memory()
     dQ, dK, dV = (torch.empty_like(t, device=dev) for t in (hQ, hK, hV))
     dO = torch.empty(hQ.shape, dtype=torch.bfloat16, device=dev)
-    ws = ops.make_workspace(w.B, w.N, w.H, w.d, dev)
+    L = w.block
+    ws = (ops.make_block_causal_workspace(w.B, w.N, w.H, w.d, L, dev) if L
+          else ops.make_workspace(w.B, w.N, w.H, w.d, dev))
 
     def one():
         dQ.copy_(hQ, non_blocking=True)
         dK.copy_(hK, non_blocking=True)
         dV.copy_(hV, non_blocking=True)
-        ops.forward(dQ, dK, dV, out_dtype=torch.bfloat16, eps=w.eps, out=dO, workspace=ws)
+        if L:
+            ops.block_causal_forward(dQ, dK, dV, L, out_dtype=torch.bfloat16, eps=w.eps, out=dO,
+                                     workspace=ws)
+        else:
+            ops.forward(dQ, dK, dV, out_dtype=torch.bfloat16, eps=w.eps, out=dO, workspace=ws)
         hO.copy_(dO, non_blocking=True)
 
     for _ in range(3):

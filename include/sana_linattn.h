@@ -140,6 +140,60 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     sana_la_stream_t stream);
 
 /*
+ * Block-causal form ("linear-diffusion-transformer-4k-efficient-generation",
+ * section "技术演进：从图像到视频与世界模型": SANA-Video's block causal linear
+ * attention; the pages give no formula). The tokens form blocks of L
+ * consecutive tokens (block j = tokens j*L .. min((j+1)*L, N) - 1, e.g. one
+ * latent video frame each); a query of block j attends to the keys of blocks
+ * 0 .. j, i.e. it uses the inclusive prefix state
+ *   P[b,h,j] = sum over tokens n < min((j+1)*L, N) of phi(K_n)^T [V_n | 1]
+ * in place of the state of sana_linattn_apply. nblk = ceil(N / L).
+ *
+ * L must be a positive multiple of 128 (SANA_LA_ERR_UNSUPPORTED otherwise; 0
+ * or negative is SANA_LA_ERR_INVALID_ARG); sizes whose per-block partial states
+ * would exceed 4 GiB of workspace are SANA_LA_ERR_UNSUPPORTED. N need not be a
+ * multiple of L. Work is spread over ceil(B*H/(128/d)) slabs times R CTAs,
+ * where R is the largest divisor of L/128 that keeps the grid within the 148
+ * SMs; L/128 with few divisors (e.g. L = 128) therefore runs on few SMs.
+ * Other arguments, layouts and errors are as for the calls above.
+ */
+
+/* Workspace bytes of the block-causal calls (0 for invalid or unsupported sizes). */
+size_t sana_linattn_block_causal_workspace_bytes(int B, int N, int H, int d, int L);
+
+/*
+ * Prefix states: `states` fp32 (B, H, nblk, d, d+1), device, written in full;
+ * entry (b, h, j, i, c) at (((b*H + h)*nblk + j)*d + i)*(d+1) + c. The blocks'
+ * partial sums are added in ascending block order (and within a block in a
+ * fixed order), so the result does not depend on scheduling.
+ */
+sana_la_status sana_linattn_block_causal_kv_state(const void* K, const void* V,
+                                                  int B, int N, int H, int d, int L,
+                                                  float* states,
+                                                  void* workspace, size_t workspace_bytes,
+                                                  sana_la_stream_t stream);
+
+/* O from the prefix states: query row (b, n, h) uses states[b, h, n / L]. */
+sana_la_status sana_linattn_block_causal_apply(const void* Q, const float* states,
+                                               int B, int N, int H, int d, int L,
+                                               void* O, sana_la_out_dtype out_dtype, float eps,
+                                               sana_la_stream_t stream);
+
+/*
+ * The whole block-causal forward (three launches: state kernel, prefix
+ * reduction, apply kernel); bit-identical to sana_linattn_block_causal_kv_state
+ * followed by sana_linattn_block_causal_apply.
+ */
+sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, const void* V,
+                                                 int B, int N, int H, int d, int L,
+                                                 void* O, sana_la_out_dtype out_dtype, float eps,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 sana_la_stream_t stream);
+
+/* Kernel launches one sana_linattn_block_causal_forward call enqueues (0 if invalid). */
+int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L);
+
+/*
  * sana_linattn_forward without a workspace argument, for callers that cannot
  * allocate device memory: code that runs under an allocator it does not own
  * (a host application or framework that hands out all device memory itself),
@@ -185,7 +239,8 @@ const char* sana_linattn_build_info(void);
  * Diagnostic: the first error code a kernel of this library recorded on the
  * current device (0 = none; 1 = a pipeline wait inside a kernel ran past its
  * ~2 s limit, after which that kernel stopped early and its outputs are not
- * valid). With clear != 0 the code is reset to 0. This call synchronises with
+ * valid; 2 = a kernel was launched with parameters it does not handle, and did
+ * nothing). With clear != 0 the code is reset to 0. This call synchronises with
  * the device; call it after the work it should cover has completed (e.g.
  * after cudaDeviceSynchronize), not in a hot loop.
  */

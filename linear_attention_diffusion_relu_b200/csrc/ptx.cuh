@@ -16,6 +16,7 @@ namespace ptx {
 enum : uint32_t {
     kErrNone = 0,
     kErrWaitTimeout = 1,
+    kErrUnsupported = 2,   // a kernel was launched with parameters it does not handle
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

@@ -41,7 +41,7 @@ struct Plan {
     sana::tc::KsParams ks;
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
-    size_t state_bytes;     // fp32 (B, H, d, d+1)
+    size_t state_bytes;     // fp32 (B, H, d, d+1); block-causal (B, H, nblk, d, d+1)
     size_t flag_bytes;      // grid-barrier flags of the single-launch forward (one per CTA)
 };
 
@@ -59,25 +59,63 @@ sana::tc::Sched make_sched(long long S, long long T) {
         q.grid = kSMs;
     }
     q.max_seg = (int)cdiv(S, q.grid);
+    q.nblk = 1;
+    q.tpb = 0;
     return q;
 }
 
-Plan make_plan(int B, int N, int H, int d) {
+// Block-causal schedule: S slabs of nblk blocks of bt tiles, R CTAs per slab
+// (R divides bt), each taking bt / R tiles of every block.
+sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int R) {
+    sana::tc::Sched q{};
+    q.S = (int)S;
+    q.T = (int)(nblk * bt);
+    q.R = R;
+    q.grid = S <= kSMs ? (int)(S * R) : kSMs;
+    q.nblk = (int)nblk;
+    q.tpb = (int)(bt / R);
+    q.max_seg = (int)(cdiv(S, q.grid) * nblk);
+    return q;
+}
+
+// CTAs per slab of the block-causal schedule: the largest divisor of the
+// 128-token tiles per block (hence also of the 64-token ones) that fits
+// S * R <= 148.
+int block_sched_r(long long S, long long tiles128) {
+    if (S > kSMs) return 1;
+    for (long long r = std::min<long long>(kSMs / S, tiles128); r > 1; --r)
+        if (tiles128 % r == 0) return (int)r;
+    return 1;
+}
+
+// L = 0: the plain forward; L > 0 (a multiple of 128): block-causal with
+// blocks of L tokens.
+Plan make_plan(int B, int N, int H, int d, int L = 0) {
     const int G = 128 / d;                        // heads per 128-row group
     const long long groups = cdiv(H, G);
+    const long long S = (long long)B * groups;
     Plan p{};
     p.ks.N = N;
     p.ks.H = H;
     p.ks.groups = (int)groups;
-    p.ks.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KS_TILE));
     p.ka.N = N;
     p.ka.H = H;
     p.ka.groups = (int)groups;
-    p.ka.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KA_TILE));
+    long long nblk = 1;
+    if (L > 0) {
+        nblk = cdiv(N, L);
+        const long long tiles128 = L / sana::tc::KA_TILE;
+        const int R = block_sched_r(S, tiles128);
+        p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, R);
+        p.ka.q = make_block_sched(S, nblk, tiles128, R);
+    } else {
+        p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE));
+        p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE));
+    }
     p.ka.eps = 0.0f;
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
-    p.state_bytes = align256((size_t)B * H * dd);
+    p.state_bytes = align256((size_t)B * H * nblk * dd);
     p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
     return p;
 }
@@ -92,6 +130,26 @@ sana_la_status check_sizes(int B, int N, int H, int d) {
     // one batch of one tensor must stay under the 2^40-byte TMA stride limit
     if ((long long)N * H * d * 2 >= (1LL << 40)) return SANA_LA_ERR_UNSUPPORTED;
     if ((long long)B * H > kMaxGrid) return SANA_LA_ERR_UNSUPPORTED;
+    return SANA_LA_OK;
+}
+
+// Block length of the block-causal form: a multiple of 128 tokens, and the
+// partial states (one per CTA, slab and block) within 4 GiB.
+constexpr size_t kMaxBlockPartialBytes = size_t(4) << 30;
+
+sana_la_status check_block(int B, int N, int H, int d, int L) {
+    if (L < 1) return SANA_LA_ERR_INVALID_ARG;
+    if (L % sana::tc::KA_TILE != 0) return SANA_LA_ERR_UNSUPPORTED;
+    // the sizes of make_plan(B, N, H, d, L), in 64-bit arithmetic first
+    const long long G = 128 / d;
+    const long long S = (long long)B * cdiv(H, G);
+    const long long nblk = cdiv(N, L);
+    const long long R = block_sched_r(S, L / sana::tc::KA_TILE);
+    const long long grid = S <= kSMs ? S * R : kSMs;
+    const long long segs = cdiv(S, grid) * nblk;             // per CTA
+    const long long per_seg = G * d * (d + 1) * (long long)sizeof(float);
+    if (segs > (long long)(kMaxBlockPartialBytes / per_seg) / grid) return SANA_LA_ERR_UNSUPPORTED;
+    if (nblk * L > 0x7fffffffLL) return SANA_LA_ERR_UNSUPPORTED;    // padded token coordinates
     return SANA_LA_OK;
 }
 
@@ -233,9 +291,9 @@ sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N,
 // stream (forward), so Q was ready before they started and the apply kernel
 // may start early; a standalone apply waits for everything before it.
 template <int D>
-sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, void* O,
+sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, int L, void* O,
                          sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
-    Plan p = make_plan(B, N, H, D);
+    Plan p = make_plan(B, N, H, D, L);
     p.ka.eps = eps;
     CUtensorMap tmQ;
     sana_la_status st;
@@ -332,10 +390,10 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     return launch_status("fwd_fused_tc");
 }
 
-sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d,
+sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d, int L,
                              float* state, void* ws, size_t ws_bytes, cudaStream_t s,
                              bool need_state_area) {
-    const Plan p = make_plan(B, N, H, d);
+    const Plan p = make_plan(B, N, H, d, L);
     const size_t need = p.partial_bytes + (need_state_area ? p.state_bytes : 0);
     if (ws_bytes < need) return SANA_LA_ERR_WORKSPACE;
     float* partial = static_cast<float*>(ws);
@@ -343,10 +401,10 @@ sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, 
                    : run_kv_state<64>(K, V, B, N, H, p, partial, state, s);
 }
 
-sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d,
+sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d, int L,
                           void* O, sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
-    return d == 32 ? run_apply<32>(Q, state, B, N, H, O, od, eps, s, overlap)
-                   : run_apply<64>(Q, state, B, N, H, O, od, eps, s, overlap);
+    return d == 32 ? run_apply<32>(Q, state, B, N, H, L, O, od, eps, s, overlap)
+                   : run_apply<64>(Q, state, B, N, H, L, O, od, eps, s, overlap);
 }
 
 }  // namespace
@@ -368,7 +426,7 @@ sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N,
     if (st != SANA_LA_OK) return st;
     if (!aligned16(K) || !aligned16(V) || !aligned16(state) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
-    return kv_state_impl(K, V, B, N, H, d, state, workspace, workspace_bytes,
+    return kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes,
                          reinterpret_cast<cudaStream_t>(stream), false);
 }
 
@@ -382,7 +440,7 @@ sana_la_status sana_linattn_apply(const void* Q, const float* state, int B, int 
     if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(Q) || !aligned16(state) || !aligned16(O)) return SANA_LA_ERR_INVALID_ARG;
-    return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps,
+    return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps,
                       reinterpret_cast<cudaStream_t>(stream), false);
 }
 
@@ -416,9 +474,75 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
     if (st != SANA_LA_ERR_UNSUPPORTED) return st;
     // the device cannot hold the whole grid at once: the same kernels as
     // kv_state + apply, overlapped by programmatic launch
-    st = kv_state_impl(K, V, B, N, H, d, state, workspace, workspace_bytes, s, true);
+    st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes, s, true);
     if (st != SANA_LA_OK) return st;
-    return apply_impl(Q, state, B, N, H, d, O, out_dtype, eps, s, true);
+    return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true);
+}
+
+// ------------------------------------------------------- block-causal ----
+size_t sana_linattn_block_causal_workspace_bytes(int B, int N, int H, int d, int L) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
+    const Plan p = make_plan(B, N, H, d, L);
+    return p.partial_bytes + p.state_bytes;
+}
+
+sana_la_status sana_linattn_block_causal_kv_state(const void* K, const void* V, int B, int N, int H,
+                                                  int d, int L, float* states, void* workspace,
+                                                  size_t workspace_bytes, sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!K || !V || !states || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    if ((st = check_block(B, N, H, d, L)) != SANA_LA_OK) return st;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(states) || !aligned16(workspace))
+        return SANA_LA_ERR_INVALID_ARG;
+    return kv_state_impl(K, V, B, N, H, d, L, states, workspace, workspace_bytes,
+                         reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+sana_la_status sana_linattn_block_causal_apply(const void* Q, const float* states, int B, int N,
+                                               int H, int d, int L, void* O,
+                                               sana_la_out_dtype out_dtype, float eps,
+                                               sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!Q || !states || !O) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    if ((st = check_block(B, N, H, d, L)) != SANA_LA_OK) return st;
+    if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
+    if ((st = check_eps(eps)) != SANA_LA_OK) return st;
+    if (!aligned16(Q) || !aligned16(states) || !aligned16(O)) return SANA_LA_ERR_INVALID_ARG;
+    return apply_impl(Q, states, B, N, H, d, L, O, out_dtype, eps,
+                      reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, const void* V,
+                                                 int B, int N, int H, int d, int L,
+                                                 void* O, sana_la_out_dtype out_dtype, float eps,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!Q || !K || !V || !O || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    if ((st = check_block(B, N, H, d, L)) != SANA_LA_OK) return st;
+    if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
+    if ((st = check_eps(eps)) != SANA_LA_OK) return st;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
+        return SANA_LA_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, N, H, d, L);
+    if (workspace_bytes < p.partial_bytes + p.state_bytes) return SANA_LA_ERR_WORKSPACE;
+    float* states = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.partial_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // state kernel + prefix reduction, then the apply kernel (programmatic launch)
+    st = kv_state_impl(K, V, B, N, H, d, L, states, workspace, workspace_bytes, s, true);
+    if (st != SANA_LA_OK) return st;
+    return apply_impl(Q, states, B, N, H, d, L, O, out_dtype, eps, s, true);
+}
+
+int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
+    return 3;   // ks_state_tc, kr_reduce_tc (prefix states), ka_apply_tc
 }
 
 int sana_linattn_forward_launches(int B, int N, int H, int d) {

@@ -34,6 +34,14 @@
 //   S >  148: CTA c takes slabs c, c + 148, ... with all their tiles.
 // Each (CTA, slab) pair is one "segment"; KS writes one partial state per
 // segment and KR adds a slab's segments in ascending CTA order.
+//
+// Block-causal form (blocks of L tokens, L a multiple of 128): the tiles of a
+// slab are padded to whole blocks and R divides the tiles per block, so every
+// CTA takes the same number of tiles, tpb, from each block (tiles past N read
+// as zeros and are not stored). A segment is then one (slab, block) pair:
+// KS writes one partial per (CTA, slab, block), KR turns them into prefix
+// states (ascending blocks, within a block ascending CTA), and KA stages the
+// prefix state of a tile's block.
 // Every mbarrier wait is bounded; a wait that runs out sets an error code and
 // the whole CTA winds down (drains its TMA loads and UMMAs, frees TMEM).
 #pragma once
@@ -105,27 +113,31 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 // =============================================================== schedule ===
 struct Sched {
     int S;          // (b, group) slabs = B * groups
-    int T;          // tiles per slab
+    int T;          // tiles per slab (block-causal: padded to whole blocks)
     int R;          // CTAs sharing one slab (1 when S > grid)
     int grid;       // CTAs
-    int max_seg;    // most slabs one CTA visits
+    int max_seg;    // most segments one CTA visits
+    int nblk;       // token blocks per slab (1 = not block-causal)
+    int tpb;        // block-causal: tiles of one block per CTA (0 otherwise)
 };
 
 // tiles per segment of CTA c
 __host__ __device__ __forceinline__ int sched_tps(int c, const Sched& q) {
+    if (q.tpb > 0) return q.tpb;
     const int r = c / q.S;
     return (q.T - r + q.R - 1) / q.R;
 }
-// segments (slabs) of CTA c
+// segments of CTA c: its slabs times the blocks of a slab
 __host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
-    return (q.S - c % q.S + q.grid - 1) / q.grid;
+    return (q.S - c % q.S + q.grid - 1) / q.grid * q.nblk;
 }
-// i-th tile of CTA c -> (slab, tile, segment index)
+// i-th tile of CTA c -> (slab, tile, segment index); the segment's block is
+// seg % q.nblk
 __host__ __device__ __forceinline__ void sched_item(int c, int i, int tps, const Sched& q,
                                                     int& slab, int& tile, int& seg) {
     seg = i / tps;
-    slab = c % q.S + seg * q.grid;
-    tile = c / q.S + (i % tps) * q.R;
+    slab = c % q.S + seg / q.nblk * q.grid;
+    tile = c / q.S + ((seg % q.nblk) * tps + i % tps) * q.R;
 }
 
 // ===================================================================== KS ===
@@ -332,11 +344,24 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
     const int slab = b * p.groups + h / G;
-    const float* src = partial + ks_slot(slab % p.q.grid, slab / p.q.grid, h % G, G, p) * DD + e;
     const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
+    // one block: the sum of the slab's R partials; block-causal: the running
+    // sum over blocks, i.e. the inclusive prefix state of every block
     float s = 0.0f;
-    for (int r = 0; r < p.q.R; ++r) s += src[r * step];
-    state[bh * DD + e] = s;
+    for (int j = 0; j < p.q.nblk; ++j) {
+        const float* src =
+            partial + ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j, h % G, G, p) * DD + e;
+        // eight loads in flight, then their additions in ascending r
+        for (int r0 = 0; r0 < p.q.R; r0 += 8) {
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (r0 + u < p.q.R) s += t[u];
+        }
+        state[(bh * p.q.nblk + j) * DD + e] = s;
+    }
 }
 
 // ===================================================================== KA ===
@@ -603,7 +628,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
 
         // stage the state of `slab` in shared memory as bf16 hi + lo parts
         bool grid_synced = false;
-        auto stage_state = [&](int slab) -> bool {
+        auto stage_state = [&](int slab, int blk) -> bool {
             if (src.state == nullptr && !grid_synced) {
                 // the partial states of every CTA must be in memory (once)
                 if (warp == 0) {
@@ -625,7 +650,8 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 for (int j = 0; j < NE; ++j) {
                     const int x = tid + j * kWorkerThreads;
                     const int h = g * G + x / DD;
-                    if (x < G * DD && h < p.H) v[j] = src.state[((long long)b * p.H + h) * DD + x % DD];
+                    if (x < G * DD && h < p.H)
+                        v[j] = src.state[(((long long)b * p.H + h) * p.q.nblk + blk) * DD + x % DD];
                 }
             } else {
                 // the same additions, in the same order, as kr_reduce_tc: the R
@@ -684,7 +710,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 }
                 int slab, tile, seg;
                 sched_item(cta, i, tps, p.q, slab, tile, seg);
-                if (!stage_state(slab)) return false;
+                if (!stage_state(slab, seg % p.q.nblk)) return false;
             }
             const int s = i % S;
             if (!warp_wait(&bar.full[s], (i / S) & 1, abort, err)) return false;
@@ -767,7 +793,8 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                     for (int k = 0; k < HALF_BOXES; ++k) {
                         const int bx = half * HALF_BOXES + k;
                         const int x = x0 + bx * L::OUT_BOX_ELEMS;
-                        if (x < p.H * D) ptx::tma_store_3d(tmO, staging + bx * KA_BOX_BYTES, x, y, b);
+                        if (x < p.H * D && y < p.N)    // (block-causal padding tiles are not stored)
+                            ptx::tma_store_3d(tmO, staging + bx * KA_BOX_BYTES, x, y, b);
                     }
                     ptx::bulk_commit_group();
                     // release the staging boxes for unit i + 1: the store that last
@@ -892,6 +919,12 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
              unsigned long long* flags, const unsigned long long epoch)
 {
     using Map = FwdMap<D, OUT_BF16>;
+    // the apply phase here sums one block's partials; prefix states over token
+    // blocks take the three-kernel path
+    if (ks.q.nblk != 1 || ka.q.nblk != 1) {
+        if (threadIdx.x == 0) atomicCAS(&g_device_error, ptx::kErrNone, ptx::kErrUnsupported);
+        return;
+    }
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF);

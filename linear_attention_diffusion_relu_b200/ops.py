@@ -11,6 +11,13 @@ The functions mirror the C ABI in ``include/sana_linattn.h``:
     kv_state(K, V, state=None, workspace=None)             -> state (B, H, d, d+1) fp32
     apply(Q, state, out_dtype=torch.bfloat16, eps=1e-15, out=None) -> O (B, N, H, d)
     forward(Q, K, V, out_dtype=torch.bfloat16, eps=1e-15, out=None, workspace=None) -> O
+
+and the block-causal form (blocks of L tokens, L a multiple of 128):
+
+    block_causal_workspace_bytes(B, N, H, d, L)
+    block_causal_kv_state(K, V, L, states=None, workspace=None) -> (B, H, nblk, d, d+1) fp32
+    block_causal_apply(Q, states, L, out_dtype=..., eps=..., out=None) -> O
+    block_causal_forward(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None) -> O
 """
 from __future__ import annotations
 
@@ -32,6 +39,11 @@ SYMBOLS = (
     "sana_linattn_apply",
     "sana_linattn_forward",
     "sana_linattn_forward_launches",
+    "sana_linattn_block_causal_workspace_bytes",
+    "sana_linattn_block_causal_kv_state",
+    "sana_linattn_block_causal_apply",
+    "sana_linattn_block_causal_forward",
+    "sana_linattn_block_causal_forward_launches",
     "sana_linattn_build_info",
     "sana_linattn_device_error",
     "sana_linattn_selftest_wait_timeout",
@@ -79,6 +91,16 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_device_error.restype = st
         lib.sana_linattn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
         lib.sana_linattn_selftest_wait_timeout.restype = st
+        lib.sana_linattn_block_causal_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_block_causal_workspace_bytes.restype = sz
+        lib.sana_linattn_block_causal_kv_state.argtypes = [vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+        lib.sana_linattn_block_causal_kv_state.restype = st
+        lib.sana_linattn_block_causal_apply.argtypes = [vp, vp, i, i, i, i, i, vp, i, f, vp]
+        lib.sana_linattn_block_causal_apply.restype = st
+        lib.sana_linattn_block_causal_forward.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_block_causal_forward.restype = st
+        lib.sana_linattn_block_causal_forward_launches.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_block_causal_forward_launches.restype = ctypes.c_int
         lib.sana_linattn_last_error.argtypes = []
         lib.sana_linattn_last_error.restype = ctypes.c_char_p
         if path == LIBRARY:
@@ -224,4 +246,89 @@ def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.b
                                   out.data_ptr(), code, float(eps), workspace.data_ptr(),
                                   workspace.numel() * workspace.element_size(), _stream(Q.device))
     _check(lib, st, "sana_linattn_forward")
+    return out
+
+
+# ------------------------------------------------------------ block-causal --
+
+def num_blocks(N: int, L: int) -> int:
+    return -(-N // L)
+
+
+def block_causal_workspace_bytes(B: int, N: int, H: int, d: int, L: int) -> int:
+    return int(load_library().sana_linattn_block_causal_workspace_bytes(B, N, H, d, L))
+
+
+def block_causal_forward_launches(B: int, N: int, H: int, d: int, L: int) -> int:
+    return int(load_library().sana_linattn_block_causal_forward_launches(B, N, H, d, L))
+
+
+def make_block_causal_workspace(B: int, N: int, H: int, d: int, L: int, device="cuda") -> torch.Tensor:
+    n = block_causal_workspace_bytes(B, N, H, d, L)
+    if n == 0:
+        raise ValueError(f"unsupported sizes B={B} N={N} H={H} d={d} L={L}")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check_states(states, B, N, H, d, L, device):
+    shape = (B, H, num_blocks(N, L), d, d + 1)
+    if (states.dtype != torch.float32 or tuple(states.shape) != shape
+            or not states.is_contiguous() or states.device != device):
+        raise ValueError(f"states must be contiguous float32 {shape} on {device}")
+
+
+def block_causal_kv_state(K: torch.Tensor, V: torch.Tensor, L: int, states: torch.Tensor | None = None,
+                          workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Inclusive prefix states over blocks of L tokens, fp32 (B, H, nblk, d, d+1)."""
+    _check_bnhd("K", K)
+    _check_bnhd("V", V, K.shape)
+    B, N, H, d = K.shape
+    if states is None:
+        states = torch.empty((B, H, num_blocks(N, L), d, d + 1), dtype=torch.float32, device=K.device)
+    _check_states(states, B, N, H, d, L, K.device)
+    if workspace is None:
+        workspace = make_block_causal_workspace(B, N, H, d, L, K.device)
+    lib = load_library()
+    st = lib.sana_linattn_block_causal_kv_state(K.data_ptr(), V.data_ptr(), B, N, H, d, int(L),
+                                                states.data_ptr(), workspace.data_ptr(),
+                                                workspace.numel() * workspace.element_size(),
+                                                _stream(K.device))
+    _check(lib, st, "sana_linattn_block_causal_kv_state")
+    return states
+
+
+def block_causal_apply(Q: torch.Tensor, states: torch.Tensor, L: int, out_dtype=torch.bfloat16,
+                       eps: float = 1e-15, out: torch.Tensor | None = None) -> torch.Tensor:
+    """O for block-causal attention: row n uses the prefix state of block n // L."""
+    _check_bnhd("Q", Q)
+    B, N, H, d = Q.shape
+    _check_states(states, B, N, H, d, L, Q.device)
+    code = _out_code(out_dtype)
+    out = _prep_out(out, Q.shape, out_dtype, Q.device)
+    lib = load_library()
+    st = lib.sana_linattn_block_causal_apply(Q.data_ptr(), states.data_ptr(), B, N, H, d, int(L),
+                                             out.data_ptr(), code, float(eps), _stream(Q.device))
+    _check(lib, st, "sana_linattn_block_causal_apply")
+    return out
+
+
+def block_causal_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: int,
+                         out_dtype=torch.bfloat16, eps: float = 1e-15, out: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Whole block-causal forward; bit-identical to block_causal_kv_state + block_causal_apply."""
+    _check_bnhd("Q", Q)
+    _check_bnhd("K", K, Q.shape)
+    _check_bnhd("V", V, Q.shape)
+    B, N, H, d = Q.shape
+    code = _out_code(out_dtype)
+    out = _prep_out(out, Q.shape, out_dtype, Q.device)
+    if workspace is None:
+        workspace = make_block_causal_workspace(B, N, H, d, L, Q.device)
+    lib = load_library()
+    st = lib.sana_linattn_block_causal_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d,
+                                               int(L), out.data_ptr(), code, float(eps),
+                                               workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(),
+                                               _stream(Q.device))
+    _check(lib, st, "sana_linattn_block_causal_forward")
     return out

@@ -14,6 +14,13 @@ with H = 36, C = 2240 with H = 70, d = 32) describe Sana-0.6B-like and
 Sana-1.6B-like widths; the walk-through's section 5 gives 2240 channels for the
 1.6B model. B = 2 is a classifier-free-guidance cond/uncond pair.
 
+The block-causal workloads stand in for latent video: ``block`` tokens per
+frame, 16 frames, after the video row of the token table in
+"08_sana高效高分辨率生成" (papers-3lj.pages.dev), section "Linear Attention 的原理"
+(4096x4096 x 16 frames = 1,048,576 tokens, i.e. 65,536 per frame; that table
+counts 4,096 tokens per 1024x1024 frame). They draw the same tensors as the
+sweep workloads of the same size (same seed and shape).
+
 Recipe (all draws from one torch generator seeded per workload):
   1. Q, K, V drawn in that order with ``torch.randn`` in float32, each shaped
      (B, N, H, d).
@@ -48,6 +55,7 @@ class Workload:
     neg_rows: tuple = field(default=())
     eps: float = 1e-15
     description: str = ""
+    block: int = 0                  # block-causal form: tokens per block (0 = not block-causal)
 
     @property
     def token_heads(self) -> int:
@@ -81,6 +89,10 @@ WORKLOADS: dict[str, Workload] = {
                               description="ragged token count, B=1, H=36, d=32"),
     "d64": Workload("d64", 1, 16384, 18, 64, seed=4,
                     description="head size 64, B=1, N=16384, H=18"),
+    "video16f_1024px": Workload("video16f_1024px", 1, 16 * 4096, 36, 32, seed=4, block=4096,
+                                description="block-causal, 16 frames of 4,096 tokens, H=36, d=32"),
+    "video16f_4096px": Workload("video16f_4096px", 1, 16 * 65536, 36, 32, seed=4, block=65536,
+                                description="block-causal, 16 frames of 65,536 tokens, H=36, d=32"),
 }
 
 

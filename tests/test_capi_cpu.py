@@ -114,3 +114,32 @@ def test_library_is_sm100a_only():
     """The build targets sm_100a and nothing else (no PTX for other archs)."""
     assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
     assert not any("compute_90" in f or "sm_90" in f for f in build.NVCC_FLAGS)
+
+
+def test_block_causal_host_checks(lib):
+    wsb = lib.sana_linattn_block_causal_workspace_bytes
+    assert wsb(2, 3572, 6, 32, 1024) > 0
+    assert wsb(2, 3572, 6, 32, 1024) % 256 == 0
+    # the prefix states alone: B * H * nblk * d * (d+1) fp32
+    assert wsb(2, 3572, 6, 32, 1024) >= 2 * 6 * 4 * 32 * 33 * 4
+    assert wsb(2, 3572, 6, 32, 100) == 0          # not a multiple of 128
+    assert wsb(2, 3572, 6, 32, 0) == 0
+    assert wsb(2, 3572, 6, 48, 1024) == 0         # head size
+    assert wsb(1, 1 << 24, 36, 32, 128) == 0      # partials beyond the 4 GiB cap
+    assert wsb(1, 1 << 24, 36, 32, 65536) > 0
+    n = lib.sana_linattn_block_causal_forward_launches
+    assert n(2, 3572, 6, 32, 1024) == 3 and n(2, 3572, 6, 32, 96) == 0
+    f = lib.sana_linattn_block_causal_forward
+    ws = wsb(1, 1024, 2, 32, 256)
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 100, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 0, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, -128, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, 1, 1e-15, FAKE, ws - 1, None) == ops.ERR_WORKSPACE
+    assert f(None, FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, 1, -1.0, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    ks = lib.sana_linattn_block_causal_kv_state
+    assert ks(FAKE, FAKE, 1, 1024, 2, 32, 192, FAKE, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert ks(FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, FAKE, 0, None) == ops.ERR_WORKSPACE
+    ap = lib.sana_linattn_block_causal_apply
+    assert ap(FAKE, FAKE, 1, 1024, 2, 32, 200, FAKE, 0, 0.0, None) == ops.ERR_UNSUPPORTED
+    assert ap(FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, 5, 0.0, None) == ops.ERR_INVALID_ARG
