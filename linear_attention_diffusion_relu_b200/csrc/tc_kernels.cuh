@@ -364,6 +364,56 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     }
 }
 
+// Block-causal prefix states: one warp per state entry; lane j takes block
+// j of a 32-block chunk, adds the block's R partials (ascending r), and a warp
+// scan (fixed shuffle pattern) plus the previous chunk's total gives the
+// inclusive prefix over blocks. Deterministic: the same additions in the same
+// order on every run.
+constexpr int KP_WARPS = 4;
+
+template <int D>
+__global__ void __launch_bounds__(KP_WARPS * 32)
+kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restrict__ states)
+{
+    constexpr int G = 128 / D;
+    constexpr int DD = D * (D + 1);
+    ptx::launch_dependents();
+    ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.y * KP_WARPS + (threadIdx.x >> 5);
+    if (e >= DD) return;                         // whole warps leave together
+    const long long bh = blockIdx.x;
+    const int b = (int)(bh / p.H);
+    const int h = (int)(bh % p.H);
+    const int slab = b * p.groups + h / G;
+    const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
+    float carry = 0.0f;
+    for (int j0 = 0; j0 < p.q.nblk; j0 += 32) {
+        const int j = j0 + lane;
+        float x = 0.0f;
+        if (j < p.q.nblk) {
+            const float* src =
+                partial + ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j, h % G, G, p) * DD + e;
+            for (int r0 = 0; r0 < p.q.R; r0 += 8) {
+                float t[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (r0 + u < p.q.R) x += t[u];
+            }
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x = y + x;
+        }
+        x = carry + x;
+        if (j < p.q.nblk) states[(bh * p.q.nblk + j) * DD + e] = x;
+        carry = __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
 // ===================================================================== KA ===
 //
 // Unit = one 128-token tile of a (b, group) slab, dealt out by the lockstep
