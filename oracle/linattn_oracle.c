@@ -45,12 +45,20 @@
  *   P[b,h,j] = sum over tokens n < min((j+1)*L, N) of phi(K_n)^T [V_n | 1]
  * in place of S. The prefix states are (B, H, nblk, d, d+1), nblk = ceil(N/L).
  *
+ * Other feature maps ("08_sana高效高分辨率生成", section "Linear Attention 的原理"
+ * names ELU+1 and cos as alternatives to ReLU). Reading: ELU with alpha = 1,
+ * plus one, i.e. phi(x) = x + 1 for x > 0 and exp(x) otherwise; cos is
+ * phi(x) = cos(x) elementwise. Everything else (state, normaliser, eps) is the
+ * same; with cos the normaliser can be zero or negative and O = num/(den+eps)
+ * is taken as it stands.
+ *
  * All arithmetic is IEEE double. Sums run in token order n = 0 .. N-1 and
  * feature order i = 0 .. d-1, nothing is blocked or reordered. OpenMP only
  * spreads independent (b, h) pairs or independent query rows over threads, which
  * does not change any sum.
  */
 #include <stddef.h>
+#include <math.h>
 #include <stdlib.h>
 #include <omp.h>
 
@@ -196,6 +204,62 @@ void oracle_block_causal_apply(const double* Q, const double* P, long B, long N,
                         num += relu(Q[at_bnhd(b, n, h, i, N, H, d)]) * P[at_prefix(b, h, j, i, c, H, nblk, d)];
                     O[at_bnhd(b, n, h, c, N, H, d)] = num / (den + eps);
                 }
+            }
+        }
+    }
+}
+
+/* feature map: 0 = ReLU, 1 = ELU + 1, 2 = cos */
+static double feature(double x, int fm)
+{
+    if (fm == 1)
+        return x > 0.0 ? x + 1.0 : exp(x);
+    if (fm == 2)
+        return cos(x);
+    return x > 0.0 ? x : 0.0;
+}
+
+/* the state with feature map fm: S[b,h,i,j] = sum_n phi(K[b,n,h,i]) * [V | 1][b,n,h,j] */
+void oracle_state_fm(const double* K, const double* V, long B, long N, long H, long d, int fm,
+                     double* S)
+{
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b) {
+        for (long h = 0; h < H; ++h) {
+            for (long i = 0; i < d; ++i)
+                for (long j = 0; j <= d; ++j)
+                    S[at_state(b, h, i, j, H, d)] = 0.0;
+            for (long n = 0; n < N; ++n) {
+                for (long i = 0; i < d; ++i) {
+                    double k = feature(K[at_bnhd(b, n, h, i, N, H, d)], fm);
+                    for (long j = 0; j < d; ++j)
+                        S[at_state(b, h, i, j, H, d)] += k * V[at_bnhd(b, n, h, j, N, H, d)];
+                    S[at_state(b, h, i, d, H, d)] += k * 1.0;
+                }
+            }
+        }
+    }
+}
+
+/* apply with feature map fm: O = (phi(Q) S[:, 0:d]) / (phi(Q) S[:, d] + eps) */
+void oracle_apply_fm(const double* Q, const double* S, long B, long N, long H, long d, int fm,
+                     double eps, double* O, double* den_out)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (long b = 0; b < B; ++b) {
+        for (long n = 0; n < N; ++n) {
+            for (long h = 0; h < H; ++h) {
+                double den = 0.0;
+                for (long i = 0; i < d; ++i)
+                    den += feature(Q[at_bnhd(b, n, h, i, N, H, d)], fm) * S[at_state(b, h, i, d, H, d)];
+                for (long j = 0; j < d; ++j) {
+                    double num = 0.0;
+                    for (long i = 0; i < d; ++i)
+                        num += feature(Q[at_bnhd(b, n, h, i, N, H, d)], fm) * S[at_state(b, h, i, j, H, d)];
+                    O[at_bnhd(b, n, h, j, N, H, d)] = num / (den + eps);
+                }
+                if (den_out)
+                    den_out[((size_t)b * N + n) * H + h] = den;
             }
         }
     }

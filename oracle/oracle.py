@@ -59,6 +59,11 @@ class Oracle:
         lib.oracle_block_causal_apply.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long,
                                                   _c_long, _c_double, _ptr]
         lib.oracle_block_causal_apply.restype = None
+        lib.oracle_state_fm.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long, ctypes.c_int, _ptr]
+        lib.oracle_state_fm.restype = None
+        lib.oracle_apply_fm.argtypes = [_ptr, _ptr, _c_long, _c_long, _c_long, _c_long, ctypes.c_int,
+                                        _c_double, _ptr, _ptr]
+        lib.oracle_apply_fm.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         self._lib = lib
@@ -101,6 +106,35 @@ class Oracle:
         S = self.state(K, V)
         return self.apply(Q, S, eps, return_den=return_den)
 
+
+    FEATURE_MAPS = {"relu": 0, "elu1": 1, "cos": 2}
+
+    def state_fm(self, K, V, feature: str) -> np.ndarray:
+        """S = phi(K)^T [V | 1] with phi = relu | elu1 (ELU + 1) | cos."""
+        K = self._f64(K)
+        V = self._f64(V)
+        if K.shape != V.shape:
+            raise ValueError("K and V must have the same shape")
+        B, N, H, d = K.shape
+        S = np.empty((B, H, d, d + 1), dtype=np.float64)
+        self._lib.oracle_state_fm(K.ctypes.data, V.ctypes.data, B, N, H, d,
+                                  self.FEATURE_MAPS[feature], S.ctypes.data)
+        return S
+
+    def apply_fm(self, Q, S, feature: str, eps: float, return_den: bool = False):
+        Q = self._f64(Q)
+        S = np.ascontiguousarray(np.asarray(S, dtype=np.float64))
+        B, N, H, d = Q.shape
+        if S.shape != (B, H, d, d + 1):
+            raise ValueError(f"state shape {S.shape} does not match Q {Q.shape}")
+        O = np.empty((B, N, H, d), dtype=np.float64)
+        den = np.empty((B, N, H), dtype=np.float64) if return_den else None
+        self._lib.oracle_apply_fm(Q.ctypes.data, S.ctypes.data, B, N, H, d, self.FEATURE_MAPS[feature],
+                                  float(eps), O.ctypes.data, den.ctypes.data if return_den else None)
+        return (O, den) if return_den else O
+
+    def forward_fm(self, Q, K, V, feature: str, eps: float, return_den: bool = False):
+        return self.apply_fm(Q, self.state_fm(K, V, feature), feature, eps, return_den=return_den)
 
     def block_causal_state(self, K, V, L: int) -> np.ndarray:
         """Inclusive prefix states of blocks of L tokens: (B, H, nblk, d, d+1)."""

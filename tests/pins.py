@@ -350,11 +350,80 @@ def pin_block_causal_no_future(orc, seed=24):
     assert np.all(np.abs(O3[:, 16:24] - O[:, 16:24]).max(axis=-1) > 0)
 
 
+# ------------------------------------------------------------ feature maps --
+# "08_sana高效高分辨率生成", section "Linear Attention 的原理": ELU+1 and cos are
+# named as alternatives to ReLU. Reading: ELU with alpha = 1, plus one.
+
+FEATURES_NP = {
+    "relu": lambda x: np.maximum(x, 0.0),
+    "elu1": lambda x: np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0))),
+    "cos": np.cos,
+}
+
+
+def bruteforce_fm(Q, K, V, eps, feature):
+    """The quadratic definition with feature map phi, in numpy."""
+    Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
+    phi = FEATURES_NP[feature]
+    B, N, H, d = Q.shape
+    O = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            W = phi(Q[b, :, h, :]) @ phi(K[b, :, h, :]).T
+            O[b, :, h, :] = (W @ V[b, :, h, :]) / (W.sum(axis=1, keepdims=True) + eps)
+    return O
+
+
+def pin_feature_maps_bruteforce(orc, seed=31):
+    """Each feature map against its n x n definition (1e-12 normwise per row;
+    cos normalisers of random inputs stay far from zero here); ReLU through the
+    feature-map entry equals the plain oracle bit for bit."""
+    Q, K, V = _rng_inputs(seed, B=2, N=37, H=3, d=8)
+    for feature in ("relu", "elu1", "cos"):
+        O, den = orc.forward_fm(Q, K, V, feature, 1e-15, return_den=True)
+        R = bruteforce_fm(Q, K, V, 1e-15, feature)
+        assert row_relerr(O, R).max() <= 1e-12, (feature, row_relerr(O, R).max())
+        if feature == "cos":
+            assert np.abs(den).min() > 1.0
+    assert np.array_equal(orc.forward_fm(Q, K, V, "relu", 1e-15), orc.forward(Q, K, V, 1e-15))
+
+
+def pin_feature_maps_closed_forms(orc, seed=32):
+    """Q = K = 0 gives phi = 1 for ELU+1 and cos, every weight equals d, so
+    O = d * sum_m V_m / (N d + eps): the mean of V up to eps. ELU+1 at hand
+    points: phi(1) = 2, phi(0) = 1, phi(-ln 2) = 1/2 (one head, d = 1)."""
+    _, _, V = _rng_inputs(seed, B=1, N=20, H=2, d=4)
+    Z = np.zeros_like(V)
+    for feature in ("elu1", "cos"):
+        O = orc.forward_fm(Z, Z, V, feature, 0.0)
+        assert np.allclose(O, np.broadcast_to(V.mean(axis=1, keepdims=True), O.shape), rtol=1e-14, atol=1e-15)
+    Q = np.array([1.0]).reshape(1, 1, 1, 1)
+    K = np.array([1.0, 0.0, -np.log(2.0)]).reshape(1, 3, 1, 1)
+    V = np.array([3.0, 5.0, 7.0]).reshape(1, 3, 1, 1)
+    # phi(Q) = 2, phi(K) = [2, 1, 1/2]: weights [4, 2, 1] -> (12 + 10 + 7) / 7
+    O = orc.forward_fm(Q, K, V, "elu1", 0.0)
+    assert np.allclose(O.ravel(), [29.0 / 7.0], rtol=1e-15), O
+
+
+def pin_feature_maps_symmetries(orc, seed=33):
+    """cos is even: negating Q and K changes nothing, bit for bit. ELU+1 keeps
+    every weight positive, so outputs stay in the hull of V (plus 0)."""
+    Q, K, V = _rng_inputs(seed, B=1, N=30, H=2, d=8)
+    assert np.array_equal(orc.forward_fm(-Q, -K, V, "cos", 1e-15), orc.forward_fm(Q, K, V, "cos", 1e-15))
+    O = orc.forward_fm(Q, K, V, "elu1", 1e-15)
+    lo = np.minimum(V.min(axis=1, keepdims=True), 0.0)
+    hi = np.maximum(V.max(axis=1, keepdims=True), 0.0)
+    assert np.all(O >= lo - 1e-12) and np.all(O <= hi + 1e-12)
+    S = orc.state_fm(K, V, "elu1")
+    assert np.allclose(S[..., -1], np.where(K > 0, K + 1, np.exp(np.minimum(K, 0))).sum(axis=1), rtol=1e-13)
+
+
 ALL_PINS = [
     pin_bruteforce_tiny, pin_bruteforce_random, pin_exact_integers, pin_hand_example,
     pin_single_token, pin_equal_keys, pin_one_hot, pin_constant_column,
     pin_key_permutation, pin_query_permutation_and_independence, pin_convex_hull,
     pin_zero_query, pin_scale_invariance, pin_linearity_in_v, pin_state_definition,
     pin_block_causal_bruteforce, pin_block_causal_exact_integers, pin_block_causal_reductions,
-    pin_block_causal_no_future,
+    pin_block_causal_no_future, pin_feature_maps_bruteforce, pin_feature_maps_closed_forms,
+    pin_feature_maps_symmetries,
 ]

@@ -72,6 +72,18 @@ MUTANTS = [
      "* P[at_prefix(b, h, j, i, 0, H, nblk, d)];", 0),
     ("bc_no_eps",
      "] = num / (den + eps);", "] = num / (den);", 1),
+    # feature maps
+    ("elu_without_plus_one",
+     "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x) - 1.0;", 0),
+    ("elu_branch_at_wrong_side",
+     "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? exp(x) : x + 1.0;", 0),
+    ("cos_as_sin",
+     "return cos(x);", "return sin(x);", 0),
+    ("fm_normaliser_without_key_feature",
+     "S[at_state(b, h, i, d, H, d)] += k * 1.0;", "S[at_state(b, h, i, d, H, d)] += 1.0;", 1),
+    ("fm_query_feature_ignored_in_num",
+     "num += feature(Q[at_bnhd(b, n, h, i, N, H, d)], fm)",
+     "num += (Q[at_bnhd(b, n, h, i, N, H, d)])", 0),
 ]
 
 
