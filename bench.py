@@ -194,6 +194,8 @@ def oracle_sample(w, seconds: float, max_heads: int | None = None):
         t0 = time.perf_counter()
         if w.block:
             O = orc.block_causal_apply(sl[0], orc.block_causal_state(sl[1], sl[2], w.block), w.block, w.eps)
+        elif w.feature != "relu":
+            O = orc.apply_fm(sl[0], orc.state_fm(sl[1], sl[2], w.feature), w.feature, w.eps)
         else:
             O = orc.apply(sl[0], orc.state(sl[1], sl[2]), w.eps)
         elapsed += time.perf_counter() - t0
@@ -273,23 +275,27 @@ def run_ours(args):
         state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=dev)
         ws = ops.make_workspace(B, N, H, d, dev)
 
+    fm = w.feature
+    if L and fm != "relu":
+        raise SystemExit("the block-causal form runs with phi = ReLU only")
+
     def step():
         if L:
             ops.block_causal_forward(Q, K, V, L, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws)
         else:
-            ops.forward(Q, K, V, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws)
+            ops.forward(Q, K, V, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws, feature_map=fm)
 
     def split_step(ev):
         ev[0].record(stream)
         if L:
             ops.block_causal_kv_state(K, V, L, states=state, workspace=ws)
         else:
-            ops.kv_state(K, V, state=state, workspace=ws)
+            ops.kv_state(K, V, state=state, workspace=ws, feature_map=fm)
         ev[1].record(stream)
         if L:
             ops.block_causal_apply(Q, state, L, out_dtype=torch.bfloat16, eps=w.eps, out=out)
         else:
-            ops.apply(Q, state, out_dtype=torch.bfloat16, eps=w.eps, out=out)
+            ops.apply(Q, state, out_dtype=torch.bfloat16, eps=w.eps, out=out, feature_map=fm)
         ev[2].record(stream)
 
     for _ in range(args.warmup):
@@ -380,6 +386,7 @@ def run_ours(args):
             "mtokens_per_s": mtok, "pct_of_hbm_peak": 100.0 * value / (hbm_peak * world),
             "config": {"workload": w.name, "B": B, "N": N, "H": H, "d": d,
                        **({"form": "block-causal", "block": L} if L else {}),
+                       **({"feature_map": fm} if fm != "relu" else {}),
                        "io": "bf16 Q/K/V in, bf16 O out, fp32 state and accumulation",
                        "eps": w.eps, "per_rank": f"one independent {w.name} batch",
                        "parallelism": f"dp{world}",
@@ -420,7 +427,8 @@ def run_e2e(args, w, dev, stream, world):
             ops.block_causal_forward(dQ, dK, dV, L, out_dtype=torch.bfloat16, eps=w.eps, out=dO,
                                      workspace=ws)
         else:
-            ops.forward(dQ, dK, dV, out_dtype=torch.bfloat16, eps=w.eps, out=dO, workspace=ws)
+            ops.forward(dQ, dK, dV, out_dtype=torch.bfloat16, eps=w.eps, out=dO, workspace=ws,
+                        feature_map=w.feature)
         hO.copy_(dO, non_blocking=True)
 
     for _ in range(3):

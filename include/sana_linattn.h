@@ -80,6 +80,15 @@ typedef enum {
     SANA_LA_OUT_BF16 = 1
 } sana_la_out_dtype;
 
+/* Feature map phi ("08_sana高效高分辨率生成", "Linear Attention 的原理": ReLU, with
+ * ELU+1 and cos named as alternatives). ELU is taken with alpha = 1:
+ * phi(x) = x + 1 for x > 0, exp(x) otherwise. */
+typedef enum {
+    SANA_LA_FEATURE_RELU = 0,
+    SANA_LA_FEATURE_ELU1 = 1,
+    SANA_LA_FEATURE_COS = 2
+} sana_la_feature_map;
+
 /*
  * Bytes of device workspace that sana_linattn_kv_state and
  * sana_linattn_forward need for these sizes (a pure function of the sizes).
@@ -138,6 +147,35 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     void* O, sana_la_out_dtype out_dtype, float eps,
                                     void* workspace, size_t workspace_bytes,
                                     sana_la_stream_t stream);
+
+/*
+ * The three calls above with another feature map phi. SANA_LA_FEATURE_RELU
+ * gives exactly the calls above. For ELU+1 and cos, phi is evaluated in fp32
+ * from the bf16 inputs (CUDA's expf and cosf) and carried into the tensor-core
+ * products as a bf16 hi + lo pair (~2^-17 relative), so the accuracy matches the
+ * ReLU path; the state kernel runs with 4 instead of 6 pipeline stages and the
+ * apply kernel issues one more product per head. With cos the normaliser
+ * phi(Q) state[:, d] can be zero or negative; O = num / (den + eps) is returned
+ * as it stands. A feature_map outside the enum is SANA_LA_ERR_INVALID_ARG. The
+ * workspace size is sana_linattn_workspace_bytes; states from
+ * sana_linattn_kv_state_fm must be applied with the same feature map.
+ */
+sana_la_status sana_linattn_kv_state_fm(const void* K, const void* V,
+                                        int B, int N, int H, int d, sana_la_feature_map feature_map,
+                                        float* state,
+                                        void* workspace, size_t workspace_bytes,
+                                        sana_la_stream_t stream);
+
+sana_la_status sana_linattn_apply_fm(const void* Q, const float* state,
+                                     int B, int N, int H, int d, sana_la_feature_map feature_map,
+                                     void* O, sana_la_out_dtype out_dtype, float eps,
+                                     sana_la_stream_t stream);
+
+sana_la_status sana_linattn_forward_fm(const void* Q, const void* K, const void* V,
+                                       int B, int N, int H, int d, sana_la_feature_map feature_map,
+                                       void* O, sana_la_out_dtype out_dtype, float eps,
+                                       void* workspace, size_t workspace_bytes,
+                                       sana_la_stream_t stream);
 
 /*
  * Block-causal form ("linear-diffusion-transformer-4k-efficient-generation",

@@ -26,6 +26,33 @@ __device__ __forceinline__ uint32_t float2_to_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Feature maps phi ("08_sana高效高分辨率生成", "Linear Attention 的原理": ReLU, with
+// ELU+1 and cos named as alternatives). ELU is taken with alpha = 1.
+enum : int { kFeatureRelu = 0, kFeatureElu1 = 1, kFeatureCos = 2 };
+
+template <int FM>
+__device__ __forceinline__ float feature_f32(float x) {
+    if constexpr (FM == kFeatureElu1) return x > 0.0f ? x + 1.0f : expf(x);
+    else if constexpr (FM == kFeatureCos) return cosf(x);
+    else return fmaxf(x, 0.0f);
+}
+
+// phi of a packed bf16 pair, split into bf16 hi and lo parts: hi = bf16(phi),
+// lo = bf16(phi - hi), so hi + lo carries phi to ~2^-17 relative and products
+// on the tensor cores keep fp32-grade accuracy (ReLU needs no split: it is
+// exact in bf16).
+template <int FM>
+__device__ __forceinline__ void feature_split_bf16x2(uint32_t packed, uint32_t& hi, uint32_t& lo) {
+    const float2 x = bf16x2_to_float2(packed);
+    const float a = feature_f32<FM>(x.x);
+    const float b = feature_f32<FM>(x.y);
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 // streaming 16-byte global load that bypasses L1 allocation (inputs are read once)
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 r;

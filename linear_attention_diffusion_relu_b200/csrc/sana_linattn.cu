@@ -255,7 +255,7 @@ sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done
 }
 
 // ------------------------------------------------------------- launches ----
-template <int D>
+template <int D, int FM>
 sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, const Plan& p,
                             float* partial, float* state, cudaStream_t s) {
     static std::atomic<uint64_t> smem_set{0};
@@ -263,9 +263,9 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
     sana_la_status st;
     if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
-    if ((st = ensure_smem(sana::tc::ks_state_tc<D>, sana::tc::KsMap::BYTES, smem_set)) != SANA_LA_OK)
+    if ((st = ensure_smem(sana::tc::ks_state_tc<D, FM>, sana::tc::KsMap::BYTES, smem_set)) != SANA_LA_OK)
         return st;
-    if ((st = launch(sana::tc::ks_state_tc<D>, dim3(p.ks.q.grid), dim3(sana::tc::kThreads),
+    if ((st = launch(sana::tc::ks_state_tc<D, FM>, dim3(p.ks.q.grid), dim3(sana::tc::kThreads),
                      sana::tc::KsMap::BYTES, s, false, "ks_state_tc", tmK, tmV, p.ks, partial)) != SANA_LA_OK)
         return st;
     // the reduction overlaps the state kernel's tail; it waits for its results
@@ -281,7 +281,7 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
                   (const float*)partial, p.ks, state);
 }
 
-template <int D, bool OUT_BF16>
+template <int D, bool OUT_BF16, int FM>
 sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N, int H,
                             const Plan& p, const float* state, cudaStream_t s, bool overlap) {
     static std::atomic<uint64_t> smem_set{0};
@@ -289,15 +289,15 @@ sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N,
     sana_la_status st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
     constexpr int smem = sana::tc::KaMap<D, OUT_BF16>::BYTES;
-    if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16>, smem, smem_set)) != SANA_LA_OK) return st;
-    return launch(sana::tc::ka_apply_tc<D, OUT_BF16>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
+    if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, smem, smem_set)) != SANA_LA_OK) return st;
+    return launch(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
                   overlap, "ka_apply_tc", tmQ, tmO, p.ka, state);
 }
 
 // `overlap`: called right after this library's own state kernels on the same
 // stream (forward), so Q was ready before they started and the apply kernel
 // may start early; a standalone apply waits for everything before it.
-template <int D>
+template <int D, int FM>
 sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, int L, void* O,
                          sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
     Plan p = make_plan(B, N, H, D, L);
@@ -305,8 +305,8 @@ sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H,
     CUtensorMap tmQ;
     sana_la_status st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
-    return od == SANA_LA_OUT_BF16 ? launch_apply<D, true>(tmQ, O, B, N, H, p, state, s, overlap)
-                                  : launch_apply<D, false>(tmQ, O, B, N, H, p, state, s, overlap);
+    return od == SANA_LA_OUT_BF16 ? launch_apply<D, true, FM>(tmQ, O, B, N, H, p, state, s, overlap)
+                                  : launch_apply<D, false, FM>(tmQ, O, B, N, H, p, state, s, overlap);
 }
 
 // The whole forward as one cooperative launch (fwd_fused_tc). Returns
@@ -336,7 +336,7 @@ int blocks_per_sm(Kernel kernel, int threads, int smem, std::atomic<int> (&cache
     return v;
 }
 
-template <int D, bool OUT_BF16>
+template <int D, bool OUT_BF16, int FM>
 sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
                                     int H, const Plan& p, float* partial, unsigned long long* flags,
                                     cudaStream_t s) {
@@ -349,7 +349,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
     constexpr int smem = sana::tc::FwdMap<D, OUT_BF16>::BYTES;
-    auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16>;
+    auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16, FM>;
     if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
     const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
     int dev = 0, sms = 0;
@@ -399,65 +399,81 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
 
 sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, int d, int L,
                              float* state, void* ws, size_t ws_bytes, cudaStream_t s,
-                             bool need_state_area) {
+                             bool need_state_area, int fm = sana::kFeatureRelu) {
     const Plan p = make_plan(B, N, H, d, L);
     const size_t need = p.partial_bytes + (need_state_area ? p.state_bytes : 0);
     if (ws_bytes < need) return SANA_LA_ERR_WORKSPACE;
     float* partial = static_cast<float*>(ws);
-    return d == 32 ? run_kv_state<32>(K, V, B, N, H, p, partial, state, s)
-                   : run_kv_state<64>(K, V, B, N, H, p, partial, state, s);
+    switch (d * 4 + fm) {
+        case 32 * 4 + sana::kFeatureRelu: return run_kv_state<32, sana::kFeatureRelu>(K, V, B, N, H, p, partial, state, s);
+        case 32 * 4 + sana::kFeatureElu1: return run_kv_state<32, sana::kFeatureElu1>(K, V, B, N, H, p, partial, state, s);
+        case 32 * 4 + sana::kFeatureCos:  return run_kv_state<32, sana::kFeatureCos>(K, V, B, N, H, p, partial, state, s);
+        case 64 * 4 + sana::kFeatureRelu: return run_kv_state<64, sana::kFeatureRelu>(K, V, B, N, H, p, partial, state, s);
+        case 64 * 4 + sana::kFeatureElu1: return run_kv_state<64, sana::kFeatureElu1>(K, V, B, N, H, p, partial, state, s);
+        case 64 * 4 + sana::kFeatureCos:  return run_kv_state<64, sana::kFeatureCos>(K, V, B, N, H, p, partial, state, s);
+    }
+    return SANA_LA_ERR_INVALID_ARG;
 }
 
 sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d, int L,
-                          void* O, sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
-    return d == 32 ? run_apply<32>(Q, state, B, N, H, L, O, od, eps, s, overlap)
-                   : run_apply<64>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+                          void* O, sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap,
+                          int fm = sana::kFeatureRelu) {
+    switch (d * 4 + fm) {
+        case 32 * 4 + sana::kFeatureRelu: return run_apply<32, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 32 * 4 + sana::kFeatureElu1: return run_apply<32, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 32 * 4 + sana::kFeatureCos:  return run_apply<32, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 64 * 4 + sana::kFeatureRelu: return run_apply<64, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 64 * 4 + sana::kFeatureElu1: return run_apply<64, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 64 * 4 + sana::kFeatureCos:  return run_apply<64, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+    }
+    return SANA_LA_ERR_INVALID_ARG;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
-    if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
-    const Plan p = make_plan(B, N, H, d);
-    return p.partial_bytes + p.state_bytes + p.flag_bytes;
+template <int FM>
+sana_la_status forward_fused_dispatch(const void* Q, const void* K, const void* V, void* O, int B, int N,
+                                      int H, int d, bool bf16, const Plan& p, float* partial,
+                                      unsigned long long* flags, cudaStream_t s) {
+    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s))
+                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s));
 }
 
-sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,
-                                     float* state, void* workspace, size_t workspace_bytes,
-                                     sana_la_stream_t stream) {
+bool valid_feature(int fm) {
+    return fm == sana::kFeatureRelu || fm == sana::kFeatureElu1 || fm == sana::kFeatureCos;
+}
+
+sana_la_status kv_state_entry(const void* K, const void* V, int B, int N, int H, int d, int fm,
+                              float* state, void* workspace, size_t workspace_bytes,
+                              sana_la_stream_t stream) {
     g_last_error[0] = '\0';
-    if (!K || !V || !state || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    if (!K || !V || !state || !workspace || !valid_feature(fm)) return SANA_LA_ERR_INVALID_ARG;
     sana_la_status st = check_sizes(B, N, H, d);
     if (st != SANA_LA_OK) return st;
     if (!aligned16(K) || !aligned16(V) || !aligned16(state) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
     return kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes,
-                         reinterpret_cast<cudaStream_t>(stream), false);
+                         reinterpret_cast<cudaStream_t>(stream), false, fm);
 }
 
-sana_la_status sana_linattn_apply(const void* Q, const float* state, int B, int N, int H, int d,
-                                  void* O, sana_la_out_dtype out_dtype, float eps,
-                                  sana_la_stream_t stream) {
+sana_la_status apply_entry(const void* Q, const float* state, int B, int N, int H, int d, int fm,
+                           void* O, sana_la_out_dtype out_dtype, float eps, sana_la_stream_t stream) {
     g_last_error[0] = '\0';
-    if (!Q || !state || !O) return SANA_LA_ERR_INVALID_ARG;
+    if (!Q || !state || !O || !valid_feature(fm)) return SANA_LA_ERR_INVALID_ARG;
     sana_la_status st = check_sizes(B, N, H, d);
     if (st != SANA_LA_OK) return st;
     if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(Q) || !aligned16(state) || !aligned16(O)) return SANA_LA_ERR_INVALID_ARG;
     return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps,
-                      reinterpret_cast<cudaStream_t>(stream), false);
+                      reinterpret_cast<cudaStream_t>(stream), false, fm);
 }
 
-sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
-                                    int B, int N, int H, int d,
-                                    void* O, sana_la_out_dtype out_dtype, float eps,
-                                    void* workspace, size_t workspace_bytes,
-                                    sana_la_stream_t stream) {
+sana_la_status forward_entry(const void* Q, const void* K, const void* V, int B, int N, int H, int d, int fm,
+                             void* O, sana_la_out_dtype out_dtype, float eps, void* workspace,
+                             size_t workspace_bytes, sana_la_stream_t stream) {
     g_last_error[0] = '\0';
-    if (!Q || !K || !V || !O || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !O || !workspace || !valid_feature(fm)) return SANA_LA_ERR_INVALID_ARG;
     sana_la_status st = check_sizes(B, N, H, d);
     if (st != SANA_LA_OK) return st;
     if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
@@ -474,16 +490,75 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
     // one cooperative launch: state phase, grid barrier, apply phase
     p.ka.eps = eps;
     const bool bf16 = out_dtype == SANA_LA_OUT_BF16;
-    st = d == 32 ? (bf16 ? launch_forward_fused<32, true>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                         : launch_forward_fused<32, false>(Q, K, V, O, B, N, H, p, partial, flags, s))
-                 : (bf16 ? launch_forward_fused<64, true>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                         : launch_forward_fused<64, false>(Q, K, V, O, B, N, H, p, partial, flags, s));
+    switch (fm) {
+        case sana::kFeatureElu1:
+            st = forward_fused_dispatch<sana::kFeatureElu1>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+            break;
+        case sana::kFeatureCos:
+            st = forward_fused_dispatch<sana::kFeatureCos>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+            break;
+        default:
+            st = forward_fused_dispatch<sana::kFeatureRelu>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+    }
     if (st != SANA_LA_ERR_UNSUPPORTED) return st;
     // the device cannot hold the whole grid at once: the same kernels as
     // kv_state + apply, overlapped by programmatic launch
-    st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes, s, true);
+    st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes, s, true, fm);
     if (st != SANA_LA_OK) return st;
-    return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true);
+    return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true, fm);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
+    const Plan p = make_plan(B, N, H, d);
+    return p.partial_bytes + p.state_bytes + p.flag_bytes;
+}
+
+sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,
+                                     float* state, void* workspace, size_t workspace_bytes,
+                                     sana_la_stream_t stream) {
+    return kv_state_entry(K, V, B, N, H, d, sana::kFeatureRelu, state, workspace, workspace_bytes, stream);
+}
+
+sana_la_status sana_linattn_apply(const void* Q, const float* state, int B, int N, int H, int d,
+                                  void* O, sana_la_out_dtype out_dtype, float eps,
+                                  sana_la_stream_t stream) {
+    return apply_entry(Q, state, B, N, H, d, sana::kFeatureRelu, O, out_dtype, eps, stream);
+}
+
+sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
+                                    int B, int N, int H, int d,
+                                    void* O, sana_la_out_dtype out_dtype, float eps,
+                                    void* workspace, size_t workspace_bytes,
+                                    sana_la_stream_t stream) {
+    return forward_entry(Q, K, V, B, N, H, d, sana::kFeatureRelu, O, out_dtype, eps, workspace,
+                         workspace_bytes, stream);
+}
+
+// ------------------------------------------------------- feature maps ----
+sana_la_status sana_linattn_kv_state_fm(const void* K, const void* V, int B, int N, int H, int d,
+                                        sana_la_feature_map feature_map, float* state, void* workspace,
+                                        size_t workspace_bytes, sana_la_stream_t stream) {
+    return kv_state_entry(K, V, B, N, H, d, (int)feature_map, state, workspace, workspace_bytes, stream);
+}
+
+sana_la_status sana_linattn_apply_fm(const void* Q, const float* state, int B, int N, int H, int d,
+                                     sana_la_feature_map feature_map, void* O, sana_la_out_dtype out_dtype,
+                                     float eps, sana_la_stream_t stream) {
+    return apply_entry(Q, state, B, N, H, d, (int)feature_map, O, out_dtype, eps, stream);
+}
+
+sana_la_status sana_linattn_forward_fm(const void* Q, const void* K, const void* V,
+                                       int B, int N, int H, int d, sana_la_feature_map feature_map,
+                                       void* O, sana_la_out_dtype out_dtype, float eps,
+                                       void* workspace, size_t workspace_bytes,
+                                       sana_la_stream_t stream) {
+    return forward_entry(Q, K, V, B, N, H, d, (int)feature_map, O, out_dtype, eps, workspace,
+                         workspace_bytes, stream);
 }
 
 // ------------------------------------------------------- block-causal ----

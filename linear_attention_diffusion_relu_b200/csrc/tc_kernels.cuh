@@ -93,6 +93,27 @@ __device__ __forceinline__ void relu_smem(uint8_t* base, int tid) {
     }
 }
 
+// phi on N16 16-byte chunks of K at base, split: hi in place, lo to the same
+// offsets at lo_base. Worker t takes chunks t, t+256, ...
+template <int FM, int N16>
+__device__ __forceinline__ void feature_split_smem(uint8_t* base, uint8_t* lo_base, int tid) {
+    constexpr int PER = N16 / kWorkerThreads;
+    static_assert(N16 % kWorkerThreads == 0, "whole chunks per worker");
+    uint4 v[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) v[j] = *reinterpret_cast<const uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        uint4 h, l;
+        feature_split_bf16x2<FM>(v[j].x, h.x, l.x);
+        feature_split_bf16x2<FM>(v[j].y, h.y, l.y);
+        feature_split_bf16x2<FM>(v[j].z, h.z, l.z);
+        feature_split_bf16x2<FM>(v[j].w, h.w, l.w);
+        *reinterpret_cast<uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16) = h;
+        *reinterpret_cast<uint4*>(lo_base + (size_t)(tid + j * kWorkerThreads) * 16) = l;
+    }
+}
+
 // Bounded wait whose outcome is the same for every lane of the warp: if any
 // lane gives up, all do. Worker code paths stay warp-uniform this way, so a
 // wind-down never leaves part of a warp at a warp-synchronous instruction.
@@ -147,12 +168,21 @@ struct KsParams {
 };
 
 constexpr int KS_TILE = 64;                                // tokens per stage
-constexpr int KS_STAGES = 6;
+constexpr int KS_STAGES = 6;                               // stages with phi = ReLU
 constexpr int KS_BOX_BYTES = KS_TILE * kBoxBytesRow;       // 8 KB
 constexpr int KS_STAGE_BYTES = 4 * KS_BOX_BYTES;           // K0 K1 V0 V1
 constexpr int KS_ONES_OFF = KS_STAGES * KS_STAGE_BYTES;
 constexpr int KS_DATA_BYTES = KS_ONES_OFF + 1024;          // stages + the ones tile
 constexpr int KS_NUM_BARS = 3 * KS_STAGES + 5;
+// Other feature maps need phi(K) as bf16 hi + lo: 4 stages, and after them a
+// lo copy of each stage's two K boxes (same swizzled layout), in the same bytes.
+constexpr int KS_STAGES_SPLIT = 4;
+constexpr int KS_LO_OFF = KS_STAGES_SPLIT * KS_STAGE_BYTES;
+constexpr int KS_LO_BYTES = 2 * KS_BOX_BYTES;
+static_assert(KS_LO_OFF + KS_STAGES_SPLIT * KS_LO_BYTES == KS_ONES_OFF, "split layout fits the ReLU one");
+
+template <int FM>
+__host__ __device__ constexpr int ks_stages() { return FM == kFeatureRelu ? KS_STAGES : KS_STAGES_SPLIT; }
 
 struct KsBars {
     uint64_t* full;        // [KS_STAGES] K and V tiles landed
@@ -194,7 +224,7 @@ __device__ __forceinline__ void ks_fill_ones(uint8_t* smem, int tid) {
 // of this phase is free again once bar.empty[s] has completed the phase of the
 // last tile that used it (the single-launch kernel's apply phase waits for
 // that before it loads into the same bytes).
-template <int D>
+template <int D, int FM>
 __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
                                          int cta, float* __restrict__ partial, uint8_t* smem,
                                          const KsBars& bar, uint32_t tmem, volatile int* abort,
@@ -202,6 +232,7 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
+    constexpr int NS = ks_stages<FM>();
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -209,14 +240,15 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
     const int tps = sched_tps(cta, p.q);
     const int ntiles = tps * sched_nseg(cta, p.q);
     auto stage_ptr = [&](int s) { return smem + (size_t)s * KS_STAGE_BYTES; };
+    auto lo_ptr = [&](int s) { return smem + KS_LO_OFF + (size_t)s * KS_LO_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int issued = 0;
             for (int i = 0; i < ntiles; ++i) {
-                const int s = i % KS_STAGES;
-                if (!ptx::mbar_wait(&bar.empty[s], ((i / KS_STAGES) & 1) ^ 1, abort, err)) break;
+                const int s = i % NS;
+                if (!ptx::mbar_wait(&bar.empty[s], ((i / NS) & 1) ^ 1, abort, err)) break;
                 int slab, tile, seg;
                 sched_item(cta, i, tps, p.q, slab, tile, seg);
                 const int b = slab / p.groups;
@@ -231,8 +263,8 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
                 issued = i + 1;
             }
             // drain: every issued load must land before the CTA may exit
-            for (int i = (issued > KS_STAGES ? issued - KS_STAGES : 0); i < issued; ++i)
-                ptx::mbar_wait(&bar.full[i % KS_STAGES], (i / KS_STAGES) & 1, nullptr, err);
+            for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+                ptx::mbar_wait(&bar.full[i % NS], (i / NS) & 1, nullptr, err);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- UMMA issuer ----
@@ -252,8 +284,8 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
                     ptx::tc_fence_after_sync();
                     first = true;
                 }
-                const int s = i % KS_STAGES;
-                if (!ptx::mbar_wait(&bar.relu_done[s], (i / KS_STAGES) & 1, abort, err)) break;
+                const int s = i % NS;
+                if (!ptx::mbar_wait(&bar.relu_done[s], (i / NS) & 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const uint32_t d_tmem = tmem + (uint32_t)(seg & 1) * 256u;
                 const uint32_t k_addr = ptx::smem_u32(stage_ptr(s));
@@ -268,6 +300,13 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
                     const bool acc = !(first && ks == 0);
                     ptx::umma_f16_ss(d_tmem, a, bv, idesc_v, acc);
                     ptx::umma_f16_ss(d_tmem + 128, a, ones_desc, idesc_1, acc);
+                    if constexpr (FM != kFeatureRelu) {
+                        // the lo part of phi(K): phi(K)^T [V | 1] = hi^T [V | 1] + lo^T [V | 1]
+                        const uint64_t al = ptx::smem_desc(ptx::smem_u32(lo_ptr(s)) + ks * 2048, KS_BOX_BYTES,
+                                                           1024, ptx::kLayoutSW128);
+                        ptx::umma_f16_ss(d_tmem, al, bv, idesc_v, true);
+                        ptx::umma_f16_ss(d_tmem + 128, al, ones_desc, idesc_1, true);
+                    }
                 }
                 first = false;
                 ptx::umma_commit(&bar.empty[s]);
@@ -281,9 +320,12 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
         for (int i = 0; i < ntiles; ++i) {
             const bool seg_end = (i % tps) == tps - 1;
             const int seg = i / tps;
-            const int s = i % KS_STAGES;
-            if (!warp_wait(&bar.full[s], (i / KS_STAGES) & 1, abort, err)) break;
-            relu_smem<2 * KS_BOX_BYTES / 16>(stage_ptr(s), tid);     // phi on the K boxes only
+            const int s = i % NS;
+            if (!warp_wait(&bar.full[s], (i / NS) & 1, abort, err)) break;
+            if constexpr (FM == kFeatureRelu)
+                relu_smem<2 * KS_BOX_BYTES / 16>(stage_ptr(s), tid);     // phi on the K boxes only
+            else
+                feature_split_smem<FM, 2 * KS_BOX_BYTES / 16>(stage_ptr(s), lo_ptr(s), tid);
             ptx::fence_proxy_async_smem();
             warp_arrive(&bar.relu_done[s]);
             if (seg_end && warp < 4) {
@@ -439,6 +481,7 @@ constexpr int KA_TILE = 128;                               // tokens = UMMA M
 constexpr int KA_BOX_BYTES = KA_TILE * kBoxBytesRow;       // 16 KB
 constexpr int KA_STAGE_BYTES = 2 * KA_BOX_BYTES;           // one group row of 128 tokens
 constexpr uint32_t KA_A_COL = 256;                         // first A buffer column
+constexpr uint32_t KA_A_LO_COL = 384;                      // lo parts of phi(Q) (feature maps other than ReLU)
 constexpr int kBarRegion = 4096;                           // barriers + control block + slack
 
 template <int D, bool OUT_BF16>
@@ -583,7 +626,7 @@ __device__ __forceinline__ bool grid_wait(const unsigned long long* flags, int n
 // `prev_empty`/`prev_tiles` (single launch): the state phase's stage barriers
 // and how many tiles it loaded; Q stage s (< 6) reuses its stage s, so the
 // first load into each waits until the state phase released that stage.
-template <int D, bool OUT_BF16>
+template <int D, bool OUT_BF16, int FM>
 __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorMap* tmO, const KaParams& p,
                                          int cta, const KaStateSrc& src, uint8_t* smem,
                                          const KaBars<D, OUT_BF16>& bar, uint32_t tmem,
@@ -607,14 +650,15 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int issued = 0;
-            static_assert(L::STAGES <= KS_STAGES && KA_STAGE_BYTES == KS_STAGE_BYTES, "stage reuse");
+            constexpr int PS = ks_stages<FM>();       // the state phase's stages (single launch)
+            static_assert(L::STAGES <= PS && KA_STAGE_BYTES == KS_STAGE_BYTES, "stage reuse");
             for (int i = 0; i < nunits; ++i) {
                 const int s = i % S;
                 if (!ptx::mbar_wait(&bar.empty[s], ((i / S) & 1) ^ 1, abort, err)) break;
                 if (prev_empty != nullptr && i < S) {
                     // the state phase's next (never issued) use of stage s
-                    const int j = prev_tiles + ((s - prev_tiles) % KS_STAGES + KS_STAGES) % KS_STAGES;
-                    if (!ptx::mbar_wait(&prev_empty[s], ((j / KS_STAGES) & 1) ^ 1, abort, err)) break;
+                    const int j = prev_tiles + ((s - prev_tiles) % PS + PS) % PS;
+                    if (!ptx::mbar_wait(&prev_empty[s], ((j / PS) & 1) ^ 1, abort, err)) break;
                 }
                 int slab, tile, seg;
                 sched_item(cta, i, tps, p.q, slab, tile, seg);
@@ -638,6 +682,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 if (!ptx::mbar_wait(bar.acc_empty, (i & 1) ^ 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
                 const uint32_t a_base = tmem + KA_A_COL + (uint32_t)(i & 1) * 64u;
+                const uint32_t a_lo_base = tmem + KA_A_LO_COL + (uint32_t)(i & 1) * 64u;
 #pragma unroll
                 for (int hh = 0; hh < G; ++hh) {
                     const uint32_t d_tmem = tmem + (uint32_t)(hh * L::ACC_COLS);
@@ -650,6 +695,12 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                                          idesc, ks > 0);
                         ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(lo, 128, L::SBO, ptx::kLayoutNone),
                                          idesc, true);
+                        if constexpr (FM != kFeatureRelu) {
+                            // phi(Q) lo x S hi (lo x lo is below fp32 rounding)
+                            const uint32_t al = a_lo_base + (uint32_t)(hh * D / 2 + ks * 8);
+                            ptx::umma_f16_ts(d_tmem, al, ptx::smem_desc(hi, 128, L::SBO, ptx::kLayoutNone),
+                                             idesc, true);
+                        }
                     }
                 }
                 ptx::umma_commit(bar.acc_full);
@@ -767,16 +818,31 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
             // row m of box `half`: logical 16-byte chunk q sits at q ^ (m % 8)
             const uint8_t* row = stage_ptr(s) + half * KA_BOX_BYTES + m * kBoxBytesRow;
             uint32_t r[32];
+            if constexpr (FM == kFeatureRelu) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row + ((q ^ (m & 7)) * 16));
-                r[4 * q + 0] = relu_bf16x2(v.x);
-                r[4 * q + 1] = relu_bf16x2(v.y);
-                r[4 * q + 2] = relu_bf16x2(v.z);
-                r[4 * q + 3] = relu_bf16x2(v.w);
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + ((q ^ (m & 7)) * 16));
+                    r[4 * q + 0] = relu_bf16x2(v.x);
+                    r[4 * q + 1] = relu_bf16x2(v.y);
+                    r[4 * q + 2] = relu_bf16x2(v.z);
+                    r[4 * q + 3] = relu_bf16x2(v.w);
+                }
+                warp_arrive(&bar.empty[s]);
+                __syncwarp();
+            } else {
+                uint32_t rl[32];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + ((q ^ (m & 7)) * 16));
+                    feature_split_bf16x2<FM>(v.x, r[4 * q + 0], rl[4 * q + 0]);
+                    feature_split_bf16x2<FM>(v.y, r[4 * q + 1], rl[4 * q + 1]);
+                    feature_split_bf16x2<FM>(v.z, r[4 * q + 2], rl[4 * q + 2]);
+                    feature_split_bf16x2<FM>(v.w, r[4 * q + 3], rl[4 * q + 3]);
+                }
+                warp_arrive(&bar.empty[s]);
+                __syncwarp();
+                ptx::tmem_st32_wait(lane_base + KA_A_LO_COL + (uint32_t)(i & 1) * 64u + (uint32_t)half * 32u, rl);
             }
-            warp_arrive(&bar.empty[s]);
-            __syncwarp();
             ptx::tmem_st32_wait(lane_base + KA_A_COL + (uint32_t)(i & 1) * 64u + (uint32_t)half * 32u, r);
             ptx::tc_fence_before_sync();
             warp_arrive(&bar.a_full[i & 1]);
@@ -896,7 +962,7 @@ template <int D, bool OUT_BF16>
 using FwdMap = SmemMap<(KaLayout<D, OUT_BF16>::DATA_BYTES > KS_DATA_BYTES ? KaLayout<D, OUT_BF16>::DATA_BYTES
                                                                           : KS_DATA_BYTES)>;
 
-template <int D>
+template <int D, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
 ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
             const KsParams p, float* __restrict__ partial)
@@ -921,11 +987,11 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     ptx::tc_fence_after_sync();
     // the reduction kernel may be scheduled now; it waits for this grid's results
     if (tid == 0) ptx::launch_dependents();
-    ks_phase<D>(&tmK, &tmV, p, blockIdx.x, partial, smem, bar, ctl->tmem_base, &ctl->abort, &g_device_error);
+    ks_phase<D, FM>(&tmK, &tmV, p, blockIdx.x, partial, smem, bar, ctl->tmem_base, &ctl->abort, &g_device_error);
     kernel_epilogue(ctl, tid);
 }
 
-template <int D, bool OUT_BF16>
+template <int D, bool OUT_BF16, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
 ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
             const KaParams p, const float* __restrict__ state)
@@ -950,7 +1016,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after_sync();
     KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, 0};
-    ka_phase<D, OUT_BF16>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
+    ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
                           &g_device_error);
     kernel_epilogue(ctl, tid);
 }
@@ -961,7 +1027,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 // start as soon as the state phase has released its shared memory, so they
 // overlap the barrier. `flags` has one slot per CTA; `epoch` is unique to the
 // launch.
-template <int D, bool OUT_BF16>
+template <int D, bool OUT_BF16, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -1001,7 +1067,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     ptx::tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
-    ks_phase<D>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error);
+    ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error);
 
     // Warps 0-3 have written this CTA's partial states (after the last
     // accumulator was complete, i.e. after every state-phase UMMA): make them
@@ -1020,7 +1086,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     KaStateSrc src{nullptr, partial, ks, flags, epoch, (int)gridDim.x};
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
-    ka_phase<D, OUT_BF16>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
+    ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
                           kbar.empty, ks_tiles);
     kernel_epilogue(ctl, tid);
 }

@@ -12,6 +12,8 @@ The functions mirror the C ABI in ``include/sana_linattn.h``:
     apply(Q, state, out_dtype=torch.bfloat16, eps=1e-15, out=None) -> O (B, N, H, d)
     forward(Q, K, V, out_dtype=torch.bfloat16, eps=1e-15, out=None, workspace=None) -> O
 
+each with ``feature_map="relu" | "elu1" | "cos"`` (the ``*_fm`` entry points),
+
 and the block-causal form (blocks of L tokens, L a multiple of 128):
 
     block_causal_workspace_bytes(B, N, H, d, L)
@@ -32,6 +34,7 @@ LIBRARY = os.path.join(_PKG, "libsana_linattn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = range(5)
 OUT_F32, OUT_BF16 = 0, 1
+FEATURE_MAPS = {"relu": 0, "elu1": 1, "cos": 2}
 
 SYMBOLS = (
     "sana_linattn_workspace_bytes",
@@ -39,6 +42,9 @@ SYMBOLS = (
     "sana_linattn_apply",
     "sana_linattn_forward",
     "sana_linattn_forward_launches",
+    "sana_linattn_kv_state_fm",
+    "sana_linattn_apply_fm",
+    "sana_linattn_forward_fm",
     "sana_linattn_block_causal_workspace_bytes",
     "sana_linattn_block_causal_kv_state",
     "sana_linattn_block_causal_apply",
@@ -91,6 +97,12 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_device_error.restype = st
         lib.sana_linattn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
         lib.sana_linattn_selftest_wait_timeout.restype = st
+        lib.sana_linattn_kv_state_fm.argtypes = [vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+        lib.sana_linattn_kv_state_fm.restype = st
+        lib.sana_linattn_apply_fm.argtypes = [vp, vp, i, i, i, i, i, vp, i, f, vp]
+        lib.sana_linattn_apply_fm.restype = st
+        lib.sana_linattn_forward_fm.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_forward_fm.restype = st
         lib.sana_linattn_block_causal_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.sana_linattn_block_causal_workspace_bytes.restype = sz
         lib.sana_linattn_block_causal_kv_state.argtypes = [vp, vp, i, i, i, i, i, vp, vp, sz, vp]
@@ -138,6 +150,12 @@ def _check_bnhd(name, t, shape=None):
         raise ValueError(f"{name} shape {tuple(t.shape)} != {tuple(shape)}")
 
 
+def _feature_code(feature_map: str) -> int:
+    if feature_map not in FEATURE_MAPS:
+        raise ValueError(f"feature_map must be one of {sorted(FEATURE_MAPS)}, got {feature_map!r}")
+    return FEATURE_MAPS[feature_map]
+
+
 def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -183,8 +201,9 @@ def make_workspace(B: int, N: int, H: int, d: int, device="cuda") -> torch.Tenso
 
 
 def kv_state(K: torch.Tensor, V: torch.Tensor, state: torch.Tensor | None = None,
-             workspace: torch.Tensor | None = None) -> torch.Tensor:
+             workspace: torch.Tensor | None = None, feature_map: str = "relu") -> torch.Tensor:
     """state = phi(K)^T [V | 1] per (b, h), fp32 (B, H, d, d+1)."""
+    fm = _feature_code(feature_map)
     _check_bnhd("K", K)
     _check_bnhd("V", V, K.shape)
     B, N, H, d = K.shape
@@ -196,10 +215,10 @@ def kv_state(K: torch.Tensor, V: torch.Tensor, state: torch.Tensor | None = None
     if workspace is None:
         workspace = make_workspace(B, N, H, d, K.device)
     lib = load_library()
-    st = lib.sana_linattn_kv_state(K.data_ptr(), V.data_ptr(), B, N, H, d, state.data_ptr(),
-                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                   _stream(K.device))
-    _check(lib, st, "sana_linattn_kv_state")
+    st = lib.sana_linattn_kv_state_fm(K.data_ptr(), V.data_ptr(), B, N, H, d, fm, state.data_ptr(),
+                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                      _stream(K.device))
+    _check(lib, st, "sana_linattn_kv_state_fm")
     return state
 
 
@@ -213,8 +232,9 @@ def _prep_out(out, shape, dtype, device):
 
 
 def apply(Q: torch.Tensor, state: torch.Tensor, out_dtype=torch.bfloat16, eps: float = 1e-15,
-          out: torch.Tensor | None = None) -> torch.Tensor:
+          out: torch.Tensor | None = None, feature_map: str = "relu") -> torch.Tensor:
     """O = (phi(Q) state[..., :d]) / (phi(Q) state[..., d] + eps)."""
+    fm = _feature_code(feature_map)
     _check_bnhd("Q", Q)
     B, N, H, d = Q.shape
     if (state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d + 1)
@@ -223,16 +243,17 @@ def apply(Q: torch.Tensor, state: torch.Tensor, out_dtype=torch.bfloat16, eps: f
     code = _out_code(out_dtype)
     out = _prep_out(out, Q.shape, out_dtype, Q.device)
     lib = load_library()
-    st = lib.sana_linattn_apply(Q.data_ptr(), state.data_ptr(), B, N, H, d, out.data_ptr(), code,
-                                float(eps), _stream(Q.device))
-    _check(lib, st, "sana_linattn_apply")
+    st = lib.sana_linattn_apply_fm(Q.data_ptr(), state.data_ptr(), B, N, H, d, fm, out.data_ptr(), code,
+                                   float(eps), _stream(Q.device))
+    _check(lib, st, "sana_linattn_apply_fm")
     return out
 
 
 def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.bfloat16,
             eps: float = 1e-15, out: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Whole ReLU linear-attention forward; bit-identical to kv_state + apply."""
+            workspace: torch.Tensor | None = None, feature_map: str = "relu") -> torch.Tensor:
+    """Whole linear-attention forward; bit-identical to kv_state + apply."""
+    fm = _feature_code(feature_map)
     _check_bnhd("Q", Q)
     _check_bnhd("K", K, Q.shape)
     _check_bnhd("V", V, Q.shape)
@@ -242,10 +263,10 @@ def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.b
     if workspace is None:
         workspace = make_workspace(B, N, H, d, Q.device)
     lib = load_library()
-    st = lib.sana_linattn_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d,
-                                  out.data_ptr(), code, float(eps), workspace.data_ptr(),
-                                  workspace.numel() * workspace.element_size(), _stream(Q.device))
-    _check(lib, st, "sana_linattn_forward")
+    st = lib.sana_linattn_forward_fm(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d, fm,
+                                     out.data_ptr(), code, float(eps), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), _stream(Q.device))
+    _check(lib, st, "sana_linattn_forward_fm")
     return out
 
 

@@ -19,7 +19,8 @@ frame, 16 frames, after the video row of the token table in
 "08_sana高效高分辨率生成" (papers-3lj.pages.dev), section "Linear Attention 的原理"
 (4096x4096 x 16 frames = 1,048,576 tokens, i.e. 65,536 per frame; that table
 counts 4,096 tokens per 1024x1024 frame). They draw the same tensors as the
-sweep workloads of the same size (same seed and shape).
+sweep workloads of the same size (same seed and shape). The ``_elu1`` and ``_cos``
+workloads draw the tensors of the 4096px one and use another feature map.
 
 Recipe (all draws from one torch generator seeded per workload):
   1. Q, K, V drawn in that order with ``torch.randn`` in float32, each shaped
@@ -56,6 +57,7 @@ class Workload:
     eps: float = 1e-15
     description: str = ""
     block: int = 0                  # block-causal form: tokens per block (0 = not block-causal)
+    feature: str = "relu"           # feature map phi: "relu" | "elu1" | "cos"
 
     @property
     def token_heads(self) -> int:
@@ -89,6 +91,10 @@ WORKLOADS: dict[str, Workload] = {
                               description="ragged token count, B=1, H=36, d=32"),
     "d64": Workload("d64", 1, 16384, 18, 64, seed=4,
                     description="head size 64, B=1, N=16384, H=18"),
+    "4096px_elu1": Workload("4096px_elu1", 2, 16384, 70, 32, seed=3, feature="elu1",
+                            description="the 4096px step with phi = ELU+1"),
+    "4096px_cos": Workload("4096px_cos", 2, 16384, 70, 32, seed=3, feature="cos",
+                           description="the 4096px step with phi = cos"),
     "video16f_1024px": Workload("video16f_1024px", 1, 16 * 4096, 36, 32, seed=4, block=4096,
                                 description="block-causal, 16 frames of 4,096 tokens, H=36, d=32"),
     "video16f_4096px": Workload("video16f_4096px", 1, 16 * 65536, 36, 32, seed=4, block=65536,

@@ -143,3 +143,21 @@ def test_block_causal_host_checks(lib):
     ap = lib.sana_linattn_block_causal_apply
     assert ap(FAKE, FAKE, 1, 1024, 2, 32, 200, FAKE, 0, 0.0, None) == ops.ERR_UNSUPPORTED
     assert ap(FAKE, FAKE, 1, 1024, 2, 32, 256, FAKE, 5, 0.0, None) == ops.ERR_INVALID_ARG
+
+
+def test_feature_map_host_checks(lib):
+    wsb = lib.sana_linattn_workspace_bytes(1, 64, 2, 32)
+    f = lib.sana_linattn_forward_fm
+    for bad in (-1, 3, 99):
+        assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, bad, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_INVALID_ARG
+        assert lib.sana_linattn_kv_state_fm(FAKE, FAKE, 1, 64, 2, 32, bad, FAKE, FAKE, wsb, None) \
+            == ops.ERR_INVALID_ARG
+        assert lib.sana_linattn_apply_fm(FAKE, FAKE, 1, 64, 2, 32, bad, FAKE, 1, 0.0, None) == ops.ERR_INVALID_ARG
+    # valid feature maps still get the ordinary checks
+    for fm in ops.FEATURE_MAPS.values():
+        assert f(FAKE, FAKE, FAKE, 1, 64, 2, 48, fm, FAKE, 1, 1e-15, FAKE, wsb, None) == ops.ERR_UNSUPPORTED
+        assert f(FAKE, FAKE, FAKE, 1, 64, 2, 32, fm, FAKE, 1, 1e-15, FAKE, wsb - 1, None) == ops.ERR_WORKSPACE
+    import torch
+    x = torch.zeros((1, 8, 1, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="feature_map"):
+        ops.forward(x, x, x, feature_map="softmax")
