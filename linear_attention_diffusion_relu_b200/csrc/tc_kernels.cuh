@@ -93,10 +93,13 @@ __device__ __forceinline__ void relu_smem(uint8_t* base, int tid) {
     }
 }
 
-// phi on N16 16-byte chunks of K at base, split: hi in place, lo to the same
-// offsets at lo_base. Worker t takes chunks t, t+256, ...
-template <int FM, int N16>
-__device__ __forceinline__ void feature_split_smem(uint8_t* base, uint8_t* lo_base, int tid) {
+// phi on the K boxes of a state-phase stage (N16 16-byte chunks of 128-byte
+// rows, one token per row), split: hi in place, lo to the same offsets at
+// lo_base. Rows at or past `valid_rows` are tokens past N, which TMA filled
+// with zeros; phi(0) is not 0 for these feature maps, so they are written as
+// zeros. Worker t takes chunks t, t+256, ...
+template <int FM, int N16, int BOX_ROWS>
+__device__ __forceinline__ void feature_split_smem(uint8_t* base, uint8_t* lo_base, int valid_rows, int tid) {
     constexpr int PER = N16 / kWorkerThreads;
     static_assert(N16 % kWorkerThreads == 0, "whole chunks per worker");
     uint4 v[PER];
@@ -104,13 +107,17 @@ __device__ __forceinline__ void feature_split_smem(uint8_t* base, uint8_t* lo_ba
     for (int j = 0; j < PER; ++j) v[j] = *reinterpret_cast<const uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16);
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
-        uint4 h, l;
-        feature_split_bf16x2<FM>(v[j].x, h.x, l.x);
-        feature_split_bf16x2<FM>(v[j].y, h.y, l.y);
-        feature_split_bf16x2<FM>(v[j].z, h.z, l.z);
-        feature_split_bf16x2<FM>(v[j].w, h.w, l.w);
-        *reinterpret_cast<uint4*>(base + (size_t)(tid + j * kWorkerThreads) * 16) = h;
-        *reinterpret_cast<uint4*>(lo_base + (size_t)(tid + j * kWorkerThreads) * 16) = l;
+        const int c = tid + j * kWorkerThreads;
+        const int row = (c % (BOX_ROWS * 8)) / 8;     // 8 chunks per 128-byte row, one box after the other
+        uint4 h = make_uint4(0u, 0u, 0u, 0u), l = make_uint4(0u, 0u, 0u, 0u);
+        if (row < valid_rows) {
+            feature_split_bf16x2<FM>(v[j].x, h.x, l.x);
+            feature_split_bf16x2<FM>(v[j].y, h.y, l.y);
+            feature_split_bf16x2<FM>(v[j].z, h.z, l.z);
+            feature_split_bf16x2<FM>(v[j].w, h.w, l.w);
+        }
+        *reinterpret_cast<uint4*>(base + (size_t)c * 16) = h;
+        *reinterpret_cast<uint4*>(lo_base + (size_t)c * 16) = l;
     }
 }
 
@@ -322,10 +329,14 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
             const int seg = i / tps;
             const int s = i % NS;
             if (!warp_wait(&bar.full[s], (i / NS) & 1, abort, err)) break;
-            if constexpr (FM == kFeatureRelu)
+            if constexpr (FM == kFeatureRelu) {
                 relu_smem<2 * KS_BOX_BYTES / 16>(stage_ptr(s), tid);     // phi on the K boxes only
-            else
-                feature_split_smem<FM, 2 * KS_BOX_BYTES / 16>(stage_ptr(s), lo_ptr(s), tid);
+            } else {
+                int slab, tile, sg;
+                sched_item(cta, i, tps, p.q, slab, tile, sg);
+                feature_split_smem<FM, 2 * KS_BOX_BYTES / 16, KS_TILE>(stage_ptr(s), lo_ptr(s),
+                                                                      p.N - tile * KS_TILE, tid);
+            }
             ptx::fence_proxy_async_smem();
             warp_arrive(&bar.relu_done[s]);
             if (seg_end && warp < 4) {
