@@ -151,9 +151,10 @@ sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
 /*
  * The three calls above with another feature map phi. SANA_LA_FEATURE_RELU
  * gives exactly the calls above. For ELU+1 and cos, phi is evaluated in fp32
- * from the bf16 inputs (CUDA's expf and cosf) and carried into the tensor-core
- * products as a bf16 hi + lo pair (~2^-17 relative), so the accuracy matches the
- * ReLU path; the state kernel runs with 4 instead of 6 pipeline stages and the
+ * from the bf16 inputs (the hardware exponential; for cos a Cody-Waite
+ * reduction to [-pi, pi] and the hardware cosine) and carried into the
+ * tensor-core products as a bf16 hi + lo pair (~2^-17 relative), so the
+ * output meets the ReLU path's tolerance; the state kernel runs with 4 instead of 6 pipeline stages and the
  * apply kernel issues one more product per head. With cos the normaliser
  * phi(Q) state[:, d] can be zero or negative; O = num / (den + eps) is returned
  * as it stands. A feature_map outside the enum is SANA_LA_ERR_INVALID_ARG. The

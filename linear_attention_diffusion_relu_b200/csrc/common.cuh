@@ -30,10 +30,29 @@ __device__ __forceinline__ uint32_t float2_to_bf16x2(float a, float b) {
 // ELU+1 and cos named as alternatives). ELU is taken with alpha = 1.
 enum : int { kFeatureRelu = 0, kFeatureElu1 = 1, kFeatureCos = 2 };
 
+// cos(x) for moderate |x|: Cody-Waite additive range reduction (W. J. Cody and
+// W. Waite, "Software Manual for the Elementary Functions", 1980) by the
+// nearest multiple of 2*pi, with 2*pi carried as a float head plus a float
+// tail and both products folded in by fma, then the hardware cosine
+// (__cosf), whose error bound holds on [-pi, pi]. Inputs are bf16 activations
+// (|x| of order 10 at most), where the reduced argument is accurate to a few
+// float ulps.
+__device__ __forceinline__ float cos_reduced(float x) {
+    constexpr float kInv2Pi = 0.159154943091895336f;          // 1 / (2 pi), rounded
+    constexpr float k2PiHi = 6.28318548202514648f;            // float(2 pi)
+    constexpr float k2PiLo = -1.74845553146951880e-07f;       // 2 pi - float(2 pi)
+    const float k = rintf(x * kInv2Pi);
+    float r = fmaf(-k, k2PiHi, x);
+    r = fmaf(-k, k2PiLo, r);
+    return __cosf(r);
+}
+
+// ELU+1 uses the hardware exponential (__expf) on x <= 0, where its relative
+// error is far below the bf16 hi/lo split's.
 template <int FM>
 __device__ __forceinline__ float feature_f32(float x) {
-    if constexpr (FM == kFeatureElu1) return x > 0.0f ? x + 1.0f : expf(x);
-    else if constexpr (FM == kFeatureCos) return cosf(x);
+    if constexpr (FM == kFeatureElu1) return x > 0.0f ? x + 1.0f : __expf(x);
+    else if constexpr (FM == kFeatureCos) return cos_reduced(x);
     else return fmaxf(x, 0.0f);
 }
 

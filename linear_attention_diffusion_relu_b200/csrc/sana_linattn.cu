@@ -270,11 +270,11 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
         return st;
     // the reduction overlaps the state kernel's tail; it waits for its results
     if (p.ks.q.nblk > 1) {
-        // block-causal: prefix states over the blocks, one warp per entry
+        // block-causal: prefix states over the blocks
         const dim3 kp_grid((unsigned)((long long)B * H),
-                           (D * (D + 1) + sana::tc::KP_WARPS - 1) / sana::tc::KP_WARPS);
-        return launch(sana::tc::kr_prefix_tc<D>, kp_grid, dim3(sana::tc::KP_WARPS * 32), 0, s, true,
-                      "kr_prefix_tc", (const float*)partial, p.ks, state);
+                           (D * (D + 1) + sana::tc::KP_ENTRIES - 1) / sana::tc::KP_ENTRIES);
+        return launch(sana::tc::kr_prefix_tc<D>, kp_grid, dim3(sana::tc::KP_ENTRIES * sana::tc::KP_LANES), 0, s,
+                      true, "kr_prefix_tc", (const float*)partial, p.ks, state);
     }
     const dim3 kr_grid((unsigned)((long long)B * H), (D * (D + 1) + sana::tc::KR_THREADS - 1) / sana::tc::KR_THREADS);
     return launch(sana::tc::kr_reduce_tc<D>, kr_grid, dim3(sana::tc::KR_THREADS), 0, s, true, "kr_reduce_tc",

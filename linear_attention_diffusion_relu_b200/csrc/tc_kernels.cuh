@@ -235,7 +235,7 @@ template <int D, int FM>
 __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
                                          int cta, float* __restrict__ partial, uint8_t* smem,
                                          const KsBars& bar, uint32_t tmem, volatile int* abort,
-                                         uint32_t* err)
+                                         uint32_t* err, bool evict_first = false)
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
@@ -263,10 +263,18 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
                 const int y = tile * KS_TILE;
                 uint8_t* st = stage_ptr(s);
                 ptx::mbar_arrive_expect_tx(&bar.full[s], KS_STAGE_BYTES);
-                ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b);
-                ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b);
-                ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b);
-                ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b);
+                if (evict_first) {
+                    const uint64_t pol = ptx::l2_policy_evict_first();
+                    ptx::tma_load_3d_hint(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b, pol);
+                    ptx::tma_load_3d_hint(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b, pol);
+                    ptx::tma_load_3d_hint(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b, pol);
+                    ptx::tma_load_3d_hint(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b, pol);
+                } else {
+                    ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b);
+                    ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b);
+                    ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b);
+                    ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b);
+                }
                 issued = i + 1;
             }
             // drain: every issued load must land before the CTA may exit
@@ -417,53 +425,60 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     }
 }
 
-// Block-causal prefix states: one warp per state entry; lane j takes block
-// j of a 32-block chunk, adds the block's R partials (ascending r), and a warp
-// scan (fixed shuffle pattern) plus the previous chunk's total gives the
-// inclusive prefix over blocks. Deterministic: the same additions in the same
-// order on every run.
-constexpr int KP_WARPS = 4;
+// Block-causal prefix states. A CTA takes 32 consecutive state entries (so
+// every load instruction reads 128 contiguous bytes) times 8 block lanes:
+// lane jl sums the R partials (ascending r) of blocks jl, jl+8, ... of a
+// 64-block chunk into shared memory, then one thread per entry walks the
+// chunk in block order: prefix_j = prefix_{j-1} + blocksum_j. The same
+// additions in the same order on every run.
+constexpr int KP_ENTRIES = 32;
+constexpr int KP_LANES = 8;
+constexpr int KP_CHUNK = 64;
 
 template <int D>
-__global__ void __launch_bounds__(KP_WARPS * 32)
+__global__ void __launch_bounds__(KP_ENTRIES * KP_LANES)
 kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restrict__ states)
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
+    __shared__ float bsum[KP_CHUNK][KP_ENTRIES];
     ptx::launch_dependents();
     ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
-    const int lane = threadIdx.x & 31;
-    const int e = blockIdx.y * KP_WARPS + (threadIdx.x >> 5);
-    if (e >= DD) return;                         // whole warps leave together
+    const int el = threadIdx.x % KP_ENTRIES;
+    const int jl = threadIdx.x / KP_ENTRIES;
+    const int e = blockIdx.y * KP_ENTRIES + el;
+    const bool live = e < DD;
     const long long bh = blockIdx.x;
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
     const int slab = b * p.groups + h / G;
     const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
     float carry = 0.0f;
-    for (int j0 = 0; j0 < p.q.nblk; j0 += 32) {
-        const int j = j0 + lane;
-        float x = 0.0f;
-        if (j < p.q.nblk) {
-            const float* src =
-                partial + ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j, h % G, G, p) * DD + e;
-            for (int r0 = 0; r0 < p.q.R; r0 += 8) {
-                float t[8];
+    for (int j0 = 0; j0 < p.q.nblk; j0 += KP_CHUNK) {
+        for (int jj = jl; jj < KP_CHUNK && j0 + jj < p.q.nblk; jj += KP_LANES) {
+            float x = 0.0f;
+            if (live) {
+                const float* src = partial +
+                    ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j0 + jj, h % G, G, p) * DD + e;
+                for (int r0 = 0; r0 < p.q.R; r0 += 8) {
+                    float t[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
+                    for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (r0 + u < p.q.R) x += t[u];
+                    for (int u = 0; u < 8; ++u)
+                        if (r0 + u < p.q.R) x += t[u];
+                }
+            }
+            bsum[jj][el] = x;
+        }
+        __syncthreads();
+        if (jl == 0 && live) {
+            for (int jj = 0; jj < KP_CHUNK && j0 + jj < p.q.nblk; ++jj) {
+                carry = carry + bsum[jj][el];
+                states[(bh * p.q.nblk + j0 + jj) * DD + e] = carry;
             }
         }
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off) x = y + x;
-        }
-        x = carry + x;
-        if (j < p.q.nblk) states[(bh * p.q.nblk + j) * DD + e] = x;
-        carry = __shfl_sync(0xffffffffu, x, 31);
+        __syncthreads();
     }
 }
 
@@ -642,7 +657,8 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                                          int cta, const KaStateSrc& src, uint8_t* smem,
                                          const KaBars<D, OUT_BF16>& bar, uint32_t tmem,
                                          volatile int* abort, uint32_t* err,
-                                         uint64_t* prev_empty = nullptr, int prev_tiles = 0)
+                                         uint64_t* prev_empty = nullptr, int prev_tiles = 0,
+                                         bool evict_first = false)
 {
     using L = KaLayout<D, OUT_BF16>;
     constexpr int G = L::G;
@@ -676,8 +692,15 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 const int b = slab / p.groups;
                 const int x0 = (slab % p.groups) * 128;
                 ptx::mbar_arrive_expect_tx(&bar.full[s], KA_STAGE_BYTES);
-                ptx::tma_load_3d(stage_ptr(s), tmQ, &bar.full[s], x0, tile * KA_TILE, b);
-                ptx::tma_load_3d(stage_ptr(s) + KA_BOX_BYTES, tmQ, &bar.full[s], x0 + 64, tile * KA_TILE, b);
+                if (evict_first) {
+                    const uint64_t pol = ptx::l2_policy_evict_first();
+                    ptx::tma_load_3d_hint(stage_ptr(s), tmQ, &bar.full[s], x0, tile * KA_TILE, b, pol);
+                    ptx::tma_load_3d_hint(stage_ptr(s) + KA_BOX_BYTES, tmQ, &bar.full[s], x0 + 64,
+                                          tile * KA_TILE, b, pol);
+                } else {
+                    ptx::tma_load_3d(stage_ptr(s), tmQ, &bar.full[s], x0, tile * KA_TILE, b);
+                    ptx::tma_load_3d(stage_ptr(s) + KA_BOX_BYTES, tmQ, &bar.full[s], x0 + 64, tile * KA_TILE, b);
+                }
                 issued = i + 1;
             }
             for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
@@ -1078,7 +1101,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     ptx::tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
-    ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error);
+    // K, V and Q are read once: their lines go first when L2 needs room, which
+    // keeps the output's lines (and the partial states) resident longer
+    ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error,
+                    true);
 
     // Warps 0-3 have written this CTA's partial states (after the last
     // accumulator was complete, i.e. after every state-phase UMMA): make them
@@ -1098,7 +1124,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
-                          kbar.empty, ks_tiles);
+                          kbar.empty, ks_tiles, true);
     kernel_epilogue(ctl, tid);
 }
 
