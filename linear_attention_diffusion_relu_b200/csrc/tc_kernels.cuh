@@ -1066,7 +1066,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
              const KsParams ks, const KaParams ka, float* __restrict__ partial,
-             unsigned long long* flags, const unsigned long long epoch)
+             unsigned long long* flags, const unsigned long long epoch, const int evict_first)
 {
     using Map = FwdMap<D, OUT_BF16>;
     // the apply phase here sums one block's partials; prefix states over token
@@ -1101,10 +1101,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     ptx::tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
-    // K, V and Q are read once: their lines go first when L2 needs room, which
-    // keeps the output's lines (and the partial states) resident longer
+    // with evict_first, K, V and Q (read once) are marked first to go when L2
+    // needs room (the host sets it for problems a few times the size of L2)
     ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error,
-                    true);
+                    evict_first != 0);
 
     // Warps 0-3 have written this CTA's partial states (after the last
     // accumulator was complete, i.e. after every state-phase UMMA): make them
@@ -1124,7 +1124,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
-                          kbar.empty, ks_tiles, true);
+                          kbar.empty, ks_tiles, evict_first != 0);
     kernel_epilogue(ctl, tid);
 }
 
