@@ -136,6 +136,39 @@ class Oracle:
     def forward_fm(self, Q, K, V, feature: str, eps: float, return_den: bool = False):
         return self.apply_fm(Q, self.state_fm(K, V, feature), feature, eps, return_den=return_den)
 
+    # ---------------------------------------------- projection-fused state --
+    # "SANA: Efficient High-Resolution Image Synthesis with Linear Diffusion
+    # Transformers" (phd-frog.tistory.com/40), section 4 "On-Device Deployment":
+    # the ReLU(K)^T V product is fused into the QKV projection, and the key-value
+    # projection stays in full precision. Reading: K = X Wk^T and V = X Wv^T
+    # (no bias), each rounded to bf16 as the projection would store it, then the
+    # state phi(K)^T [V | 1] as above; the fused kernel never writes K or V.
+
+    @staticmethod
+    def round_bf16(x) -> np.ndarray:
+        """Round to the nearest bfloat16 value (8 significant bits, ties to even), as float64."""
+        x = np.asarray(x, dtype=np.float64)
+        m, e = np.frexp(x)                      # x = m * 2**e, 0.5 <= |m| < 1
+        return np.ldexp(np.round(np.ldexp(m, 8)), e - 8)   # np.round: half to even
+
+    def project_kv(self, X, Wk, Wv, H: int):
+        """K, V (B, N, H, d) = bf16(X Wk^T), bf16(X Wv^T) for X (B, N, C) and W (H*d, C)."""
+        X = np.asarray(X, dtype=np.float64)
+        Wk = np.asarray(Wk, dtype=np.float64)
+        Wv = np.asarray(Wv, dtype=np.float64)
+        B, N, C = X.shape
+        HD = Wk.shape[0]
+        if Wk.shape != (HD, C) or Wv.shape != (HD, C) or HD % H:
+            raise ValueError("weights must be (H*d, C) with C matching X")
+        K = self.round_bf16(X @ Wk.T).reshape(B, N, H, HD // H)
+        V = self.round_bf16(X @ Wv.T).reshape(B, N, H, HD // H)
+        return K, V
+
+    def projected_state(self, X, Wk, Wv, H: int) -> np.ndarray:
+        """phi(K)^T [V | 1] with K, V from the key-value projection of X."""
+        K, V = self.project_kv(X, Wk, Wv, H)
+        return self.state(K, V)
+
     def block_causal_state(self, K, V, L: int) -> np.ndarray:
         """Inclusive prefix states of blocks of L tokens: (B, H, nblk, d, d+1)."""
         K = self._f64(K)

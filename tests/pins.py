@@ -418,6 +418,50 @@ def pin_feature_maps_symmetries(orc, seed=33):
     assert np.allclose(S[..., -1], np.where(K > 0, K + 1, np.exp(np.minimum(K, 0))).sum(axis=1), rtol=1e-13)
 
 
+# ------------------------------------------------- projection-fused state --
+# Section 4 "On-Device Deployment" of the SANA walk-through: ReLU(K)^T V fused
+# into the QKV projection.
+
+def pin_round_bf16(orc):
+    """The oracle's bf16 rounding equals torch's float32 -> bfloat16 cast
+    (round to nearest even) on float32 values, including exact ties and values
+    that carry into the next binade."""
+    import torch
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(3.0)
+    ties = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 255.5 / 128.0, -(1.0 + 2.0 ** -8),
+                     1.0 - 2.0 ** -10, 0.0, -0.0], dtype=np.float32)
+    x = np.concatenate([x, ties])
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = orc.round_bf16(x.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def pin_projected_state_integers(orc, seed=42):
+    """Small-integer X and weights: the projections are exact integers; with
+    |values| < 256 they are exact in bf16 too, so the projected state equals the
+    state of the explicitly computed integer K and V (triple loop), bit for bit."""
+    rng = np.random.default_rng(seed)
+    B, N, H, d, C = 2, 9, 3, 4, 5
+    X = rng.integers(-3, 4, size=(B, N, C)).astype(np.float64)
+    Wk = rng.integers(-3, 4, size=(H * d, C)).astype(np.float64)
+    Wv = rng.integers(-3, 4, size=(H * d, C)).astype(np.float64)
+    K = np.zeros((B, N, H * d))
+    V = np.zeros((B, N, H * d))
+    for b in range(B):
+        for n in range(N):
+            for o in range(H * d):
+                K[b, n, o] = sum(X[b, n, c] * Wk[o, c] for c in range(C))
+                V[b, n, o] = sum(X[b, n, c] * Wv[o, c] for c in range(C))
+    S = orc.projected_state(X, Wk, Wv, H)
+    assert np.array_equal(S, orc.state(K.reshape(B, N, H, d), V.reshape(B, N, H, d)))
+    # the rounding step is applied: a projection that is not a bf16 value
+    X2 = np.ones((1, 1, 1))
+    W2 = np.full((1, 1), 1.0 + 2.0 ** -9)      # 1 + 2^-9 rounds to 1 (tie to even)
+    K2, _ = orc.project_kv(X2, W2, W2, 1)
+    assert K2.ravel()[0] == 1.0
+
+
 ALL_PINS = [
     pin_bruteforce_tiny, pin_bruteforce_random, pin_exact_integers, pin_hand_example,
     pin_single_token, pin_equal_keys, pin_one_hot, pin_constant_column,
@@ -425,5 +469,5 @@ ALL_PINS = [
     pin_zero_query, pin_scale_invariance, pin_linearity_in_v, pin_state_definition,
     pin_block_causal_bruteforce, pin_block_causal_exact_integers, pin_block_causal_reductions,
     pin_block_causal_no_future, pin_feature_maps_bruteforce, pin_feature_maps_closed_forms,
-    pin_feature_maps_symmetries,
+    pin_feature_maps_symmetries, pin_round_bf16, pin_projected_state_integers,
 ]
