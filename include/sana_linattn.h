@@ -179,6 +179,35 @@ sana_la_status sana_linattn_forward_fm(const void* Q, const void* K, const void*
                                        sana_la_stream_t stream);
 
 /*
+ * The state built inside the key-value projection ("SANA: Efficient
+ * High-Resolution Image Synthesis with Linear Diffusion Transformers", section 4
+ * "On-Device Deployment": the ReLU(K)^T V product is fused into the QKV
+ * projection, which stays in full precision):
+ *   K = X Wk^T, V = X Wv^T   (bf16 inputs, fp32 accumulation on the tensor cores,
+ *                            then rounded to bf16 as a stored K and V would be)
+ *   state = phi(K)^T [V | 1] per (b, h), as sana_linattn_kv_state would give
+ *                            for those K and V (up to the summation order)
+ * K and V are never written to memory. No bias. phi = ReLU.
+ *   X         bf16 (B, N, C) row-major (token-major activations), device.
+ *   Wk, Wv    bf16 (H*d, C) row-major (the layout of a linear layer's weight:
+ *             output feature h*d + i is row h*d + i), device.
+ *   state     fp32 (B, H, d, d+1), device, written in full.
+ *   workspace at least sana_linattn_kv_projection_workspace_bytes(...) bytes.
+ * C must be a multiple of 8 (SANA_LA_ERR_UNSUPPORTED otherwise). The queries
+ * are a plain projection (Q = X Wq^T, any GEMM); sana_linattn_apply then gives O.
+ */
+size_t sana_linattn_kv_projection_workspace_bytes(int B, int N, int C, int H, int d);
+
+sana_la_status sana_linattn_kv_projection_state(const void* X, const void* Wk, const void* Wv,
+                                                int B, int N, int C, int H, int d,
+                                                float* state,
+                                                void* workspace, size_t workspace_bytes,
+                                                sana_la_stream_t stream);
+
+/* Kernel launches one sana_linattn_kv_projection_state call enqueues (0 if invalid). */
+int sana_linattn_kv_projection_state_launches(int B, int N, int C, int H, int d);
+
+/*
  * Block-causal form ("linear-diffusion-transformer-4k-efficient-generation",
  * section "技术演进：从图像到视频与世界模型": SANA-Video's block causal linear
  * attention; the pages give no formula). The tokens form blocks of L

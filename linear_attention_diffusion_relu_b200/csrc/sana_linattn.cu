@@ -16,6 +16,7 @@
 #include "../../include/sana_linattn.h"
 #include "common.cuh"
 #include "tc_kernels.cuh"
+#include "kvproj_kernel.cuh"
 
 namespace {
 
@@ -449,6 +450,64 @@ bool valid_feature(int fm) {
     return fm == sana::kFeatureRelu || fm == sana::kFeatureElu1 || fm == sana::kFeatureCos;
 }
 
+// ------------------------------------------- key-value projection + state ----
+struct KpPlan {
+    sana::tc::KpParams kp;
+    size_t partial_bytes;
+};
+
+KpPlan make_kp_plan(int B, int N, int C, int H, int d) {
+    const int G = 128 / d;
+    const long long groups = cdiv(H, G);
+    KpPlan p{};
+    p.kp.N = N;
+    p.kp.H = H;
+    p.kp.groups = (int)groups;
+    p.kp.C = C;
+    p.kp.kblocks = (int)cdiv(C, 64);
+    p.kp.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KP_TILE));
+    const size_t dd = (size_t)d * (d + 1) * sizeof(float);
+    p.partial_bytes = align256((size_t)p.kp.q.grid * p.kp.q.max_seg * G * dd);
+    return p;
+}
+
+sana_la_status check_projection(int B, int N, int C, int H, int d) {
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    if (C < 1) return SANA_LA_ERR_INVALID_ARG;
+    if (C % 8 != 0) return SANA_LA_ERR_UNSUPPORTED;          // TMA row strides are multiples of 16 bytes
+    if ((long long)B * N > kMaxElems / C) return SANA_LA_ERR_INVALID_ARG;
+    if ((long long)N * C * 2 >= (1LL << 40) || (long long)H * d * C * 2 >= (1LL << 40))
+        return SANA_LA_ERR_UNSUPPORTED;
+    return SANA_LA_OK;
+}
+
+template <int D>
+sana_la_status run_kvproj_state(const void* X, const void* Wk, const void* Wv, int B, int N, int C, int H,
+                                const KpPlan& p, float* partial, float* state, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmX, tmWk, tmWv;
+    sana_la_status st;
+    // X as {C, N, B}; the weights as {C, H*d, 1}: 64 features x 128 rows per box
+    if ((st = make_tmap(&tmX, X, B, N, 1, C, sana::tc::KP_TILE)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmWk, Wk, 1, H * D, 1, C, 128)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmWv, Wv, 1, H * D, 1, C, 128)) != SANA_LA_OK) return st;
+    if ((st = ensure_smem(sana::tc::kvproj_state_tc<D>, sana::tc::KpMap::BYTES, smem_set)) != SANA_LA_OK)
+        return st;
+    if ((st = launch(sana::tc::kvproj_state_tc<D>, dim3(p.kp.q.grid), dim3(sana::tc::kThreads),
+                     sana::tc::KpMap::BYTES, s, false, "kvproj_state_tc", tmX, tmWk, tmWv, p.kp,
+                     partial)) != SANA_LA_OK)
+        return st;
+    sana::tc::KsParams ksp{};
+    ksp.N = N;
+    ksp.H = H;
+    ksp.groups = p.kp.groups;
+    ksp.q = p.kp.q;
+    const dim3 kr_grid((unsigned)((long long)B * H), (D * (D + 1) + sana::tc::KR_THREADS - 1) / sana::tc::KR_THREADS);
+    return launch(sana::tc::kr_reduce_tc<D>, kr_grid, dim3(sana::tc::KR_THREADS), 0, s, true, "kr_reduce_tc",
+                  (const float*)partial, ksp, state);
+}
+
 sana_la_status kv_state_entry(const void* K, const void* V, int B, int N, int H, int d, int fm,
                               float* state, void* workspace, size_t workspace_bytes,
                               sana_la_stream_t stream) {
@@ -565,6 +624,34 @@ sana_la_status sana_linattn_forward_fm(const void* Q, const void* K, const void*
                                        sana_la_stream_t stream) {
     return forward_entry(Q, K, V, B, N, H, d, (int)feature_map, O, out_dtype, eps, workspace,
                          workspace_bytes, stream);
+}
+
+// ------------------------------------------- key-value projection + state ----
+size_t sana_linattn_kv_projection_workspace_bytes(int B, int N, int C, int H, int d) {
+    if (check_projection(B, N, C, H, d) != SANA_LA_OK) return 0;
+    return make_kp_plan(B, N, C, H, d).partial_bytes;
+}
+
+sana_la_status sana_linattn_kv_projection_state(const void* X, const void* Wk, const void* Wv,
+                                                int B, int N, int C, int H, int d, float* state,
+                                                void* workspace, size_t workspace_bytes,
+                                                sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!X || !Wk || !Wv || !state || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_projection(B, N, C, H, d);
+    if (st != SANA_LA_OK) return st;
+    if (!aligned16(X) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(state) || !aligned16(workspace))
+        return SANA_LA_ERR_INVALID_ARG;
+    const KpPlan p = make_kp_plan(B, N, C, H, d);
+    if (workspace_bytes < p.partial_bytes) return SANA_LA_ERR_WORKSPACE;
+    float* partial = static_cast<float*>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return d == 32 ? run_kvproj_state<32>(X, Wk, Wv, B, N, C, H, p, partial, state, s)
+                   : run_kvproj_state<64>(X, Wk, Wv, B, N, C, H, p, partial, state, s);
+}
+
+int sana_linattn_kv_projection_state_launches(int B, int N, int C, int H, int d) {
+    return check_projection(B, N, C, H, d) == SANA_LA_OK ? 2 : 0;   // kvproj_state_tc, kr_reduce_tc
 }
 
 // ------------------------------------------------------- block-causal ----

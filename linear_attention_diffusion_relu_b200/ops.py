@@ -14,6 +14,10 @@ The functions mirror the C ABI in ``include/sana_linattn.h``:
 
 each with ``feature_map="relu" | "elu1" | "cos"`` (the ``*_fm`` entry points),
 
+the state built inside the key-value projection (K and V never stored):
+
+    kv_projection_state(X, Wk, Wv, H, state=None, workspace=None) -> (B, H, d, d+1) fp32
+
 and the block-causal form (blocks of L tokens, L a multiple of 128):
 
     block_causal_workspace_bytes(B, N, H, d, L)
@@ -45,6 +49,9 @@ SYMBOLS = (
     "sana_linattn_kv_state_fm",
     "sana_linattn_apply_fm",
     "sana_linattn_forward_fm",
+    "sana_linattn_kv_projection_workspace_bytes",
+    "sana_linattn_kv_projection_state",
+    "sana_linattn_kv_projection_state_launches",
     "sana_linattn_block_causal_workspace_bytes",
     "sana_linattn_block_causal_kv_state",
     "sana_linattn_block_causal_apply",
@@ -103,6 +110,12 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_apply_fm.restype = st
         lib.sana_linattn_forward_fm.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
         lib.sana_linattn_forward_fm.restype = st
+        lib.sana_linattn_kv_projection_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_kv_projection_workspace_bytes.restype = sz
+        lib.sana_linattn_kv_projection_state.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+        lib.sana_linattn_kv_projection_state.restype = st
+        lib.sana_linattn_kv_projection_state_launches.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_kv_projection_state_launches.restype = ctypes.c_int
         lib.sana_linattn_block_causal_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.sana_linattn_block_causal_workspace_bytes.restype = sz
         lib.sana_linattn_block_causal_kv_state.argtypes = [vp, vp, i, i, i, i, i, vp, vp, sz, vp]
@@ -353,3 +366,43 @@ def block_causal_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: i
                                                _stream(Q.device))
     _check(lib, st, "sana_linattn_block_causal_forward")
     return out
+
+
+# ------------------------------------------------ key-value projection + state --
+
+def kv_projection_workspace_bytes(B: int, N: int, C: int, H: int, d: int) -> int:
+    return int(load_library().sana_linattn_kv_projection_workspace_bytes(B, N, C, H, d))
+
+
+def kv_projection_state(X: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor, H: int,
+                        state: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """state = phi(K)^T [V | 1] with K = bf16(X Wk^T), V = bf16(X Wv^T), computed
+    without storing K or V. X bf16 (B, N, C); Wk, Wv bf16 (H*d, C)."""
+    for name, t in (("X", X), ("Wk", Wk), ("Wv", Wv)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous bfloat16")
+    if X.dim() != 3:
+        raise ValueError(f"X must have shape (B, N, C), got {tuple(X.shape)}")
+    B, N, C = X.shape
+    if Wk.dim() != 2 or Wk.shape[1] != C or Wk.shape[0] % H or tuple(Wv.shape) != tuple(Wk.shape):
+        raise ValueError("Wk and Wv must both have shape (H*d, C)")
+    d = Wk.shape[0] // H
+    if state is None:
+        state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=X.device)
+    elif (state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d + 1)
+          or not state.is_contiguous() or state.device != X.device):
+        raise ValueError("state must be contiguous float32 (B, H, d, d+1) on X's device")
+    if workspace is None:
+        n = kv_projection_workspace_bytes(B, N, C, H, d)
+        if n == 0:
+            raise ValueError(f"unsupported sizes B={B} N={N} C={C} H={H} d={d}")
+        workspace = torch.empty(n, dtype=torch.uint8, device=X.device)
+    lib = load_library()
+    st = lib.sana_linattn_kv_projection_state(X.data_ptr(), Wk.data_ptr(), Wv.data_ptr(), B, N, C, H, d,
+                                              state.data_ptr(), workspace.data_ptr(),
+                                              workspace.numel() * workspace.element_size(), _stream(X.device))
+    _check(lib, st, "sana_linattn_kv_projection_state")
+    return state

@@ -161,3 +161,21 @@ def test_feature_map_host_checks(lib):
     x = torch.zeros((1, 8, 1, 32), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="feature_map"):
         ops.forward(x, x, x, feature_map="softmax")
+
+
+def test_kv_projection_host_checks(lib):
+    wsb = lib.sana_linattn_kv_projection_workspace_bytes
+    assert wsb(2, 16384, 2240, 70, 32) > 0
+    assert wsb(2, 16384, 2240, 70, 32) % 256 == 0
+    assert wsb(2, 16384, 2244, 70, 32) == 0     # C not a multiple of 8
+    assert wsb(2, 16384, 0, 70, 32) == 0
+    assert wsb(2, 16384, 2240, 70, 48) == 0     # head size
+    f = lib.sana_linattn_kv_projection_state
+    ws = wsb(1, 300, 128, 4, 32)
+    assert f(None, FAKE, FAKE, 1, 300, 128, 4, 32, FAKE, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 300, 124, 4, 32, FAKE, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, 300, 128, 4, 48, FAKE, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE + 8, FAKE, 1, 300, 128, 4, 32, FAKE, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 300, 128, 4, 32, FAKE, FAKE, ws - 1, None) == ops.ERR_WORKSPACE
+    assert lib.sana_linattn_kv_projection_state_launches(1, 300, 128, 4, 32) == 2
+    assert lib.sana_linattn_kv_projection_state_launches(1, 300, 124, 4, 32) == 0
