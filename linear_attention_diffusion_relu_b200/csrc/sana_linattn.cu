@@ -29,7 +29,6 @@ void set_last_error(const char* where, cudaError_t e) {
 
 constexpr int kSMs = 148;             // B200: one persistent CTA per SM
 constexpr int kMaxDevicesCached = 64; // per-device caches of launch properties
-constexpr long long kEvictFirstMaxBytes = 2LL << 30;   // inputs per forward (see launch_forward_fused)
 constexpr long long kMaxElems = 1LL << 62;
 constexpr long long kMaxGrid = 0x7fffffffLL;
 
@@ -391,11 +390,10 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // Evict-first L2 policy on the input loads: measured faster back to back at
-    // 0.6 GB per step (112 vs 120 us at 4096px) and slower at 9.7 GB (1641 vs
-    // 1556 us at N = 1,048,576), so it is used below kEvictFirstMaxBytes.
-    const long long in_bytes = 3LL * B * N * H * D * 2;
-    const int evict_first = in_bytes <= kEvictFirstMaxBytes ? 1 : 0;
+    // Evict-first L2 policy on the input loads. Measured back to back on B200
+    // (same process, A/B): 111.9 vs 119.3 us at 4096px (0.44 GB of inputs),
+    // 400.7 vs 404.3 us at N = 262,144 and 1598 vs 1608 us at N = 1,048,576.
+    const int evict_first = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch, evict_first);
     if (e != cudaSuccess) {
         set_last_error("fwd_fused_tc", e);

@@ -1102,7 +1102,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const uint32_t tmem = ctl->tmem_base;
 
     // with evict_first, K, V and Q (read once) are marked first to go when L2
-    // needs room (the host sets it for problems a few times the size of L2)
+    // needs room
     ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error,
                     evict_first != 0);
 
