@@ -35,6 +35,7 @@ METRIC = "ReLU linear-attn GB/s (% of B200 HBM peak) and Mtokens/s at 4096px sha
 UNIT = "GB/s"
 WORKLOAD = "4096px"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
 # the same build (profiles/), keyed by (kernel set, workload, kernel); None when
 # the kernels changed since the counters were taken
@@ -54,6 +55,9 @@ def parse_args(argv=None):
                    help="timed steps (about 1 s at 4096px, long enough to sample clocks)")
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--op", choices=["forward", "kvproj"], default="forward",
+                   help="kvproj: the key-value projection with the state in its epilogue (one GPU), "
+                        "against a cuBLAS projection followed by kv_state")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -447,10 +451,90 @@ def run_e2e(args, w, dev, stream, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
 
 
+def run_kvproj(args):
+    """The key-value projection with the state in its epilogue at a Sana
+    shape (X (B, N, C) with C = H*d), timed per call with CUDA events, next to
+    the unfused pipeline it replaces: K and V from torch's bf16 matmul (cuBLAS,
+    stored), then kv_state. Metric: TFLOP/s of the projection GEMM (the state
+    product adds < 1 %), roofline against the measured cuBLAS bf16 peak."""
+    import torch
+    from linear_attention_diffusion_relu_b200 import ops
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS
+    if args.gpus != 1:
+        raise SystemExit("--op kvproj runs on one GPU")
+    w = WORKLOADS[args.workload]
+    B, N, H, d = w.B, w.N, w.H, w.d
+    C = H * d
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device="cuda").manual_seed(w.seed)
+    X = torch.randn((B, N, C), generator=g, device=dev).to(torch.bfloat16)
+    Wk = (torch.randn((H * d, C), generator=g, device=dev) / C ** 0.5).to(torch.bfloat16)
+    Wv = (torch.randn((H * d, C), generator=g, device=dev) / C ** 0.5).to(torch.bfloat16)
+    state = torch.empty((B, H, d, d + 1), dtype=torch.float32, device=dev)
+    ws = torch.empty(ops.kv_projection_workspace_bytes(B, N, C, H, d), dtype=torch.uint8, device=dev)
+    K = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    ws2 = ops.make_workspace(B, N, H, d, dev)
+
+    def fused():
+        ops.kv_projection_state(X, Wk, Wv, H, state=state, workspace=ws)
+
+    def unfused():
+        torch.matmul(X, Wk.T, out=K.view(B, N, H * d))
+        torch.matmul(X, Wv.T, out=V.view(B, N, H * d))
+        ops.kv_state(K, V, state=state, workspace=ws2)
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    steps = max(1, min(args.steps, 200))
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = timed(fused, steps)
+    clk = clocks.stop()
+    ms_unfused = timed(unfused, steps)
+    flops = 2.0 * B * N * C * (2 * H * d)
+    tflops = flops / (ms / 1e3) / 1e12
+    peak = FALLBACK_BF16_TFLOPS
+    src = "fallback"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        pass
+    line = {
+        "metric": "key-value projection with the state in its epilogue, TFLOP/s", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} key-value projection", "B": B, "N": N, "C": C, "H": H, "d": d},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "kernel": "kvproj_state_tc",
+                     "peak_source": f"{src} cuBLAS bf16 (burst)"},
+        "unfused": {"ms_per_step": ms_unfused, "what": "torch bf16 matmul for K and V (stored) + kv_state",
+                    "tflops": flops / (ms_unfused / 1e3) / 1e12},
+        "clocks": clk,
+        "gpu_launches": ops.load_library().sana_linattn_kv_projection_state_launches(B, N, C, H, d) * steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "kvproj":
+        return run_kvproj(args)
     return run_ours(args)
 
 
