@@ -3,11 +3,13 @@ ReLU(K)^T V product fused into the QKV projection: SANA walk-through, section 4
 "On-Device Deployment") with the oracle, through the C ABI.
 
 The oracle projects in fp64 and rounds K and V to bf16; the kernel accumulates
-the projection in fp32 before the same rounding, so a small fraction of K and
-V elements can land one bf16 step apart. State entries are therefore held to
-1e-4 of the sum of |terms| they add up (an O(1) error from a wrong layout,
-head, token or feature fails by orders of magnitude). End to end, apply() on
-that state meets the output tolerance of the forward."""
+the projection in fp32 before the same rounding, so a small fraction (~1e-4 to
+1e-3, growing with C) of K and V elements land one bf16 step (at most 2^-7
+relative) apart. A state entry sum_n t_n, t_n = phi(K_ni) [V | 1]_nj, is
+therefore held to 1e-4 of sum_n |t_n| plus four such steps of its largest term
+(an O(1) error from a wrong layout, head, token or feature fails by orders of
+magnitude). End to end, apply() on that state is held to 1e-3 per row (fp32)
+and to the forward's bf16 output tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -36,13 +38,31 @@ def _inputs(B, N, C, H, d, seed):
     return X.cuda(), Wk.cuda(), Wv.cuda()
 
 
-def _check_state(oracle, S, X, Wk, Wv, H, tol=1e-4):
+def _max_term(K, V):
+    """max_n |phi(K_ni)| |[V | 1]_nj| per state entry (B, H, d, d+1)."""
+    B, N, H, d = K.shape
+    out = np.zeros((B, H, d, d + 1))
+    pk = np.maximum(K, 0.0)
+    v1 = np.concatenate([np.abs(V), np.ones((B, N, H, 1))], axis=-1)
+    for b in range(B):
+        for h in range(H):
+            for n0 in range(0, N, 512):
+                t = pk[b, n0:n0 + 512, h, :, None] * v1[b, n0:n0 + 512, h, None, :]
+                out[b, h] = np.maximum(out[b, h], t.max(axis=0))
+    return out
+
+
+def _bound(K, V, mag):
+    return 1e-4 * mag + 4 * 2.0 ** -7 * _max_term(K, V) + 1e-30
+
+
+def _check_state(oracle, S, X, Wk, Wv, H):
     K, V = oracle.project_kv(to_f64(X), to_f64(Wk), to_f64(Wv), H)
     ref = oracle.state(K, V)
     mag = oracle.state(K, np.abs(V))
     err = np.abs(to_f64(S) - ref)
-    worst = (err / (mag + 1e-30)).max()
-    assert np.all(err <= tol * mag + 1e-30), worst
+    bound = _bound(K, V, mag)
+    assert np.all(err <= bound), (err / bound).max()
     return K, V
 
 
@@ -69,11 +89,16 @@ def test_projected_state_end_to_end_and_deterministic(oracle):
     Q = torch.randn((B, N, H, d), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).cuda()
     S1 = ops.kv_projection_state(X, Wk, Wv, H)
     S2 = ops.kv_projection_state(X, Wk, Wv, H)
-    O = ops.apply(Q, S1, out_dtype=torch.float32)
+    O32 = ops.apply(Q, S1, out_dtype=torch.float32)
+    O16 = ops.apply(Q, S1, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert torch.equal(S1.view(torch.int32), S2.view(torch.int32))
     K, V = oracle.project_kv(to_f64(X), to_f64(Wk), to_f64(Wv), H)
-    check_output(O, oracle.forward(to_f64(Q), K, V, 1e-15), "projected state, end to end")
+    ref = oracle.forward(to_f64(Q), K, V, 1e-15)
+    check_output(O16, ref, "projected state, end to end (bf16 out)")
+    got = to_f64(O32)
+    rel = np.linalg.norm(got - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
+    assert rel.max() <= 1e-3, rel.max()
 
 
 def test_projected_state_agrees_with_unfused_path():
@@ -88,5 +113,6 @@ def test_projected_state_agrees_with_unfused_path():
     S_ref = ops.kv_state(K, V)
     mag = ops.kv_state(K, V.abs())
     torch.cuda.synchronize()
-    err = (S - S_ref).abs()
-    assert bool(torch.all(err <= 1e-4 * mag + 1e-30)), float((err / (mag + 1e-30)).max())
+    err = to_f64(S - S_ref)
+    bound = _bound(to_f64(K), to_f64(V), to_f64(mag))
+    assert np.all(np.abs(err) <= bound), (np.abs(err) / bound).max()
