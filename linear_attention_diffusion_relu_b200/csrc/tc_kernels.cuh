@@ -2,8 +2,14 @@
 //
 // KS  ks_state_tc   partial states  phi(K)^T [V | 1]  on UMMA, fp32 in TMEM
 // KR  kr_reduce_tc  fixed-order sum of the partials of each (b, h)
+//     kr_prefix_tc  block-causal: fixed-order prefix sums over token blocks
 // KA  ka_apply_tc   phi(Q) S on UMMA (S split into bf16 hi + lo), then
 //                   O = num / (den + eps) in the epilogue, stored by TMA
+// KF  fwd_fused_tc  KS, a grid-wide barrier and KA in one cooperative launch
+//
+// The feature map phi is a template parameter (ReLU, ELU+1, cos; the latter
+// two carried as bf16 hi + lo pairs); the block-causal form is a runtime
+// property of the schedule (see below).
 //
 // The two contractions ("08_sana高效高分辨率生成", "Linear Attention 的原理":
 // KV = phi(K)^T V, A = phi(Q) KV; the normaliser of the normalised form in
