@@ -5,7 +5,7 @@
 //     kr_prefix_tc  block-causal: fixed-order prefix sums over token blocks
 // KA  ka_apply_tc   phi(Q) S on UMMA (S split into bf16 hi + lo), then
 //                   O = num / (den + eps) in the epilogue, stored by TMA
-// KF  fwd_fused_tc  KS, a grid-wide barrier and KA in one cooperative launch
+// KF  fwd_fused_tc  KS, per-slab readiness flags and KA in one cooperative launch
 //
 // The feature map phi is a template parameter (ReLU, ELU+1, cos; the latter
 // two carried as bf16 hi + lo pairs); the block-causal form is a runtime
@@ -166,7 +166,10 @@ __host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
     return (q.S - c % q.S + q.grid - 1) / q.grid * q.nblk;
 }
 // i-th tile of CTA c -> (slab, tile, segment index); the segment's block is
-// seg % q.nblk
+// seg % q.nblk. In round k the R CTAs of a slab take tiles kR .. kR + R - 1,
+// CTA r always position r. (Rotating the positions from round to round made
+// every CTA finish the state phase together, but all of them at the time the
+// last position finished before: slower overall, measured on B200.)
 __host__ __device__ __forceinline__ void sched_item(int c, int i, int tps, const Sched& q,
                                                     int& slab, int& tile, int& seg) {
     seg = i / tps;
@@ -557,7 +560,7 @@ struct KaBars {
     uint64_t* stg_free;    // [2 halves] this half's staging boxes may be written
     uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
     uint64_t* mma_done;
-    uint64_t* grid_ready;  // (single launch) every CTA's partial states are in memory
+    uint64_t* grid_ready;  // (single launch) the staged slab's partial states are in memory
     uint64_t* p1_written;  // (single launch) this CTA's partial states are written
     __device__ void init() const {
         for (int s = 0; s < L::STAGES; ++s) {
@@ -605,39 +608,40 @@ __device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid) {
 // Where the apply phase gets the state of a slab from:
 //   state != nullptr   the reduced fp32 state (B, H, d, d+1) of the reduction kernel
 //   otherwise          the partial states of the state phase (same launch), summed
-//                      here in the reduction kernel's order, once every CTA's
-//                      arrival flag holds this launch's epoch
+//                      here in the reduction kernel's order, once the arrival
+//                      flags of the CTAs that wrote them hold this launch's epoch
 struct KaStateSrc {
     const float* state;
     const float* partial;
     KsParams ks;
     const unsigned long long* flags;   // one arrival flag per CTA of the grid
     unsigned long long epoch;          // unique to this launch (set by the host)
-    int nflags;
 };
 
-// Grid-wide barrier of the single-launch forward. CTA c announces that its
+// Readiness flags of the single-launch forward. CTA c announces that all its
 // partial states are in memory by storing the launch's epoch into flags[c]
-// (after a fence); the barrier is passed when every flag holds the epoch.
-// The host draws a new 64-bit epoch for every launch, so flags left by earlier
-// launches (or any other bytes) never pass for this one and the flag array
-// needs no reset between launches.
+// (after a fence). Before staging a slab's state, a CTA waits only for the
+// flags of the CTAs that wrote that slab's partials (its R siblings), not for
+// the whole grid. The host draws a new 64-bit epoch for every launch, so flags
+// left by earlier launches (or any other bytes) never pass for this one and
+// the flag array needs no reset between launches.
 __device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned long long epoch) {
     __threadfence();
     asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
 }
 
-// Bounded spin of one whole warp until every flag holds `epoch` (warp-uniform
-// result). On a timeout it records the error code and sets *abort.
-__device__ __forceinline__ bool grid_wait(const unsigned long long* flags, int nflags,
-                                          unsigned long long epoch, volatile int* abort, uint32_t* err) {
+// Bounded spin of one whole warp until flags[first + r * stride] hold `epoch`
+// for r < count (warp-uniform result). On a timeout it records the error code
+// and sets *abort.
+__device__ __forceinline__ bool flags_wait(const unsigned long long* flags, int first, int stride, int count,
+                                           unsigned long long epoch, volatile int* abort, uint32_t* err) {
     const int lane = threadIdx.x & 31;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (;;) {
         bool mine = true;
-        for (int c = lane; c < nflags; c += 32) {
+        for (int r = lane; r < count; r += 32) {
             unsigned long long v;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + c) : "memory");
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + first + r * stride) : "memory");
             mine = mine && v == epoch;
         }
         if (__all_sync(0xffffffffu, mine)) return true;
@@ -768,16 +772,18 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         if (src.state != nullptr) ptx::wait_prerequisite_grid();
 
         // stage the state of `slab` in shared memory as bf16 hi + lo parts
-        bool grid_synced = false;
+        int nsync = 0;      // slabs staged from partial states so far
         auto stage_state = [&](int slab, int blk) -> bool {
-            if (src.state == nullptr && !grid_synced) {
-                // the partial states of every CTA must be in memory (once)
+            if (src.state == nullptr) {
+                // the CTAs that wrote this slab's partials (slab % grid + r S,
+                // r < R) must be done; warp 0 waits and tells the others
                 if (warp == 0) {
-                    if (grid_wait(src.flags, src.nflags, src.epoch, abort, err) && lane == 0)
+                    if (flags_wait(src.flags, slab % src.ks.q.grid, src.ks.q.S, src.ks.q.R, src.epoch, abort, err)
+                        && lane == 0)
                         ptx::mbar_arrive(bar.grid_ready);
                 }
-                if (!warp_wait(bar.grid_ready, 0, abort, err)) return false;
-                grid_synced = true;
+                if (!warp_wait(bar.grid_ready, nsync & 1, abort, err)) return false;
+                ++nsync;
             }
             const int b = slab / p.groups;
             const int g = slab % p.groups;
@@ -1055,18 +1061,19 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, 0};
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull};
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
                           &g_device_error);
     kernel_epilogue(ctl, tid);
 }
 
-// The whole forward in one cooperative launch: the state phase, a grid-wide
-// barrier (bounded), then the apply phase, which sums each slab's partial
-// states itself in the reduction kernel's order. The apply phase's Q loads
-// start as soon as the state phase has released its shared memory, so they
-// overlap the barrier. `flags` has one slot per CTA; `epoch` is unique to the
-// launch.
+// The whole forward in one cooperative launch (all CTAs resident, so a CTA
+// may wait for another): the state phase; a readiness flag per CTA; then the
+// apply phase, which waits (bounded) for the flags of the CTAs that wrote its
+// slab's partial states and sums them itself in the reduction kernel's order.
+// The apply phase's Q loads start as soon as the state phase has released its
+// shared memory, so they overlap that wait. `flags` has one slot per CTA;
+// `epoch` is unique to the launch.
 template <int D, bool OUT_BF16, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -1122,11 +1129,11 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     }
     if (warp < kWorkerWarps) {
         warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
-        // every CTA arrives at the grid barrier, with or without apply work
+        // every CTA raises its readiness flag, with or without apply work
         if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
         ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     }
-    KaStateSrc src{nullptr, partial, ks, flags, epoch, (int)gridDim.x};
+    KaStateSrc src{nullptr, partial, ks, flags, epoch};
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
