@@ -15,10 +15,12 @@
 //   producer  TMA: per 64-feature k-block, the X tile (128 tokens) and the
 //             group's 128 rows of Wk and of Wv (K-major, 128-byte swizzle)
 //   UMMA      GEMM D[128 x 256] = X [Wk_g; Wv_g]^T into TMEM columns 0-255
-//   workers   D -> registers, bf16(K) -> phi, bf16(V), into two staging tiles
-//             laid out like the state kernel's TMA tiles (tokens as rows)
-//   UMMA      state += phi(K)^T V and phi(K)^T 1 (TMEM columns 256-399),
-//             issued while the next unit's GEMM runs
+//   workers   D -> registers, bf16(K) -> phi, bf16(V), into staging tiles
+//             laid out like the state kernel's TMA tiles (tokens as rows), one
+//             64-token half after the other through the same 32 KB (so the
+//             GEMM keeps 4 pipeline stages)
+//   UMMA      state += phi(K)^T V and phi(K)^T 1 (TMEM columns 256-399) per
+//             half, issued between the next unit's k-blocks
 // At the end of a segment warps 0-3 write the partial states.
 #pragma once
 
@@ -37,20 +39,29 @@ struct KpParams {
 constexpr int KP_TILE = 128;                                // tokens per unit = GEMM M
 constexpr int KP_BOX_BYTES = 128 * kBoxBytesRow;            // 128 rows x 128 bytes = 16 KB
 constexpr int KP_STAGE_BYTES = 3 * KP_BOX_BYTES;            // X, Wk rows, Wv rows
-constexpr int KP_STAGES = 3;
-constexpr int KP_STG_OFF = KP_STAGES * KP_STAGE_BYTES;      // staging: phi(K) 0/1, V 0/1
-constexpr int KP_ONES_OFF = KP_STG_OFF + 4 * KP_BOX_BYTES;
+constexpr int KP_STAGES = 4;
+constexpr int KP_HALF = KP_TILE / 2;                        // tokens per staging half
+constexpr int KP_HBOX_BYTES = KP_HALF * kBoxBytesRow;       // 64 token rows x 128 bytes = 8 KB
+constexpr int KP_STG_OFF = KP_STAGES * KP_STAGE_BYTES;      // staging: phi(K) boxes 0/1, V boxes 0/1
+constexpr int KP_ONES_OFF = KP_STG_OFF + 4 * KP_HBOX_BYTES;
 constexpr int KP_DATA_BYTES = KP_ONES_OFF + 1024;
 constexpr uint32_t KP_STATE_COL = 256;                      // state accumulator columns 256-399
-using KpMap = SmemMap<KP_DATA_BYTES>;
+// shared memory: data, 256 bytes of barriers, the control block, 1 KB of
+// alignment slack (tighter than SmemMap to fit 4 stages)
+struct KpMap {
+    static constexpr int BAR_OFF = KP_DATA_BYTES;
+    static constexpr int CTL_OFF = BAR_OFF + 256;
+    static constexpr int BYTES = CTL_OFF + 64 + 1024;
+    static_assert(BYTES <= kSmemLimit, "shared memory");
+};
 
 struct KpBars {
     uint64_t* full;        // [KP_STAGES] X and weight boxes landed
     uint64_t* empty;       // [KP_STAGES] read by the GEMM UMMAs
     uint64_t* acc_full;    // a unit's GEMM accumulator complete
     uint64_t* acc_empty;   // GEMM accumulator read by every worker warp
-    uint64_t* staged;      // phi(K) and V of a unit written by every worker warp
-    uint64_t* stg_free;    // the state UMMAs of a unit have read the staging tiles
+    uint64_t* staged;      // [2 halves] a half's phi(K) and V written by its 4 warps
+    uint64_t* stg_free;    // [2 halves] the state UMMAs of a half have read the staging
     uint64_t* state_full;  // a segment's state accumulator complete
     uint64_t* state_empty; // state accumulator read by warps 0-3
     uint64_t* mma_done;
@@ -61,8 +72,10 @@ struct KpBars {
         }
         ptx::mbar_init(acc_full, 1);
         ptx::mbar_init(acc_empty, kWorkerWarps);
-        ptx::mbar_init(staged, kWorkerWarps);
-        ptx::mbar_init(stg_free, 1);
+        for (int h = 0; h < 2; ++h) {
+            ptx::mbar_init(&staged[h], kWorkerWarps / 2);
+            ptx::mbar_init(&stg_free[h], 1);
+        }
         ptx::mbar_init(state_full, 1);
         ptx::mbar_init(state_empty, 4);
         ptx::mbar_init(mma_done, 1);
@@ -71,7 +84,7 @@ struct KpBars {
 
 __device__ __forceinline__ KpBars kp_bars(uint64_t* b) {
     uint64_t* a = b + 2 * KP_STAGES;
-    return KpBars{b, b + KP_STAGES, a, a + 1, a + 2, a + 3, a + 4, a + 5, a + 6};
+    return KpBars{b, b + KP_STAGES, a, a + 1, a + 2, a + 4, a + 6, a + 7, a + 8};
 }
 
 template <int D>
@@ -153,31 +166,32 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             const uint64_t ones_desc =
                 ptx::smem_desc(ptx::smem_u32(smem + KP_ONES_OFF), 256, 128, ptx::kLayoutNone);
             const uint32_t kstg = ptx::smem_u32(stg);
-            const uint32_t vstg = kstg + 2 * KP_BOX_BYTES;
-            // state UMMAs of unit u: phi(K)^T [V | 1] over its 128 tokens
-            auto issue_state = [&](int u) -> bool {
+            const uint32_t vstg = kstg + 2 * KP_HBOX_BYTES;
+            // state UMMAs of half h of unit u: phi(K)^T [V | 1] over its 64 tokens
+            auto issue_state = [&](int u, int h) -> bool {
                 const int seg = u / tps;
-                const bool first = (u % tps) == 0;
+                const bool first = (u % tps) == 0 && h == 0;
                 if (first && seg > 0) {
                     // warps 0-3 have read the previous segment's state
                     if (!ptx::mbar_wait(bar.state_empty, (seg & 1) ^ 1, abort, err)) return false;
                 }
                 ptx::tc_fence_after_sync();
 #pragma unroll
-                for (int ks = 0; ks < KP_TILE / 16; ++ks) {
+                for (int ks = 0; ks < KP_HALF / 16; ++ks) {
                     // 16 tokens = two 8-row groups of 1024 B in the swizzled tiles
-                    const uint64_t a = ptx::smem_desc(kstg + ks * 2048, KP_BOX_BYTES, 1024, ptx::kLayoutSW128);
-                    const uint64_t bv = ptx::smem_desc(vstg + ks * 2048, KP_BOX_BYTES, 1024, ptx::kLayoutSW128);
+                    const uint64_t a = ptx::smem_desc(kstg + ks * 2048, KP_HBOX_BYTES, 1024, ptx::kLayoutSW128);
+                    const uint64_t bv = ptx::smem_desc(vstg + ks * 2048, KP_HBOX_BYTES, 1024, ptx::kLayoutSW128);
                     const bool acc = !(first && ks == 0);
                     ptx::umma_f16_ss(tmem + KP_STATE_COL, a, bv, idesc_v, acc);
                     ptx::umma_f16_ss(tmem + KP_STATE_COL + 128, a, ones_desc, idesc_1, acc);
                 }
-                ptx::umma_commit(bar.stg_free);
-                if ((u % tps) == tps - 1) ptx::umma_commit(bar.state_full);
+                ptx::umma_commit(&bar.stg_free[h]);
+                if (h == 1 && (u % tps) == tps - 1) ptx::umma_commit(bar.state_full);
                 return true;
             };
             int k = 0;
-            int pending = -1;              // unit whose state UMMAs are still to issue
+            int pending = -1;              // unit whose state halves are still to issue
+            int pending_h = 0;             // its next half
             bool ok = true;
             for (int i = 0; i < nunits && ok; ++i) {
                 // the workers have read the previous unit's accumulator
@@ -197,23 +211,30 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         ptx::umma_f16_ss(tmem, a, bw, idesc_gemm, (kb | kk) != 0);
                     }
                     ptx::umma_commit(&bar.empty[s]);
-                    if (pending >= 0 && ptx::mbar_test_wait(bar.staged, pending & 1)) {
-                        if (!issue_state(pending)) { ok = false; break; }
-                        pending = -1;
+                    if (pending >= 0 && ptx::mbar_test_wait(&bar.staged[pending_h], pending & 1)) {
+                        if (!issue_state(pending, pending_h)) { ok = false; break; }
+                        if (++pending_h == 2) { pending = -1; pending_h = 0; }
                     }
                 }
                 if (!ok) break;
                 ptx::umma_commit(bar.acc_full);
-                if (pending >= 0) {
-                    if (!ptx::mbar_wait(bar.staged, pending & 1, abort, err) || !issue_state(pending)) {
+                while (ok && pending >= 0) {
+                    if (!ptx::mbar_wait(&bar.staged[pending_h], pending & 1, abort, err) ||
+                        !issue_state(pending, pending_h)) {
                         ok = false;
                         break;
                     }
+                    if (++pending_h == 2) { pending = -1; pending_h = 0; }
                 }
+                if (!ok) break;
                 pending = i;
+                pending_h = 0;
             }
-            if (ok && pending >= 0) {
-                if (ptx::mbar_wait(bar.staged, pending & 1, abort, err)) issue_state(pending);
+            while (ok && pending >= 0) {
+                if (!ptx::mbar_wait(&bar.staged[pending_h], pending & 1, abort, err) ||
+                    !issue_state(pending, pending_h))
+                    break;
+                if (++pending_h == 2) pending = -1;
             }
             ptx::umma_commit(bar.mma_done);
             ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
@@ -223,7 +244,8 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         // Warp w reads TMEM lanes 32*(w%4).. (its 32 tokens) and half w/4 of the
         // accumulator: columns 0-127 (K) or 128-255 (V).
         const int t = (warp & 3) * 32 + lane;           // token row of the tile
-        const int half = warp >> 2;
+        const int half = warp >> 2;                     // 0: K columns, 1: V columns
+        const int th = (warp & 3) >> 1;                 // token half of this warp
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         for (int i = 0; i < nunits; ++i) {
             if (!warp_wait(bar.acc_full, i & 1, abort, err)) break;
@@ -234,11 +256,16 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             for (int c = 0; c < 4; ++c) ptx::tmem_ld32(lane_base + (uint32_t)(half * 128 + c * 32), v + c * 32);
             ptx::tc_fence_before_sync();
             warp_arrive(bar.acc_empty);
-            // the previous unit's state UMMAs must be done reading the staging
-            if (!warp_wait(bar.stg_free, (i & 1) ^ 1, abort, err)) break;
+            // the staging's previous contents must have been read by the state
+            // UMMAs: the other token half of the previous unit for half 0, half
+            // 0 of this unit for half 1
+            const bool free_ok = th == 0 ? warp_wait(&bar.stg_free[1], (i & 1) ^ 1, abort, err)
+                                         : warp_wait(&bar.stg_free[0], i & 1, abort, err);
+            if (!free_ok) break;
             // bf16 as a stored projection would hold it; phi = ReLU on K (it
             // commutes with the rounding)
-            uint8_t* base = stg + half * 2 * KP_BOX_BYTES + t * kBoxBytesRow;
+            const int row = t & (KP_HALF - 1);
+            uint8_t* base = stg + half * 2 * KP_HBOX_BYTES + row * kBoxBytesRow;
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
                 const float* x = v + q * 8;
@@ -254,11 +281,11 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     w.z = float2_to_bf16x2(x[4], x[5]);
                     w.w = float2_to_bf16x2(x[6], x[7]);
                 }
-                // features 64*(q/8).. in box q/8; 16-byte chunk q%8 of the row at (q%8) ^ (t%8)
-                *reinterpret_cast<uint4*>(base + (q >> 3) * KP_BOX_BYTES + (((q & 7) ^ (t & 7)) * 16)) = w;
+                // features 64*(q/8).. in box q/8; 16-byte chunk q%8 of the row at (q%8) ^ (row%8)
+                *reinterpret_cast<uint4*>(base + (q >> 3) * KP_HBOX_BYTES + (((q & 7) ^ (row & 7)) * 16)) = w;
             }
             ptx::fence_proxy_async_smem();
-            warp_arrive(bar.staged);
+            warp_arrive(&bar.staged[th]);
             if ((i % tps) == tps - 1 && warp < 4) {
                 // end of a segment: the partial states, TMEM -> workspace
                 const int seg = i / tps;
