@@ -169,6 +169,50 @@ class Oracle:
         K, V = self.project_kv(X, Wk, Wv, H)
         return self.state(K, V)
 
+    # ------------------------------------------------------------- Mix-FFN --
+    # "SANA: Efficient High-Resolution Image Synthesis with Linear Diffusion
+    # Transformers" (phd-frog.tistory.com/40), section 2.2 "선형 어텐션 블럭":
+    # Mix-FFN = an inverted residual block (1x1 expand, 3x3 depthwise conv over
+    # the 2-D token grid, 1x1 project) with a GLU; section 4: the GLU is fused
+    # into the Mix-FFN kernel. Readings: tokens n = y * W + x on an (Hg, W)
+    # grid; expand X -> U = X W1^T with 2*Ch channels; depthwise 3x3 with zero
+    # padding; GLU with the original sigmoid gate on the channel halves,
+    # Z = D[:, :Ch] * sigmoid(D[:, Ch:]); project Y = Z W2^T. No biases, no
+    # other activation, no residual inside the block. U and Z are rounded to
+    # bf16 as the stored intermediates of a kernel pipeline would be.
+
+    @staticmethod
+    def depthwise3x3(U, Kdw, hw) -> np.ndarray:
+        """D[b, y, x, c] = sum_{dy, dx in 0..2} U[b, y+dy-1, x+dx-1, c] Kdw[c, dy, dx]
+        (zero outside the grid); U (B, Hg*W, Cc) -> D (B, Hg*W, Cc)."""
+        U = np.asarray(U, dtype=np.float64)
+        Kdw = np.asarray(Kdw, dtype=np.float64)
+        Hg, W = hw
+        B, N, Cc = U.shape
+        if N != Hg * W or Kdw.shape != (Cc, 3, 3):
+            raise ValueError("grid or kernel shape mismatch")
+        G = np.zeros((B, Hg + 2, W + 2, Cc))
+        G[:, 1:-1, 1:-1, :] = U.reshape(B, Hg, W, Cc)
+        D = np.zeros((B, Hg, W, Cc))
+        for dy in range(3):
+            for dx in range(3):
+                D += G[:, dy:dy + Hg, dx:dx + W, :] * Kdw[:, dy, dx]
+        return D.reshape(B, N, Cc)
+
+    def mix_ffn(self, X, W1, Kdw, W2, hw) -> np.ndarray:
+        """Y (B, N, C) for X (B, N, C), W1 (2 Ch, C), Kdw (2 Ch, 3, 3), W2 (C, Ch)."""
+        X = np.asarray(X, dtype=np.float64)
+        W1 = np.asarray(W1, dtype=np.float64)
+        W2 = np.asarray(W2, dtype=np.float64)
+        Ch2 = W1.shape[0]
+        if Ch2 % 2 or W2.shape[1] * 2 != Ch2 or W1.shape[1] != X.shape[2]:
+            raise ValueError("weight shapes do not match")
+        Ch = Ch2 // 2
+        U = self.round_bf16(X @ W1.T)
+        D = self.depthwise3x3(U, Kdw, hw)
+        Z = self.round_bf16(D[..., :Ch] / (1.0 + np.exp(-D[..., Ch:])))
+        return Z @ W2.T
+
     def block_causal_state(self, K, V, L: int) -> np.ndarray:
         """Inclusive prefix states of blocks of L tokens: (B, H, nblk, d, d+1)."""
         K = self._f64(K)

@@ -462,6 +462,96 @@ def pin_projected_state_integers(orc, seed=42):
     assert K2.ravel()[0] == 1.0
 
 
+# ---------------------------------------------------------------- Mix-FFN --
+# SANA walk-through, section 2.2: inverted residual + 3x3 depthwise conv + GLU.
+
+def pin_depthwise_loops(orc, seed=51):
+    """The depthwise 3x3 conv against explicit loops over taps with bounds
+    checks, on a small non-square grid."""
+    rng = np.random.default_rng(seed)
+    B, Hg, W, Cc = 2, 3, 5, 4
+    U = rng.standard_normal((B, Hg * W, Cc))
+    Kd = rng.standard_normal((Cc, 3, 3))
+    D = orc.depthwise3x3(U, Kd, (Hg, W))
+    for b in range(B):
+        for y in range(Hg):
+            for x in range(W):
+                for c in range(Cc):
+                    acc = 0.0
+                    for dy in range(3):
+                        for dx in range(3):
+                            yy, xx = y + dy - 1, x + dx - 1
+                            if 0 <= yy < Hg and 0 <= xx < W:
+                                acc += U[b, yy * W + xx, c] * Kd[c, dy, dx]
+                    assert abs(D[b, y * W + x, c] - acc) <= 1e-12 * (1 + abs(acc))
+
+
+def pin_depthwise_shift_and_identity(orc, seed=52):
+    """A centre-only kernel returns U; a kernel with only the (dy, dx) = (0, 2)
+    tap shifts the grid by (+1 row, -1 column) with zeros entering at the edges."""
+    rng = np.random.default_rng(seed)
+    B, Hg, W, Cc = 1, 4, 3, 2
+    U = rng.standard_normal((B, Hg * W, Cc))
+    ident = np.zeros((Cc, 3, 3)); ident[:, 1, 1] = 1.0
+    assert np.array_equal(orc.depthwise3x3(U, ident, (Hg, W)), U)
+    shift = np.zeros((Cc, 3, 3)); shift[:, 0, 2] = 1.0
+    D = orc.depthwise3x3(U, shift, (Hg, W)).reshape(Hg, W, Cc)
+    G = U.reshape(Hg, W, Cc)
+    for y in range(Hg):
+        for x in range(W):
+            want = G[y - 1, x + 1] if (y >= 1 and x + 1 < W) else np.zeros(Cc)
+            assert np.array_equal(D[y, x], want)
+
+
+def pin_mix_ffn_gate(orc):
+    """With identity-like weights and a centre-only kernel, the block reduces to
+    the GLU: Y = bf16(a * sigmoid(g)) for the channel halves a, g of X. Small
+    integer a and g: g = 0 halves a exactly; g = 40 passes a (sigmoid rounds to 1)."""
+    C = Ch = 2
+    X = np.array([[[3.0, -5.0], [7.0, 1.0], [2.0, 4.0]]])        # B=1, N=3 tokens, C=2
+    W1 = np.zeros((2 * Ch, C)); W1[0, 0] = W1[1, 1] = 1.0          # a = X, g = 0
+    ident = np.zeros((2 * Ch, 3, 3)); ident[:, 1, 1] = 1.0
+    W2 = np.eye(C)
+    Y = orc.mix_ffn(X, W1, ident, W2, (1, 3))
+    assert np.array_equal(Y, X / 2.0)
+    Xg = np.concatenate([X, np.full((1, 3, C), 40.0)], axis=-1)     # C_in = 4: a = X, g = 40
+    W1c = np.zeros((2 * Ch, 4)); W1c[0, 0] = W1c[1, 1] = 1.0; W1c[2, 2] = W1c[3, 3] = 1.0
+    Y2 = orc.mix_ffn(Xg, W1c, ident, W2, (1, 3))
+    assert np.array_equal(Y2, X)
+
+
+def pin_mix_ffn_bruteforce(orc, seed=53):
+    """The whole block against explicit per-token loops (expand, 3x3 taps,
+    sigmoid gate, project) with the same two bf16 roundings."""
+    rng = np.random.default_rng(seed)
+    B, Hg, W, C, Ch = 1, 3, 4, 5, 3
+    X = rng.standard_normal((B, Hg * W, C))
+    W1 = rng.standard_normal((2 * Ch, C)) / np.sqrt(C)
+    Kd = rng.standard_normal((2 * Ch, 3, 3)) / 3.0
+    W2 = rng.standard_normal((C, Ch)) / np.sqrt(Ch)
+    Y = orc.mix_ffn(X, W1, Kd, W2, (Hg, W))
+    rb = orc.round_bf16
+    U = np.zeros((B, Hg * W, 2 * Ch))
+    for n in range(Hg * W):
+        for o in range(2 * Ch):
+            U[0, n, o] = rb(sum(X[0, n, c] * W1[o, c] for c in range(C)))
+    for n in range(Hg * W):
+        y, x = divmod(n, W)
+        z = []
+        for c in range(Ch):
+            da = dg = 0.0
+            for dy in range(3):
+                for dx in range(3):
+                    yy, xx = y + dy - 1, x + dx - 1
+                    if 0 <= yy < Hg and 0 <= xx < W:
+                        da += U[0, yy * W + xx, c] * Kd[c, dy, dx]
+                        dg += U[0, yy * W + xx, Ch + c] * Kd[Ch + c, dy, dx]
+            z.append(rb(da * (1.0 / (1.0 + np.exp(-dg)))))
+        for o in range(C):
+            want = sum(z[c] * W2[o, c] for c in range(Ch))
+            assert abs(Y[0, n, o] - want) <= 1e-12 * (1 + abs(want)), (n, o)
+
+
 ALL_PINS = [
     pin_bruteforce_tiny, pin_bruteforce_random, pin_exact_integers, pin_hand_example,
     pin_single_token, pin_equal_keys, pin_one_hot, pin_constant_column,
@@ -470,4 +560,5 @@ ALL_PINS = [
     pin_block_causal_bruteforce, pin_block_causal_exact_integers, pin_block_causal_reductions,
     pin_block_causal_no_future, pin_feature_maps_bruteforce, pin_feature_maps_closed_forms,
     pin_feature_maps_symmetries, pin_round_bf16, pin_projected_state_integers,
+    pin_depthwise_loops, pin_depthwise_shift_and_identity, pin_mix_ffn_gate, pin_mix_ffn_bruteforce,
 ]
