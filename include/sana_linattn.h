@@ -208,6 +208,37 @@ sana_la_status sana_linattn_kv_projection_state(const void* X, const void* Wk, c
 int sana_linattn_kv_projection_state_launches(int B, int N, int C, int H, int d);
 
 /*
+ * Mix-FFN, the step after the attention in a Sana block ("SANA: Efficient
+ * High-Resolution Image Synthesis with Linear Diffusion Transformers", section
+ * 2.2 "선형 어텐션 블럭": an inverted residual block with a 3x3 depthwise
+ * convolution and a GLU; section 4: the GLU fused into the Mix-FFN kernel):
+ *   U = X W1^T                      1x1 expand to 2*Ch channels (bf16 out)
+ *   D = depthwise3x3(U)             per channel over the Hg x Wg token grid
+ *                                   (token n = y*Wg + x), zero padding
+ *   Z = D[:, :Ch] * sigmoid(D[:, Ch:])   GLU, fused with the convolution (bf16 out)
+ *   Y = Z W2^T                      1x1 project back to C channels (bf16 out)
+ * No biases, no other activation, no residual inside the block.
+ *   X    bf16 (B, Hg*Wg, C) row-major, device.
+ *   W1   bf16 (2*Ch, C) row-major (a linear layer's weight), device.
+ *   Kdw  fp32 (2*Ch, 3, 3): tap (dy, dx) of channel c at c*9 + dy*3 + dx, device.
+ *   W2   bf16 (C, Ch) row-major, device.
+ *   Y    bf16 (B, Hg*Wg, C), device, written in full.
+ *   workspace at least sana_linattn_mix_ffn_workspace_bytes(...) bytes; after
+ *        the call it holds U (B*Hg*Wg x 2*Ch bf16) at offset 0 and Z (B*Hg*Wg x
+ *        Ch bf16) at the next 256-byte boundary.
+ * C and Ch must be multiples of 8 (SANA_LA_ERR_UNSUPPORTED otherwise). Three
+ * launches: tcgen05 GEMM, fused depthwise + GLU, tcgen05 GEMM.
+ */
+size_t sana_linattn_mix_ffn_workspace_bytes(int B, int Hg, int Wg, int C, int Ch);
+
+sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* Kdw, const void* W2,
+                                    int B, int Hg, int Wg, int C, int Ch, void* Y,
+                                    void* workspace, size_t workspace_bytes, sana_la_stream_t stream);
+
+/* Kernel launches one sana_linattn_mix_ffn call enqueues (0 if invalid). */
+int sana_linattn_mix_ffn_launches(int B, int Hg, int Wg, int C, int Ch);
+
+/*
  * Block-causal form ("linear-diffusion-transformer-4k-efficient-generation",
  * section "技术演进：从图像到视频与世界模型": SANA-Video's block causal linear
  * attention; the pages give no formula). The tokens form blocks of L

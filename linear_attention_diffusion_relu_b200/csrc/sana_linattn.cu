@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "tc_kernels.cuh"
 #include "kvproj_kernel.cuh"
+#include "ffn_kernels.cuh"
 
 namespace {
 
@@ -506,6 +507,49 @@ sana_la_status run_kvproj_state(const void* X, const void* Wk, const void* Wv, i
                   (const float*)partial, ksp, state);
 }
 
+// ------------------------------------------------------------- Mix-FFN ----
+struct FfnPlan {
+    size_t u_bytes, z_bytes;
+};
+
+FfnPlan make_ffn_plan(int B, int Hg, int Wg, int Ch) {
+    const size_t tokens = (size_t)B * Hg * Wg;
+    return FfnPlan{align256(tokens * 2 * Ch * 2), align256(tokens * Ch * 2)};
+}
+
+sana_la_status check_ffn(int B, int Hg, int Wg, int C, int Ch) {
+    if (B < 1 || Hg < 1 || Wg < 1 || C < 1 || Ch < 1) return SANA_LA_ERR_INVALID_ARG;
+    if (C % 8 != 0 || Ch % 8 != 0) return SANA_LA_ERR_UNSUPPORTED;   // 16-byte rows and vectors
+    const long long tokens = (long long)B * Hg * Wg;
+    if (tokens > 0x7fffffffLL) return SANA_LA_ERR_UNSUPPORTED;
+    if (tokens > kMaxElems / (2LL * Ch) || tokens > kMaxElems / C) return SANA_LA_ERR_INVALID_ARG;
+    if (tokens * 2LL * Ch * 2 >= (1LL << 40) || tokens * (long long)C * 2 >= (1LL << 40))
+        return SANA_LA_ERR_UNSUPPORTED;
+    return SANA_LA_OK;
+}
+
+// C (M x N, row stride ldc) = A (M x K) B^T (B is N x K), bf16 in and out
+sana_la_status launch_gemm(const void* A, const void* Bm, void* C, int M, int N, int K, int ldc, cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmA, tmB;
+    sana_la_status st;
+    if ((st = make_tmap(&tmA, A, 1, M, 1, K, sana::tc::GM_TILE_M)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmB, Bm, 1, N, 1, K, sana::tc::GM_TILE_N)) != SANA_LA_OK) return st;
+    if ((st = ensure_smem(sana::tc::gemm_bf16_tc, sana::tc::GemmMap::BYTES, smem_set)) != SANA_LA_OK) return st;
+    sana::tc::GemmParams gp{};
+    gp.M = M;
+    gp.N = N;
+    gp.K = K;
+    gp.ldc = ldc;
+    gp.kblocks = (int)cdiv(K, 64);
+    gp.mtiles = (int)cdiv(M, sana::tc::GM_TILE_M);
+    gp.ntiles = (int)cdiv(N, sana::tc::GM_TILE_N);
+    const long long tiles = (long long)gp.mtiles * gp.ntiles;
+    const int grid = (int)std::min<long long>(tiles, kSMs);
+    return launch(sana::tc::gemm_bf16_tc, dim3(grid), dim3(sana::tc::kThreads), sana::tc::GemmMap::BYTES, s,
+                  false, "gemm_bf16_tc", tmA, tmB, gp, static_cast<__nv_bfloat16*>(C));
+}
+
 sana_la_status kv_state_entry(const void* K, const void* V, int B, int N, int H, int d, int fm,
                               float* state, void* workspace, size_t workspace_bytes,
                               sana_la_stream_t stream) {
@@ -650,6 +694,47 @@ sana_la_status sana_linattn_kv_projection_state(const void* X, const void* Wk, c
 
 int sana_linattn_kv_projection_state_launches(int B, int N, int C, int H, int d) {
     return check_projection(B, N, C, H, d) == SANA_LA_OK ? 2 : 0;   // kvproj_state_tc, kr_reduce_tc
+}
+
+// ------------------------------------------------------------- Mix-FFN ----
+size_t sana_linattn_mix_ffn_workspace_bytes(int B, int Hg, int Wg, int C, int Ch) {
+    if (check_ffn(B, Hg, Wg, C, Ch) != SANA_LA_OK) return 0;
+    const FfnPlan p = make_ffn_plan(B, Hg, Wg, Ch);
+    return p.u_bytes + p.z_bytes;
+}
+
+sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* Kdw, const void* W2,
+                                    int B, int Hg, int Wg, int C, int Ch, void* Y,
+                                    void* workspace, size_t workspace_bytes, sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!X || !W1 || !Kdw || !W2 || !Y || !workspace) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_ffn(B, Hg, Wg, C, Ch);
+    if (st != SANA_LA_OK) return st;
+    if (!aligned16(X) || !aligned16(W1) || !aligned16(W2) || !aligned16(Y) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(Kdw) & 3) != 0)
+        return SANA_LA_ERR_INVALID_ARG;
+    const FfnPlan p = make_ffn_plan(B, Hg, Wg, Ch);
+    if (workspace_bytes < p.u_bytes + p.z_bytes) return SANA_LA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    void* U = ws;
+    void* Z = ws + p.u_bytes;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int M = B * Hg * Wg;
+    // 1x1 expand: U = X W1^T (2 Ch channels)
+    if ((st = launch_gemm(X, W1, U, M, 2 * Ch, C, 2 * Ch, s)) != SANA_LA_OK) return st;
+    // 3x3 depthwise over the grid and the GLU, fused
+    const long long threads = (long long)M * (Ch / 8);
+    const int blocks = (int)std::min<long long>(cdiv(threads, 256), 148LL * 16);
+    if ((st = launch(sana::tc::dwconv_glu, dim3(blocks), dim3(256), 0, s, false, "dwconv_glu",
+                     static_cast<const __nv_bfloat16*>(U), Kdw, B, Hg, Wg, Ch,
+                     static_cast<__nv_bfloat16*>(Z))) != SANA_LA_OK)
+        return st;
+    // 1x1 project: Y = Z W2^T
+    return launch_gemm(Z, W2, Y, M, C, Ch, C, s);
+}
+
+int sana_linattn_mix_ffn_launches(int B, int Hg, int Wg, int C, int Ch) {
+    return check_ffn(B, Hg, Wg, C, Ch) == SANA_LA_OK ? 3 : 0;   // gemm, dwconv_glu, gemm
 }
 
 // ------------------------------------------------------- block-causal ----

@@ -18,6 +18,10 @@ the state built inside the key-value projection (K and V never stored):
 
     kv_projection_state(X, Wk, Wv, H, state=None, workspace=None) -> (B, H, d, d+1) fp32
 
+the Mix-FFN that follows the attention in a Sana block:
+
+    mix_ffn(X, W1, Kdw, W2, grid_hw, out=None, workspace=None) -> Y (B, N, C) bf16
+
 and the block-causal form (blocks of L tokens, L a multiple of 128):
 
     block_causal_workspace_bytes(B, N, H, d, L)
@@ -49,6 +53,9 @@ SYMBOLS = (
     "sana_linattn_kv_state_fm",
     "sana_linattn_apply_fm",
     "sana_linattn_forward_fm",
+    "sana_linattn_mix_ffn_workspace_bytes",
+    "sana_linattn_mix_ffn",
+    "sana_linattn_mix_ffn_launches",
     "sana_linattn_kv_projection_workspace_bytes",
     "sana_linattn_kv_projection_state",
     "sana_linattn_kv_projection_state_launches",
@@ -110,6 +117,12 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_apply_fm.restype = st
         lib.sana_linattn_forward_fm.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
         lib.sana_linattn_forward_fm.restype = st
+        lib.sana_linattn_mix_ffn_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_mix_ffn_workspace_bytes.restype = sz
+        lib.sana_linattn_mix_ffn.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+        lib.sana_linattn_mix_ffn.restype = st
+        lib.sana_linattn_mix_ffn_launches.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_mix_ffn_launches.restype = ctypes.c_int
         lib.sana_linattn_kv_projection_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.sana_linattn_kv_projection_workspace_bytes.restype = sz
         lib.sana_linattn_kv_projection_state.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
@@ -406,3 +419,40 @@ def kv_projection_state(X: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor, H: 
                                               workspace.numel() * workspace.element_size(), _stream(X.device))
     _check(lib, st, "sana_linattn_kv_projection_state")
     return state
+
+
+# ---------------------------------------------------------------------- Mix-FFN --
+
+def mix_ffn_workspace_bytes(B: int, Hg: int, Wg: int, C: int, Ch: int) -> int:
+    return int(load_library().sana_linattn_mix_ffn_workspace_bytes(B, Hg, Wg, C, Ch))
+
+
+def mix_ffn(X: torch.Tensor, W1: torch.Tensor, Kdw: torch.Tensor, W2: torch.Tensor, grid_hw,
+            out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = (a * sigmoid(g)) W2^T with [a | g] = depthwise3x3(X W1^T) over the token
+    grid. X bf16 (B, Hg*Wg, C); W1 bf16 (2*Ch, C); Kdw fp32 (2*Ch, 3, 3); W2 bf16 (C, Ch)."""
+    for name, t, dt in (("X", X, torch.bfloat16), ("W1", W1, torch.bfloat16), ("Kdw", Kdw, torch.float32),
+                        ("W2", W2, torch.bfloat16)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+        if t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous {dt}")
+    Hg, Wg = grid_hw
+    B, N, C = X.shape
+    Ch2 = W1.shape[0]
+    if N != Hg * Wg or W1.shape != (Ch2, C) or Ch2 % 2 or tuple(Kdw.shape) != (Ch2, 3, 3) \
+            or tuple(W2.shape) != (C, Ch2 // 2):
+        raise ValueError("shapes do not match: X (B, Hg*Wg, C), W1 (2Ch, C), Kdw (2Ch, 3, 3), W2 (C, Ch)")
+    Ch = Ch2 // 2
+    out = _prep_out(out, (B, N, C), torch.bfloat16, X.device)
+    if workspace is None:
+        n = mix_ffn_workspace_bytes(B, Hg, Wg, C, Ch)
+        if n == 0:
+            raise ValueError(f"unsupported sizes B={B} grid={grid_hw} C={C} Ch={Ch}")
+        workspace = torch.empty(n, dtype=torch.uint8, device=X.device)
+    lib = load_library()
+    st = lib.sana_linattn_mix_ffn(X.data_ptr(), W1.data_ptr(), Kdw.data_ptr(), W2.data_ptr(), B, Hg, Wg, C, Ch,
+                                  out.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream(X.device))
+    _check(lib, st, "sana_linattn_mix_ffn")
+    return out

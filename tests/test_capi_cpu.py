@@ -179,3 +179,20 @@ def test_kv_projection_host_checks(lib):
     assert f(FAKE, FAKE, FAKE, 1, 300, 128, 4, 32, FAKE, FAKE, ws - 1, None) == ops.ERR_WORKSPACE
     assert lib.sana_linattn_kv_projection_state_launches(1, 300, 128, 4, 32) == 2
     assert lib.sana_linattn_kv_projection_state_launches(1, 300, 124, 4, 32) == 0
+
+
+def test_mix_ffn_host_checks(lib):
+    wsb = lib.sana_linattn_mix_ffn_workspace_bytes
+    assert wsb(2, 128, 128, 2240, 5600) > 0
+    assert wsb(2, 128, 128, 2244, 5600) == 0        # C not a multiple of 8
+    assert wsb(2, 128, 128, 2240, 5604) == 0        # Ch not a multiple of 8
+    assert wsb(0, 128, 128, 2240, 5600) == 0
+    # U (2 Ch bf16) and Z (Ch bf16) per token
+    assert wsb(1, 4, 4, 64, 32) >= 16 * (64 + 32) * 2
+    f = lib.sana_linattn_mix_ffn
+    ws = wsb(1, 4, 4, 64, 32)
+    assert f(None, FAKE, FAKE, FAKE, 1, 4, 4, 64, 32, FAKE, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 60, 32, FAKE, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE + 2, FAKE, 1, 4, 4, 64, 32, FAKE, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 64, 32, FAKE, FAKE, ws - 1, None) == ops.ERR_WORKSPACE
+    assert lib.sana_linattn_mix_ffn_launches(1, 4, 4, 64, 32) == 3
