@@ -55,9 +55,10 @@ def parse_args(argv=None):
                    help="timed steps (about 1 s at 4096px, long enough to sample clocks)")
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--op", choices=["forward", "kvproj"], default="forward",
+    p.add_argument("--op", choices=["forward", "kvproj", "mixffn"], default="forward",
                    help="kvproj: the key-value projection with the state in its epilogue (one GPU), "
-                        "against a cuBLAS projection followed by kv_state")
+                        "against a cuBLAS projection followed by kv_state; mixffn: the Mix-FFN after "
+                        "the attention (one GPU), against torch (cuBLAS + cuDNN depthwise conv)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -529,12 +530,96 @@ def run_kvproj(args):
     return 0
 
 
+def run_mixffn(args):
+    """The Mix-FFN at a Sana shape: tokens on a square grid (N = Hg * Wg), C = H*d,
+    hidden Ch = 2.5 C (a workload choice; the pages give no expansion ratio).
+    Metric: TFLOP/s of the two 1x1 convolutions (the depthwise conv adds < 1 %),
+    roofline against the measured cuBLAS bf16 peak; torch's unfused pipeline
+    (cuBLAS, cuDNN depthwise conv, GLU) is timed beside it."""
+    import math
+    import torch
+    from linear_attention_diffusion_relu_b200 import ops
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS
+    if args.gpus != 1:
+        raise SystemExit("--op mixffn runs on one GPU")
+    w = WORKLOADS[args.workload]
+    B, N = w.B, w.N
+    C = w.H * w.d
+    Ch = int(round(2.5 * C / 8)) * 8
+    Hg = Wg = int(math.isqrt(N))
+    if Hg * Wg != N:
+        raise SystemExit(f"{w.name}: N = {N} is not a square grid")
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device="cuda").manual_seed(w.seed)
+    X = torch.randn((B, N, C), generator=g, device=dev).to(torch.bfloat16)
+    W1 = (torch.randn((2 * Ch, C), generator=g, device=dev) / C ** 0.5).to(torch.bfloat16)
+    Kdw = (torch.randn((2 * Ch, 3, 3), generator=g, device=dev) / 3.0).float()
+    W2 = (torch.randn((C, Ch), generator=g, device=dev) / Ch ** 0.5).to(torch.bfloat16)
+    Y = torch.empty((B, N, C), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ops.mix_ffn_workspace_bytes(B, Hg, Wg, C, Ch), dtype=torch.uint8, device=dev)
+    Kt = Kdw.to(torch.bfloat16).view(2 * Ch, 1, 3, 3)
+
+    def ours():
+        ops.mix_ffn(X, W1, Kdw, W2, (Hg, Wg), out=Y, workspace=ws)
+
+    def torch_ref():
+        U = (X @ W1.T).view(B, Hg, Wg, 2 * Ch).permute(0, 3, 1, 2)
+        D = torch.nn.functional.conv2d(U, Kt, padding=1, groups=2 * Ch)
+        a, gt = D.permute(0, 2, 3, 1).reshape(B, N, 2 * Ch).chunk(2, dim=-1)
+        return (a * torch.sigmoid(gt)) @ W2.T
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    steps = max(1, min(args.steps, 100))
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = timed(ours, steps)
+    clk = clocks.stop()
+    ms_torch = timed(torch_ref, max(1, steps // 4))
+    flops = 2.0 * B * N * C * (2 * Ch) + 2.0 * B * N * Ch * C
+    tflops = flops / (ms / 1e3) / 1e12
+    peak, src = FALLBACK_BF16_TFLOPS, "fallback"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        pass
+    line = {
+        "metric": "Mix-FFN (expand, depthwise 3x3 + GLU, project), TFLOP/s", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} Mix-FFN", "B": B, "grid": [Hg, Wg], "C": C, "Ch": Ch},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "kernel": "gemm_bf16_tc (x2) + dwconv_glu",
+                     "peak_source": f"{src} cuBLAS bf16 (burst)"},
+        "torch_unfused": {"ms_per_step": ms_torch,
+                          "what": "cuBLAS matmul, cuDNN depthwise conv2d, sigmoid gate, cuBLAS matmul"},
+        "clocks": clk,
+        "gpu_launches": ops.load_library().sana_linattn_mix_ffn_launches(B, Hg, Wg, C, Ch) * steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "kvproj":
         return run_kvproj(args)
+    if args.op == "mixffn":
+        return run_mixffn(args)
     return run_ours(args)
 
 
