@@ -5,8 +5,9 @@ The workspace keeps the two bf16 intermediates (U after the expand, Z after
 the depthwise conv and the GLU), so each stage is checked against the oracle
 applied to the GPU's own input of that stage: the GEMMs accumulate in fp32
 and the oracle in fp64 before the same bf16 rounding, so an element may land
-one bf16 step (2^-7 relative) apart; the project's output is held to one bf16
-rounding plus an fp32 accumulation bound. End to end, rows of Y are held to 2e-2
+one bf16 step (2^-7 relative) apart, or, where the sum cancels, differ by the
+fp32 accumulation error; the project's output is held to one bf16 rounding plus
+an fp32 accumulation bound. End to end, rows of Y are held to 2e-2
 of their norm (the two intermediate roundings compound)."""
 import numpy as np
 import pytest
@@ -60,7 +61,10 @@ def test_mix_ffn_stages_match_oracle(oracle, shape):
     # expand: one bf16 step at most, on few elements
     U_ref = oracle.round_bf16(Xd @ W1d.T)
     dU = np.abs(U - U_ref)
-    assert np.all(dU <= 2.0 ** -7 * np.abs(U_ref) + 1e-30), (dU / (np.abs(U_ref) + 1e-30)).max()
+    # one bf16 step, or (for sums that cancel) the fp32 accumulation error
+    # K * 2^-24 * sum |x w| carrying the rounding across a boundary
+    boundU = 2.0 ** -7 * np.abs(U_ref) + C * 2.0 ** -23 * (np.abs(Xd) @ np.abs(W1d).T) + 1e-30
+    assert np.all(dU <= boundU), (dU / boundU).max()
     assert np.mean(dU > 0) < 1e-2
     # depthwise + GLU on the GPU's own U
     D = oracle.depthwise3x3(U, Kd, (Hg, Wg))
@@ -71,7 +75,7 @@ def test_mix_ffn_stages_match_oracle(oracle, shape):
     assert np.mean(dZ > 0) < 1e-2
     # project on the GPU's own Z: one bf16 rounding plus fp32 accumulation
     Y_ref = Z @ W2d.T
-    bound = 2.0 ** -8 * np.abs(Y_ref) + 1e-5 * (np.abs(Z) @ np.abs(W2d).T) + 1e-30
+    bound = 2.0 ** -8 * np.abs(Y_ref) + Ch * 2.0 ** -23 * (np.abs(Z) @ np.abs(W2d).T) + 1e-30
     assert np.all(np.abs(to_f64(Y) - Y_ref) <= bound)
     # end to end
     Y_e2e = oracle.mix_ffn(Xd, W1d, Kd, W2d, (Hg, Wg))
