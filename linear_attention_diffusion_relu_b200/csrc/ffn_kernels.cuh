@@ -187,28 +187,45 @@ gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 }
 
 // ====================================================== depthwise + GLU ===
-// One thread per (token, 8 channels of the gated half): for each of the 9
-// taps it reads 8 channels of the value half a and the gate half g of U
-// (16 bytes each), accumulates in fp32 in tap order (dy, dx), and writes
-// Z = a * sigmoid(g) as 8 bf16. Neighbour tokens are read through L1/L2.
+// A CTA is 32 channel chunks (8 channels each, both halves) x 8 token lanes.
+// Each thread keeps its chunk's 2 x 8 x 9 taps in registers and walks the
+// tokens t0 + lane_y, t0 + lane_y + 8, ... of its CTA's token range: for each
+// of the 9 taps it reads 8 channels of the value half a and of the gate half g
+// of U (16 bytes each; the 32 chunk lanes of a token read 512 contiguous
+// bytes), accumulates in fp32 in tap order (dy, dx) and writes
+// Z = a * sigmoid(g) as 8 bf16. Neighbour tokens come through L1/L2.
 // U: (B, Hg*Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z: (B, Hg*Wg, Ch) bf16.
-__global__ void __launch_bounds__(256)
+constexpr int DW_CHUNKS = 32;      // channel chunks per CTA
+constexpr int DW_LANES = 8;        // token lanes per CTA
+constexpr int DW_TOKENS = 64;      // tokens per CTA
+
+__global__ void __launch_bounds__(DW_CHUNKS * DW_LANES)
 dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, int B, int Hg, int Wg, int Ch,
            __nv_bfloat16* __restrict__ Z)
 {
     const int chunks = Ch / 8;
-    const long long total = (long long)B * Hg * Wg * chunks;
-    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
-         idx += (long long)gridDim.x * blockDim.x) {
-        const int ck = (int)(idx % chunks);
-        const long long tok = idx / chunks;              // b * Hg * Wg + y * Wg + x
+    const int ck = blockIdx.x * DW_CHUNKS + (threadIdx.x % DW_CHUNKS);
+    const int ly = threadIdx.x / DW_CHUNKS;
+    if (ck >= chunks) return;
+    const int c0 = ck * 8;
+    float ka[8][9], kg[8][9];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int t = 0; t < 9; ++t) {
+            ka[j][t] = Kdw[(c0 + j) * 9 + t];
+            kg[j][t] = Kdw[(Ch + c0 + j) * 9 + t];
+        }
+    }
+    const long long ntok = (long long)B * Hg * Wg;
+    const long long t_begin = (long long)blockIdx.y * DW_TOKENS;
+    for (long long tok = t_begin + ly; tok < ntok && tok < t_begin + DW_TOKENS; tok += DW_LANES) {
         const int x = (int)(tok % Wg);
         const int y = (int)((tok / Wg) % Hg);
-        const long long b0 = tok - (long long)y * Wg - x; // first token of this batch's grid
+        const long long base = tok - (long long)y * Wg - x;    // first token of this batch's grid
         float a[8], g[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) a[j] = g[j] = 0.0f;
-        const int c0 = ck * 8;
 #pragma unroll
         for (int dy = 0; dy < 3; ++dy) {
             const int yy = y + dy - 1;
@@ -216,19 +233,20 @@ dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, i
             for (int dx = 0; dx < 3; ++dx) {
                 const int xx = x + dx - 1;
                 if (yy < 0 || yy >= Hg || xx < 0 || xx >= Wg) continue;
-                const __nv_bfloat16* u = U + (b0 + (long long)yy * Wg + xx) * (2LL * Ch);
+                const __nv_bfloat16* u = U + (base + (long long)yy * Wg + xx) * (2LL * Ch);
                 const uint4 va = *reinterpret_cast<const uint4*>(u + c0);
                 const uint4 vg = *reinterpret_cast<const uint4*>(u + Ch + c0);
                 const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
                 const uint32_t wg[4] = {vg.x, vg.y, vg.z, vg.w};
+                const int t = dy * 3 + dx;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float2 fa = bf16x2_to_float2(wa[j]);
                     const float2 fg = bf16x2_to_float2(wg[j]);
-                    a[2 * j] = fmaf(fa.x, Kdw[(c0 + 2 * j) * 9 + dy * 3 + dx], a[2 * j]);
-                    a[2 * j + 1] = fmaf(fa.y, Kdw[(c0 + 2 * j + 1) * 9 + dy * 3 + dx], a[2 * j + 1]);
-                    g[2 * j] = fmaf(fg.x, Kdw[(Ch + c0 + 2 * j) * 9 + dy * 3 + dx], g[2 * j]);
-                    g[2 * j + 1] = fmaf(fg.y, Kdw[(Ch + c0 + 2 * j + 1) * 9 + dy * 3 + dx], g[2 * j + 1]);
+                    a[2 * j] = fmaf(fa.x, ka[2 * j][t], a[2 * j]);
+                    a[2 * j + 1] = fmaf(fa.y, ka[2 * j + 1][t], a[2 * j + 1]);
+                    g[2 * j] = fmaf(fg.x, kg[2 * j][t], g[2 * j]);
+                    g[2 * j + 1] = fmaf(fg.y, kg[2 * j + 1][t], g[2 * j + 1]);
                 }
             }
         }
