@@ -187,66 +187,87 @@ gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 }
 
 // ====================================================== depthwise + GLU ===
-// A CTA is 32 channel chunks (8 channels each, both halves) x 8 token lanes.
-// Each thread keeps its chunk's 2 x 8 x 9 taps in registers and walks the
-// tokens t0 + lane_y, t0 + lane_y + 8, ... of its CTA's token range: for each
-// of the 9 taps it reads 8 channels of the value half a and of the gate half g
-// of U (16 bytes each; the 32 chunk lanes of a token read 512 contiguous
-// bytes), accumulates in fp32 in tap order (dy, dx) and writes
-// Z = a * sigmoid(g) as 8 bf16. Neighbour tokens come through L1/L2.
+// A CTA takes one batch image's tile of DW_TY grid rows x DW_TX columns and 64
+// channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). It
+// copies the tile plus a one-token halo of U into shared memory (zeros outside
+// the grid) and the 128 channels' taps, then each thread computes 8 outputs of
+// one 8-channel chunk: for each of the 9 taps (order dy, dx) it reads 16 bytes
+// of a and of g of the neighbour from shared memory and accumulates in fp32;
+// Z = a * sigmoid(g) is stored as 8 bf16 (8 lanes = one token's 128 bytes).
 // U: (B, Hg*Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z: (B, Hg*Wg, Ch) bf16.
-constexpr int DW_CHUNKS = 32;      // channel chunks per CTA
-constexpr int DW_LANES = 8;        // token lanes per CTA
-constexpr int DW_TOKENS = 64;      // tokens per CTA
+constexpr int DW_TY = 4;                        // grid rows per CTA
+constexpr int DW_TX = 64;                       // grid columns per CTA
+constexpr int DW_CH = 64;                       // channels of each half per CTA
+constexpr int DW_THREADS = 256;
+constexpr int DW_ROW_BYTES = 2 * DW_CH * 2;     // a and g of one token: 256 bytes
+constexpr int DW_SMEM = (DW_TY + 2) * (DW_TX + 2) * DW_ROW_BYTES + 2 * DW_CH * 9 * 4;
 
-__global__ void __launch_bounds__(DW_CHUNKS * DW_LANES)
+__global__ void __launch_bounds__(DW_THREADS)
 dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, int B, int Hg, int Wg, int Ch,
            __nv_bfloat16* __restrict__ Z)
 {
-    const int chunks = Ch / 8;
-    const int ck = blockIdx.x * DW_CHUNKS + (threadIdx.x % DW_CHUNKS);
-    const int ly = threadIdx.x / DW_CHUNKS;
-    if (ck >= chunks) return;
-    const int c0 = ck * 8;
-    float ka[8][9], kg[8][9];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-        for (int t = 0; t < 9; ++t) {
-            ka[j][t] = Kdw[(c0 + j) * 9 + t];
-            kg[j][t] = Kdw[(Ch + c0 + j) * 9 + t];
-        }
+    extern __shared__ __align__(16) uint8_t dsm[];
+    float* taps = reinterpret_cast<float*>(dsm + (DW_TY + 2) * (DW_TX + 2) * DW_ROW_BYTES);  // [tap][128 ch]
+    const int tid = threadIdx.x;
+    const int tiles_x = (Wg + DW_TX - 1) / DW_TX;
+    const int tiles_y = (Hg + DW_TY - 1) / DW_TY;
+    const int c0 = blockIdx.x * DW_CH;                       // first channel of the group (each half)
+    const int b = blockIdx.y / (tiles_y * tiles_x);
+    const int ty = (blockIdx.y / tiles_x) % tiles_y;
+    const int tx = blockIdx.y % tiles_x;
+    const int y0 = ty * DW_TY, x0 = tx * DW_TX;
+    const int nch = min(DW_CH, Ch - c0);                     // channels of this group (multiple of 8)
+    const long long img = (long long)b * Hg * Wg;
+    // taps: entry t * 128 + j, j < 64 the value half, j >= 64 the gate half
+    for (int e = tid; e < 2 * DW_CH * 9; e += DW_THREADS) {
+        const int t = e / (2 * DW_CH), j = e % (2 * DW_CH);
+        const int c = j < DW_CH ? c0 + j : Ch + c0 + (j - DW_CH);
+        taps[e] = (j % DW_CH) < nch ? Kdw[(size_t)c * 9 + t] : 0.0f;
     }
-    const long long ntok = (long long)B * Hg * Wg;
-    const long long t_begin = (long long)blockIdx.y * DW_TOKENS;
-    for (long long tok = t_begin + ly; tok < ntok && tok < t_begin + DW_TOKENS; tok += DW_LANES) {
-        const int x = (int)(tok % Wg);
-        const int y = (int)((tok / Wg) % Hg);
-        const long long base = tok - (long long)y * Wg - x;    // first token of this batch's grid
+    // the tile and its halo: (DW_TY + 2) x (DW_TX + 2) tokens, 16 chunks of 16 bytes each
+    constexpr int TOK = (DW_TY + 2) * (DW_TX + 2);
+    for (int e = tid; e < TOK * 16; e += DW_THREADS) {
+        const int tok = e / 16, q = e % 16;                  // q < 8: value half, else gate half
+        const int yy = y0 - 1 + tok / (DW_TX + 2);
+        const int xx = x0 - 1 + tok % (DW_TX + 2);
+        const int ch = (q & 7) * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (yy >= 0 && yy < Hg && xx >= 0 && xx < Wg && ch < nch) {
+            const __nv_bfloat16* u = U + (img + (long long)yy * Wg + xx) * (2LL * Ch) + (q < 8 ? c0 : Ch + c0) + ch;
+            v = *reinterpret_cast<const uint4*>(u);
+        }
+        *reinterpret_cast<uint4*>(dsm + (size_t)tok * DW_ROW_BYTES + q * 16) = v;
+    }
+    __syncthreads();
+    // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8, tokens tid / 8 + 32 k
+    const int ck = tid % 8;
+    if (ck * 8 >= nch) return;
+    for (int o = tid / 8; o < DW_TY * DW_TX; o += DW_THREADS / 8) {
+        const int ly = o / DW_TX, lx = o % DW_TX;
+        const int y = y0 + ly, x = x0 + lx;
+        if (y >= Hg || x >= Wg) continue;
         float a[8], g[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) a[j] = g[j] = 0.0f;
 #pragma unroll
         for (int dy = 0; dy < 3; ++dy) {
-            const int yy = y + dy - 1;
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-                const int xx = x + dx - 1;
-                if (yy < 0 || yy >= Hg || xx < 0 || xx >= Wg) continue;
-                const __nv_bfloat16* u = U + (base + (long long)yy * Wg + xx) * (2LL * Ch);
-                const uint4 va = *reinterpret_cast<const uint4*>(u + c0);
-                const uint4 vg = *reinterpret_cast<const uint4*>(u + Ch + c0);
+                const uint8_t* row = dsm + (size_t)((ly + dy) * (DW_TX + 2) + (lx + dx)) * DW_ROW_BYTES;
+                const uint4 va = *reinterpret_cast<const uint4*>(row + ck * 16);
+                const uint4 vg = *reinterpret_cast<const uint4*>(row + 128 + ck * 16);
+                const float* ta = taps + (dy * 3 + dx) * (2 * DW_CH) + ck * 8;
+                const float* tg = ta + DW_CH;
                 const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
                 const uint32_t wg[4] = {vg.x, vg.y, vg.z, vg.w};
-                const int t = dy * 3 + dx;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float2 fa = bf16x2_to_float2(wa[j]);
                     const float2 fg = bf16x2_to_float2(wg[j]);
-                    a[2 * j] = fmaf(fa.x, ka[2 * j][t], a[2 * j]);
-                    a[2 * j + 1] = fmaf(fa.y, ka[2 * j + 1][t], a[2 * j + 1]);
-                    g[2 * j] = fmaf(fg.x, kg[2 * j][t], g[2 * j]);
-                    g[2 * j + 1] = fmaf(fg.y, kg[2 * j + 1][t], g[2 * j + 1]);
+                    a[2 * j] = fmaf(fa.x, ta[2 * j], a[2 * j]);
+                    a[2 * j + 1] = fmaf(fa.y, ta[2 * j + 1], a[2 * j + 1]);
+                    g[2 * j] = fmaf(fg.x, tg[2 * j], g[2 * j]);
+                    g[2 * j + 1] = fmaf(fg.y, tg[2 * j + 1], g[2 * j + 1]);
                 }
             }
         }
@@ -258,7 +279,7 @@ dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, i
         out.y = float2_to_bf16x2(z[2], z[3]);
         out.z = float2_to_bf16x2(z[4], z[5]);
         out.w = float2_to_bf16x2(z[6], z[7]);
-        *reinterpret_cast<uint4*>(Z + tok * Ch + c0) = out;
+        *reinterpret_cast<uint4*>(Z + (img + (long long)y * Wg + x) * Ch + c0 + ck * 8) = out;
     }
 }
 

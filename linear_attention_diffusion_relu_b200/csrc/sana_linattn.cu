@@ -723,9 +723,12 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
     // 1x1 expand: U = X W1^T (2 Ch channels)
     if ((st = launch_gemm(X, W1, U, M, 2 * Ch, C, 2 * Ch, s)) != SANA_LA_OK) return st;
     // 3x3 depthwise over the grid and the GLU, fused
-    const dim3 dw_grid((unsigned)cdiv(Ch / 8, sana::tc::DW_CHUNKS), (unsigned)cdiv(M, sana::tc::DW_TOKENS));
-    if (dw_grid.y > 65535u) return SANA_LA_ERR_UNSUPPORTED;
-    if ((st = launch(sana::tc::dwconv_glu, dw_grid, dim3(sana::tc::DW_CHUNKS * sana::tc::DW_LANES), 0, s,
+    static std::atomic<uint64_t> dw_smem_set{0};
+    if ((st = ensure_smem(sana::tc::dwconv_glu, sana::tc::DW_SMEM, dw_smem_set)) != SANA_LA_OK) return st;
+    const long long dw_tiles = (long long)B * cdiv(Hg, sana::tc::DW_TY) * cdiv(Wg, sana::tc::DW_TX);
+    if (dw_tiles > 65535) return SANA_LA_ERR_UNSUPPORTED;
+    const dim3 dw_grid((unsigned)cdiv(Ch, sana::tc::DW_CH), (unsigned)dw_tiles);
+    if ((st = launch(sana::tc::dwconv_glu, dw_grid, dim3(sana::tc::DW_THREADS), sana::tc::DW_SMEM, s,
                      false, "dwconv_glu",
                      static_cast<const __nv_bfloat16*>(U), Kdw, B, Hg, Wg, Ch,
                      static_cast<__nv_bfloat16*>(Z))) != SANA_LA_OK)
