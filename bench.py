@@ -16,6 +16,11 @@ divided by the slowest rank's time. Multi-GPU runs give every rank its own
 
 `--impl reference` times the fp64 CPU oracle (the only reference there is) on
 bounded samples of the same workload, on the host cores, rank 0 only.
+
+`--workload` selects another named workload (other sizes, the ELU+1 and cos
+feature maps, the block-causal video shapes). `--op kvproj` times the key-value
+projection with the state in its epilogue and `--op mixffn` the Mix-FFN, each
+next to the unfused pipeline it replaces (one GPU, TFLOP/s).
 """
 from __future__ import annotations
 
