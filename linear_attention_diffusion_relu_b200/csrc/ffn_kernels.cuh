@@ -224,20 +224,23 @@ dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, i
         const int c = j < DW_CH ? c0 + j : Ch + c0 + (j - DW_CH);
         taps[e] = (j % DW_CH) < nch ? Kdw[(size_t)c * 9 + t] : 0.0f;
     }
-    // the tile and its halo: (DW_TY + 2) x (DW_TX + 2) tokens, 16 chunks of 16 bytes each
+    // the tile and its halo: (DW_TY + 2) x (DW_TX + 2) tokens, 16 chunks of 16 bytes
+    // each, copied with cp.async (all in flight together; a source size of 0
+    // writes zeros for positions outside the grid)
     constexpr int TOK = (DW_TY + 2) * (DW_TX + 2);
     for (int e = tid; e < TOK * 16; e += DW_THREADS) {
         const int tok = e / 16, q = e % 16;                  // q < 8: value half, else gate half
         const int yy = y0 - 1 + tok / (DW_TX + 2);
         const int xx = x0 - 1 + tok % (DW_TX + 2);
         const int ch = (q & 7) * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (yy >= 0 && yy < Hg && xx >= 0 && xx < Wg && ch < nch) {
-            const __nv_bfloat16* u = U + (img + (long long)yy * Wg + xx) * (2LL * Ch) + (q < 8 ? c0 : Ch + c0) + ch;
-            v = *reinterpret_cast<const uint4*>(u);
-        }
-        *reinterpret_cast<uint4*>(dsm + (size_t)tok * DW_ROW_BYTES + q * 16) = v;
+        const bool in = yy >= 0 && yy < Hg && xx >= 0 && xx < Wg && ch < nch;
+        const __nv_bfloat16* u = in ? U + (img + (long long)yy * Wg + xx) * (2LL * Ch) + (q < 8 ? c0 : Ch + c0) + ch
+                                    : U;
+        const uint32_t dst = ptx::smem_u32(dsm + (size_t)tok * DW_ROW_BYTES + q * 16);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                     :: "r"(dst), "l"(u), "r"(in ? 16 : 0) : "memory");
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8, tokens tid / 8 + 32 k
     const int ck = tid % 8;
