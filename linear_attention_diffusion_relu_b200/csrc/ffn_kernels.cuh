@@ -188,26 +188,33 @@ gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 
 // ====================================================== depthwise + GLU ===
 // A CTA takes one batch image's tile of DW_TY grid rows x DW_TX columns and 64
-// channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). It
-// copies the tile plus a one-token halo of U into shared memory (zeros outside
-// the grid) and the 128 channels' taps, then each thread computes 8 outputs of
-// one 8-channel chunk: for each of the 9 taps (order dy, dx) it reads 16 bytes
-// of a and of g of the neighbour from shared memory and accumulates in fp32;
-// Z = a * sigmoid(g) is stored as 8 bf16 (8 lanes = one token's 128 bytes).
-// U: (B, Hg*Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z: (B, Hg*Wg, Ch) bf16.
+// channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). Two
+// TMA loads bring the tile plus a one-token halo of each half into shared
+// memory ([row][column][64 channels], zeros outside the grid: the load starts
+// at column x0-1 and row y0-1); the 128 channels' taps go beside them. Each
+// thread then computes 8 outputs of one 8-channel chunk: for each of the 9
+// taps (order dy, dx) it reads 16 bytes of a and of g of the neighbour and
+// accumulates in fp32; Z = a * sigmoid(g) is stored as 8 bf16 (8 lanes = one
+// token's 128 bytes).
+// U (tensor map): (B, Hg, Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z: (B, Hg*Wg, Ch) bf16.
 constexpr int DW_TY = 4;                        // grid rows per CTA
 constexpr int DW_TX = 64;                       // grid columns per CTA
 constexpr int DW_CH = 64;                       // channels of each half per CTA
 constexpr int DW_THREADS = 256;
-constexpr int DW_ROW_BYTES = 2 * DW_CH * 2;     // a and g of one token: 256 bytes
-constexpr int DW_SMEM = (DW_TY + 2) * (DW_TX + 2) * DW_ROW_BYTES + 2 * DW_CH * 9 * 4;
+constexpr int DW_HALF_BYTES = (DW_TY + 2) * (DW_TX + 2) * DW_CH * 2;   // one half's box: 50,688 B
+constexpr int DW_TAPS_OFF = 2 * DW_HALF_BYTES;
+constexpr int DW_BAR_OFF = DW_TAPS_OFF + 2 * DW_CH * 9 * 4;
+constexpr int DW_SMEM = DW_BAR_OFF + 16 + 128;  // barrier, flag, alignment slack
 
 __global__ void __launch_bounds__(DW_THREADS)
-dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, int B, int Hg, int Wg, int Ch,
+dwconv_glu(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Kdw, int B, int Hg, int Wg, int Ch,
            __nv_bfloat16* __restrict__ Z)
 {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    float* taps = reinterpret_cast<float*>(dsm + (DW_TY + 2) * (DW_TX + 2) * DW_ROW_BYTES);  // [tap][128 ch]
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+    float* taps = reinterpret_cast<float*>(dsm + DW_TAPS_OFF);     // [tap][128 ch]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + DW_BAR_OFF);
+    int* loaded = reinterpret_cast<int*>(dsm + DW_BAR_OFF + 8);
     const int tid = threadIdx.x;
     const int tiles_x = (Wg + DW_TX - 1) / DW_TX;
     const int tiles_y = (Hg + DW_TY - 1) / DW_TY;
@@ -217,34 +224,35 @@ dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, i
     const int tx = blockIdx.y % tiles_x;
     const int y0 = ty * DW_TY, x0 = tx * DW_TX;
     const int nch = min(DW_CH, Ch - c0);                     // channels of this group (multiple of 8)
-    const long long img = (long long)b * Hg * Wg;
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(bar, 2 * DW_HALF_BYTES);
+        ptx::tma_load_4d(dsm, &tmU, bar, c0, x0 - 1, y0 - 1, b);
+        ptx::tma_load_4d(dsm + DW_HALF_BYTES, &tmU, bar, Ch + c0, x0 - 1, y0 - 1, b);
+    }
     // taps: entry t * 128 + j, j < 64 the value half, j >= 64 the gate half
     for (int e = tid; e < 2 * DW_CH * 9; e += DW_THREADS) {
         const int t = e / (2 * DW_CH), j = e % (2 * DW_CH);
         const int c = j < DW_CH ? c0 + j : Ch + c0 + (j - DW_CH);
         taps[e] = (j % DW_CH) < nch ? Kdw[(size_t)c * 9 + t] : 0.0f;
     }
-    // the tile and its halo: (DW_TY + 2) x (DW_TX + 2) tokens, 16 chunks of 16 bytes
-    // each, copied with cp.async (all in flight together; a source size of 0
-    // writes zeros for positions outside the grid)
-    constexpr int TOK = (DW_TY + 2) * (DW_TX + 2);
-    for (int e = tid; e < TOK * 16; e += DW_THREADS) {
-        const int tok = e / 16, q = e % 16;                  // q < 8: value half, else gate half
-        const int yy = y0 - 1 + tok / (DW_TX + 2);
-        const int xx = x0 - 1 + tok % (DW_TX + 2);
-        const int ch = (q & 7) * 8;
-        const bool in = yy >= 0 && yy < Hg && xx >= 0 && xx < Wg && ch < nch;
-        const __nv_bfloat16* u = in ? U + (img + (long long)yy * Wg + xx) * (2LL * Ch) + (q < 8 ? c0 : Ch + c0) + ch
-                                    : U;
-        const uint32_t dst = ptx::smem_u32(dsm + (size_t)tok * DW_ROW_BYTES + q * 16);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                     :: "r"(dst), "l"(u), "r"(in ? 16 : 0) : "memory");
+    // thread 0 waits for the tile (bounded) and tells the others, so the
+    // decision to go on is the same for every thread
+    if (tid == 0) {
+        const bool ok = ptx::mbar_wait(bar, 0, nullptr, &g_device_error);
+        if (!ok) ptx::mbar_wait(bar, 0, nullptr, &g_device_error);   // let the copies land before leaving
+        *loaded = ok ? 1 : 0;
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
+    if (!*loaded) return;
     // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8, tokens tid / 8 + 32 k
     const int ck = tid % 8;
     if (ck * 8 >= nch) return;
+    const long long img = (long long)b * Hg * Wg;
     for (int o = tid / 8; o < DW_TY * DW_TX; o += DW_THREADS / 8) {
         const int ly = o / DW_TX, lx = o % DW_TX;
         const int y = y0 + ly, x = x0 + lx;
@@ -256,9 +264,9 @@ dwconv_glu(const __nv_bfloat16* __restrict__ U, const float* __restrict__ Kdw, i
         for (int dy = 0; dy < 3; ++dy) {
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-                const uint8_t* row = dsm + (size_t)((ly + dy) * (DW_TX + 2) + (lx + dx)) * DW_ROW_BYTES;
-                const uint4 va = *reinterpret_cast<const uint4*>(row + ck * 16);
-                const uint4 vg = *reinterpret_cast<const uint4*>(row + 128 + ck * 16);
+                const size_t off = (size_t)((ly + dy) * (DW_TX + 2) + (lx + dx)) * (DW_CH * 2) + ck * 16;
+                const uint4 va = *reinterpret_cast<const uint4*>(dsm + off);
+                const uint4 vg = *reinterpret_cast<const uint4*>(dsm + DW_HALF_BYTES + off);
                 const float* ta = taps + (dy * 3 + dx) * (2 * DW_CH) + ck * 8;
                 const float* tg = ta + DW_CH;
                 const uint32_t wa[4] = {va.x, va.y, va.z, va.w};

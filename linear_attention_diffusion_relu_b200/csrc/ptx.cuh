@@ -100,6 +100,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
+// 4-D tiled bulk-tensor load (no swizzle here), completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, uint64_t* bar,
+                                            int c, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        :: "r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 // An L2 policy that marks lines as first to evict (for inputs read once).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
