@@ -249,48 +249,69 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Kd
     }
     __syncthreads();
     if (!*loaded) return;
-    // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8, tokens tid / 8 + 32 k
+    // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8 and the
+    // tokens tid / 8 + 32 k, taken two at a time so that each tap's 16 weights
+    // (four 16-byte loads) serve two tokens
     const int ck = tid % 8;
     if (ck * 8 >= nch) return;
     const long long img = (long long)b * Hg * Wg;
-    for (int o = tid / 8; o < DW_TY * DW_TX; o += DW_THREADS / 8) {
-        const int ly = o / DW_TX, lx = o % DW_TX;
-        const int y = y0 + ly, x = x0 + lx;
-        if (y >= Hg || x >= Wg) continue;
-        float a[8], g[8];
+    for (int o0 = tid / 8; o0 < DW_TY * DW_TX; o0 += 2 * (DW_THREADS / 8)) {
+        int ly[2], lx[2];
+        bool live[2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a[j] = g[j] = 0.0f;
+        for (int p = 0; p < 2; ++p) {
+            const int o = o0 + p * (DW_THREADS / 8);
+            ly[p] = o / DW_TX;
+            lx[p] = o % DW_TX;
+            live[p] = o < DW_TY * DW_TX && y0 + ly[p] < Hg && x0 + lx[p] < Wg;
+        }
+        float a[2][8], g[2][8];
 #pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[p][j] = g[p][j] = 0.0f;
+#pragma unroll 1
         for (int dy = 0; dy < 3; ++dy) {
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-                const size_t off = (size_t)((ly + dy) * (DW_TX + 2) + (lx + dx)) * (DW_CH * 2) + ck * 16;
-                const uint4 va = *reinterpret_cast<const uint4*>(dsm + off);
-                const uint4 vg = *reinterpret_cast<const uint4*>(dsm + DW_HALF_BYTES + off);
-                const float* ta = taps + (dy * 3 + dx) * (2 * DW_CH) + ck * 8;
-                const float* tg = ta + DW_CH;
-                const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-                const uint32_t wg[4] = {vg.x, vg.y, vg.z, vg.w};
+                const float4* tp = reinterpret_cast<const float4*>(taps + (dy * 3 + dx) * (2 * DW_CH) + ck * 8);
+                const float4 ta0 = tp[0], ta1 = tp[1];                  // value channels
+                const float4 tg0 = tp[DW_CH / 4], tg1 = tp[DW_CH / 4 + 1];   // gate channels
+                const float ta[8] = {ta0.x, ta0.y, ta0.z, ta0.w, ta1.x, ta1.y, ta1.z, ta1.w};
+                const float tg[8] = {tg0.x, tg0.y, tg0.z, tg0.w, tg1.x, tg1.y, tg1.z, tg1.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 fa = bf16x2_to_float2(wa[j]);
-                    const float2 fg = bf16x2_to_float2(wg[j]);
-                    a[2 * j] = fmaf(fa.x, ta[2 * j], a[2 * j]);
-                    a[2 * j + 1] = fmaf(fa.y, ta[2 * j + 1], a[2 * j + 1]);
-                    g[2 * j] = fmaf(fg.x, tg[2 * j], g[2 * j]);
-                    g[2 * j + 1] = fmaf(fg.y, tg[2 * j + 1], g[2 * j + 1]);
+                for (int p = 0; p < 2; ++p) {
+                    const size_t off = (size_t)((min(ly[p], DW_TY - 1) + dy) * (DW_TX + 2) + (lx[p] + dx)) *
+                                       (DW_CH * 2) + ck * 16;
+                    const uint4 va = *reinterpret_cast<const uint4*>(dsm + off);
+                    const uint4 vg = *reinterpret_cast<const uint4*>(dsm + DW_HALF_BYTES + off);
+                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+                    const uint32_t wg[4] = {vg.x, vg.y, vg.z, vg.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 fa = bf16x2_to_float2(wa[j]);
+                        const float2 fg = bf16x2_to_float2(wg[j]);
+                        a[p][2 * j] = fmaf(fa.x, ta[2 * j], a[p][2 * j]);
+                        a[p][2 * j + 1] = fmaf(fa.y, ta[2 * j + 1], a[p][2 * j + 1]);
+                        g[p][2 * j] = fmaf(fg.x, tg[2 * j], g[p][2 * j]);
+                        g[p][2 * j + 1] = fmaf(fg.y, tg[2 * j + 1], g[p][2 * j + 1]);
+                    }
                 }
             }
         }
-        float z[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) z[j] = a[j] / (1.0f + __expf(-g[j]));   // a * sigmoid(g)
-        uint4 out;
-        out.x = float2_to_bf16x2(z[0], z[1]);
-        out.y = float2_to_bf16x2(z[2], z[3]);
-        out.z = float2_to_bf16x2(z[4], z[5]);
-        out.w = float2_to_bf16x2(z[6], z[7]);
-        *reinterpret_cast<uint4*>(Z + (img + (long long)y * Wg + x) * Ch + c0 + ck * 8) = out;
+        for (int p = 0; p < 2; ++p) {
+            if (!live[p]) continue;
+            float z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) z[j] = a[p][j] / (1.0f + __expf(-g[p][j]));   // a * sigmoid(g)
+            uint4 out;
+            out.x = float2_to_bf16x2(z[0], z[1]);
+            out.y = float2_to_bf16x2(z[2], z[3]);
+            out.z = float2_to_bf16x2(z[4], z[5]);
+            out.w = float2_to_bf16x2(z[6], z[7]);
+            *reinterpret_cast<uint4*>(Z + (img + (long long)(y0 + ly[p]) * Wg + (x0 + lx[p])) * Ch + c0 + ck * 8) = out;
+        }
     }
 }
 
