@@ -191,31 +191,45 @@ gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 // channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). Two
 // TMA loads bring the tile plus a one-token halo of each half into shared
 // memory ([row][column][64 channels], zeros outside the grid: the load starts
-// at column x0-1 and row y0-1); the 128 channels' taps go beside them. Each
-// thread then computes 8 outputs of one 8-channel chunk: for each of the 9
-// taps (order dy, dx) it reads 16 bytes of a and of g of the neighbour and
-// accumulates in fp32; Z = a * sigmoid(g) is stored as 8 bf16 (8 lanes = one
-// token's 128 bytes).
-// U (tensor map): (B, Hg, Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z: (B, Hg*Wg, Ch) bf16.
+// at column x0-1 and row y0-1). Lane l owns channels 2l and 2l+1 of both
+// halves, with their 2 x 2 x 9 fp32 taps in registers; warp w owns one output
+// row and a strip of DW_SX columns, along which it slides a 3 x 3 window of
+// unpacked values: each output column loads only the window's new column
+// (3 rows x 2 halves, 4 bytes per lane, one 128-byte line per warp) and
+// accumulates the 9 taps of both channels with packed fp32x2 FMAs. Then
+// Z = a * sigmoid(g) as bf16x2, kept in registers until every warp is done
+// with the input tile, written over it ([row][column][64 channels]) and
+// stored with one TMA store, which leaves out what lies outside the grid or
+// past the last channel.
+// U (tensor map): (B, Hg, Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z (tensor
+// map): (B, Hg, Wg, Ch) bf16.
 constexpr int DW_TY = 4;                        // grid rows per CTA
 constexpr int DW_TX = 64;                       // grid columns per CTA
+constexpr int DW_SX = 32;                       // columns per warp strip
 constexpr int DW_CH = 64;                       // channels of each half per CTA
 constexpr int DW_THREADS = 256;
-constexpr int DW_HALF_BYTES = (DW_TY + 2) * (DW_TX + 2) * DW_CH * 2;   // one half's box: 50,688 B
-constexpr int DW_TAPS_OFF = 2 * DW_HALF_BYTES;
-constexpr int DW_BAR_OFF = DW_TAPS_OFF + 2 * DW_CH * 9 * 4;
+constexpr int DW_ROW_BYTES = (DW_TX + 2) * DW_CH * 2;                  // one halo row of one half
+constexpr int DW_HALF_BYTES = (DW_TY + 2) * DW_ROW_BYTES;              // one half's box: 50,688 B
+constexpr int DW_BAR_OFF = 2 * DW_HALF_BYTES;
 constexpr int DW_SMEM = DW_BAR_OFF + 16 + 128;  // barrier, flag, alignment slack
+static_assert(DW_TY * (DW_TX / DW_SX) == DW_THREADS / 32, "one strip per warp");
+static_assert(DW_TY * DW_TX * DW_CH * 2 <= DW_HALF_BYTES, "the output tile fits over the value half");
 
-__global__ void __launch_bounds__(DW_THREADS)
-dwconv_glu(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Kdw, int B, int Hg, int Wg, int Ch,
-           __nv_bfloat16* __restrict__ Z)
+__device__ __forceinline__ float2 bf16x2_unpack(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+__global__ void __launch_bounds__(DW_THREADS, 2)
+dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmZ,
+           const float* __restrict__ Kdw, int Hg, int Wg, int Ch)
 {
     extern __shared__ uint8_t dsm_raw[];
     uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
-    float* taps = reinterpret_cast<float*>(dsm + DW_TAPS_OFF);     // [tap][128 ch]
     uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + DW_BAR_OFF);
     int* loaded = reinterpret_cast<int*>(dsm + DW_BAR_OFF + 8);
     const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int tiles_x = (Wg + DW_TX - 1) / DW_TX;
     const int tiles_y = (Hg + DW_TY - 1) / DW_TY;
     const int c0 = blockIdx.x * DW_CH;                       // first channel of the group (each half)
@@ -234,11 +248,18 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Kd
         ptx::tma_load_4d(dsm, &tmU, bar, c0, x0 - 1, y0 - 1, b);
         ptx::tma_load_4d(dsm + DW_HALF_BYTES, &tmU, bar, Ch + c0, x0 - 1, y0 - 1, b);
     }
-    // taps: entry t * 128 + j, j < 64 the value half, j >= 64 the gate half
-    for (int e = tid; e < 2 * DW_CH * 9; e += DW_THREADS) {
-        const int t = e / (2 * DW_CH), j = e % (2 * DW_CH);
-        const int c = j < DW_CH ? c0 + j : Ch + c0 + (j - DW_CH);
-        taps[e] = (j % DW_CH) < nch ? Kdw[(size_t)c * 9 + t] : 0.0f;
+    // this lane's channel pair and its taps (tap t = 3 dy + dx), both halves;
+    // lanes past the group's channels compute zeros that the store leaves out
+    const int cp = 2 * lane;
+    const bool ch_live = cp < nch;
+    float2 wa[9], wg[9];
+#pragma unroll
+    for (int t = 0; t < 9; ++t) {
+        wa[t] = ch_live ? make_float2(__ldg(Kdw + (size_t)(c0 + cp) * 9 + t), __ldg(Kdw + (size_t)(c0 + cp + 1) * 9 + t))
+                        : make_float2(0.0f, 0.0f);
+        wg[t] = ch_live ? make_float2(__ldg(Kdw + (size_t)(Ch + c0 + cp) * 9 + t),
+                                      __ldg(Kdw + (size_t)(Ch + c0 + cp + 1) * 9 + t))
+                        : make_float2(0.0f, 0.0f);
     }
     // thread 0 waits for the tile (bounded) and tells the others, so the
     // decision to go on is the same for every thread
@@ -249,69 +270,53 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Kd
     }
     __syncthreads();
     if (!*loaded) return;
-    // outputs: DW_TY * DW_TX tokens x 8 chunks; thread -> chunk tid % 8 and the
-    // tokens tid / 8 + 32 k, taken two at a time so that each tap's 16 weights
-    // (four 16-byte loads) serve two tokens
-    const int ck = tid % 8;
-    if (ck * 8 >= nch) return;
-    const long long img = (long long)b * Hg * Wg;
-    for (int o0 = tid / 8; o0 < DW_TY * DW_TX; o0 += 2 * (DW_THREADS / 8)) {
-        int ly[2], lx[2];
-        bool live[2];
+    constexpr int STRIPS = DW_TX / DW_SX;
+    const int ly = warp / STRIPS;                           // output row y0 + ly = halo row ly + 1
+    const int sx = (warp % STRIPS) * DW_SX;                 // first output column of the strip
+    // halo row ly + r, halo column sx + j holds grid (y0 + ly - 1 + r, x0 + sx - 1 + j)
+    const uint8_t* base = dsm + (size_t)ly * DW_ROW_BYTES + (size_t)sx * (DW_CH * 2) + lane * 4;
+    float2 win[2][3][3];                                    // [half][row][column slot]
+    auto load_col = [&](int j, int slot) {
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int o = o0 + p * (DW_THREADS / 8);
-            ly[p] = o / DW_TX;
-            lx[p] = o % DW_TX;
-            live[p] = o < DW_TY * DW_TX && y0 + ly[p] < Hg && x0 + lx[p] < Wg;
+        for (int r = 0; r < 3; ++r) {
+            const uint8_t* q = base + r * DW_ROW_BYTES + j * (DW_CH * 2);
+            win[0][r][slot] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q));
+            win[1][r][slot] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q + DW_HALF_BYTES));
         }
-        float a[2][8], g[2][8];
+    };
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint32_t zo[DW_SX];
+    load_col(0, 0);
+    load_col(1, 1);
 #pragma unroll
-        for (int p = 0; p < 2; ++p)
+    for (int k = 0; k < DW_SX; ++k) {
+        load_col(k + 2, (k + 2) % 3);
+        float2 a = make_float2(0.0f, 0.0f), g = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a[p][j] = g[p][j] = 0.0f;
-#pragma unroll 1
         for (int dy = 0; dy < 3; ++dy) {
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-                const float4* tp = reinterpret_cast<const float4*>(taps + (dy * 3 + dx) * (2 * DW_CH) + ck * 8);
-                const float4 ta0 = tp[0], ta1 = tp[1];                  // value channels
-                const float4 tg0 = tp[DW_CH / 4], tg1 = tp[DW_CH / 4 + 1];   // gate channels
-                const float ta[8] = {ta0.x, ta0.y, ta0.z, ta0.w, ta1.x, ta1.y, ta1.z, ta1.w};
-                const float tg[8] = {tg0.x, tg0.y, tg0.z, tg0.w, tg1.x, tg1.y, tg1.z, tg1.w};
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const size_t off = (size_t)((min(ly[p], DW_TY - 1) + dy) * (DW_TX + 2) + (lx[p] + dx)) *
-                                       (DW_CH * 2) + ck * 16;
-                    const uint4 va = *reinterpret_cast<const uint4*>(dsm + off);
-                    const uint4 vg = *reinterpret_cast<const uint4*>(dsm + DW_HALF_BYTES + off);
-                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-                    const uint32_t wg[4] = {vg.x, vg.y, vg.z, vg.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 fa = bf16x2_to_float2(wa[j]);
-                        const float2 fg = bf16x2_to_float2(wg[j]);
-                        a[p][2 * j] = fmaf(fa.x, ta[2 * j], a[p][2 * j]);
-                        a[p][2 * j + 1] = fmaf(fa.y, ta[2 * j + 1], a[p][2 * j + 1]);
-                        g[p][2 * j] = fmaf(fg.x, tg[2 * j], g[p][2 * j]);
-                        g[p][2 * j + 1] = fmaf(fg.y, tg[2 * j + 1], g[p][2 * j + 1]);
-                    }
-                }
+                a = __ffma2_rn(win[0][dy][(k + dx) % 3], wa[dy * 3 + dx], a);
+                g = __ffma2_rn(win[1][dy][(k + dx) % 3], wg[dy * 3 + dx], g);
             }
         }
+        // sigmoid(g) = 1 / (1 + 2^(-g log2 e))
+        const float2 t = __fmul2_rn(g, make_float2(-kLog2e, -kLog2e));
+        const float2 d = __fadd2_rn(make_float2(ptx::ex2_approx(t.x), ptx::ex2_approx(t.y)), make_float2(1.0f, 1.0f));
+        const float2 z = __fmul2_rn(a, make_float2(ptx::rcp_approx(d.x), ptx::rcp_approx(d.y)));
+        zo[k] = float2_to_bf16x2(z.x, z.y);
+    }
+    __syncthreads();                                        // every warp is done with the input tile
+    // output tile [row][column][64 channels] over the value half
+    uint8_t* zt = dsm + ((size_t)ly * DW_TX + sx) * (DW_CH * 2) + lane * 4;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            if (!live[p]) continue;
-            float z[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) z[j] = a[p][j] / (1.0f + __expf(-g[p][j]));   // a * sigmoid(g)
-            uint4 out;
-            out.x = float2_to_bf16x2(z[0], z[1]);
-            out.y = float2_to_bf16x2(z[2], z[3]);
-            out.z = float2_to_bf16x2(z[4], z[5]);
-            out.w = float2_to_bf16x2(z[6], z[7]);
-            *reinterpret_cast<uint4*>(Z + (img + (long long)(y0 + ly[p]) * Wg + (x0 + lx[p])) * Ch + c0 + ck * 8) = out;
-        }
+    for (int k = 0; k < DW_SX; ++k) *reinterpret_cast<uint32_t*>(zt + k * (DW_CH * 2)) = zo[k];
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        ptx::tma_store_4d(&tmZ, dsm, c0, x0, y0, b);
+        ptx::bulk_commit_group();
+        ptx::bulk_wait_group<0>();                          // written before the CTA retires
     }
 }
 

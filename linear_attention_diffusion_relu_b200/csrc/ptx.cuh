@@ -110,6 +110,18 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
+// 2^x and 1/x on the special-function unit (approximate, subnormals flushed)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // An L2 policy that marks lines as first to evict (for inputs read once).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
@@ -133,6 +145,14 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_
     asm volatile(
         "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
         :: "l"(tmap), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
+// 4-D tiled bulk-tensor store from this CTA's shared memory (bulk-group
+// completion). Parts of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const void* tmap, const void* smem_src, int c, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        :: "l"(tmap), "r"(smem_u32(smem_src)), "r"(c), "r"(x), "r"(y), "r"(z) : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit_group() {

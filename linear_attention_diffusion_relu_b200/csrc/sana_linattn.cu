@@ -725,31 +725,35 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
     // 3x3 depthwise over the grid and the GLU, fused
     static std::atomic<uint64_t> dw_smem_set{0};
     if ((st = ensure_smem(sana::tc::dwconv_glu, sana::tc::DW_SMEM, dw_smem_set)) != SANA_LA_OK) return st;
-    // U as {2 Ch, Wg, Hg, B}; a box is 64 channels x (64 + 2) columns x (4 + 2) rows
-    CUtensorMap tmU;
+    // U as {2 Ch, Wg, Hg, B}: a load box is 64 channels x (DW_TX + 2) columns x
+    // (DW_TY + 2) rows; Z as {Ch, Wg, Hg, B}: a store box is 64 x DW_TX x DW_TY
+    CUtensorMap tmU, tmZ;
     {
         auto encode = tensor_map_encoder();
         if (encode == nullptr) return SANA_LA_ERR_CUDA;
-        cuuint64_t dims[4] = {(cuuint64_t)2 * Ch, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
-        cuuint64_t strides[3] = {(cuuint64_t)2 * Ch * 2, (cuuint64_t)2 * Ch * 2 * Wg,
-                                 (cuuint64_t)2 * Ch * 2 * Wg * Hg};
-        cuuint32_t box[4] = {(cuuint32_t)sana::tc::DW_CH, (cuuint32_t)(sana::tc::DW_TX + 2),
-                             (cuuint32_t)(sana::tc::DW_TY + 2), 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
-        CUresult r = encode(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, U, dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
-            return SANA_LA_ERR_CUDA;
+        for (int which = 0; which < 2; ++which) {
+            const cuuint64_t ch = which == 0 ? (cuuint64_t)2 * Ch : (cuuint64_t)Ch;
+            cuuint64_t dims[4] = {ch, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
+            cuuint64_t strides[3] = {ch * 2, ch * 2 * Wg, ch * 2 * Wg * Hg};
+            const int halo = which == 0 ? 2 : 0;
+            cuuint32_t box[4] = {(cuuint32_t)sana::tc::DW_CH, (cuuint32_t)(sana::tc::DW_TX + halo),
+                                 (cuuint32_t)(sana::tc::DW_TY + halo), 1};
+            CUresult r = encode(which == 0 ? &tmU : &tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                                which == 0 ? U : Z, dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+                return SANA_LA_ERR_CUDA;
+            }
         }
     }
     const long long dw_tiles = (long long)B * cdiv(Hg, sana::tc::DW_TY) * cdiv(Wg, sana::tc::DW_TX);
     if (dw_tiles > 65535) return SANA_LA_ERR_UNSUPPORTED;
     const dim3 dw_grid((unsigned)cdiv(Ch, sana::tc::DW_CH), (unsigned)dw_tiles);
     if ((st = launch(sana::tc::dwconv_glu, dw_grid, dim3(sana::tc::DW_THREADS), sana::tc::DW_SMEM, s,
-                     false, "dwconv_glu", tmU, Kdw, B, Hg, Wg, Ch,
-                     static_cast<__nv_bfloat16*>(Z))) != SANA_LA_OK)
+                     false, "dwconv_glu", tmU, tmZ, Kdw, Hg, Wg, Ch)) != SANA_LA_OK)
         return st;
     // 1x1 project: Y = Z W2^T
     return launch_gemm(Z, W2, Y, M, C, Ch, C, s);

@@ -45,7 +45,9 @@ def _intermediates(ws, B, N, Ch):
     return U, Z
 
 
-SHAPES = [(1, 4, 4, 64, 32), (2, 16, 24, 256, 320), (1, 32, 32, 1152, 2880), (2, 7, 5, 136, 24)]
+# (1, 9, 70, 128, 104): a last channel group of 40, a 6-column and a 1-row tile
+SHAPES = [(1, 4, 4, 64, 32), (2, 16, 24, 256, 320), (1, 32, 32, 1152, 2880), (2, 7, 5, 136, 24),
+          (1, 9, 70, 128, 104)]
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}G{}x{}C{}Ch{}".format(*s))
