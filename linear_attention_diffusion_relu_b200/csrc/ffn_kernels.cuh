@@ -186,6 +186,211 @@ gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     kernel_epilogue(ctl, tid);
 }
 
+// ======================================================= GEMM, CTA pairs ===
+// The same product on a cluster of two CTAs (the two SMs of a TPC): a tile is
+// 256 rows of A x 256 rows of B; CTA r of the pair loads A rows 128r .. and B
+// rows 128r .. of it into its own shared memory, and the even CTA issues
+// tcgen05.mma.cta_group::2 with M = 256, which reads both CTAs' operands and
+// leaves rows 128r .. of the product in CTA r's TMEM. Per CTA that halves the
+// B bytes staged and read per flop against the one-CTA kernel.
+// Both CTAs' loads complete on the even CTA's full barrier (it expects the
+// pair's bytes); its UMMA commits arrive on the empty and accumulator barriers
+// of both CTAs; the odd CTA's epilogue warps release the accumulator on the
+// even CTA's barrier. The pair ends with a bounded handshake before TMEM is
+// freed, so neither CTA leaves while the other may still use its memory.
+constexpr int G2_TILE_M = 256;
+constexpr int G2_TILE_N = 256;
+constexpr int G2_HALF_BYTES = 128 * kBoxBytesRow;          // 128 rows x 64 bf16
+constexpr int G2_STAGE_BYTES = 2 * G2_HALF_BYTES;          // this CTA's A half + B half
+constexpr int G2_STAGES = 6;
+using Gemm2Map = SmemMap<G2_STAGES * G2_STAGE_BYTES>;
+
+struct Gemm2Bars {
+    uint64_t* full;        // [G2_STAGES] both CTAs' tiles landed (even CTA's copy used)
+    uint64_t* empty;       // [G2_STAGES] the pair's UMMAs have read the stage
+    uint64_t* acc_full;    // [2] a tile's accumulator complete
+    uint64_t* acc_empty;   // [2] read by the worker warps of both CTAs (even CTA's copy used)
+    uint64_t* mma_done;
+    uint64_t* pair_done;   // the other CTA of the pair has finished
+    __device__ void init() const {
+        for (int s = 0; s < G2_STAGES; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int j = 0; j < 2; ++j) {
+            ptx::mbar_init(&acc_full[j], 1);
+            ptx::mbar_init(&acc_empty[j], 2 * kWorkerWarps);
+        }
+        ptx::mbar_init(mma_done, 1);
+        ptx::mbar_init(pair_done, 1);
+    }
+};
+
+__device__ __forceinline__ Gemm2Bars gemm2_bars(uint64_t* b) {
+    uint64_t* a = b + 2 * G2_STAGES;
+    return Gemm2Bars{b, b + G2_STAGES, a, a + 2, a + 4, a + 5};
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_bf16_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const GemmParams p, __nv_bfloat16* __restrict__ C)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    const Gemm2Bars bar = gemm2_bars(reinterpret_cast<uint64_t*>(smem + Gemm2Map::BAR_OFF));
+    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Gemm2Map::CTL_OFF);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    volatile int* abort = &ctl->abort;
+    uint32_t* err = &g_device_error;
+    if (tid == 0) {
+        ctl->abort = 0;
+        bar.init();
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+        ptx::tmem_relinquish_pair();
+    }
+    if (tid == kProducerWarp * 32) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+    }
+    // both CTAs' barriers initialised and TMEM allocated before either uses
+    // the other's
+    ptx::tc_fence_before_sync();
+    ptx::cluster_sync();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const int pair = (int)blockIdx.x / 2;
+    const int npairs = (int)gridDim.x / 2;
+    const int tiles = p.mtiles * p.ntiles;
+    const int ntl = pair < tiles ? (tiles - pair + npairs - 1) / npairs : 0;
+    auto tile_of = [&](int i, int& m0, int& n0) {
+        const int t = pair + i * npairs;
+        m0 = (t / p.ntiles) * G2_TILE_M;
+        n0 = (t % p.ntiles) * G2_TILE_N;
+    };
+    auto stage_ptr = [&](int s) { return smem + (size_t)s * G2_STAGE_BYTES; };
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            const uint32_t full0 = ptx::mapa_shared(&bar.full[0], 0);    // the even CTA's full[0]
+            int k = 0, issued = 0;
+            bool ok = true;
+            for (int i = 0; i < ntl && ok; ++i) {
+                int m0, n0;
+                tile_of(i, m0, n0);
+                for (int kb = 0; kb < p.kblocks; ++kb, ++k) {
+                    const int s = k % G2_STAGES;
+                    if (!ptx::mbar_wait(&bar.empty[s], ((k / G2_STAGES) & 1) ^ 1, abort, err)) { ok = false; break; }
+                    if (leader) ptx::mbar_arrive_expect_tx(&bar.full[s], 2 * G2_STAGE_BYTES);
+                    uint8_t* st = stage_ptr(s);
+                    const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
+                    ptx::tma_load_3d_pair(st, &tmA, fb, kb * 64, m0 + (int)rank * 128, 0);
+                    ptx::tma_load_3d_pair(st + G2_HALF_BYTES, &tmB, fb, kb * 64, n0 + (int)rank * 128, 0);
+                    issued = k + 1;
+                }
+            }
+            // every issued load must land before the CTA may leave: the even
+            // CTA sees them on its full barriers; the odd CTA's stages are
+            // released (empty) only after the pair's UMMAs have read them
+            for (int j = (issued > G2_STAGES ? issued - G2_STAGES : 0); j < issued; ++j) {
+                if (leader) ptx::mbar_wait(&bar.full[j % G2_STAGES], (j / G2_STAGES) & 1, nullptr, err);
+                else ptx::mbar_wait(&bar.empty[j % G2_STAGES], (j / G2_STAGES) & 1, nullptr, err);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(G2_TILE_M, G2_TILE_N, 0, 0);
+            int k = 0;
+            bool ok = true;
+            for (int i = 0; i < ntl && ok; ++i) {
+                const int buf = i & 1;
+                if (!ptx::mbar_wait(&bar.acc_empty[buf], ((i >> 1) & 1) ^ 1, abort, err)) break;
+                ptx::tc_fence_after_sync();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * G2_TILE_N);
+                for (int kb = 0; kb < p.kblocks; ++kb, ++k) {
+                    const int s = k % G2_STAGES;
+                    if (!ptx::mbar_wait(&bar.full[s], (k / G2_STAGES) & 1, abort, err)) { ok = false; break; }
+                    ptx::tc_fence_after_sync();
+                    const uint32_t a0 = ptx::smem_u32(stage_ptr(s));
+                    const uint32_t b0 = a0 + G2_HALF_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a = ptx::smem_desc(a0 + kk * 32, 16, 1024, ptx::kLayoutSW128);
+                        const uint64_t b = ptx::smem_desc(b0 + kk * 32, 16, 1024, ptx::kLayoutSW128);
+                        ptx::umma_f16_ss_pair(d_tmem, a, b, idesc, (kb | kk) != 0);
+                    }
+                    ptx::umma_commit_pair(&bar.empty[s], 0x3);
+                }
+                if (ok) ptx::umma_commit_pair(&bar.acc_full[buf], 0x3);
+            }
+            ptx::umma_commit_pair(bar.mma_done, 0x1);
+            ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
+        }
+    } else {
+        // workers: warp w reads TMEM lanes 32*(w%4).. (its 32 rows of this
+        // CTA's 128) and columns 128*(w/4).. of the tile
+        const int r = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        for (int i = 0; i < ntl; ++i) {
+            const int buf = i & 1;
+            if (!warp_wait(&bar.acc_full[buf], (i >> 1) & 1, abort, err)) break;
+            ptx::tc_fence_after_sync();
+            float v[128];
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                ptx::tmem_ld32(lane_base + (uint32_t)(buf * G2_TILE_N + half * 128 + c * 32), v + c * 32);
+            ptx::tc_fence_before_sync();
+            if (leader) {
+                warp_arrive(&bar.acc_empty[buf]);
+            } else {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(&bar.acc_empty[buf], 0));
+            }
+            int m0, n0;
+            tile_of(i, m0, n0);
+            const int m = m0 + (int)rank * 128 + r;
+            if (m < p.M) {
+                __nv_bfloat16* row = C + (size_t)m * p.ldc;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int n = n0 + half * 128 + q * 8;
+                    if (n < p.N) {
+                        const float* x = v + q * 8;
+                        uint4 w;
+                        w.x = float2_to_bf16x2(x[0], x[1]);
+                        w.y = float2_to_bf16x2(x[2], x[3]);
+                        w.z = float2_to_bf16x2(x[4], x[5]);
+                        w.w = float2_to_bf16x2(x[6], x[7]);
+                        *reinterpret_cast<uint4*>(row + n) = w;
+                    }
+                }
+            }
+        }
+    }
+    // the pair: each CTA tells the other it is done (bounded wait), then both
+    // free the shared TMEM allocation
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        ptx::mbar_arrive_cluster(ptx::mapa_shared(bar.pair_done, rank ^ 1u));
+        ptx::mbar_wait(bar.pair_done, 0, nullptr, err);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
 // ====================================================== depthwise + GLU ===
 // A CTA takes one batch image's tile of DW_TY grid rows x DW_TX columns and 64
 // channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). Two
@@ -210,7 +415,8 @@ constexpr int DW_CH = 64;                       // channels of each half per CTA
 constexpr int DW_THREADS = 256;
 constexpr int DW_ROW_BYTES = (DW_TX + 2) * DW_CH * 2;                  // one halo row of one half
 constexpr int DW_HALF_BYTES = (DW_TY + 2) * DW_ROW_BYTES;              // one half's box: 50,688 B
-constexpr int DW_BAR_OFF = 2 * DW_HALF_BYTES;
+constexpr int DW_TAPS_OFF = 2 * DW_HALF_BYTES;                        // fp32 [half][tap][64 channels]
+constexpr int DW_BAR_OFF = DW_TAPS_OFF + 2 * 9 * DW_CH * 4;
 constexpr int DW_SMEM = DW_BAR_OFF + 16 + 128;  // barrier, flag, alignment slack
 static_assert(DW_TY * (DW_TX / DW_SX) == DW_THREADS / 32, "one strip per warp");
 static_assert(DW_TY * DW_TX * DW_CH * 2 <= DW_HALF_BYTES, "the output tile fits over the value half");
@@ -248,18 +454,14 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUte
         ptx::tma_load_4d(dsm, &tmU, bar, c0, x0 - 1, y0 - 1, b);
         ptx::tma_load_4d(dsm + DW_HALF_BYTES, &tmU, bar, Ch + c0, x0 - 1, y0 - 1, b);
     }
-    // this lane's channel pair and its taps (tap t = 3 dy + dx), both halves;
-    // lanes past the group's channels compute zeros that the store leaves out
-    const int cp = 2 * lane;
-    const bool ch_live = cp < nch;
-    float2 wa[9], wg[9];
-#pragma unroll
-    for (int t = 0; t < 9; ++t) {
-        wa[t] = ch_live ? make_float2(__ldg(Kdw + (size_t)(c0 + cp) * 9 + t), __ldg(Kdw + (size_t)(c0 + cp + 1) * 9 + t))
-                        : make_float2(0.0f, 0.0f);
-        wg[t] = ch_live ? make_float2(__ldg(Kdw + (size_t)(Ch + c0 + cp) * 9 + t),
-                                      __ldg(Kdw + (size_t)(Ch + c0 + cp + 1) * 9 + t))
-                        : make_float2(0.0f, 0.0f);
+    // the group's taps, read in address order (each half's 64 x 9 block is
+    // contiguous) into [half][tap][channel]; zeros past the group's channels
+    float* taps = reinterpret_cast<float*>(dsm + DW_TAPS_OFF);
+    for (int e = tid; e < 2 * DW_CH * 9; e += DW_THREADS) {
+        const int half = e / (DW_CH * 9), j = e % (DW_CH * 9);
+        const int ch = j / 9, t = j % 9;
+        taps[(half * 9 + t) * DW_CH + ch] =
+            ch < nch ? __ldg(Kdw + (size_t)(half * Ch + c0) * 9 + j) : 0.0f;
     }
     // thread 0 waits for the tile (bounded) and tells the others, so the
     // decision to go on is the same for every thread
@@ -270,6 +472,15 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUte
     }
     __syncthreads();
     if (!*loaded) return;
+    // this lane's channel pair and its taps (tap t = 3 dy + dx), both halves;
+    // lanes past the group's channels compute zeros that the store leaves out
+    const int cp = 2 * lane;
+    float2 wa[9], wg[9];
+#pragma unroll
+    for (int t = 0; t < 9; ++t) {
+        wa[t] = *reinterpret_cast<const float2*>(taps + t * DW_CH + cp);
+        wg[t] = *reinterpret_cast<const float2*>(taps + (9 + t) * DW_CH + cp);
+    }
     constexpr int STRIPS = DW_TX / DW_SX;
     const int ly = warp / STRIPS;                           // output row y0 + ly = halo row ly + 1
     const int sx = (warp % STRIPS) * DW_SX;                 // first output column of the strip

@@ -529,7 +529,34 @@ sana_la_status check_ffn(int B, int Hg, int Wg, int C, int Ch) {
 }
 
 // C (M x N, row stride ldc) = A (M x K) B^T (B is N x K), bf16 in and out
+// C = A B^T on CTA pairs (256 x 256 tiles, tcgen05.mma.cta_group::2) or, with
+// kGemmPairs = false, on single CTAs (128 x 256 tiles).
+constexpr bool kGemmPairs = true;
+
+sana_la_status launch_gemm_pairs(const void* A, const void* Bm, void* C, int M, int N, int K, int ldc,
+                                 cudaStream_t s) {
+    static std::atomic<uint64_t> smem_set{0};
+    CUtensorMap tmA, tmB;
+    sana_la_status st;
+    if ((st = make_tmap(&tmA, A, 1, M, 1, K, 128)) != SANA_LA_OK) return st;
+    if ((st = make_tmap(&tmB, Bm, 1, N, 1, K, 128)) != SANA_LA_OK) return st;
+    if ((st = ensure_smem(sana::tc::gemm_bf16_tc2, sana::tc::Gemm2Map::BYTES, smem_set)) != SANA_LA_OK) return st;
+    sana::tc::GemmParams gp{};
+    gp.M = M;
+    gp.N = N;
+    gp.K = K;
+    gp.ldc = ldc;
+    gp.kblocks = (int)cdiv(K, 64);
+    gp.mtiles = (int)cdiv(M, sana::tc::G2_TILE_M);
+    gp.ntiles = (int)cdiv(N, sana::tc::G2_TILE_N);
+    const long long tiles = (long long)gp.mtiles * gp.ntiles;
+    const int pairs = (int)std::min<long long>(tiles, kSMs / 2);
+    return launch(sana::tc::gemm_bf16_tc2, dim3(2 * pairs), dim3(sana::tc::kThreads), sana::tc::Gemm2Map::BYTES, s,
+                  false, "gemm_bf16_tc2", tmA, tmB, gp, static_cast<__nv_bfloat16*>(C));
+}
+
 sana_la_status launch_gemm(const void* A, const void* Bm, void* C, int M, int N, int K, int ldc, cudaStream_t s) {
+    if (kGemmPairs) return launch_gemm_pairs(A, Bm, C, M, N, K, ldc, s);
     static std::atomic<uint64_t> smem_set{0};
     CUtensorMap tmA, tmB;
     sana_la_status st;
