@@ -63,31 +63,54 @@ sana::tc::Sched make_sched(long long S, long long T) {
     q.max_seg = (int)cdiv(S, q.grid);
     q.nblk = 1;
     q.tpb = 0;
+    q.rb = 1;
     return q;
 }
 
-// Block-causal schedule: S slabs of nblk blocks of bt tiles, R CTAs per slab
-// (R divides bt), each taking bt / R tiles of every block.
-sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int R) {
+// Block-causal schedule: S slabs of nblk blocks of bt tiles; a slab's
+// rb * rt CTAs split its blocks rb ways and each block's tiles rt ways (rt
+// divides bt).
+sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int rb, int rt) {
     sana::tc::Sched q{};
     q.S = (int)S;
     q.T = (int)(nblk * bt);
-    q.R = R;
-    q.grid = S <= kSMs ? (int)(S * R) : kSMs;
+    q.R = rb * rt;
+    q.grid = S <= kSMs ? (int)(S * q.R) : kSMs;
     q.nblk = (int)nblk;
-    q.tpb = (int)(bt / R);
-    q.max_seg = (int)(cdiv(S, q.grid) * nblk);
+    q.tpb = (int)(bt / rt);
+    q.rb = rb;
+    q.max_seg = (int)(cdiv(S, q.grid) * cdiv(nblk, rb));
     return q;
 }
 
-// CTAs per slab of the block-causal schedule: the largest divisor of the
-// 128-token tiles per block (hence also of the 64-token ones) that fits
-// S * R <= 148.
-int block_sched_r(long long S, long long tiles128) {
-    if (S > kSMs) return 1;
-    for (long long r = std::min<long long>(kSMs / S, tiles128); r > 1; --r)
-        if (tiles128 % r == 0) return (int)r;
-    return 1;
+// How the CTAs of a slab split a block-causal slab (S slabs, nblk blocks of
+// tiles128 128-token tiles; at most 148 CTAs): the split (rb, rt), rb * rt <=
+// 148 / S and rt dividing tiles128, that minimises the tiles of the busiest
+// CTA plus three tiles' worth for each state it stages (one per block it
+// visits), times 1.06 when rb > 1; ties go to fewer partial states per block
+// (smaller rt). The factor is what reading rb token regions at once instead
+// of one cost on B200: at 16 frames of 256 x 256 tokens (16 blocks of 512
+// tiles, 18 slabs) rb = 8, rt = 1 took 1796 us against 1703 us for rb = 1,
+// rt = 8; at 16 frames of 64 x 64 tokens (16 blocks of 32 tiles, 9 slabs)
+// rb = 16, rt = 1 took 138 us against 198 us for rb = 1, rt = 16.
+struct BlockSplit {
+    int rb, rt;
+};
+BlockSplit block_split(long long S, long long nblk, long long tiles128) {
+    if (S > kSMs) return BlockSplit{1, 1};
+    const long long rmax = kSMs / S;
+    BlockSplit best{1, 1};
+    long long best_cost = -1;
+    for (long long rt = 1; rt <= std::min(rmax, tiles128); ++rt) {
+        if (tiles128 % rt != 0) continue;
+        const long long rb = std::min(nblk, rmax / rt);
+        const long long cost = cdiv(nblk, rb) * (tiles128 / rt + 3) * (rb > 1 ? 106 : 100);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = BlockSplit{(int)rb, (int)rt};
+        }
+    }
+    return best;
 }
 
 // L = 0: the plain forward; L > 0 (a multiple of 128): block-causal with
@@ -107,9 +130,9 @@ Plan make_plan(int B, int N, int H, int d, int L = 0) {
     if (L > 0) {
         nblk = cdiv(N, L);
         const long long tiles128 = L / sana::tc::KA_TILE;
-        const int R = block_sched_r(S, tiles128);
-        p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, R);
-        p.ka.q = make_block_sched(S, nblk, tiles128, R);
+        const BlockSplit sp = block_split(S, nblk, tiles128);
+        p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, sp.rb, sp.rt);
+        p.ka.q = make_block_sched(S, nblk, tiles128, sp.rb, sp.rt);
     } else {
         p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE));
         p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE));
@@ -146,9 +169,9 @@ sana_la_status check_block(int B, int N, int H, int d, int L) {
     const long long G = 128 / d;
     const long long S = (long long)B * cdiv(H, G);
     const long long nblk = cdiv(N, L);
-    const long long R = block_sched_r(S, L / sana::tc::KA_TILE);
-    const long long grid = S <= kSMs ? S * R : kSMs;
-    const long long segs = cdiv(S, grid) * nblk;             // per CTA
+    const BlockSplit sp = block_split(S, nblk, L / sana::tc::KA_TILE);
+    const long long grid = S <= kSMs ? S * sp.rb * sp.rt : kSMs;
+    const long long segs = cdiv(S, grid) * cdiv(nblk, sp.rb);   // per CTA
     const long long per_seg = G * d * (d + 1) * (long long)sizeof(float);
     if (segs > (long long)(kMaxBlockPartialBytes / per_seg) / grid) return SANA_LA_ERR_UNSUPPORTED;
     if (nblk * L > 0x7fffffffLL) return SANA_LA_ERR_UNSUPPORTED;    // padded token coordinates

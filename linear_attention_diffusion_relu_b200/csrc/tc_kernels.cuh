@@ -42,12 +42,14 @@
 // segment and KR adds a slab's segments in ascending CTA order.
 //
 // Block-causal form (blocks of L tokens, L a multiple of 128): the tiles of a
-// slab are padded to whole blocks and R divides the tiles per block, so every
-// CTA takes the same number of tiles, tpb, from each block (tiles past N read
-// as zeros and are not stored). A segment is then one (slab, block) pair:
-// KS writes one partial per (CTA, slab, block), KR turns them into prefix
-// states (ascending blocks, within a block ascending CTA), and KA stages the
-// prefix state of a tile's block.
+// slab are padded to whole blocks, and its R = Rb * Rt CTAs split the blocks
+// first: CTA r takes blocks r % Rb, r % Rb + Rb, ... and, of each, the tiles
+// r / Rb, r / Rb + Rt, ... (Rt divides the tiles per block, so every CTA takes
+// tpb of them; tiles past N read as zeros and are not stored). A segment is
+// then one (slab, block) pair: KS writes one partial per (CTA, slab, block),
+// KR turns them into prefix states (ascending blocks, within a block the Rt
+// partials in ascending r), and KA stages the prefix state of a segment's
+// block once for its tpb tiles.
 // Every mbarrier wait is bounded; a wait that runs out sets an error code and
 // the whole CTA winds down (drains its TMA loads and UMMAs, frees TMEM).
 #pragma once
@@ -153,6 +155,7 @@ struct Sched {
     int max_seg;    // most segments one CTA visits
     int nblk;       // token blocks per slab (1 = not block-causal)
     int tpb;        // block-causal: tiles of one block per CTA (0 otherwise)
+    int rb;         // block-causal: CTAs of a slab that split its blocks (R / rb split each block)
 };
 
 // tiles per segment of CTA c
@@ -161,20 +164,33 @@ __host__ __device__ __forceinline__ int sched_tps(int c, const Sched& q) {
     const int r = c / q.S;
     return (q.T - r + q.R - 1) / q.R;
 }
-// segments of CTA c: its slabs times the blocks of a slab
-__host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
-    return (q.S - c % q.S + q.grid - 1) / q.grid * q.nblk;
+// blocks of one slab that CTA c visits (1 unless block-causal)
+__host__ __device__ __forceinline__ int sched_nb(int c, const Sched& q) {
+    const int rb = (c / q.S) % q.rb;
+    return (q.nblk - rb + q.rb - 1) / q.rb;
 }
-// i-th tile of CTA c -> (slab, tile, segment index); the segment's block is
-// seg % q.nblk. In round k the R CTAs of a slab take tiles kR .. kR + R - 1,
-// CTA r always position r. (Rotating the positions from round to round made
-// every CTA finish the state phase together, but all of them at the time the
-// last position finished before: slower overall, measured on B200.)
+// segments of CTA c: its slabs times the blocks it visits in each
+__host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
+    return (q.S - c % q.S + q.grid - 1) / q.grid * sched_nb(c, q);
+}
+// token block of segment `seg` of CTA c
+__host__ __device__ __forceinline__ int sched_block(int c, int seg, const Sched& q) {
+    return (c / q.S) % q.rb + (seg % sched_nb(c, q)) * q.rb;
+}
+// i-th tile of CTA c -> (slab, tile, segment index). In round k the R CTAs of
+// a slab take tiles kR .. kR + R - 1, CTA r always position r. (Rotating the
+// positions from round to round made every CTA finish the state phase
+// together, but all of them at the time the last position finished before:
+// slower overall, measured on B200.) Block-causal: see the comment at the top.
 __host__ __device__ __forceinline__ void sched_item(int c, int i, int tps, const Sched& q,
                                                     int& slab, int& tile, int& seg) {
     seg = i / tps;
-    slab = c % q.S + seg / q.nblk * q.grid;
-    tile = c / q.S + ((seg % q.nblk) * tps + i % tps) * q.R;
+    const int r = c / q.S;
+    slab = c % q.S + seg / sched_nb(c, q) * q.grid;
+    if (q.tpb > 0)
+        tile = sched_block(c, seg, q) * (q.T / q.nblk) + r / q.rb + (i % tps) * (q.R / q.rb);
+    else
+        tile = r + (i % tps) * q.R;
 }
 
 // ===================================================================== KS ===
@@ -386,10 +402,20 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
 }
 
 // Partial-state slot of segment `seg` of CTA `c` for head hh of the group.
-// A slab's R partials are those of CTAs (slab % grid) + r * S, r = 0 .. R-1,
-// segment slab / grid; they are always added in ascending r.
 __device__ __forceinline__ long long ks_slot(long long c, int seg, int hh, int G, const KsParams& p) {
     return (c * p.q.max_seg + seg) * G + hh;
+}
+// Slot of the first of the R / rb partials of block `blk` of `slab` (those of
+// CTAs (slab % grid) + (blk % rb + t rb) S, t = 0, 1, ...; they are always
+// added in ascending t, ks_block_step slots apart).
+__device__ __forceinline__ long long ks_block_slot(int slab, int blk, int hh, int G, const KsParams& p) {
+    const int rbi = blk % p.q.rb;
+    const long long c = slab % p.q.grid + (long long)rbi * p.q.S;
+    const int nb = (p.q.nblk - rbi + p.q.rb - 1) / p.q.rb;
+    return ks_slot(c, slab / p.q.grid * nb + blk / p.q.rb, hh, G, p);
+}
+__device__ __forceinline__ long long ks_block_step(int G, const KsParams& p) {
+    return (long long)p.q.rb * p.q.S * p.q.max_seg * G;
 }
 
 // ===================================================================== KR ===
@@ -414,21 +440,21 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
     const int slab = b * p.groups + h / G;
-    const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
-    // one block: the sum of the slab's R partials; block-causal: the running
+    const long long step = ks_block_step(G, p) * DD;
+    const int nr = p.q.R / p.q.rb;                  // partials per block
+    // one block: the sum of the slab's partials; block-causal: the running
     // sum over blocks, i.e. the inclusive prefix state of every block
     float s = 0.0f;
     for (int j = 0; j < p.q.nblk; ++j) {
-        const float* src =
-            partial + ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j, h % G, G, p) * DD + e;
-        // eight loads in flight, then their additions in ascending r
-        for (int r0 = 0; r0 < p.q.R; r0 += 8) {
+        const float* src = partial + ks_block_slot(slab, j, h % G, G, p) * DD + e;
+        // eight loads in flight, then their additions in ascending order
+        for (int r0 = 0; r0 < nr; r0 += 8) {
             float t[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
+            for (int u = 0; u < 8; ++u) t[u] = r0 + u < nr ? src[(r0 + u) * step] : 0.0f;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (r0 + u < p.q.R) s += t[u];
+                if (r0 + u < nr) s += t[u];
         }
         state[(bh * p.q.nblk + j) * DD + e] = s;
     }
@@ -436,7 +462,7 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 
 // Block-causal prefix states. A CTA takes 32 consecutive state entries (so
 // every load instruction reads 128 contiguous bytes) times 8 block lanes:
-// lane jl sums the R partials (ascending r) of blocks jl, jl+8, ... of a
+// lane jl sums the partials (ascending CTA) of blocks jl, jl+8, ... of a
 // 64-block chunk into shared memory, then one thread per entry walks the
 // chunk in block order: prefix_j = prefix_{j-1} + blocksum_j. The same
 // additions in the same order on every run.
@@ -461,21 +487,21 @@ kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
     const int slab = b * p.groups + h / G;
-    const long long step = (long long)p.q.S * p.q.max_seg * G * DD;   // next r: CTA c + S
+    const long long step = ks_block_step(G, p) * DD;
+    const int nr = p.q.R / p.q.rb;                  // partials per block
     float carry = 0.0f;
     for (int j0 = 0; j0 < p.q.nblk; j0 += KP_CHUNK) {
         for (int jj = jl; jj < KP_CHUNK && j0 + jj < p.q.nblk; jj += KP_LANES) {
             float x = 0.0f;
             if (live) {
-                const float* src = partial +
-                    ks_slot(slab % p.q.grid, slab / p.q.grid * p.q.nblk + j0 + jj, h % G, G, p) * DD + e;
-                for (int r0 = 0; r0 < p.q.R; r0 += 8) {
+                const float* src = partial + ks_block_slot(slab, j0 + jj, h % G, G, p) * DD + e;
+                for (int r0 = 0; r0 < nr; r0 += 8) {
                     float t[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) t[u] = r0 + u < p.q.R ? src[(r0 + u) * step] : 0.0f;
+                    for (int u = 0; u < 8; ++u) t[u] = r0 + u < nr ? src[(r0 + u) * step] : 0.0f;
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
-                        if (r0 + u < p.q.R) x += t[u];
+                        if (r0 + u < nr) x += t[u];
                 }
             }
             bsum[jj][el] = x;
@@ -857,7 +883,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 }
                 int slab, tile, seg;
                 sched_item(cta, i, tps, p.q, slab, tile, seg);
-                if (!stage_state(slab, seg % p.q.nblk)) return false;
+                if (!stage_state(slab, sched_block(cta, seg, p.q))) return false;
             }
             const int s = i % S;
             if (!warp_wait(&bar.full[s], (i / S) & 1, abort, err)) return false;

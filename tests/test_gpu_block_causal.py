@@ -45,6 +45,8 @@ SHAPES = [
     (1, 500, 3, 32, 1024),       # L > N: one block
     (1, 17281, 9, 32, 5760),     # L / 128 = 45: R = 45 CTAs per slab
     (2, 16384, 70, 32, 1024),    # 16 frames of 32x32 tokens at the 1.6B width
+    (1, 1280, 80, 32, 128),      # 7 CTAs per slab over 10 blocks: some take two
+    (1, 4600, 120, 32, 1024),    # 2 x 2 CTAs per slab: 5 ragged blocks over 2, tiles split 2 ways
 ]
 
 
@@ -77,7 +79,7 @@ def test_block_causal_prefix_states(oracle):
     assert np.all(err <= 1e-5 * mag + 1e-30), (err / (mag + 1e-30)).max()
 
 
-@pytest.mark.parametrize("shape", [SHAPES[1], SHAPES[3], SHAPES[4], SHAPES[7]], ids=_ids)
+@pytest.mark.parametrize("shape", [SHAPES[1], SHAPES[3], SHAPES[4], SHAPES[7], SHAPES[10]], ids=_ids)
 def test_block_causal_forward_equals_two_calls_and_is_deterministic(shape):
     B, N, H, d, L = shape
     Q, K, V = make_inputs(Workload("bcb", B, N, H, d, seed=3), device="cuda")
