@@ -321,6 +321,44 @@ sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const 
                                             sana_la_stream_t stream);
 
 /*
+ * The forward of sana_linattn_forward_fm from and to HOST memory ("08_sana
+ * 高效高分辨率生成", "Linear Attention 的原理": the state sum over all tokens,
+ * then each token's row against it).
+ *   Q, K, V   host, (B, N, H, d) bf16 row-major (as for sana_linattn_forward)
+ *   O         host, (B, N, H, d) fp32 or bf16 by out_dtype
+ *   workspace device, sana_linattn_forward_host_workspace_bytes(B, N, H, d,
+ *             out_dtype) bytes, 16-byte aligned; holds device copies of Q, K,
+ *             V and O, the state and the state kernels' partials
+ * K and V are copied in and the state is computed over all tokens; then Q is
+ * streamed in chunks of about an eighth of the tokens (at least 1024 tokens,
+ * whole batches when a batch is shorter): each chunk is copied in and applied
+ * on `stream`, and copied out on a stream of this library's (one per device,
+ * made on first use) while the next chunk is copied in, so the two copy
+ * directions overlap. `stream` waits for the last copy out before anything
+ * enqueued after this call: once `stream` is done, O is in host memory. O is
+ * bit-identical to sana_linattn_forward_fm's on the same inputs (the apply of
+ * a token does not depend on the chunk it is in). For the copies to be
+ * asynchronous and to overlap, the host buffers must be page-locked
+ * (cudaHostAlloc, cudaHostRegister); with pageable memory the copies still
+ * happen, but CUDA completes them before the copy calls return. Host buffers
+ * stay owned by the caller and must stay valid until `stream` has finished.
+ * Errors as for sana_linattn_forward (null pointers, bad sizes, an unaligned
+ * workspace: SANA_LA_ERR_INVALID_ARG; a short workspace:
+ * SANA_LA_ERR_WORKSPACE; a failed CUDA call: SANA_LA_ERR_CUDA).
+ */
+size_t sana_linattn_forward_host_workspace_bytes(int B, int N, int H, int d, sana_la_out_dtype out_dtype);
+
+sana_la_status sana_linattn_forward_host(const void* Q, const void* K, const void* V,
+                                         int B, int N, int H, int d, sana_la_feature_map feature_map,
+                                         void* O, sana_la_out_dtype out_dtype, float eps,
+                                         void* workspace, size_t workspace_bytes,
+                                         sana_la_stream_t stream);
+
+/* Kernel launches of one sana_linattn_forward_host call (0 for invalid sizes):
+ * the state, its reduction, and one apply per chunk of Q. */
+int sana_linattn_forward_host_launches(int B, int N, int H, int d);
+
+/*
  * Number of kernel launches one sana_linattn_forward call enqueues for these
  * sizes (0 for invalid or unsupported sizes): 1 (the single cooperative
  * launch; a captured call adds one memset node). Useful for counting launches

@@ -87,12 +87,12 @@ sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int 
 // tiles128 128-token tiles; at most 148 CTAs): the split (rb, rt), rb * rt <=
 // 148 / S and rt dividing tiles128, that minimises the tiles of the busiest
 // CTA plus three tiles' worth for each state it stages (one per block it
-// visits), times 1.06 when rb > 1; ties go to fewer partial states per block
-// (smaller rt). The factor is what reading rb token regions at once instead
-// of one cost on B200: at 16 frames of 256 x 256 tokens (16 blocks of 512
-// tiles, 18 slabs) rb = 8, rt = 1 took 1796 us against 1703 us for rb = 1,
-// rt = 8; at 16 frames of 64 x 64 tokens (16 blocks of 32 tiles, 9 slabs)
-// rb = 16, rt = 1 took 138 us against 198 us for rb = 1, rt = 16.
+// visits), times 1.15 when rb > 1; ties go to fewer partial states per block
+// (smaller rt). The factor stands for what reading rb token regions at once
+// instead of one cost on B200, fitted to two measurements with 9 slabs of 16
+// blocks: 512 tiles per block, rb = 16, rt = 1 took 1796-1817 us against
+// 1703 us for rb = 1, rt = 16; 32 tiles per block, rb = 16, rt = 1 took 138 us
+// against 198 us for rb = 1, rt = 16.
 struct BlockSplit {
     int rb, rt;
 };
@@ -104,7 +104,7 @@ BlockSplit block_split(long long S, long long nblk, long long tiles128) {
     for (long long rt = 1; rt <= std::min(rmax, tiles128); ++rt) {
         if (tiles128 % rt != 0) continue;
         const long long rb = std::min(nblk, rmax / rt);
-        const long long cost = cdiv(nblk, rb) * (tiles128 / rt + 3) * (rb > 1 ? 106 : 100);
+        const long long cost = cdiv(nblk, rb) * (tiles128 / rt + 3) * (rb > 1 ? 115 : 100);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = BlockSplit{(int)rb, (int)rt};
@@ -665,6 +665,169 @@ sana_la_status forward_entry(const void* Q, const void* K, const void* V, int B,
     return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true, fm);
 }
 
+// ------------------------------------------------- host-buffer forward ----
+// Device layout of the host-buffer forward's workspace: Q, K, V and O staging,
+// the state, and the state kernels' partials, each 256-byte aligned.
+struct HostPlan {
+    size_t q, kv, o, state, partial, total;
+};
+
+HostPlan make_host_plan(int B, int N, int H, int d, sana_la_out_dtype od) {
+    const Plan p = make_plan(B, N, H, d);
+    const size_t elems = (size_t)B * N * H * d;
+    HostPlan h{};
+    h.q = align256(elems * 2);
+    h.kv = align256(elems * 2);
+    h.o = align256(elems * (od == SANA_LA_OUT_F32 ? 4 : 2));
+    h.state = align256((size_t)B * H * d * (d + 1) * sizeof(float));
+    h.partial = p.partial_bytes;
+    h.total = h.q + 2 * h.kv + h.o + h.state + h.partial;
+    return h;
+}
+
+// Q is streamed in chunks of about 1/8 of the tokens (at least 1024): chunks
+// of whole batches when a batch is shorter, else pieces of one batch.
+struct HostChunks {
+    long long tokens;   // tokens per chunk within a batch (N when chunks are whole batches)
+    int batches;        // batches per chunk (1 when a batch is split)
+    int count;
+};
+
+HostChunks host_chunks(int B, int N) {
+    const long long target = std::max<long long>(1024, cdiv((long long)B * N, 8));
+    HostChunks c{};
+    if (N >= target) {
+        c.tokens = cdiv(target, 128) * 128;
+        c.batches = 1;
+        c.count = (int)(B * cdiv(N, c.tokens));
+    } else {
+        c.tokens = N;
+        c.batches = (int)std::max<long long>(1, target / N);
+        c.count = (int)cdiv(B, c.batches);
+    }
+    return c;
+}
+
+// The library's device-to-host copy stream and a small ring of events, per
+// device, made on first use.
+constexpr int kHostEvents = 16;
+struct CopyCtx {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t ev[kHostEvents] = {};
+    cudaEvent_t join = nullptr;
+    bool ready = false;
+};
+CopyCtx g_copy_ctx[kMaxDevicesCached];
+std::mutex g_copy_ctx_mutex;
+
+sana_la_status copy_ctx(CopyCtx** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_last_error("cudaGetDevice", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevicesCached) return SANA_LA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_copy_ctx_mutex);
+    CopyCtx& c = g_copy_ctx[dev];
+    if (!c.ready) {
+        e = cudaStreamCreateWithFlags(&c.stream, cudaStreamNonBlocking);
+        for (int i = 0; i < kHostEvents && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&c.ev[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            set_last_error("copy stream and events", e);
+            return SANA_LA_ERR_CUDA;
+        }
+        c.ready = true;
+    }
+    *out = &c;
+    return SANA_LA_OK;
+}
+
+sana_la_status copy_async(void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyAsync(dst, src, bytes, kind, s);
+    if (e != cudaSuccess) {
+        set_last_error(kind == cudaMemcpyHostToDevice ? "cudaMemcpyAsync (to device)" : "cudaMemcpyAsync (to host)", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    return SANA_LA_OK;
+}
+
+sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV, int B, int N, int H, int d,
+                                  int fm, void* hO, sana_la_out_dtype out_dtype, float eps, void* workspace,
+                                  size_t workspace_bytes, sana_la_stream_t stream) {
+    g_last_error[0] = '\0';
+    if (!hQ || !hK || !hV || !hO || !workspace || !valid_feature(fm)) return SANA_LA_ERR_INVALID_ARG;
+    sana_la_status st = check_sizes(B, N, H, d);
+    if (st != SANA_LA_OK) return st;
+    if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
+    if ((st = check_eps(eps)) != SANA_LA_OK) return st;
+    if (!aligned16(workspace)) return SANA_LA_ERR_INVALID_ARG;
+    const HostPlan hp = make_host_plan(B, N, H, d, out_dtype);
+    if (workspace_bytes < hp.total) return SANA_LA_ERR_WORKSPACE;
+    CopyCtx* cc = nullptr;
+    if ((st = copy_ctx(&cc)) != SANA_LA_OK) return st;
+    char* ws = static_cast<char*>(workspace);
+    char* dQ = ws;
+    char* dK = dQ + hp.q;
+    char* dV = dK + hp.kv;
+    char* dO = dV + hp.kv;
+    float* state = reinterpret_cast<float*>(dO + hp.o);
+    void* partial = dO + hp.o + hp.state;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t row_in = (size_t)H * d * 2;                                  // bytes per token
+    const size_t row_out = (size_t)H * d * (out_dtype == SANA_LA_OUT_F32 ? 4 : 2);
+    const size_t tokens = (size_t)B * N;
+    // K and V in, then the state over all tokens
+    if ((st = copy_async(dK, hK, tokens * row_in, cudaMemcpyHostToDevice, s)) != SANA_LA_OK) return st;
+    if ((st = copy_async(dV, hV, tokens * row_in, cudaMemcpyHostToDevice, s)) != SANA_LA_OK) return st;
+    if ((st = kv_state_impl(dK, dV, B, N, H, d, 0, state, partial, hp.partial, s, false, fm)) != SANA_LA_OK)
+        return st;
+    // Q in chunk by chunk; each chunk applied on `s`, then copied out on the
+    // copy stream while the next chunk comes in
+    const HostChunks hc = host_chunks(B, N);
+    const long long per_batch = cdiv(N, hc.tokens);
+    const size_t state_stride = (size_t)H * d * (d + 1);
+    cudaError_t e = cudaSuccess;
+    for (int c = 0; c < hc.count; ++c) {
+        int b0, nb, t0, nt;
+        if (hc.batches > 1 || hc.tokens >= N) {
+            b0 = c * hc.batches;
+            nb = std::min(hc.batches, B - b0);
+            t0 = 0;
+            nt = N;
+        } else {
+            b0 = (int)(c / per_batch);
+            nb = 1;
+            t0 = (int)((c % per_batch) * hc.tokens);
+            nt = (int)std::min<long long>(hc.tokens, N - t0);
+        }
+        const size_t first = (size_t)b0 * N + t0;                       // first token of the chunk
+        const size_t rows = (size_t)nb * nt;                             // tokens in the chunk
+        if ((st = copy_async(dQ + first * row_in, static_cast<const char*>(hQ) + first * row_in, rows * row_in,
+                             cudaMemcpyHostToDevice, s)) != SANA_LA_OK)
+            return st;
+        if ((st = apply_impl(dQ + first * row_in, state + (size_t)b0 * state_stride, nb, nt, H, d, 0,
+                             dO + first * row_out, out_dtype, eps, s, false, fm)) != SANA_LA_OK)
+            return st;
+        cudaEvent_t ev = cc->ev[c % kHostEvents];
+        if ((e = cudaEventRecord(ev, s)) != cudaSuccess || (e = cudaStreamWaitEvent(cc->stream, ev, 0)) != cudaSuccess) {
+            set_last_error("chunk event", e);
+            return SANA_LA_ERR_CUDA;
+        }
+        if ((st = copy_async(static_cast<char*>(hO) + first * row_out, dO + first * row_out, rows * row_out,
+                             cudaMemcpyDeviceToHost, cc->stream)) != SANA_LA_OK)
+            return st;
+    }
+    // `s` ends after the last copy out
+    if ((e = cudaEventRecord(cc->join, cc->stream)) != cudaSuccess || (e = cudaStreamWaitEvent(s, cc->join, 0)) != cudaSuccess) {
+        set_last_error("join event", e);
+        return SANA_LA_ERR_CUDA;
+    }
+    return SANA_LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -877,6 +1040,25 @@ sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, c
 int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
     return 3;   // ks_state_tc, kr_reduce_tc (prefix states), ka_apply_tc
+}
+
+size_t sana_linattn_forward_host_workspace_bytes(int B, int N, int H, int d, sana_la_out_dtype out_dtype) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
+    if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return 0;
+    return make_host_plan(B, N, H, d, out_dtype).total;
+}
+
+sana_la_status sana_linattn_forward_host(const void* Q, const void* K, const void* V, int B, int N, int H, int d,
+                                         sana_la_feature_map feature_map, void* O, sana_la_out_dtype out_dtype,
+                                         float eps, void* workspace, size_t workspace_bytes,
+                                         sana_la_stream_t stream) {
+    return forward_host_entry(Q, K, V, B, N, H, d, (int)feature_map, O, out_dtype, eps, workspace,
+                              workspace_bytes, stream);
+}
+
+int sana_linattn_forward_host_launches(int B, int N, int H, int d) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
+    return 2 + host_chunks(B, N).count;          // state, reduction, one apply per chunk
 }
 
 int sana_linattn_forward_launches(int B, int N, int H, int d) {

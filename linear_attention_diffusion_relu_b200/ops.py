@@ -3,7 +3,8 @@
 Every step of the computation runs in the library's CUDA kernels; this module
 checks torch tensors (dtype, shape, contiguity, device), passes raw device
 pointers and the current CUDA stream, and raises on any non-OK status. There is
-no CPU path: CPU tensors are rejected and a missing library raises.
+no CPU path: CPU tensors are rejected (except by forward_host, whose host
+buffers the library copies to the device itself) and a missing library raises.
 
 The functions mirror the C ABI in ``include/sana_linattn.h``:
 
@@ -13,6 +14,10 @@ The functions mirror the C ABI in ``include/sana_linattn.h``:
     forward(Q, K, V, out_dtype=torch.bfloat16, eps=1e-15, out=None, workspace=None) -> O
 
 each with ``feature_map="relu" | "elu1" | "cos"`` (the ``*_fm`` entry points),
+
+the forward from and to host memory, copies overlapped by the library:
+
+    forward_host(Q, K, V, out_dtype=..., eps=..., out=None, workspace=None) -> O (CPU)
 
 the state built inside the key-value projection (K and V never stored):
 
@@ -64,6 +69,9 @@ SYMBOLS = (
     "sana_linattn_block_causal_apply",
     "sana_linattn_block_causal_forward",
     "sana_linattn_block_causal_forward_launches",
+    "sana_linattn_forward_host_workspace_bytes",
+    "sana_linattn_forward_host",
+    "sana_linattn_forward_host_launches",
     "sana_linattn_build_info",
     "sana_linattn_device_error",
     "sana_linattn_selftest_wait_timeout",
@@ -117,6 +125,12 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_apply_fm.restype = st
         lib.sana_linattn_forward_fm.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
         lib.sana_linattn_forward_fm.restype = st
+        lib.sana_linattn_forward_host_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_forward_host_workspace_bytes.restype = sz
+        lib.sana_linattn_forward_host.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_forward_host.restype = st
+        lib.sana_linattn_forward_host_launches.argtypes = [i, i, i, i]
+        lib.sana_linattn_forward_host_launches.restype = ctypes.c_int
         lib.sana_linattn_mix_ffn_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.sana_linattn_mix_ffn_workspace_bytes.restype = sz
         lib.sana_linattn_mix_ffn.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp, sz, vp]
@@ -293,6 +307,54 @@ def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.b
                                      out.data_ptr(), code, float(eps), workspace.data_ptr(),
                                      workspace.numel() * workspace.element_size(), _stream(Q.device))
     _check(lib, st, "sana_linattn_forward_fm")
+    return out
+
+
+def forward_host_workspace_bytes(B: int, N: int, H: int, d: int, out_dtype=torch.bfloat16) -> int:
+    return int(load_library().sana_linattn_forward_host_workspace_bytes(B, N, H, d, _out_code(out_dtype)))
+
+
+def forward_host_launches(B: int, N: int, H: int, d: int) -> int:
+    return int(load_library().sana_linattn_forward_host_launches(B, N, H, d))
+
+
+def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=torch.bfloat16,
+                 eps: float = 1e-15, out: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, feature_map: str = "relu",
+                 device=None) -> torch.Tensor:
+    """The forward from host tensors to a host tensor, with the copies done by the
+    library (K, V in; the state; Q streamed through in chunks whose outputs are
+    copied back while the next chunk comes in). Q, K, V: CPU (B, N, H, d) bf16,
+    page-locked for the copies to overlap; out: CPU, allocated page-locked when
+    None. Enqueued on the current stream of `device` (default: the current CUDA
+    device); the result is ready once that stream is done. Bit-identical to
+    forward() on the same inputs."""
+    fm = _feature_code(feature_map)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    for name, t in (("Q", Q), ("K", K), ("V", V)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+            raise ValueError(f"{name} must be a CPU tensor (the device copy is made by the library)")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous (B, N, H, d) bf16 tensor")
+        if t.shape != Q.shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(Q.shape)}")
+    B, N, H, d = Q.shape
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty(Q.shape, dtype=out_dtype).pin_memory()
+    elif (out.device.type != "cpu" or out.dtype != out_dtype or tuple(out.shape) != tuple(Q.shape)
+          or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous CPU {out_dtype} tensor of shape {tuple(Q.shape)}")
+    if workspace is None:
+        n = forward_host_workspace_bytes(B, N, H, d, out_dtype)
+        if n == 0:
+            raise ValueError(f"unsupported sizes B={B} N={N} H={H} d={d}")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    lib = load_library()
+    st = lib.sana_linattn_forward_host(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d, fm,
+                                       out.data_ptr(), code, float(eps), workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(lib, st, "sana_linattn_forward_host")
     return out
 
 

@@ -196,3 +196,28 @@ def test_mix_ffn_host_checks(lib):
     assert f(FAKE, FAKE, FAKE + 2, FAKE, 1, 4, 4, 64, 32, FAKE, FAKE, ws, None) == ops.ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 64, 32, FAKE, FAKE, ws - 1, None) == ops.ERR_WORKSPACE
     assert lib.sana_linattn_mix_ffn_launches(1, 4, 4, 64, 32) == 3
+
+
+def test_forward_host_host_checks(lib):
+    wsb = lib.sana_linattn_forward_host_workspace_bytes
+    n16 = wsb(2, 1000, 6, 32, ops.OUT_BF16)
+    n32 = wsb(2, 1000, 6, 32, ops.OUT_F32)
+    assert n16 > 0 and n16 % 256 == 0 and n32 > n16
+    # at least the four device copies and the state
+    assert n16 >= 4 * (2 * 1000 * 6 * 32 * 2) + 2 * 6 * 32 * 33 * 4
+    assert wsb(2, 1000, 6, 48, ops.OUT_BF16) == 0
+    assert wsb(2, 1000, 6, 32, 7) == 0
+    n = lib.sana_linattn_forward_host_launches
+    assert n(2, 16384, 70, 32) == 2 + 8          # 4096 tokens per chunk
+    assert n(1, 256, 4, 32) == 3                 # one chunk
+    assert n(8, 300, 4, 32) == 2 + 3             # three batches per chunk
+    assert n(0, 1, 1, 32) == 0
+    f = lib.sana_linattn_forward_host
+    ws = wsb(1, 1024, 2, 32, ops.OUT_BF16)
+    # argument errors come back before any CUDA call
+    assert f(None, FAKE, FAKE, 1, 1024, 2, 32, 0, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 3, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 0, FAKE, 1, -1.0, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 0, FAKE, 5, 1e-15, FAKE, ws, None) == ops.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 48, 0, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 0, FAKE, 1, 1e-15, FAKE, ws - 256, None) == ops.ERR_WORKSPACE

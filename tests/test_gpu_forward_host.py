@@ -1,0 +1,71 @@
+"""The forward from host buffers (sana_linattn_forward_host): the library copies
+K and V in, computes the state, and streams Q through in chunks whose outputs
+are copied back on its own stream while the next chunk comes in. The apply of a
+token does not depend on the chunk it is in, so the result must be
+bit-identical to the device forward on the same inputs, for every way the
+tokens are cut into chunks; and the caller's stream must cover the last copy
+out."""
+import pytest
+import torch
+
+from linear_attention_diffusion_relu_b200 import ops
+from linear_attention_diffusion_relu_b200.workloads import Workload, make_inputs
+from tests.parity import check_output, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from linear_attention_diffusion_relu_b200 import build
+    build.build()
+    ops.load_library()
+
+
+# chunks: one; pieces of a batch (ragged last); whole batches; several batches
+# per chunk; the 4096px shape (8 chunks of 4096 tokens)
+SHAPES = [(1, 256, 4, 32), (2, 5000, 6, 32), (3, 700, 5, 64), (8, 300, 4, 32), (2, 16384, 70, 32)]
+BITS = {torch.float32: torch.int32, torch.bfloat16: torch.int16}
+
+
+def _host(B, N, H, d, seed, pinned=True):
+    Q, K, V = make_inputs(Workload("host", B, N, H, d, seed=seed))
+    return tuple(t.pin_memory() if pinned else t for t in (Q, K, V))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}N{}H{}d{}".format(*s))
+def test_forward_host_equals_device_forward(shape, dtype):
+    B, N, H, d = shape
+    hQ, hK, hV = _host(B, N, H, d, seed=N + H)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        O = ops.forward_host(hQ, hK, hV, out_dtype=dtype)
+    side.synchronize()               # the caller's stream covers the copies out
+    Od = ops.forward(hQ.cuda(), hK.cuda(), hV.cuda(), out_dtype=dtype)
+    assert O.device.type == "cpu" and O.is_pinned()
+    assert torch.equal(O.view(BITS[dtype]), Od.cpu().view(BITS[dtype]))
+    assert ops.device_error() == 0
+
+
+def test_forward_host_pageable_buffers_and_feature_map():
+    B, N, H, d = 2, 3000, 3, 32
+    hQ, hK, hV = _host(B, N, H, d, seed=5, pinned=False)
+    out = torch.empty((B, N, H, d), dtype=torch.bfloat16)
+    O = ops.forward_host(hQ, hK, hV, out=out, feature_map="elu1")
+    torch.cuda.synchronize()
+    Od = ops.forward(hQ.cuda(), hK.cuda(), hV.cuda(), feature_map="elu1")
+    assert O.data_ptr() == out.data_ptr()
+    assert torch.equal(O.view(torch.int16), Od.cpu().view(torch.int16))
+
+
+def test_forward_host_matches_oracle(oracle):
+    B, N, H, d = 2, 2500, 4, 32
+    hQ, hK, hV = _host(B, N, H, d, seed=11)
+    ws = torch.empty(ops.forward_host_workspace_bytes(B, N, H, d, torch.float32), dtype=torch.uint8, device="cuda")
+    O = ops.forward_host(hQ, hK, hV, out_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle.forward(to_f64(hQ), to_f64(hK), to_f64(hV), 1e-15)
+    check_output(O, ref, "forward_host")
