@@ -166,6 +166,7 @@ __host__ __device__ __forceinline__ int sched_tps(int c, const Sched& q) {
 }
 // blocks of one slab that CTA c visits (1 unless block-causal)
 __host__ __device__ __forceinline__ int sched_nb(int c, const Sched& q) {
+    if (q.rb == 1) return q.nblk;
     const int rb = (c / q.S) % q.rb;
     return (q.nblk - rb + q.rb - 1) / q.rb;
 }
@@ -175,6 +176,7 @@ __host__ __device__ __forceinline__ int sched_nseg(int c, const Sched& q) {
 }
 // token block of segment `seg` of CTA c
 __host__ __device__ __forceinline__ int sched_block(int c, int seg, const Sched& q) {
+    if (q.rb == 1) return seg % q.nblk;
     return (c / q.S) % q.rb + (seg % sched_nb(c, q)) * q.rb;
 }
 // i-th tile of CTA c -> (slab, tile, segment index). In round k the R CTAs of
@@ -186,11 +188,15 @@ __host__ __device__ __forceinline__ void sched_item(int c, int i, int tps, const
                                                     int& slab, int& tile, int& seg) {
     seg = i / tps;
     const int r = c / q.S;
+    if (q.rb == 1) {
+        // every CTA of the slab in every block (and the plain forward): the
+        // general form below with rb = 1, in fewer divisions
+        slab = c % q.S + seg / q.nblk * q.grid;
+        tile = r + ((seg % q.nblk) * tps + i % tps) * q.R;
+        return;
+    }
     slab = c % q.S + seg / sched_nb(c, q) * q.grid;
-    if (q.tpb > 0)
-        tile = sched_block(c, seg, q) * (q.T / q.nblk) + r / q.rb + (i % tps) * (q.R / q.rb);
-    else
-        tile = r + (i % tps) * q.R;
+    tile = sched_block(c, seg, q) * (q.T / q.nblk) + r / q.rb + (i % tps) * (q.R / q.rb);
 }
 
 // ===================================================================== KS ===
