@@ -330,11 +330,13 @@ sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const 
  *             out_dtype) bytes, 16-byte aligned; holds device copies of Q, K,
  *             V and O, the state and the state kernels' partials
  * K and V are copied in and the state is computed over all tokens; then Q is
- * streamed in chunks of about an eighth of the tokens (at least 1024 tokens,
- * whole batches when a batch is shorter): each chunk is copied in and applied
- * on `stream`, and copied out on a stream of this library's (one per device,
- * made on first use) while the next chunk is copied in, so the two copy
- * directions overlap. `stream` waits for the last copy out before anything
+ * streamed in chunks of about a sixteenth of the tokens (at least 1024 tokens,
+ * whole batches when a batch is shorter). The copies in run back to back on a
+ * host-to-device stream of this library's, each chunk is applied on `stream`
+ * as soon as it is in, and its O is copied out on a device-to-host stream of
+ * this library's while later chunks are copied in, so the two copy directions
+ * overlap (both streams and a few events per device are made on first use;
+ * the copies in wait for the work enqueued on `stream` before this call). `stream` waits for the last copy out before anything
  * enqueued after this call: once `stream` is done, O is in host memory. O is
  * bit-identical to sana_linattn_forward_fm's on the same inputs (the apply of
  * a token does not depend on the chunk it is in). For the copies to be

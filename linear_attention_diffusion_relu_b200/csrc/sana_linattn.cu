@@ -685,7 +685,7 @@ HostPlan make_host_plan(int B, int N, int H, int d, sana_la_out_dtype od) {
     return h;
 }
 
-// Q is streamed in chunks of about 1/8 of the tokens (at least 1024): chunks
+// Q is streamed in chunks of about 1/16 of the tokens (at least 1024): chunks
 // of whole batches when a batch is shorter, else pieces of one batch.
 struct HostChunks {
     long long tokens;   // tokens per chunk within a batch (N when chunks are whole batches)
@@ -694,7 +694,7 @@ struct HostChunks {
 };
 
 HostChunks host_chunks(int B, int N) {
-    const long long target = std::max<long long>(1024, cdiv((long long)B * N, 8));
+    const long long target = std::max<long long>(1024, cdiv((long long)B * N, 16));
     HostChunks c{};
     if (N >= target) {
         c.tokens = cdiv(target, 128) * 128;
@@ -708,13 +708,17 @@ HostChunks host_chunks(int B, int N) {
     return c;
 }
 
-// The library's device-to-host copy stream and a small ring of events, per
-// device, made on first use.
-constexpr int kHostEvents = 16;
+// The library's copy streams (host to device, device to host) and rings of
+// events, per device, made on first use. A ring entry is recorded and waited
+// for right away, so reusing it later (a newer record) is safe.
+constexpr int kHostEvents = 32;
 struct CopyCtx {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t ev[kHostEvents] = {};
-    cudaEvent_t join = nullptr;
+    cudaStream_t h2d = nullptr;
+    cudaStream_t d2h = nullptr;
+    cudaEvent_t in[kHostEvents] = {};       // a chunk of Q (or K and V) is on the device
+    cudaEvent_t out[kHostEvents] = {};      // a chunk's O is ready to be copied back
+    cudaEvent_t start = nullptr;            // the caller's earlier work on its stream is done
+    cudaEvent_t join = nullptr;             // the last copy back is done
     bool ready = false;
 };
 CopyCtx g_copy_ctx[kMaxDevicesCached];
@@ -731,9 +735,13 @@ sana_la_status copy_ctx(CopyCtx** out) {
     std::lock_guard<std::mutex> lock(g_copy_ctx_mutex);
     CopyCtx& c = g_copy_ctx[dev];
     if (!c.ready) {
-        e = cudaStreamCreateWithFlags(&c.stream, cudaStreamNonBlocking);
-        for (int i = 0; i < kHostEvents && e == cudaSuccess; ++i)
-            e = cudaEventCreateWithFlags(&c.ev[i], cudaEventDisableTiming);
+        e = cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking);
+        for (int i = 0; i < kHostEvents && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&c.in[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.out[i], cudaEventDisableTiming);
+        }
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.start, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming);
         if (e != cudaSuccess) {
             set_last_error("copy stream and events", e);
@@ -742,6 +750,17 @@ sana_la_status copy_ctx(CopyCtx** out) {
         c.ready = true;
     }
     *out = &c;
+    return SANA_LA_OK;
+}
+
+// `waiter` waits for the work enqueued on `signaler` so far (through `ev`).
+sana_la_status stream_after(cudaStream_t waiter, cudaStream_t signaler, cudaEvent_t ev, const char* what) {
+    cudaError_t e = cudaEventRecord(ev, signaler);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(waiter, ev, 0);
+    if (e != cudaSuccess) {
+        set_last_error(what, e);
+        return SANA_LA_ERR_CUDA;
+    }
     return SANA_LA_OK;
 }
 
@@ -779,19 +798,21 @@ sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV
     const size_t row_in = (size_t)H * d * 2;                                  // bytes per token
     const size_t row_out = (size_t)H * d * (out_dtype == SANA_LA_OUT_F32 ? 4 : 2);
     const size_t tokens = (size_t)B * N;
-    // K and V in, then the state over all tokens
-    if ((st = copy_async(dK, hK, tokens * row_in, cudaMemcpyHostToDevice, s)) != SANA_LA_OK) return st;
-    if ((st = copy_async(dV, hV, tokens * row_in, cudaMemcpyHostToDevice, s)) != SANA_LA_OK) return st;
+    // Three queues: host-to-device copies on the library's h2d stream, the
+    // kernels on `s`, device-to-host copies on its d2h stream. The copies in
+    // start after the caller's earlier work on `s` (which may still use the
+    // workspace); K and V go first, then every chunk of Q back to back, so
+    // the host-to-device direction never waits for a kernel.
+    if ((st = stream_after(cc->h2d, s, cc->start, "start event")) != SANA_LA_OK) return st;
+    if ((st = copy_async(dK, hK, tokens * row_in, cudaMemcpyHostToDevice, cc->h2d)) != SANA_LA_OK) return st;
+    if ((st = copy_async(dV, hV, tokens * row_in, cudaMemcpyHostToDevice, cc->h2d)) != SANA_LA_OK) return st;
+    if ((st = stream_after(s, cc->h2d, cc->in[0], "K, V event")) != SANA_LA_OK) return st;
     if ((st = kv_state_impl(dK, dV, B, N, H, d, 0, state, partial, hp.partial, s, false, fm)) != SANA_LA_OK)
         return st;
-    // Q in chunk by chunk; each chunk applied on `s`, then copied out on the
-    // copy stream while the next chunk comes in
     const HostChunks hc = host_chunks(B, N);
     const long long per_batch = cdiv(N, hc.tokens);
     const size_t state_stride = (size_t)H * d * (d + 1);
-    cudaError_t e = cudaSuccess;
-    for (int c = 0; c < hc.count; ++c) {
-        int b0, nb, t0, nt;
+    auto chunk = [&](int c, int& b0, int& nb, int& t0, int& nt) {
         if (hc.batches > 1 || hc.tokens >= N) {
             b0 = c * hc.batches;
             nb = std::min(hc.batches, B - b0);
@@ -803,28 +824,29 @@ sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV
             t0 = (int)((c % per_batch) * hc.tokens);
             nt = (int)std::min<long long>(hc.tokens, N - t0);
         }
+    };
+    for (int c = 0; c < hc.count; ++c) {
+        int b0, nb, t0, nt;
+        chunk(c, b0, nb, t0, nt);
         const size_t first = (size_t)b0 * N + t0;                       // first token of the chunk
         const size_t rows = (size_t)nb * nt;                             // tokens in the chunk
+        // Q of the chunk in (h2d), its apply (s), its O back (d2h)
         if ((st = copy_async(dQ + first * row_in, static_cast<const char*>(hQ) + first * row_in, rows * row_in,
-                             cudaMemcpyHostToDevice, s)) != SANA_LA_OK)
+                             cudaMemcpyHostToDevice, cc->h2d)) != SANA_LA_OK)
+            return st;
+        if ((st = stream_after(s, cc->h2d, cc->in[(c + 1) % kHostEvents], "chunk in event")) != SANA_LA_OK)
             return st;
         if ((st = apply_impl(dQ + first * row_in, state + (size_t)b0 * state_stride, nb, nt, H, d, 0,
                              dO + first * row_out, out_dtype, eps, s, false, fm)) != SANA_LA_OK)
             return st;
-        cudaEvent_t ev = cc->ev[c % kHostEvents];
-        if ((e = cudaEventRecord(ev, s)) != cudaSuccess || (e = cudaStreamWaitEvent(cc->stream, ev, 0)) != cudaSuccess) {
-            set_last_error("chunk event", e);
-            return SANA_LA_ERR_CUDA;
-        }
+        if ((st = stream_after(cc->d2h, s, cc->out[c % kHostEvents], "chunk out event")) != SANA_LA_OK)
+            return st;
         if ((st = copy_async(static_cast<char*>(hO) + first * row_out, dO + first * row_out, rows * row_out,
-                             cudaMemcpyDeviceToHost, cc->stream)) != SANA_LA_OK)
+                             cudaMemcpyDeviceToHost, cc->d2h)) != SANA_LA_OK)
             return st;
     }
-    // `s` ends after the last copy out
-    if ((e = cudaEventRecord(cc->join, cc->stream)) != cudaSuccess || (e = cudaStreamWaitEvent(s, cc->join, 0)) != cudaSuccess) {
-        set_last_error("join event", e);
-        return SANA_LA_ERR_CUDA;
-    }
+    // `s` ends after the last copy back
+    if ((st = stream_after(s, cc->d2h, cc->join, "join event")) != SANA_LA_OK) return st;
     return SANA_LA_OK;
 }
 

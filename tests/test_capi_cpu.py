@@ -208,7 +208,7 @@ def test_forward_host_host_checks(lib):
     assert wsb(2, 1000, 6, 48, ops.OUT_BF16) == 0
     assert wsb(2, 1000, 6, 32, 7) == 0
     n = lib.sana_linattn_forward_host_launches
-    assert n(2, 16384, 70, 32) == 2 + 8          # 4096 tokens per chunk
+    assert n(2, 16384, 70, 32) == 2 + 16         # 2048 tokens per chunk
     assert n(1, 256, 4, 32) == 3                 # one chunk
     assert n(8, 300, 4, 32) == 2 + 3             # three batches per chunk
     assert n(0, 1, 1, 32) == 0

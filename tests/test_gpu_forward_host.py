@@ -25,7 +25,7 @@ def _cuda():
 
 
 # chunks: one; pieces of a batch (ragged last); whole batches; several batches
-# per chunk; the 4096px shape (8 chunks of 4096 tokens)
+# per chunk; the 4096px shape (16 chunks of 2048 tokens)
 SHAPES = [(1, 256, 4, 32), (2, 5000, 6, 32), (3, 700, 5, 64), (8, 300, 4, 32), (2, 16384, 70, 32)]
 BITS = {torch.float32: torch.int32, torch.bfloat16: torch.int16}
 
