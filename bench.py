@@ -45,9 +45,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the same build (profiles/), keyed by (kernel set, workload, kernel); None when
 # the kernels changed since the counters were taken
 TRAFFIC_PER_LAUNCH = {
-    # profiles/fwd_fused_tc_sweep_N65536.md: (453.1 + 94.0) MB at B=1, N=65536, H=36,
-    # scaled by token-heads to 4096px (x 0.9722)
-    ("tcgen05-tma", "4096px", "fwd_fused_tc"): 531.9e6,
+    # profiles/fwd_fused_tc_sweep_N65536.md: (453.09 + 93.36) MB at B=1, N=65536, H=36
+    # (DRAM counters of the current kernel), scaled by token-heads to 4096px (x 0.9722)
+    ("tcgen05-tma", "4096px", "fwd_fused_tc"): 531.3e6,
 }
 SMS = 148
 FP32_LANES_PER_SM = 128
