@@ -251,9 +251,11 @@ int sana_linattn_mix_ffn_launches(int B, int Hg, int Wg, int C, int Ch);
  * L must be a positive multiple of 128 (SANA_LA_ERR_UNSUPPORTED otherwise; 0
  * or negative is SANA_LA_ERR_INVALID_ARG); sizes whose per-block partial states
  * would exceed 4 GiB of workspace are SANA_LA_ERR_UNSUPPORTED. N need not be a
- * multiple of L. Work is spread over ceil(B*H/(128/d)) slabs times R CTAs,
- * where R is the largest divisor of L/128 that keeps the grid within the 148
- * SMs; L/128 with few divisors (e.g. L = 128) therefore runs on few SMs.
+ * multiple of L. Work is spread over ceil(B*H/(128/d)) slabs times R = rb*rt
+ * CTAs (at most 148 in all): the CTAs of a slab split its blocks rb ways and
+ * each block's 128-token tiles rt ways (rt divides L/128), chosen on the host
+ * from the tiles of the busiest CTA and the states it stages. Few blocks with
+ * an L/128 of few divisors (e.g. one block of L = 128) still run on few SMs.
  * Other arguments, layouts and errors are as for the calls above.
  */
 

@@ -43,7 +43,7 @@ SHAPES = [
     (16, 900, 20, 64, 256),
     (1, 777, 2, 64, 640),
     (1, 500, 3, 32, 1024),       # L > N: one block
-    (1, 17281, 9, 32, 5760),     # L / 128 = 45: R = 45 CTAs per slab
+    (1, 17281, 9, 32, 5760),     # L / 128 = 45: 4 x 9 CTAs per slab over 4 blocks
     (2, 16384, 70, 32, 1024),    # 16 frames of 32x32 tokens at the 1.6B width
     (1, 1280, 80, 32, 128),      # 7 CTAs per slab over 10 blocks: some take two
     (1, 4600, 120, 32, 1024),    # 2 x 2 CTAs per slab: 5 ragged blocks over 2, tiles split 2 ways
