@@ -116,3 +116,23 @@ def test_projected_state_agrees_with_unfused_path():
     err = to_f64(S - S_ref)
     bound = _bound(to_f64(K), to_f64(V), to_f64(mag))
     assert np.all(np.abs(err) <= bound), (np.abs(err) / bound).max()
+
+
+def test_projected_state_4096px_sampled_heads(oracle):
+    """The bench's 4096px shape (B = 2, N = 16384, C = 2240, H = 70), in the
+    launch configuration the bench times: three heads' states (first, middle,
+    last group) against the oracle's projection and state of those heads."""
+    B, N, C, H, d = 2, 16384, 2240, 70, 32
+    X, Wk, Wv = _inputs(B, N, C, H, d, seed=N + C)
+    S = ops.kv_projection_state(X, Wk, Wv, H)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    Xd = to_f64(X)
+    for h in (0, 37, H - 1):
+        rows = slice(h * d, (h + 1) * d)
+        K, V = oracle.project_kv(Xd, to_f64(Wk[rows]), to_f64(Wv[rows]), 1)
+        ref = oracle.state(K, V)[:, 0]
+        mag = oracle.state(K, np.abs(V))[:, 0]
+        err = np.abs(to_f64(S[:, h]) - ref)
+        bound = _bound(K, V, mag[:, None])[:, 0]
+        assert np.all(err <= bound), (h, (err / bound).max())

@@ -93,3 +93,53 @@ def test_mix_ffn_deterministic():
     Y2 = ops.mix_ffn(X, W1, Kdw, W2, (Hg, Wg))
     torch.cuda.synchronize()
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_mix_ffn_4096px_sampled_tokens(oracle):
+    """The bench's 4096px Mix-FFN (B = 2, 128 x 128 grid, C = 2240, Ch = 5600), in
+    the launch configuration the bench times, stage by stage on eight tokens
+    (corners, edges, interior): U on each token's 3 x 3 neighbourhood against the
+    oracle's expand of those rows; Z from the oracle's depthwise conv of the
+    GPU's own U cropped to the neighbourhood (at the grid's edge the crop's zero
+    padding is the grid's); Y from the GPU's own Z row. Same bounds as above."""
+    B, Hg, Wg, C, Ch = 2, 128, 128, 2240, 5600
+    N = Hg * Wg
+    X, W1, Kdw, W2 = _inputs(B, Hg, Wg, C, Ch, seed=4096)
+    ws = torch.empty(ops.mix_ffn_workspace_bytes(B, Hg, Wg, C, Ch), dtype=torch.uint8, device="cuda")
+    Y = ops.mix_ffn(X, W1, Kdw, W2, (Hg, Wg), workspace=ws)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    U, Z = _intermediates(ws, B, N, Ch)
+    W1d, Kd, W2d = to_f64(W1), to_f64(Kdw), to_f64(W2)
+    samples = [(0, 0, 0), (0, 0, Wg - 1), (0, Hg - 1, 0), (1, Hg - 1, Wg - 1),
+               (0, 63, 64), (1, 5, 77), (1, 64, 0), (0, 100, Wg - 1)]
+    changed_u = changed_z = total_u = total_z = 0
+    for b, y, x in samples:
+        ys = list(range(max(0, y - 1), min(Hg, y + 2)))
+        xs = list(range(max(0, x - 1), min(Wg, x + 2)))
+        rows = [yy * Wg + xx for yy in ys for xx in xs]
+        # expand on the neighbourhood
+        Xr = to_f64(X[b, rows])
+        U_ref = oracle.round_bf16(Xr @ W1d.T)
+        Ur = to_f64(U[b, rows])
+        dU = np.abs(Ur - U_ref)
+        boundU = 2.0 ** -7 * np.abs(U_ref) + C * 2.0 ** -23 * (np.abs(Xr) @ np.abs(W1d).T) + 1e-30
+        assert np.all(dU <= boundU), ((b, y, x), (dU / boundU).max())
+        changed_u += int(np.sum(dU > 0))
+        total_u += dU.size
+        # depthwise + GLU at the token, on the GPU's U
+        crop = Ur.reshape(1, len(rows), 2 * Ch)
+        ci = (y - ys[0]) * len(xs) + (x - xs[0])
+        D = oracle.depthwise3x3(crop, Kd, (len(ys), len(xs)))[0, ci]
+        Z_ref = oracle.round_bf16(D[:Ch] / (1.0 + np.exp(-D[Ch:])))
+        mag = oracle.depthwise3x3(np.abs(crop), np.abs(Kd), (len(ys), len(xs)))[0, ci, :Ch]
+        Zg = to_f64(Z[b, y * Wg + x])
+        dZ = np.abs(Zg - Z_ref)
+        assert np.all(dZ <= 2.0 ** -7 * np.abs(Z_ref) + 1e-5 * mag + 1e-30), (b, y, x)
+        changed_z += int(np.sum(dZ > 0))
+        total_z += dZ.size
+        # project on the GPU's Z row
+        Y_ref = Zg @ W2d.T
+        bound = 2.0 ** -8 * np.abs(Y_ref) + Ch * 2.0 ** -23 * (np.abs(Zg) @ np.abs(W2d).T) + 1e-30
+        assert np.all(np.abs(to_f64(Y[b, y * Wg + x]) - Y_ref) <= bound), (b, y, x)
+    assert changed_u / total_u < 1e-2 and changed_z / total_z < 1e-2
