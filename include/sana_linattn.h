@@ -346,6 +346,8 @@ sana_la_status sana_linattn_forward_noalloc(const void* Q, const void* K, const 
  * (cudaHostAlloc, cudaHostRegister); with pageable memory the copies still
  * happen, but CUDA completes them before the copy calls return. Host buffers
  * stay owned by the caller and must stay valid until `stream` has finished.
+ * Calls from several host threads on one device are safe; they take turns to
+ * enqueue their work and share the two copy streams.
  * Errors as for sana_linattn_forward (null pointers, bad sizes, an unaligned
  * workspace: SANA_LA_ERR_INVALID_ARG; a short workspace:
  * SANA_LA_ERR_WORKSPACE; a failed CUDA call: SANA_LA_ERR_CUDA).

@@ -720,6 +720,9 @@ struct CopyCtx {
     cudaEvent_t start = nullptr;            // the caller's earlier work on its stream is done
     cudaEvent_t join = nullptr;             // the last copy back is done
     bool ready = false;
+    // Held while a call enqueues: an event must be waited for before another
+    // call records it again from a different stream.
+    std::mutex enqueue;
 };
 CopyCtx g_copy_ctx[kMaxDevicesCached];
 std::mutex g_copy_ctx_mutex;
@@ -745,6 +748,23 @@ sana_la_status copy_ctx(CopyCtx** out) {
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming);
         if (e != cudaSuccess) {
             set_last_error("copy stream and events", e);
+            // free what was made, so that a later call starts over cleanly
+            auto drop_event = [](cudaEvent_t& ev) {
+                if (ev != nullptr) cudaEventDestroy(ev);
+                ev = nullptr;
+            };
+            auto drop_stream = [](cudaStream_t& st) {
+                if (st != nullptr) cudaStreamDestroy(st);
+                st = nullptr;
+            };
+            drop_event(c.start);
+            drop_event(c.join);
+            for (int i = 0; i < kHostEvents; ++i) {
+                drop_event(c.in[i]);
+                drop_event(c.out[i]);
+            }
+            drop_stream(c.h2d);
+            drop_stream(c.d2h);
             return SANA_LA_ERR_CUDA;
         }
         c.ready = true;
@@ -787,6 +807,7 @@ sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV
     if (workspace_bytes < hp.total) return SANA_LA_ERR_WORKSPACE;
     CopyCtx* cc = nullptr;
     if ((st = copy_ctx(&cc)) != SANA_LA_OK) return st;
+    std::lock_guard<std::mutex> enqueue_lock(cc->enqueue);
     char* ws = static_cast<char*>(workspace);
     char* dQ = ws;
     char* dK = dQ + hp.q;

@@ -69,3 +69,36 @@ def test_forward_host_matches_oracle(oracle):
     torch.cuda.synchronize()
     ref = oracle.forward(to_f64(hQ), to_f64(hK), to_f64(hV), 1e-15)
     check_output(O, ref, "forward_host")
+
+
+def test_forward_host_from_two_threads():
+    """Two host threads, each on its own stream, call forward_host on the same
+    device at the same time (they share the library's copy streams and events);
+    both results are bit-identical to the device forward."""
+    import threading
+    shapes = [(2, 5000, 6, 32), (1, 9000, 4, 32)]
+    inputs = [_host(*sh, seed=40 + i) for i, sh in enumerate(shapes)]
+    outs = [None, None]
+    errors = []
+
+    def run(i):
+        try:
+            side = torch.cuda.Stream()
+            with torch.cuda.stream(side):
+                for _ in range(3):
+                    outs[i] = ops.forward_host(*inputs[i])
+            side.synchronize()
+        except Exception as exc:      # reported below, on the main thread
+            errors.append(exc)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for i in range(2):
+        hQ, hK, hV = inputs[i]
+        Od = ops.forward(hQ.cuda(), hK.cuda(), hV.cuda())
+        assert torch.equal(outs[i].view(torch.int16), Od.cpu().view(torch.int16))
+    assert ops.device_error() == 0
