@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ptx.cuh"
+
 namespace sana {
 
 // phi = ReLU on a packed pair of bf16 values. max(x, 0) is exact in bf16, so
@@ -30,44 +32,47 @@ __device__ __forceinline__ uint32_t float2_to_bf16x2(float a, float b) {
 // ELU+1 and cos named as alternatives). ELU is taken with alpha = 1.
 enum : int { kFeatureRelu = 0, kFeatureElu1 = 1, kFeatureCos = 2 };
 
-// cos(x) for moderate |x|: Cody-Waite additive range reduction (W. J. Cody and
-// W. Waite, "Software Manual for the Elementary Functions", 1980) by the
-// nearest multiple of 2*pi, with 2*pi carried as a float head plus a float
-// tail and both products folded in by fma, then the hardware cosine
-// (__cosf), whose error bound holds on [-pi, pi]. Inputs are bf16 activations
-// (|x| of order 10 at most), where the reduced argument is accurate to a few
-// float ulps.
-__device__ __forceinline__ float cos_reduced(float x) {
-    constexpr float kInv2Pi = 0.159154943091895336f;          // 1 / (2 pi), rounded
-    constexpr float k2PiHi = 6.28318548202514648f;            // float(2 pi)
-    constexpr float k2PiLo = -1.74845553146951880e-07f;       // 2 pi - float(2 pi)
-    const float k = rintf(x * kInv2Pi);
-    float r = fmaf(-k, k2PiHi, x);
-    r = fmaf(-k, k2PiLo, r);
-    return __cosf(r);
-}
-
-// ELU+1 uses the hardware exponential (__expf) on x <= 0, where its relative
-// error is far below the bf16 hi/lo split's.
+// phi on a pair of values, with packed fp32x2 arithmetic where a step allows.
+// ELU+1 = max(x, 0) + e^min(x, 0): x + 1 above zero, e^x at or below, with
+// e^y = 2^(y log2 e) on the special-function unit (its relative error is far
+// below the bf16 hi/lo split's). cos: Cody-Waite additive range reduction
+// (W. J. Cody and W. Waite, "Software Manual for the Elementary Functions",
+// 1980) by the nearest multiple of 2*pi, with 2*pi carried as a float head
+// plus a float tail and both products folded in by fma, then the hardware
+// cosine (__cosf), whose error bound holds on [-pi, pi]. Inputs are bf16
+// activations (|x| of order 10 at most), where the reduced argument is
+// accurate to a few float ulps.
 template <int FM>
-__device__ __forceinline__ float feature_f32(float x) {
-    if constexpr (FM == kFeatureElu1) return x > 0.0f ? x + 1.0f : __expf(x);
-    else if constexpr (FM == kFeatureCos) return cos_reduced(x);
-    else return fmaxf(x, 0.0f);
+__device__ __forceinline__ float2 feature_f32x2(float2 x) {
+    if constexpr (FM == kFeatureElu1) {
+        constexpr float kLog2e = 1.4426950408889634f;
+        const float2 t = __fmul2_rn(make_float2(fminf(x.x, 0.0f), fminf(x.y, 0.0f)), make_float2(kLog2e, kLog2e));
+        return __fadd2_rn(make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f)),
+                          make_float2(ptx::ex2_approx(t.x), ptx::ex2_approx(t.y)));
+    } else if constexpr (FM == kFeatureCos) {
+        constexpr float kInv2Pi = 0.159154943091895336f;          // 1 / (2 pi), rounded
+        constexpr float k2PiHi = 6.28318548202514648f;            // float(2 pi)
+        constexpr float k2PiLo = -1.74845553146951880e-07f;       // 2 pi - float(2 pi)
+        const float2 q = __fmul2_rn(x, make_float2(kInv2Pi, kInv2Pi));
+        const float2 k = make_float2(rintf(q.x), rintf(q.y));
+        float2 r = __ffma2_rn(k, make_float2(-k2PiHi, -k2PiHi), x);   // x - k * head
+        r = __ffma2_rn(k, make_float2(-k2PiLo, -k2PiLo), r);          // ... - k * tail
+        return make_float2(__cosf(r.x), __cosf(r.y));
+    } else {
+        return make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f));
+    }
 }
 
 // phi of a packed bf16 pair, split into bf16 hi and lo parts: hi = bf16(phi),
 // lo = bf16(phi - hi), so hi + lo carries phi to ~2^-17 relative and products
 // on the tensor cores keep fp32-grade accuracy (ReLU needs no split: it is
-// exact in bf16).
+// exact in bf16). phi - hi is exact in fp32 and comes from one packed fma.
 template <int FM>
 __device__ __forceinline__ void feature_split_bf16x2(uint32_t packed, uint32_t& hi, uint32_t& lo) {
-    const float2 x = bf16x2_to_float2(packed);
-    const float a = feature_f32<FM>(x.x);
-    const float b = feature_f32<FM>(x.y);
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    const float2 hf = __bfloat1622float2(h);
-    __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    const float2 p = feature_f32x2<FM>(bf16x2_to_float2(packed));
+    __nv_bfloat162 h = __floats2bfloat162_rn(p.x, p.y);
+    const float2 d = __ffma2_rn(__bfloat1622float2(h), make_float2(-1.0f, -1.0f), p);
+    __nv_bfloat162 l = __floats2bfloat162_rn(d.x, d.y);
     hi = *reinterpret_cast<uint32_t*>(&h);
     lo = *reinterpret_cast<uint32_t*>(&l);
 }
