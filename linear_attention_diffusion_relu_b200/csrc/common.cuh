@@ -53,8 +53,11 @@ __device__ __forceinline__ float2 feature_f32x2(float2 x) {
         constexpr float kInv2Pi = 0.159154943091895336f;          // 1 / (2 pi), rounded
         constexpr float k2PiHi = 6.28318548202514648f;            // float(2 pi)
         constexpr float k2PiLo = -1.74845553146951880e-07f;       // 2 pi - float(2 pi)
+        // k = nearest integer to x / (2 pi): adding and subtracting 1.5 * 2^23
+        // rounds any |q| < 2^22 to an integer (ties to even) on the FMA pipe
+        constexpr float kRound = 12582912.0f;                     // 1.5 * 2^23
         const float2 q = __fmul2_rn(x, make_float2(kInv2Pi, kInv2Pi));
-        const float2 k = make_float2(rintf(q.x), rintf(q.y));
+        const float2 k = __fadd2_rn(__fadd2_rn(q, make_float2(kRound, kRound)), make_float2(-kRound, -kRound));
         float2 r = __ffma2_rn(k, make_float2(-k2PiHi, -k2PiHi), x);   // x - k * head
         r = __ffma2_rn(k, make_float2(-k2PiLo, -k2PiLo), r);          // ... - k * tail
         return make_float2(__cosf(r.x), __cosf(r.y));
