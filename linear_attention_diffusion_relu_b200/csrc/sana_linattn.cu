@@ -1144,7 +1144,8 @@ const char* sana_linattn_status_string(sana_la_status status) {
     switch (status) {
         case SANA_LA_OK: return "ok";
         case SANA_LA_ERR_INVALID_ARG: return "invalid argument";
-        case SANA_LA_ERR_UNSUPPORTED: return "unsupported head size (d must be 32 or 64)";
+        case SANA_LA_ERR_UNSUPPORTED:
+            return "unsupported sizes (d must be 32 or 64; the other limits are in the header)";
         case SANA_LA_ERR_WORKSPACE: return "workspace too small";
         case SANA_LA_ERR_CUDA: return "CUDA error";
     }
@@ -1184,7 +1185,12 @@ sana_la_status static_scratch_address(void** out) {
         set_last_error("cudaGetDevice", e);
         return SANA_LA_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) return SANA_LA_ERR_UNSUPPORTED;
+    if (dev < 0 || dev >= kMaxDevices) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "device ordinal %d is beyond the %d devices the static scratch address table holds",
+                      dev, kMaxDevices);
+        return SANA_LA_ERR_UNSUPPORTED;
+    }
     std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
     if (g_static_scratch_ptr[dev] == nullptr) {
         void* p = nullptr;
@@ -1221,7 +1227,3 @@ extern "C" sana_la_status sana_linattn_forward_noalloc(const void* Q, const void
     return sana_linattn_forward(Q, K, V, B, N, H, d, O, out_dtype, eps, scratch,
                                 kStaticScratchBytes, stream);
 }
-
-extern "C" {
-
-}  // extern "C"

@@ -199,18 +199,35 @@ class Oracle:
                 D += G[:, dy:dy + Hg, dx:dx + W, :] * Kdw[:, dy, dx]
         return D.reshape(B, N, Cc)
 
+    def expand(self, X, W1) -> np.ndarray:
+        """The 1x1 expand, stored as bf16: U = bf16(X W1^T), (B, N, 2 Ch)."""
+        X = np.asarray(X, dtype=np.float64)
+        W1 = np.asarray(W1, dtype=np.float64)
+        if W1.shape[1] != X.shape[-1]:
+            raise ValueError("W1 must be (2 Ch, C) with C matching X")
+        return self.round_bf16(X @ W1.T)
+
+    def depthwise_glu(self, U, Kdw, hw) -> np.ndarray:
+        """The 3x3 depthwise conv of U followed by the GLU with the sigmoid gate
+        on the channel halves, stored as bf16:
+        Z = bf16(D[..., :Ch] * sigmoid(D[..., Ch:])), D = depthwise3x3(U)."""
+        D = self.depthwise3x3(U, Kdw, hw)
+        Ch2 = D.shape[-1]
+        if Ch2 % 2:
+            raise ValueError("U must have an even channel count (2 Ch)")
+        Ch = Ch2 // 2
+        return self.round_bf16(D[..., :Ch] / (1.0 + np.exp(-D[..., Ch:])))
+
     def mix_ffn(self, X, W1, Kdw, W2, hw) -> np.ndarray:
-        """Y (B, N, C) for X (B, N, C), W1 (2 Ch, C), Kdw (2 Ch, 3, 3), W2 (C, Ch)."""
+        """Y (B, N, C) for X (B, N, C), W1 (2 Ch, C), Kdw (2 Ch, 3, 3), W2 (C, Ch):
+        expand, depthwise conv + GLU, then the 1x1 project Y = Z W2^T."""
         X = np.asarray(X, dtype=np.float64)
         W1 = np.asarray(W1, dtype=np.float64)
         W2 = np.asarray(W2, dtype=np.float64)
         Ch2 = W1.shape[0]
         if Ch2 % 2 or W2.shape[1] * 2 != Ch2 or W1.shape[1] != X.shape[2]:
             raise ValueError("weight shapes do not match")
-        Ch = Ch2 // 2
-        U = self.round_bf16(X @ W1.T)
-        D = self.depthwise3x3(U, Kdw, hw)
-        Z = self.round_bf16(D[..., :Ch] / (1.0 + np.exp(-D[..., Ch:])))
+        Z = self.depthwise_glu(self.expand(X, W1), Kdw, hw)
         return Z @ W2.T
 
     def block_causal_state(self, K, V, L: int) -> np.ndarray:

@@ -68,6 +68,15 @@ def _mix_ffn(orc, X, W1, Kdw, W2, hw, gate="glu", round_u=True, round_z=True, de
     return Z @ W2.T
 
 
+def _glu_stage(orc, U, Kdw, hw, gate="glu", rnd=True):
+    D = orc.depthwise3x3(U, Kdw, hw)
+    Ch = D.shape[-1] // 2
+    a, g = D[..., :Ch], D[..., Ch:]
+    sig = lambda t: 1.0 / (1.0 + np.exp(-t))
+    Z = {"glu": a * sig(g), "swapped": sig(a) * g, "silu": a * g * sig(g)}[gate]
+    return orc.round_bf16(Z) if rnd else Z
+
+
 # name -> (method replaced, factory of the replacement given the instance)
 MUTANTS = {
     "round_truncates": ("round_bf16", lambda o: lambda x: _round_bits(x, 8, np.trunc)),
@@ -89,6 +98,13 @@ MUTANTS = {
     "mix_ffn_u_not_rounded": ("mix_ffn", lambda o: lambda *a: _mix_ffn(o, *a, round_u=False)),
     "mix_ffn_z_not_rounded": ("mix_ffn", lambda o: lambda *a: _mix_ffn(o, *a, round_z=False)),
     "mix_ffn_no_depthwise": ("mix_ffn", lambda o: lambda *a: _mix_ffn(o, *a, depthwise=False)),
+    "stage_glu_halves_swapped": ("depthwise_glu", lambda o: lambda U, K, hw: _glu_stage(o, U, K, hw, gate="swapped")),
+    "stage_glu_silu_gate": ("depthwise_glu", lambda o: lambda U, K, hw: _glu_stage(o, U, K, hw, gate="silu")),
+    "stage_glu_not_rounded": ("depthwise_glu", lambda o: lambda U, K, hw: _glu_stage(o, U, K, hw, rnd=False)),
+    "stage_expand_not_rounded": ("expand", lambda o: lambda X, W1: np.asarray(X, dtype=np.float64)
+                                 @ np.asarray(W1, dtype=np.float64).T),
+    "stage_expand_transposed_weights": ("expand", lambda o: lambda X, W1: o.round_bf16(
+        np.asarray(X, dtype=np.float64) @ np.asarray(W1, dtype=np.float64).reshape(-1, W1.shape[0]))),
 }
 
 
@@ -108,6 +124,8 @@ def test_unmutated_copies_pass_every_pin():
     Kd2 = rng.standard_normal((6, 3, 3))
     assert np.allclose(_mix_ffn(orc, X2, W1, Kd2, W2, (3, 4)), orc.mix_ffn(X2, W1, Kd2, W2, (3, 4)),
                        rtol=1e-13, atol=1e-13)
+    U2 = orc.expand(X2, W1)
+    assert np.array_equal(_glu_stage(orc, U2, Kd2, (3, 4)), orc.depthwise_glu(U2, Kd2, (3, 4)))
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
