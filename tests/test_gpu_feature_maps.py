@@ -1,7 +1,7 @@
 """Parity of the ELU+1 and cos feature maps ("08_sana高效高分辨率生成", section
 "Linear Attention 的原理": alternatives to ReLU) with the fp64 oracle, through the
 C ABI: every element at small and mid-size shapes (ragged, head size 64, more
-slabs than SMs), sampled heads at the 4096px shape, the states themselves,
+slabs than SMs; the 4096px shape is in test_gpu_headline_full.py), the states themselves,
 forward == kv_state + apply bit for bit, and ReLU through the feature-map
 entry points == the plain calls bit for bit."""
 from dataclasses import replace
@@ -12,7 +12,7 @@ import torch
 
 from linear_attention_diffusion_relu_b200 import ops
 from linear_attention_diffusion_relu_b200.workloads import WORKLOADS, Workload, make_inputs
-from tests.parity import check_output, head_slice, to_f64
+from tests.parity import check_output, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -64,19 +64,6 @@ def test_feature_map_state(oracle, feature):
     mag = np.einsum("bnhi,bnhj->bhij", phi, v1)
     err = np.abs(to_f64(S) - ref)
     assert np.all(err <= 1e-5 * mag + 1e-30), (err / (mag + 1e-30)).max()
-
-
-@pytest.mark.parametrize("feature", FEATURES)
-@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
-def test_feature_map_4096px_sampled_heads(oracle, feature, dtype):
-    w = WORKLOADS["4096px"]
-    Q, K, V = make_inputs(w, device="cuda")
-    heads = [0, w.H // 2, w.H - 1]
-    O = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps, feature_map=feature)
-    torch.cuda.synchronize()
-    Qh, Kh, Vh = (head_slice(t, heads) for t in (Q, K, V))
-    ref = oracle.forward_fm(Qh, Kh, Vh, feature, w.eps)
-    check_output(O[:, :, heads, :], ref, f"4096px {feature} heads {heads}")
 
 
 @pytest.mark.parametrize("feature", FEATURES)

@@ -3,13 +3,23 @@ ReLU(K)^T V product fused into the QKV projection: SANA walk-through, section 4
 "On-Device Deployment") with the oracle, through the C ABI.
 
 The oracle projects in fp64 and rounds K and V to bf16; the kernel accumulates
-the projection in fp32 before the same rounding, so a small fraction (~1e-4 to
-1e-3, growing with C) of K and V elements land one bf16 step (at most 2^-7
-relative) apart. A state entry sum_n t_n, t_n = phi(K_ni) [V | 1]_nj, is
-therefore held to 1e-4 of sum_n |t_n| plus four such steps of its largest term
-(an O(1) error from a wrong layout, head, token or feature fails by orders of
-magnitude). End to end, apply() on that state is held to 1e-3 per row (fp32)
-and to the forward's bf16 output tolerance."""
+the projection in fp32 before the same rounding, so a small fraction f (~1e-4
+to 1e-3, growing with C; measured below) of K and V elements land one bf16
+step (at most 2^-7 relative) apart ("flips"). A state entry sum_n t_n,
+t_n = phi(K_ni) [V | 1]_nj, is therefore held to 1e-4 of sum_n |t_n| plus four
+such steps of its largest term (an O(1) error from a wrong layout, head, token
+or feature fails by orders of magnitude).
+
+End to end the flips do not cancel the way the state's own terms do: a
+numerator entry sum_n t_n over zero-mean V is a random walk of size
+sqrt(N) rms(t), and the flips add sqrt(f N) 2^-8 rms(t) to it, so the output
+rows move by about sqrt(f) 2^-8 of their norm (~1e-4 at f = 1e-3), which is as
+large as the forward's own 1e-4 bar. So the end-to-end check has two parts:
+apply() on the GPU's state is held to the forward's tolerance against the
+oracle's apply of that same state, and the output against the oracle's
+end-to-end forward is held to that tolerance plus the first-order propagation
+of the state's measured deviation, |dO_i| <= (phi(Q) |dS[:, i]| +
+|O_i| phi(Q) |dS[:, d]|) / (den + eps), whose entries the state check bounds."""
 import numpy as np
 import pytest
 import torch
@@ -82,9 +92,12 @@ def test_projected_state_matches_oracle(oracle, shape):
 
 
 def test_projected_state_end_to_end_and_deterministic(oracle):
-    """apply() on the fused state meets the forward's output tolerance against
-    the oracle forward of the projected K and V; repeated calls give the same bits."""
+    """apply() on the fused state meets the forward's tolerance against the
+    oracle's apply of the same state; against the oracle's whole forward of the
+    projected K and V it meets that tolerance plus the propagated state
+    deviation; repeated calls give the same bits."""
     B, N, C, H, d = 2, 777, 512, 8, 32
+    eps = 1e-15
     X, Wk, Wv = _inputs(B, N, C, H, d, seed=5)
     Q = torch.randn((B, N, H, d), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).cuda()
     S1 = ops.kv_projection_state(X, Wk, Wv, H)
@@ -93,12 +106,47 @@ def test_projected_state_end_to_end_and_deterministic(oracle):
     O16 = ops.apply(Q, S1, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert torch.equal(S1.view(torch.int32), S2.view(torch.int32))
+    Qd, Sd = to_f64(Q), to_f64(S1)
+    _check_state(oracle, S1, X, Wk, Wv, H)
+    # the apply on the GPU's own state: the forward's tolerance
+    same = oracle.apply(Qd, Sd, eps)
+    check_output(O32, same, "apply on the projected state (fp32 out)")
+    check_output(O16, same, "apply on the projected state (bf16 out)")
+    # end to end: that tolerance plus the state's deviation carried through the apply
     K, V = oracle.project_kv(to_f64(X), to_f64(Wk), to_f64(Wv), H)
-    ref = oracle.forward(to_f64(Q), K, V, 1e-15)
-    check_output(O16, ref, "projected state, end to end (bf16 out)")
+    S_ref = oracle.state(K, V)
+    ref, den = oracle.apply(Qd, S_ref, eps, return_den=True)
+    dS = np.abs(Sd - S_ref)
+    phiQ = np.maximum(Qd, 0.0)
+    d_num = np.einsum("bnhk,bhki->bnhi", phiQ, dS[..., :d])
+    d_den = np.einsum("bnhk,bhk->bnh", phiQ, dS[..., d])
+    prop = (d_num + np.abs(ref) * d_den[..., None]) / (den + eps)[..., None]
     got = to_f64(O32)
-    rel = np.linalg.norm(got - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
-    assert rel.max() <= 1e-3, rel.max()
+    err = np.linalg.norm(got - ref, axis=-1)
+    bound = 1e-4 * np.linalg.norm(ref, axis=-1) + 1.01 * np.linalg.norm(prop, axis=-1) + 1e-30
+    assert np.all(err <= bound), (err / bound).max()
+
+
+def test_flip_fraction_of_fp32_projection(oracle):
+    """The mechanism behind the bounds above, measured: K from an fp32
+    accumulation (cuBLAS bf16 matmul) against the oracle's fp64 projection,
+    both rounded to bf16, differ in a small fraction of elements, each by one
+    bf16 step of the value or, where the dot product cancels to near zero, by
+    the fp32 accumulation error C 2^-24 sum |x w| carrying the rounding across
+    a step (the bound of the Mix-FFN expand check)."""
+    B, N, C, H, d = 2, 2048, 2240, 70, 32
+    X, Wk, Wv = _inputs(B, N, C, H, d, seed=11)
+    K = (X @ Wk.T).view(B, N, H, d)
+    torch.cuda.synchronize()
+    Xd, Wd = to_f64(X), to_f64(Wk)
+    Kr, _ = oracle.project_kv(Xd, Wd, Wd, H)
+    Kg = to_f64(K)
+    diff = Kg != Kr
+    f = float(diff.mean())
+    assert f < 1e-2, f
+    mag = (np.abs(Xd) @ np.abs(Wd).T).reshape(B, N, H, d)
+    bound = 2.0 ** -7 * np.abs(Kr) + C * 2.0 ** -23 * mag
+    assert np.all(np.abs(Kg - Kr) <= bound), (np.abs(Kg - Kr) / bound).max()
 
 
 def test_projected_state_agrees_with_unfused_path():
@@ -118,21 +166,23 @@ def test_projected_state_agrees_with_unfused_path():
     assert np.all(np.abs(err) <= bound), (np.abs(err) / bound).max()
 
 
-def test_projected_state_4096px_sampled_heads(oracle):
+def test_projected_state_4096px_every_head(oracle):
     """The bench's 4096px shape (B = 2, N = 16384, C = 2240, H = 70), in the
-    launch configuration the bench times: three heads' states (first, middle,
-    last group) against the oracle's projection and state of those heads."""
+    launch configuration the bench times: every head's state against the
+    oracle's projection and state of that head (ten heads at a time)."""
     B, N, C, H, d = 2, 16384, 2240, 70, 32
     X, Wk, Wv = _inputs(B, N, C, H, d, seed=N + C)
     S = ops.kv_projection_state(X, Wk, Wv, H)
     torch.cuda.synchronize()
     assert ops.device_error() == 0
     Xd = to_f64(X)
-    for h in (0, 37, H - 1):
-        rows = slice(h * d, (h + 1) * d)
-        K, V = oracle.project_kv(Xd, to_f64(Wk[rows]), to_f64(Wv[rows]), 1)
-        ref = oracle.state(K, V)[:, 0]
-        mag = oracle.state(K, np.abs(V))[:, 0]
-        err = np.abs(to_f64(S[:, h]) - ref)
-        bound = _bound(K, V, mag[:, None])[:, 0]
-        assert np.all(err <= bound), (h, (err / bound).max())
+    Sd = to_f64(S)
+    for h0 in range(0, H, 10):
+        h1 = min(H, h0 + 10)
+        rows = slice(h0 * d, h1 * d)
+        K, V = oracle.project_kv(Xd, to_f64(Wk[rows]), to_f64(Wv[rows]), h1 - h0)
+        ref = oracle.state(K, V)
+        mag = oracle.state(K, np.abs(V))
+        err = np.abs(Sd[:, h0:h1] - ref)
+        bound = _bound(K, V, mag)
+        assert np.all(err <= bound), (h0, (err / bound).max())

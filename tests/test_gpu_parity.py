@@ -1,8 +1,8 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
-Small and mid-size shapes compare every output element; the full-size Sana
-shapes compare every row of sampled heads (the oracle rebuilds those heads'
-states from all N tokens). Also: determinism, forward == kv_state + apply bit
+Every output element is compared, from single tokens up to the N = 65536
+sweep point (the 4096px shapes and the longest sweep points are in
+test_gpu_headline_full.py). Also: determinism, forward == kv_state + apply bit
 for bit, guard bands around outputs and workspace, streams, error paths."""
 from dataclasses import replace
 
@@ -12,7 +12,7 @@ import torch
 
 from linear_attention_diffusion_relu_b200 import ops
 from linear_attention_diffusion_relu_b200.workloads import WORKLOADS, Workload, make_inputs
-from tests.parity import check_output, head_slice, to_f64
+from tests.parity import check_output, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -42,8 +42,12 @@ def _full_check(oracle, Q, K, V, eps, dtype, what):
 
 SMALL = [(1, 1, 1, 32), (1, 7, 3, 32), (2, 31, 2, 64), (1, 129, 5, 32), (2, 1000, 3, 32),
          (1, 4097, 2, 64), (3, 513, 7, 32), (1, 2048, 70, 32), (2, 300, 18, 64),
+         # two slab sets with an odd slab count: one position holds a single slab
+         (1, 3000, 60, 32), (1, 1000, 68, 32),
          # more (b, head-group) slabs than CTAs: several segments per CTA
-         (5, 100, 150, 32), (16, 200, 20, 64)]
+         (5, 100, 150, 32), (16, 200, 20, 64),
+         # more than two segments per CTA: the three-kernel path
+         (40, 64, 70, 32)]
 
 
 @pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
@@ -66,42 +70,21 @@ def test_named_configs_every_element(oracle, name, dtype):
         assert torch.all(O[0, rows] == 0)
 
 
-def _sampled_heads_check(oracle, w, Q, K, V, dtype, heads, rows=None):
-    O = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps)
-    torch.cuda.synchronize()
-    Qh, Kh, Vh = (head_slice(t, heads) for t in (Q, K, V))
-    S = oracle.state(Kh, Vh)
-    if rows is not None:
-        Qh = Qh[:, rows]
-    ref = oracle.apply(Qh, S, w.eps)
-    got = O[:, :, list(heads), :]
-    if rows is not None:
-        got = got[:, torch.as_tensor(rows, device=O.device)]
-    check_output(got, ref, f"{w.name} heads {heads}")
+FULL = ["ragged_N16381", "d64", "sweep_N1024", "sweep_N16384", "sweep_N65536"]
 
 
-FULL = ["4096px", "ragged_N16381", "d64", "sweep_N1024", "sweep_N16384", "sweep_N65536"]
-
-
-@pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled_heads(oracle, name, dtype):
+def test_full_size_every_element(oracle, name):
+    """Every element of the mid-size workloads (ragged N, head size 64, the
+    sweep up to N = 65536) for both output dtypes; the 4096px shapes and the
+    longest sweep points are in test_gpu_headline_full.py."""
     w = WORKLOADS[name]
     Q, K, V = make_inputs(w, device="cuda")
-    heads = sorted({0, w.H // 2, w.H - 1})
-    _sampled_heads_check(oracle, w, Q, K, V, dtype, heads)
-
-
-@pytest.mark.parametrize("name", ["sweep_N262144", "sweep_N1048576"])
-def test_longest_sweep_sampled_rows(oracle, name):
-    """Largest token counts: inputs drawn with the seeded CUDA generator; the
-    oracle rebuilds two heads' states from all N tokens and checks 4096 rows."""
-    w = WORKLOADS[name]
-    Q, K, V = make_inputs(w, device="cuda", generator_device="cuda")
-    rows = np.sort(np.random.default_rng(0).choice(w.N, size=4096, replace=False))
-    rows[0], rows[-1] = 0, w.N - 1
+    ref = oracle.forward(to_f64(Q), to_f64(K), to_f64(V), w.eps)
     for dtype in OUT_DTYPES:
-        _sampled_heads_check(oracle, w, Q, K, V, dtype, [1, w.H - 2], rows=rows)
+        O = ops.forward(Q, K, V, out_dtype=dtype, eps=w.eps)
+        torch.cuda.synchronize()
+        check_output(O, ref, f"{name} {dtype}")
 
 
 def test_state_matches_oracle(oracle):
@@ -135,7 +118,7 @@ def test_deterministic_and_split_equals_forward(dtype):
 
 
 BITWISE = [(1, 1, 1, 32), (2, 31, 2, 64), (2, 1531, 6, 32), (5, 100, 150, 32), (16, 200, 20, 64),
-           (1, 16381, 36, 32)]
+           (1, 16381, 36, 32), (1, 3000, 60, 32), (40, 64, 70, 32)]
 
 
 @pytest.mark.parametrize("dtype", OUT_DTYPES, ids=_dt)
