@@ -42,12 +42,10 @@ WORKLOAD = "4096px"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
-# the same build (profiles/), keyed by (kernel set, workload, kernel); None when
-# the kernels changed since the counters were taken
+# the same build and workload, keyed by (kernel set, workload, kernel, output
+# bytes per element); absent when the kernels changed since the counters were
+# taken
 TRAFFIC_PER_LAUNCH = {
-    # profiles/fwd_fused_tc_sweep_N65536.md: (453.09 + 93.36) MB at B=1, N=65536, H=36
-    # (DRAM counters of the current kernel), scaled by token-heads to 4096px (x 0.9722)
-    ("tcgen05-tma", "4096px", "fwd_fused_tc"): 531.3e6,
 }
 SMS = 148
 FP32_LANES_PER_SM = 128
@@ -321,9 +319,12 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
     start.record(stream)
-    for _ in range(args.steps):
+    for k in range(args.steps):
         step()
+        if k < args.steps - 1:
+            marks[k].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -331,6 +332,8 @@ def run_ours(args):
     clk = clocks.stop()
 
     ms = start.elapsed_time(end) / args.steps
+    bounds = [start, *marks, end]
+    per_step = [bounds[k].elapsed_time(bounds[k + 1]) for k in range(args.steps)]
     ms_max = max_over_ranks(ms, dev)
     bytes_per_step = w.algorithmic_bytes(2)
     value = aggregate_gbs(bytes_per_step, world, ms_max / 1e3)
@@ -370,14 +373,19 @@ def run_ours(args):
     else:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": TRAFFIC_PER_LAUNCH.get((impl["name"], w.name, dom)),
+                "frac": achieved / hbm_peak, "traffic": TRAFFIC_PER_LAUNCH.get((impl["name"], w.name, dom, 2)),
                 "kernel": dom, "peak_source": f"{peak_src} copy bandwidth (burst)"}
     roof["ms_per_launch"] = dom_ms
     roof["algorithmic_bytes_per_launch"] = dom_bytes
+    if launches == 1:
+        roof["ms_per_launch_median"] = statistics.median(per_step)
+        roof["ms_per_launch_min"] = min(per_step)
     roof["split_api_ms"] = {"kv_state(KS+KR)": ks_ms, "apply(KA)": ka_ms}
     roof["timing"] = ("launch duration: CUDA events over the timed region / steps (one launch per "
                       "step); split_api_ms: events around kv_state and apply in a "
                       f"{n_split}-step loop of the two-call API after the timed region")
+
+    fp32 = None if L else run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl)
 
     e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, world)
 
@@ -403,7 +411,8 @@ def run_ours(args):
                        "l2": (f"inputs {w.token_heads * d * 6 / 1e6:.0f} MB + output "
                               f"{w.token_heads * d * 2 / 1e6:.0f} MB per step vs the 126 MB L2; no flush"),
                        "kernel_impl": impl["name"]},
-            "roofline": roof, "e2e": e2e, "clocks": clk,
+            "ms_per_step_median": statistics.median(per_step), "ms_per_step_min": min(per_step),
+            "roofline": roof, "fp32_out": fp32, "e2e": e2e, "clocks": clk,
             "gpu_launches": launches * args.steps,
         }
         if cpu is not None:
@@ -415,36 +424,67 @@ def run_ours(args):
     return 0
 
 
+def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl):
+    """The same forward with O in fp32 (the output type the 1e-4 per-row
+    tolerance is stated for): its own timed loop after the main one, the same
+    step count and per-step events, algorithmic bytes with 4-byte outputs."""
+    import torch
+    from linear_attention_diffusion_relu_b200 import ops
+    out32 = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.float32, device=dev)
+
+    def step():
+        ops.forward(Q, K, V, out_dtype=torch.float32, eps=w.eps, out=out32, workspace=ws, feature_map=w.feature)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for k in range(args.steps):
+        step()
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per_step = [ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)]
+    ms = ev[0].elapsed_time(ev[-1]) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+    nbytes = w.algorithmic_bytes(4)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {
+        "value": aggregate_gbs(nbytes, world, ms_max / 1e3), "unit": UNIT, "ms_per_step": ms_max,
+        "ms_per_step_median": statistics.median(per_step), "ms_per_step_min": min(per_step),
+        "mtokens_per_s": w.B * w.N * world / (ms_max / 1e3) / 1e6,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "kernel": "fwd_fused_tc",
+                     "traffic": TRAFFIC_PER_LAUNCH.get((impl["name"], w.name, "fwd_fused_tc", 4)),
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "peak_source": f"{peak_src} copy bandwidth (burst)"},
+        "io": "bf16 Q/K/V in, fp32 O out",
+    }
+
+
 def run_e2e(args, w, dev, stream, world):
     """Same metric through the public call with host buffers: every step copies
-    Q, K, V from pinned host memory to the device and O back. The plain forward
-    goes through ops.forward_host (the library makes the copies: K and V in, the
-    state, then Q streamed through in chunks whose outputs are copied back while
-    the next chunk comes in); the block-causal form copies with torch around
-    block_causal_forward."""
+    Q, K, V from pinned host memory to the device and O back, the copies made
+    by the library (ops.forward_host, or ops.block_causal_forward_host): K and
+    V in, the state (or the blocks' prefix states), then Q streamed through in
+    chunks whose outputs are copied back while the next chunk comes in."""
     import torch
     from linear_attention_diffusion_relu_b200 import ops
     from linear_attention_diffusion_relu_b200.workloads import make_inputs
     hQ, hK, hV = (t.cpu().pin_memory() for t in make_inputs(w, generator_device=input_generator(w)))
     hO = torch.empty(hQ.shape, dtype=torch.bfloat16).pin_memory()
-    dQ, dK, dV = (torch.empty_like(t, device=dev) for t in (hQ, hK, hV))
-    dO = torch.empty(hQ.shape, dtype=torch.bfloat16, device=dev)
     L = w.block
     if L:
-        ws = ops.make_block_causal_workspace(w.B, w.N, w.H, w.d, L, dev)
+        ws = torch.empty(ops.block_causal_forward_host_workspace_bytes(w.B, w.N, w.H, w.d, L, torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
     else:
-        del dQ, dK, dV, dO
         ws = torch.empty(ops.forward_host_workspace_bytes(w.B, w.N, w.H, w.d, torch.bfloat16),
                          dtype=torch.uint8, device=dev)
 
     def one():
         if L:
-            dQ.copy_(hQ, non_blocking=True)
-            dK.copy_(hK, non_blocking=True)
-            dV.copy_(hV, non_blocking=True)
-            ops.block_causal_forward(dQ, dK, dV, L, out_dtype=torch.bfloat16, eps=w.eps, out=dO,
-                                     workspace=ws)
-            hO.copy_(dO, non_blocking=True)
+            ops.block_causal_forward_host(hQ, hK, hV, L, out_dtype=torch.bfloat16, eps=w.eps, out=hO,
+                                          workspace=ws, device=dev)
         else:
             ops.forward_host(hQ, hK, hV, out_dtype=torch.bfloat16, eps=w.eps, out=hO, workspace=ws,
                              feature_map=w.feature, device=dev)
@@ -463,7 +503,7 @@ def run_e2e(args, w, dev, stream, world):
     d2h = hO.numel() * hO.element_size()
     return {"value": aggregate_gbs(w.algorithmic_bytes(2), world, ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "call": "block_causal_forward, torch copies" if L else "forward_host (copies by the library)"}
+            "call": ("block_causal_forward_host" if L else "forward_host") + " (copies by the library)"}
 
 
 def run_kvproj(args):

@@ -36,9 +36,10 @@
  *   allocates, frees or synchronises. All work is enqueued on `stream`
  *   (NULL = the legacy default stream) and the calls return as soon as it is
  *   enqueued. Inputs must not alias outputs. The result is deterministic: the
- *   same inputs and sizes give bit-identical outputs on every run, and
- *   sana_linattn_forward gives exactly the bits of sana_linattn_kv_state
- *   followed by sana_linattn_apply.
+ *   same inputs and sizes give bit-identical outputs on every run (on devices
+ *   with the same number of SMs: the work is split into one persistent CTA
+ *   per SM), and sana_linattn_forward gives exactly the bits of
+ *   sana_linattn_kv_state followed by sana_linattn_apply.
  *
  * Errors
  *   Arguments are checked on the host before anything is launched; on any
@@ -47,7 +48,8 @@
  *                              aligned, eps negative or not finite, an unknown
  *                              output dtype, or sizes whose element count
  *                              overflows 63 bits;
- *     SANA_LA_ERR_UNSUPPORTED  d not 32 or 64;
+ *     SANA_LA_ERR_UNSUPPORTED  d not 32 or 64 (the calls below state their
+ *                              other limits);
  *     SANA_LA_ERR_WORKSPACE    workspace smaller than sana_linattn_workspace_bytes;
  *     SANA_LA_ERR_CUDA         a CUDA call or launch failed (details from
  *                              sana_linattn_last_error()).
@@ -91,9 +93,12 @@ typedef enum {
 
 /*
  * Bytes of device workspace that sana_linattn_kv_state and
- * sana_linattn_forward need for these sizes (a pure function of the sizes).
- * The workspace holds the fp32 partial states of the token chunks, and for
- * sana_linattn_forward also the reduced state. Returns 0 for invalid or
+ * sana_linattn_forward need for these sizes on the current device (a function
+ * of the sizes and of the device's SM count; with no device to ask, the
+ * B200's 148). The workspace holds the fp32 partial states of the token
+ * chunks, and for sana_linattn_forward also the reduced states (staged as
+ * bf16 hi + lo parts for the apply), the fp32 state of the three-kernel
+ * fallback and four readiness flags per CTA. Returns 0 for invalid or
  * unsupported sizes. Any content is acceptable on entry; it is scratch.
  */
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d);
@@ -134,13 +139,18 @@ sana_la_status sana_linattn_apply(const void* Q, const float* state,
  * The whole forward: sana_linattn_kv_state into the workspace, then
  * sana_linattn_apply. Same arguments and rules as the two calls above; the
  * result is bit-identical to calling them in sequence.
- * It runs as one cooperative kernel launch (state phase, grid-wide barrier,
- * apply phase). The barrier uses per-CTA flags in the workspace tagged with a
- * number unique to the call, so the workspace needs no initialisation. Under
- * stream capture the call also records a memset of those flags before the
- * kernel, because a replayed graph reuses the captured number. Where the
- * device cannot hold the whole grid at once, the call falls back to the
- * kernels of the two calls above.
+ * It runs as one cooperative kernel launch: the state phase, a reduction of
+ * each (b, head group)'s partial states shared by the CTAs that made them (in
+ * the order sana_linattn_kv_state sums them), and the apply phase. The head
+ * groups are taken in two sets, so the first set's reduction runs while the
+ * second set's keys stream in and the second set's while the first set's
+ * queries are applied. CTAs signal each other through flags in the workspace
+ * tagged with a number unique to the call, so the workspace needs no
+ * initialisation. Under stream capture the call also records a memset of
+ * those flags before the kernel, because a replayed graph reuses the captured
+ * number. Where the device cannot hold the whole grid at once, or B times the
+ * head groups exceeds twice the SM count, the call runs the kernels of the
+ * two calls above instead.
  */
 sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     int B, int N, int H, int d,
@@ -293,6 +303,38 @@ sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, c
 
 /* Kernel launches one sana_linattn_block_causal_forward call enqueues (0 if invalid). */
 int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L);
+
+/*
+ * sana_linattn_block_causal_forward from and to HOST memory, with the copies
+ * overlapped by the library as in sana_linattn_forward_host (below): K and V
+ * are copied in and the prefix states computed over all blocks; then Q is
+ * streamed in chunks of whole blocks of one batch (about a sixteenth of the
+ * tokens, at least one block), each chunk applied against its blocks' prefix
+ * states as soon as it is in, its O copied out on the library's
+ * device-to-host stream while later chunks come in.
+ *   Q, K, V   host, (B, N, H, d) bf16 row-major
+ *   O         host, (B, N, H, d) fp32 or bf16 by out_dtype
+ *   workspace device, sana_linattn_block_causal_forward_host_workspace_bytes
+ *             (B, N, H, d, L, out_dtype) bytes, 16-byte aligned: device
+ *             copies of Q, K, V and O, the prefix states and the partials
+ * O is bit-identical to sana_linattn_block_causal_forward's on the same
+ * inputs (the apply of a token depends only on its block's prefix state).
+ * Page-locked host buffers make the copies asynchronous; ownership, streams
+ * and errors as for sana_linattn_forward_host; L as for the block-causal
+ * calls above (L < 1: SANA_LA_ERR_INVALID_ARG; not a multiple of 128:
+ * SANA_LA_ERR_UNSUPPORTED).
+ */
+size_t sana_linattn_block_causal_forward_host_workspace_bytes(int B, int N, int H, int d, int L,
+                                                              sana_la_out_dtype out_dtype);
+
+sana_la_status sana_linattn_block_causal_forward_host(const void* Q, const void* K, const void* V,
+                                                      int B, int N, int H, int d, int L,
+                                                      void* O, sana_la_out_dtype out_dtype, float eps,
+                                                      void* workspace, size_t workspace_bytes,
+                                                      sana_la_stream_t stream);
+
+/* Kernel launches one sana_linattn_block_causal_forward_host call enqueues (0 if invalid). */
+int sana_linattn_block_causal_forward_host_launches(int B, int N, int H, int d, int L);
 
 /*
  * sana_linattn_forward without a workspace argument, for callers that cannot

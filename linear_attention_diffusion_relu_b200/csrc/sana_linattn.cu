@@ -28,54 +28,123 @@ void set_last_error(const char* where, cudaError_t e) {
                   cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-constexpr int kSMs = 148;             // B200: one persistent CTA per SM
+constexpr int kDefaultSMs = 148;      // B200; the plans' CTA count when no device can be asked
 constexpr int kMaxDevicesCached = 64; // per-device caches of launch properties
+
+// Streaming multiprocessors of the current device (one persistent CTA runs on
+// each), asked once per device; kDefaultSMs when no device answers (the size
+// queries work on a host without a GPU). The work plans, and so the workspace
+// size and the order of the partial sums, follow this count: results are
+// bit-reproducible on devices with the same number of SMs.
+int device_sms() {
+    static std::atomic<int> cache[kMaxDevicesCached];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return kDefaultSMs;
+    }
+    if (dev >= 0 && dev < kMaxDevicesCached) {
+        const int v = cache[dev].load(std::memory_order_acquire);
+        if (v > 0) return v;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return kDefaultSMs;
+    }
+    if (dev >= 0 && dev < kMaxDevicesCached) cache[dev].store(sms, std::memory_order_release);
+    return sms;
+}
+
+// A unique id of the calling thread's current CUDA context (cuCtxGetId), or
+// 0 when there is none or the driver cannot be asked. The per-device caches
+// below (function attributes, copy streams and events, the scratch address)
+// remember the context they were made in and are made again when it changed,
+// e.g. after cudaDeviceReset destroyed the primary context.
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static std::once_flag once;
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+        return 0;
+    unsigned long long id = 0;
+    return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
 constexpr long long kMaxElems = 1LL << 62;
 constexpr long long kMaxGrid = 0x7fffffffLL;
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Work plans of the three kernels. A pure function of the sizes: the
-// workspace size and the order in which partial states are summed never
-// depend on the device or on timing.
+// Work plans of the kernels. A pure function of the sizes: the workspace
+// size and the order in which partial states are summed never depend on the
+// device or on timing.
 struct Plan {
     sana::tc::KsParams ks;
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
+    size_t staged_bytes;    // single launch: one reduced state per slab, staged as bf16 hi + lo
     size_t state_bytes;     // fp32 (B, H, d, d+1); block-causal (B, H, nblk, d, d+1)
-    size_t flag_bytes;      // grid-barrier flags of the single-launch forward (one per CTA)
+    size_t flag_bytes;      // single launch: four readiness flags per CTA
 };
 
-// Lockstep schedule of S slabs of T tiles over at most kSMs CTAs (see the
-// comment at the top of tc_kernels.cuh).
-sana::tc::Sched make_sched(long long S, long long T) {
+// Lockstep schedule of S slabs of T tiles over at most `sms` CTAs, in one or
+// two sets (see the comment at the top of tc_kernels.cuh).
+sana::tc::Sched make_sched(long long S, long long T, int sms, int nset = 1) {
     sana::tc::Sched q{};
     q.S = (int)S;
     q.T = (int)T;
-    if (S <= kSMs) {
-        q.R = (int)std::min<long long>(kSMs / S, T);
-        q.grid = (int)(S * q.R);
+    if (nset == 2) {
+        q.P = (int)cdiv(S, 2);
+        q.R = (int)std::max<long long>(1, std::min<long long>(sms / q.P, T));
+        q.max_seg = 2;
+    } else if (S <= sms) {
+        q.P = (int)S;
+        q.R = (int)std::min<long long>(sms / S, T);
+        q.max_seg = 1;
     } else {
+        q.P = sms;
         q.R = 1;
-        q.grid = kSMs;
+        q.max_seg = (int)cdiv(S, sms);
     }
-    q.max_seg = (int)cdiv(S, q.grid);
+    q.grid = q.P * q.R;
     q.nblk = 1;
     q.tpb = 0;
     q.rb = 1;
     return q;
 }
 
+// Two sets when every position then holds two slabs (even S), or when the one
+// position with a single slab idles little (S >= 15), and the single launch can
+// still give every CTA at most two segments.
+int plan_sets(long long S, int sms) {
+    return (S >= 2 && S <= 2LL * sms && (S % 2 == 0 || S >= 15)) ? 2 : 1;
+}
+
 // Block-causal schedule: S slabs of nblk blocks of bt tiles; a slab's
 // rb * rt CTAs split its blocks rb ways and each block's tiles rt ways (rt
 // divides bt).
-sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int rb, int rt) {
+sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int rb, int rt, int sms) {
     sana::tc::Sched q{};
     q.S = (int)S;
     q.T = (int)(nblk * bt);
     q.R = rb * rt;
-    q.grid = S <= kSMs ? (int)(S * q.R) : kSMs;
+    q.P = S <= sms ? (int)S : sms;
+    q.grid = S <= sms ? (int)(S * q.R) : sms;
     q.nblk = (int)nblk;
     q.tpb = (int)(bt / rt);
     q.rb = rb;
@@ -84,8 +153,8 @@ sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int 
 }
 
 // How the CTAs of a slab split a block-causal slab (S slabs, nblk blocks of
-// tiles128 128-token tiles; at most 148 CTAs): the split (rb, rt), rb * rt <=
-// 148 / S and rt dividing tiles128, that minimises the tiles of the busiest
+// tiles128 128-token tiles; at most `sms` CTAs): the split (rb, rt), rb * rt <=
+// sms / S and rt dividing tiles128, that minimises the tiles of the busiest
 // CTA plus three tiles' worth for each state it stages (one per block it
 // visits), times 1.15 when rb > 1; ties go to fewer partial states per block
 // (smaller rt). The factor stands for what reading rb token regions at once
@@ -96,9 +165,9 @@ sana::tc::Sched make_block_sched(long long S, long long nblk, long long bt, int 
 struct BlockSplit {
     int rb, rt;
 };
-BlockSplit block_split(long long S, long long nblk, long long tiles128) {
-    if (S > kSMs) return BlockSplit{1, 1};
-    const long long rmax = kSMs / S;
+BlockSplit block_split(long long S, long long nblk, long long tiles128, int sms) {
+    if (S > sms) return BlockSplit{1, 1};
+    const long long rmax = sms / S;
     BlockSplit best{1, 1};
     long long best_cost = -1;
     for (long long rt = 1; rt <= std::min(rmax, tiles128); ++rt) {
@@ -115,7 +184,7 @@ BlockSplit block_split(long long S, long long nblk, long long tiles128) {
 
 // L = 0: the plain forward; L > 0 (a multiple of 128): block-causal with
 // blocks of L tokens.
-Plan make_plan(int B, int N, int H, int d, int L = 0) {
+Plan make_plan(int B, int N, int H, int d, int L = 0, int sms = device_sms()) {
     const int G = 128 / d;                        // heads per 128-row group
     const long long groups = cdiv(H, G);
     const long long S = (long long)B * groups;
@@ -130,20 +199,28 @@ Plan make_plan(int B, int N, int H, int d, int L = 0) {
     if (L > 0) {
         nblk = cdiv(N, L);
         const long long tiles128 = L / sana::tc::KA_TILE;
-        const BlockSplit sp = block_split(S, nblk, tiles128);
-        p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, sp.rb, sp.rt);
-        p.ka.q = make_block_sched(S, nblk, tiles128, sp.rb, sp.rt);
+        const BlockSplit sp = block_split(S, nblk, tiles128, sms);
+        p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, sp.rb, sp.rt, sms);
+        p.ka.q = make_block_sched(S, nblk, tiles128, sp.rb, sp.rt, sms);
     } else {
-        p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE));
-        p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE));
+        const int nset = plan_sets(S, sms);
+        p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE), sms, nset);
+        p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE), sms, nset);
     }
     p.ka.eps = 0.0f;
+    p.ka.state_nblk = (int)nblk;
+    p.ka.blk0 = 0;
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
+    const size_t staged = d == 32 ? sana::tc::StateLayout<32>::BYTES : sana::tc::StateLayout<64>::BYTES;
+    p.staged_bytes = L > 0 ? 0 : align256((size_t)S * staged);
     p.state_bytes = align256((size_t)B * H * nblk * dd);
-    p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
+    p.flag_bytes = align256(4 * sizeof(unsigned long long) * (size_t)p.ks.q.grid);
     return p;
 }
+
+// The single launch handles one token block and at most two segments per CTA.
+bool fused_ok(const Plan& p) { return p.ks.q.nblk == 1 && p.ks.q.max_seg <= 2; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -162,15 +239,15 @@ sana_la_status check_sizes(int B, int N, int H, int d) {
 // partial states (one per CTA, slab and block) within 4 GiB.
 constexpr size_t kMaxBlockPartialBytes = size_t(4) << 30;
 
-sana_la_status check_block(int B, int N, int H, int d, int L) {
+sana_la_status check_block(int B, int N, int H, int d, int L, int sms = device_sms()) {
     if (L < 1) return SANA_LA_ERR_INVALID_ARG;
     if (L % sana::tc::KA_TILE != 0) return SANA_LA_ERR_UNSUPPORTED;
     // the sizes of make_plan(B, N, H, d, L), in 64-bit arithmetic first
     const long long G = 128 / d;
     const long long S = (long long)B * cdiv(H, G);
     const long long nblk = cdiv(N, L);
-    const BlockSplit sp = block_split(S, nblk, L / sana::tc::KA_TILE);
-    const long long grid = S <= kSMs ? S * sp.rb * sp.rt : kSMs;
+    const BlockSplit sp = block_split(S, nblk, L / sana::tc::KA_TILE, sms);
+    const long long grid = S <= sms ? S * sp.rb * sp.rt : sms;
     const long long segs = cdiv(S, grid) * cdiv(nblk, sp.rb);   // per CTA
     const long long per_seg = G * d * (d + 1) * (long long)sizeof(float);
     if (segs > (long long)(kMaxBlockPartialBytes / per_seg) / grid) return SANA_LA_ERR_UNSUPPORTED;
@@ -259,23 +336,25 @@ sana_la_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return launch_status(name);
 }
 
-// Opt a kernel into its dynamic shared memory size, once per device.
+// Opt a kernel into its dynamic shared memory size, once per device and
+// context (the attribute lives in the context).
 template <typename Kernel>
-sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<unsigned long long> (&done)[kMaxDevicesCached]) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
         set_last_error("cudaGetDevice", e);
         return SANA_LA_ERR_CUDA;
     }
-    const uint64_t bit = 1ull << (dev & 63);
-    if (done.load(std::memory_order_acquire) & bit) return SANA_LA_OK;
+    const bool cached = dev >= 0 && dev < kMaxDevicesCached;
+    const unsigned long long ctx = current_context_id();
+    if (cached && ctx != 0 && done[dev].load(std::memory_order_acquire) == ctx) return SANA_LA_OK;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) {
         set_last_error("cudaFuncSetAttribute", e);
         return SANA_LA_ERR_CUDA;
     }
-    done.fetch_or(bit, std::memory_order_acq_rel);
+    if (cached) done[dev].store(current_context_id(), std::memory_order_release);
     return SANA_LA_OK;
 }
 
@@ -283,7 +362,7 @@ sana_la_status ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done
 template <int D, int FM>
 sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, const Plan& p,
                             float* partial, float* state, cudaStream_t s) {
-    static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     CUtensorMap tmK, tmV;
     sana_la_status st;
     if ((st = make_tmap(&tmK, K, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
@@ -309,11 +388,11 @@ sana_la_status run_kv_state(const void* K, const void* V, int B, int N, int H, c
 template <int D, bool OUT_BF16, int FM>
 sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N, int H,
                             const Plan& p, const float* state, cudaStream_t s, bool overlap) {
-    static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     CUtensorMap tmO;
     sana_la_status st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::KaMap<D, OUT_BF16>::BYTES;
+    constexpr int smem = sana::tc::KaMap<D, OUT_BF16, FM>::BYTES;
     if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, smem, smem_set)) != SANA_LA_OK) return st;
     return launch(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
                   overlap, "ka_apply_tc", tmQ, tmO, p.ka, state);
@@ -324,9 +403,14 @@ sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N,
 // may start early; a standalone apply waits for everything before it.
 template <int D, int FM>
 sana_la_status run_apply(const void* Q, const float* state, int B, int N, int H, int L, void* O,
-                         sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap) {
+                         sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap, int state_nblk,
+                         int blk0) {
     Plan p = make_plan(B, N, H, D, L);
     p.ka.eps = eps;
+    if (state_nblk > 0) {
+        p.ka.state_nblk = state_nblk;
+        p.ka.blk0 = blk0;
+    }
     CUtensorMap tmQ;
     sana_la_status st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
@@ -363,9 +447,9 @@ int blocks_per_sm(Kernel kernel, int threads, int smem, std::atomic<int> (&cache
 
 template <int D, bool OUT_BF16, int FM>
 sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
-                                    int H, const Plan& p, float* partial, unsigned long long* flags,
-                                    cudaStream_t s) {
-    static std::atomic<uint64_t> smem_set{0};
+                                    int H, const Plan& p, float* partial, uint8_t* staged,
+                                    unsigned long long* flags, cudaStream_t s) {
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     static std::atomic<int> per_sm_cache[kMaxDevicesCached];
     CUtensorMap tmK, tmV, tmQ, tmO;
     sana_la_status st;
@@ -373,17 +457,18 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::FwdMap<D, OUT_BF16>::BYTES;
+    constexpr int smem = sana::tc::FwdMap<D, OUT_BF16, FM>::BYTES;
     auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16, FM>;
     if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
-    const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
+    if (!fused_ok(p)) return SANA_LA_ERR_UNSUPPORTED;
+    const int grid = p.ks.q.grid;        // the apply phase's grid is never larger
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
         return SANA_LA_ERR_UNSUPPORTED;
     }
-    const int per_sm = blocks_per_sm(kernel, sana::tc::kThreads, smem, per_sm_cache, dev);
+    const int per_sm = blocks_per_sm(kernel, sana::tc::kFusedThreads, smem, per_sm_cache, dev);
     if (per_sm <= 0 || (long long)sms * per_sm < grid) {
         cudaGetLastError();
         return SANA_LA_ERR_UNSUPPORTED;
@@ -398,7 +483,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
         return SANA_LA_ERR_CUDA;
     }
     if (capture != cudaStreamCaptureStatusNone) {
-        e = cudaMemsetAsync(flags, 0, sizeof(unsigned long long) * (size_t)grid, s);
+        e = cudaMemsetAsync(flags, 0, 4 * sizeof(unsigned long long) * (size_t)grid, s);
         if (e != cudaSuccess) {
             set_last_error("cudaMemsetAsync(grid barrier flags)", e);
             return SANA_LA_ERR_CUDA;
@@ -406,7 +491,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(sana::tc::kThreads);
+    cfg.blockDim = dim3(sana::tc::kFusedThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -418,7 +503,8 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     // (same process, A/B): 111.9 vs 119.3 us at 4096px (0.44 GB of inputs),
     // 400.7 vs 404.3 us at N = 262,144 and 1598 vs 1608 us at N = 1,048,576.
     const int evict_first = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch, evict_first);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, staged, flags, epoch,
+                           evict_first);
     if (e != cudaSuccess) {
         set_last_error("fwd_fused_tc", e);
         return SANA_LA_ERR_CUDA;
@@ -444,28 +530,31 @@ sana_la_status kv_state_impl(const void* K, const void* V, int B, int N, int H, 
     return SANA_LA_ERR_INVALID_ARG;
 }
 
+// state_nblk > 0: the states are (B, H, state_nblk, d, d+1) and this call
+// applies blocks blk0, blk0 + 1, ... of them (block-causal host-buffer chunks)
 sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H, int d, int L,
                           void* O, sana_la_out_dtype od, float eps, cudaStream_t s, bool overlap,
-                          int fm = sana::kFeatureRelu) {
+                          int fm = sana::kFeatureRelu, int state_nblk = 0, int blk0 = 0) {
+    const int sn = state_nblk, b0 = blk0;
     switch (d * 4 + fm) {
-        case 32 * 4 + sana::kFeatureRelu: return run_apply<32, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap);
-        case 32 * 4 + sana::kFeatureElu1: return run_apply<32, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap);
-        case 32 * 4 + sana::kFeatureCos:  return run_apply<32, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap);
-        case 64 * 4 + sana::kFeatureRelu: return run_apply<64, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap);
-        case 64 * 4 + sana::kFeatureElu1: return run_apply<64, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap);
-        case 64 * 4 + sana::kFeatureCos:  return run_apply<64, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap);
+        case 32 * 4 + sana::kFeatureRelu: return run_apply<32, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
+        case 32 * 4 + sana::kFeatureElu1: return run_apply<32, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
+        case 32 * 4 + sana::kFeatureCos:  return run_apply<32, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
+        case 64 * 4 + sana::kFeatureRelu: return run_apply<64, sana::kFeatureRelu>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
+        case 64 * 4 + sana::kFeatureElu1: return run_apply<64, sana::kFeatureElu1>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
+        case 64 * 4 + sana::kFeatureCos:  return run_apply<64, sana::kFeatureCos>(Q, state, B, N, H, L, O, od, eps, s, overlap, sn, b0);
     }
     return SANA_LA_ERR_INVALID_ARG;
 }
 
 template <int FM>
 sana_la_status forward_fused_dispatch(const void* Q, const void* K, const void* V, void* O, int B, int N,
-                                      int H, int d, bool bf16, const Plan& p, float* partial,
+                                      int H, int d, bool bf16, const Plan& p, float* partial, uint8_t* staged,
                                       unsigned long long* flags, cudaStream_t s) {
-    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s))
-                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s));
+    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s)
+                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s))
+                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s)
+                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s));
 }
 
 bool valid_feature(int fm) {
@@ -487,7 +576,7 @@ KpPlan make_kp_plan(int B, int N, int C, int H, int d) {
     p.kp.groups = (int)groups;
     p.kp.C = C;
     p.kp.kblocks = (int)cdiv(C, 64);
-    p.kp.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KP_TILE));
+    p.kp.q = make_sched((long long)B * groups, cdiv(N, sana::tc::KP_TILE), device_sms());
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.kp.q.grid * p.kp.q.max_seg * G * dd);
     return p;
@@ -507,7 +596,7 @@ sana_la_status check_projection(int B, int N, int C, int H, int d) {
 template <int D>
 sana_la_status run_kvproj_state(const void* X, const void* Wk, const void* Wv, int B, int N, int C, int H,
                                 const KpPlan& p, float* partial, float* state, cudaStream_t s) {
-    static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     CUtensorMap tmX, tmWk, tmWv;
     sana_la_status st;
     // X as {C, N, B}; the weights as {C, H*d, 1}: 64 features x 128 rows per box
@@ -558,7 +647,7 @@ constexpr bool kGemmPairs = true;
 
 sana_la_status launch_gemm_pairs(const void* A, const void* Bm, void* C, int M, int N, int K, int ldc,
                                  cudaStream_t s) {
-    static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     CUtensorMap tmA, tmB;
     sana_la_status st;
     if ((st = make_tmap(&tmA, A, 1, M, 1, K, 128)) != SANA_LA_OK) return st;
@@ -573,14 +662,14 @@ sana_la_status launch_gemm_pairs(const void* A, const void* Bm, void* C, int M, 
     gp.mtiles = (int)cdiv(M, sana::tc::G2_TILE_M);
     gp.ntiles = (int)cdiv(N, sana::tc::G2_TILE_N);
     const long long tiles = (long long)gp.mtiles * gp.ntiles;
-    const int pairs = (int)std::min<long long>(tiles, kSMs / 2);
+    const int pairs = (int)std::min<long long>(tiles, device_sms() / 2);
     return launch(sana::tc::gemm_bf16_tc2, dim3(2 * pairs), dim3(sana::tc::kThreads), sana::tc::Gemm2Map::BYTES, s,
                   false, "gemm_bf16_tc2", tmA, tmB, gp, static_cast<__nv_bfloat16*>(C));
 }
 
 sana_la_status launch_gemm(const void* A, const void* Bm, void* C, int M, int N, int K, int ldc, cudaStream_t s) {
     if (kGemmPairs) return launch_gemm_pairs(A, Bm, C, M, N, K, ldc, s);
-    static std::atomic<uint64_t> smem_set{0};
+    static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     CUtensorMap tmA, tmB;
     sana_la_status st;
     if ((st = make_tmap(&tmA, A, 1, M, 1, K, sana::tc::GM_TILE_M)) != SANA_LA_OK) return st;
@@ -595,7 +684,7 @@ sana_la_status launch_gemm(const void* A, const void* Bm, void* C, int M, int N,
     gp.mtiles = (int)cdiv(M, sana::tc::GM_TILE_M);
     gp.ntiles = (int)cdiv(N, sana::tc::GM_TILE_N);
     const long long tiles = (long long)gp.mtiles * gp.ntiles;
-    const int grid = (int)std::min<long long>(tiles, kSMs);
+    const int grid = (int)std::min<long long>(tiles, device_sms());
     return launch(sana::tc::gemm_bf16_tc, dim3(grid), dim3(sana::tc::kThreads), sana::tc::GemmMap::BYTES, s,
                   false, "gemm_bf16_tc", tmA, tmB, gp, static_cast<__nv_bfloat16*>(C));
 }
@@ -638,29 +727,35 @@ sana_la_status forward_entry(const void* Q, const void* K, const void* V, int B,
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
     Plan p = make_plan(B, N, H, d);
-    if (workspace_bytes < p.partial_bytes + p.state_bytes + p.flag_bytes) return SANA_LA_ERR_WORKSPACE;
+    if (workspace_bytes < p.partial_bytes + p.staged_bytes + p.state_bytes + p.flag_bytes)
+        return SANA_LA_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     float* partial = reinterpret_cast<float*>(ws);
-    float* state = reinterpret_cast<float*>(ws + p.partial_bytes);
-    auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes + p.state_bytes);
+    auto* staged = reinterpret_cast<uint8_t*>(ws + p.partial_bytes);
+    float* state = reinterpret_cast<float*>(ws + p.partial_bytes + p.staged_bytes);
+    auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes + p.staged_bytes + p.state_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // one cooperative launch: state phase, grid barrier, apply phase
+    // one cooperative launch: state phase, distributed reduction, apply phase
     p.ka.eps = eps;
     const bool bf16 = out_dtype == SANA_LA_OUT_BF16;
     switch (fm) {
         case sana::kFeatureElu1:
-            st = forward_fused_dispatch<sana::kFeatureElu1>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+            st = forward_fused_dispatch<sana::kFeatureElu1>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
+                                                            flags, s);
             break;
         case sana::kFeatureCos:
-            st = forward_fused_dispatch<sana::kFeatureCos>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+            st = forward_fused_dispatch<sana::kFeatureCos>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
+                                                           flags, s);
             break;
         default:
-            st = forward_fused_dispatch<sana::kFeatureRelu>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
+            st = forward_fused_dispatch<sana::kFeatureRelu>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
+                                                            flags, s);
     }
     if (st != SANA_LA_ERR_UNSUPPORTED) return st;
-    // the device cannot hold the whole grid at once: the same kernels as
-    // kv_state + apply, overlapped by programmatic launch
-    st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, workspace_bytes, s, true, fm);
+    // the device cannot hold the whole grid at once, or the CTAs would have
+    // more than two segments: the same kernels as kv_state + apply, overlapped
+    // by programmatic launch
+    st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, p.partial_bytes, s, false, fm);
     if (st != SANA_LA_OK) return st;
     return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true, fm);
 }
@@ -672,14 +767,16 @@ struct HostPlan {
     size_t q, kv, o, state, partial, total;
 };
 
-HostPlan make_host_plan(int B, int N, int H, int d, sana_la_out_dtype od) {
-    const Plan p = make_plan(B, N, H, d);
+// L > 0: the block-causal form (prefix states of blocks of L tokens)
+HostPlan make_host_plan(int B, int N, int H, int d, sana_la_out_dtype od, int L = 0) {
+    const Plan p = make_plan(B, N, H, d, L);
     const size_t elems = (size_t)B * N * H * d;
+    const size_t nblk = L > 0 ? (size_t)cdiv(N, L) : 1;
     HostPlan h{};
     h.q = align256(elems * 2);
     h.kv = align256(elems * 2);
     h.o = align256(elems * (od == SANA_LA_OUT_F32 ? 4 : 2));
-    h.state = align256((size_t)B * H * d * (d + 1) * sizeof(float));
+    h.state = align256((size_t)B * H * nblk * d * (d + 1) * sizeof(float));
     h.partial = p.partial_bytes;
     h.total = h.q + 2 * h.kv + h.o + h.state + h.partial;
     return h;
@@ -693,9 +790,19 @@ struct HostChunks {
     int count;
 };
 
-HostChunks host_chunks(int B, int N) {
+HostChunks host_chunks(int B, int N, int L = 0) {
     const long long target = std::max<long long>(1024, cdiv((long long)B * N, 16));
     HostChunks c{};
+    if (L > 0) {
+        // block-causal: whole blocks of one batch (each block's queries use
+        // that block's prefix state), about `target` tokens per chunk
+        const long long nblk = cdiv(N, L);
+        const long long bpc = std::min<long long>(nblk, std::max<long long>(1, target / L));
+        c.tokens = bpc * L;
+        c.batches = 1;
+        c.count = (int)(B * cdiv(nblk, bpc));
+        return c;
+    }
     if (N >= target) {
         c.tokens = cdiv(target, 128) * 128;
         c.batches = 1;
@@ -720,6 +827,7 @@ struct CopyCtx {
     cudaEvent_t start = nullptr;            // the caller's earlier work on its stream is done
     cudaEvent_t join = nullptr;             // the last copy back is done
     bool ready = false;
+    unsigned long long context = 0;         // the context the streams and events belong to
     // Held while a call enqueues: an event must be waited for before another
     // call records it again from a different stream.
     std::mutex enqueue;
@@ -737,6 +845,15 @@ sana_la_status copy_ctx(CopyCtx** out) {
     if (dev < 0 || dev >= kMaxDevicesCached) return SANA_LA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_copy_ctx_mutex);
     CopyCtx& c = g_copy_ctx[dev];
+    const unsigned long long context = current_context_id();
+    if (c.ready && context != 0 && context != c.context) {
+        // made in a context that has since been destroyed: its handles went
+        // with it (they are not destroyed here); make new ones in this context
+        c.h2d = c.d2h = nullptr;
+        for (int i = 0; i < kHostEvents; ++i) c.in[i] = c.out[i] = nullptr;
+        c.start = c.join = nullptr;
+        c.ready = false;
+    }
     if (!c.ready) {
         e = cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking);
@@ -768,6 +885,7 @@ sana_la_status copy_ctx(CopyCtx** out) {
             return SANA_LA_ERR_CUDA;
         }
         c.ready = true;
+        c.context = current_context_id();
     }
     *out = &c;
     return SANA_LA_OK;
@@ -793,17 +911,19 @@ sana_la_status copy_async(void* dst, const void* src, size_t bytes, cudaMemcpyKi
     return SANA_LA_OK;
 }
 
+// L > 0: the block-causal form (phi = ReLU)
 sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV, int B, int N, int H, int d,
                                   int fm, void* hO, sana_la_out_dtype out_dtype, float eps, void* workspace,
-                                  size_t workspace_bytes, sana_la_stream_t stream) {
+                                  size_t workspace_bytes, sana_la_stream_t stream, int L = 0) {
     g_last_error[0] = '\0';
     if (!hQ || !hK || !hV || !hO || !workspace || !valid_feature(fm)) return SANA_LA_ERR_INVALID_ARG;
     sana_la_status st = check_sizes(B, N, H, d);
     if (st != SANA_LA_OK) return st;
+    if (L != 0 && (st = check_block(B, N, H, d, L)) != SANA_LA_OK) return st;
     if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return SANA_LA_ERR_INVALID_ARG;
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(workspace)) return SANA_LA_ERR_INVALID_ARG;
-    const HostPlan hp = make_host_plan(B, N, H, d, out_dtype);
+    const HostPlan hp = make_host_plan(B, N, H, d, out_dtype, L);
     if (workspace_bytes < hp.total) return SANA_LA_ERR_WORKSPACE;
     CopyCtx* cc = nullptr;
     if ((st = copy_ctx(&cc)) != SANA_LA_OK) return st;
@@ -828,11 +948,12 @@ sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV
     if ((st = copy_async(dK, hK, tokens * row_in, cudaMemcpyHostToDevice, cc->h2d)) != SANA_LA_OK) return st;
     if ((st = copy_async(dV, hV, tokens * row_in, cudaMemcpyHostToDevice, cc->h2d)) != SANA_LA_OK) return st;
     if ((st = stream_after(s, cc->h2d, cc->in[0], "K, V event")) != SANA_LA_OK) return st;
-    if ((st = kv_state_impl(dK, dV, B, N, H, d, 0, state, partial, hp.partial, s, false, fm)) != SANA_LA_OK)
+    if ((st = kv_state_impl(dK, dV, B, N, H, d, L, state, partial, hp.partial, s, false, fm)) != SANA_LA_OK)
         return st;
-    const HostChunks hc = host_chunks(B, N);
+    const HostChunks hc = host_chunks(B, N, L);
     const long long per_batch = cdiv(N, hc.tokens);
-    const size_t state_stride = (size_t)H * d * (d + 1);
+    const int nblk = L > 0 ? (int)cdiv(N, L) : 1;
+    const size_t state_stride = (size_t)H * nblk * d * (d + 1);     // one batch's states
     auto chunk = [&](int c, int& b0, int& nb, int& t0, int& nt) {
         if (hc.batches > 1 || hc.tokens >= N) {
             b0 = c * hc.batches;
@@ -857,8 +978,11 @@ sana_la_status forward_host_entry(const void* hQ, const void* hK, const void* hV
             return st;
         if ((st = stream_after(s, cc->h2d, cc->in[(c + 1) % kHostEvents], "chunk in event")) != SANA_LA_OK)
             return st;
-        if ((st = apply_impl(dQ + first * row_in, state + (size_t)b0 * state_stride, nb, nt, H, d, 0,
-                             dO + first * row_out, out_dtype, eps, s, false, fm)) != SANA_LA_OK)
+        // block-causal: the chunk is blocks t0 / L, ... of batch b0, applied
+        // against that batch's prefix states (nblk of them, from block t0 / L)
+        if ((st = apply_impl(dQ + first * row_in, state + (size_t)b0 * state_stride, nb, nt, H, d, L,
+                             dO + first * row_out, out_dtype, eps, s, false, fm, L > 0 ? nblk : 0,
+                             L > 0 ? t0 / L : 0)) != SANA_LA_OK)
             return st;
         if ((st = stream_after(cc->d2h, s, cc->out[c % kHostEvents], "chunk out event")) != SANA_LA_OK)
             return st;
@@ -878,7 +1002,7 @@ extern "C" {
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
     const Plan p = make_plan(B, N, H, d);
-    return p.partial_bytes + p.state_bytes + p.flag_bytes;
+    return p.partial_bytes + p.staged_bytes + p.state_bytes + p.flag_bytes;
 }
 
 sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,
@@ -979,7 +1103,7 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
     // 1x1 expand: U = X W1^T (2 Ch channels)
     if ((st = launch_gemm(X, W1, U, M, 2 * Ch, C, 2 * Ch, s)) != SANA_LA_OK) return st;
     // 3x3 depthwise over the grid and the GLU, fused
-    static std::atomic<uint64_t> dw_smem_set{0};
+    static std::atomic<unsigned long long> dw_smem_set[kMaxDevicesCached];
     if ((st = ensure_smem(sana::tc::dwconv_glu, sana::tc::DW_SMEM, dw_smem_set)) != SANA_LA_OK) return st;
     // U as {2 Ch, Wg, Hg, B}: a load box is 64 channels x (DW_TX + 2) columns x
     // (DW_TY + 2) rows; Z as {Ch, Wg, Hg, B}: a store box is 64 x DW_TX x DW_TY
@@ -1085,6 +1209,30 @@ int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L
     return 3;   // ks_state_tc, kr_reduce_tc (prefix states), ka_apply_tc
 }
 
+size_t sana_linattn_block_causal_forward_host_workspace_bytes(int B, int N, int H, int d, int L,
+                                                              sana_la_out_dtype out_dtype) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
+    if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return 0;
+    return make_host_plan(B, N, H, d, out_dtype, L).total;
+}
+
+sana_la_status sana_linattn_block_causal_forward_host(const void* Q, const void* K, const void* V, int B, int N,
+                                                      int H, int d, int L, void* O, sana_la_out_dtype out_dtype,
+                                                      float eps, void* workspace, size_t workspace_bytes,
+                                                      sana_la_stream_t stream) {
+    if (L < 1) {
+        g_last_error[0] = '\0';
+        return SANA_LA_ERR_INVALID_ARG;
+    }
+    return forward_host_entry(Q, K, V, B, N, H, d, sana::kFeatureRelu, O, out_dtype, eps, workspace,
+                              workspace_bytes, stream, L);
+}
+
+int sana_linattn_block_causal_forward_host_launches(int B, int N, int H, int d, int L) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
+    return 2 + host_chunks(B, N, L).count;       // state, prefix states, one apply per chunk
+}
+
 size_t sana_linattn_forward_host_workspace_bytes(int B, int N, int H, int d, sana_la_out_dtype out_dtype) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
     if (out_dtype != SANA_LA_OUT_F32 && out_dtype != SANA_LA_OUT_BF16) return 0;
@@ -1174,10 +1322,13 @@ __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 std::mutex g_static_scratch_mutex;
 void* g_static_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_static_scratch_context[kMaxDevices] = {};
 
 // Device address of g_static_scratch on the current device. The host-side
 // name is only a stand-in; the address comes from cudaGetSymbolAddress, asked
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached with the context it
+// belongs to, and asked again when the device's context changed (a context
+// destroyed and made anew, e.g. by cudaDeviceReset, reloads the module).
 sana_la_status static_scratch_address(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1192,7 +1343,9 @@ sana_la_status static_scratch_address(void** out) {
         return SANA_LA_ERR_UNSUPPORTED;
     }
     std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-    if (g_static_scratch_ptr[dev] == nullptr) {
+    const unsigned long long context = current_context_id();
+    if (g_static_scratch_ptr[dev] == nullptr ||
+        (context != 0 && context != g_static_scratch_context[dev])) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_scratch);
         if (e != cudaSuccess || p == nullptr) {
@@ -1200,6 +1353,7 @@ sana_la_status static_scratch_address(void** out) {
             return SANA_LA_ERR_CUDA;
         }
         g_static_scratch_ptr[dev] = p;
+        g_static_scratch_context[dev] = current_context_id();
     }
     *out = g_static_scratch_ptr[dev];
     return SANA_LA_OK;

@@ -33,6 +33,7 @@ and the block-causal form (blocks of L tokens, L a multiple of 128):
     block_causal_kv_state(K, V, L, states=None, workspace=None) -> (B, H, nblk, d, d+1) fp32
     block_causal_apply(Q, states, L, out_dtype=..., eps=..., out=None) -> O
     block_causal_forward(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None) -> O
+    block_causal_forward_host(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None) -> O (CPU)
 """
 from __future__ import annotations
 
@@ -69,6 +70,9 @@ SYMBOLS = (
     "sana_linattn_block_causal_apply",
     "sana_linattn_block_causal_forward",
     "sana_linattn_block_causal_forward_launches",
+    "sana_linattn_block_causal_forward_host_workspace_bytes",
+    "sana_linattn_block_causal_forward_host",
+    "sana_linattn_block_causal_forward_host_launches",
     "sana_linattn_forward_host_workspace_bytes",
     "sana_linattn_forward_host",
     "sana_linattn_forward_host_launches",
@@ -153,6 +157,12 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_block_causal_forward.restype = st
         lib.sana_linattn_block_causal_forward_launches.argtypes = [i, i, i, i, i]
         lib.sana_linattn_block_causal_forward_launches.restype = ctypes.c_int
+        lib.sana_linattn_block_causal_forward_host_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        lib.sana_linattn_block_causal_forward_host_workspace_bytes.restype = sz
+        lib.sana_linattn_block_causal_forward_host.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_block_causal_forward_host.restype = st
+        lib.sana_linattn_block_causal_forward_host_launches.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_block_causal_forward_host_launches.restype = ctypes.c_int
         lib.sana_linattn_last_error.argtypes = []
         lib.sana_linattn_last_error.restype = ctypes.c_char_p
         if path == LIBRARY:
@@ -358,6 +368,22 @@ def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out_dtype=to
     return out
 
 
+def _host_inputs(Q, K, V, out, out_dtype):
+    for name, t in (("Q", Q), ("K", K), ("V", V)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+            raise ValueError(f"{name} must be a CPU tensor (the device copy is made by the library)")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous (B, N, H, d) bf16 tensor")
+        if t.shape != Q.shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(Q.shape)}")
+    if out is None:
+        return torch.empty(Q.shape, dtype=out_dtype).pin_memory()
+    if (out.device.type != "cpu" or out.dtype != out_dtype or tuple(out.shape) != tuple(Q.shape)
+            or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous CPU {out_dtype} tensor of shape {tuple(Q.shape)}")
+    return out
+
+
 # ------------------------------------------------------------ block-causal --
 
 def num_blocks(N: int, L: int) -> int:
@@ -440,6 +466,40 @@ def block_causal_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: i
                                                workspace.numel() * workspace.element_size(),
                                                _stream(Q.device))
     _check(lib, st, "sana_linattn_block_causal_forward")
+    return out
+
+
+def block_causal_forward_host_workspace_bytes(B: int, N: int, H: int, d: int, L: int,
+                                             out_dtype=torch.bfloat16) -> int:
+    return int(load_library().sana_linattn_block_causal_forward_host_workspace_bytes(
+        B, N, H, d, int(L), _out_code(out_dtype)))
+
+
+def block_causal_forward_host_launches(B: int, N: int, H: int, d: int, L: int) -> int:
+    return int(load_library().sana_linattn_block_causal_forward_host_launches(B, N, H, d, int(L)))
+
+
+def block_causal_forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: int,
+                              out_dtype=torch.bfloat16, eps: float = 1e-15, out: torch.Tensor | None = None,
+                              workspace: torch.Tensor | None = None, device=None) -> torch.Tensor:
+    """The block-causal forward from host tensors to a host tensor, with the
+    copies done by the library (K, V in; the prefix states; Q streamed through
+    in chunks of whole blocks whose outputs are copied back while the next chunk
+    comes in). Bit-identical to block_causal_forward() on the same inputs."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = _host_inputs(Q, K, V, out, out_dtype)
+    B, N, H, d = Q.shape
+    code = _out_code(out_dtype)
+    if workspace is None:
+        n = block_causal_forward_host_workspace_bytes(B, N, H, d, L, out_dtype)
+        if n == 0:
+            raise ValueError(f"unsupported sizes B={B} N={N} H={H} d={d} L={L}")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    lib = load_library()
+    st = lib.sana_linattn_block_causal_forward_host(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d, int(L),
+                                                    out.data_ptr(), code, float(eps), workspace.data_ptr(),
+                                                    workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(lib, st, "sana_linattn_block_causal_forward_host")
     return out
 
 
