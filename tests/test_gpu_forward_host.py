@@ -1,10 +1,10 @@
-"""The forward from host buffers (sana_linattn_forward_host): the library copies
-K and V in, computes the state, and streams Q through in chunks whose outputs
-are copied back on its own stream while the next chunk comes in. The apply of a
-token does not depend on the chunk it is in, so the result must be
-bit-identical to the device forward on the same inputs, for every way the
-tokens are cut into chunks; and the caller's stream must cover the last copy
-out."""
+"""The forward from host buffers (sana_linattn_forward_host and its block-causal
+form): the library copies K and V in, computes the state (or the blocks'
+prefix states), and streams Q through in chunks whose outputs are copied back
+on its own stream while the next chunk comes in. The apply of a token does not
+depend on the chunk it is in, so the result must be bit-identical to the
+device forward on the same inputs, for every way the tokens are cut into
+chunks; and the caller's stream must cover the last copy out."""
 import pytest
 import torch
 
@@ -102,3 +102,33 @@ def test_forward_host_from_two_threads():
         Od = ops.forward(hQ.cuda(), hK.cuda(), hV.cuda())
         assert torch.equal(outs[i].view(torch.int16), Od.cpu().view(torch.int16))
     assert ops.device_error() == 0
+
+
+# block-causal: one block per chunk (16 blocks); several blocks per chunk; a
+# ragged last block; more blocks than chunks in two batches; N shorter than L
+BLOCK_SHAPES = [(1, 16 * 1024, 4, 32, 1024), (1, 5000, 3, 32, 128), (2, 3000, 5, 64, 256),
+                (3, 2000, 6, 32, 384), (1, 100, 4, 32, 128)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", BLOCK_SHAPES, ids=lambda s: "B{}N{}H{}d{}L{}".format(*s))
+def test_block_causal_forward_host_equals_device_forward(shape, dtype):
+    B, N, H, d, L = shape
+    hQ, hK, hV = _host(B, N, H, d, seed=N + L)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        O = ops.block_causal_forward_host(hQ, hK, hV, L, out_dtype=dtype)
+    side.synchronize()
+    Od = ops.block_causal_forward(hQ.cuda(), hK.cuda(), hV.cuda(), L, out_dtype=dtype)
+    assert O.device.type == "cpu" and O.is_pinned()
+    assert torch.equal(O.view(BITS[dtype]), Od.cpu().view(BITS[dtype]))
+    assert ops.device_error() == 0
+
+
+def test_block_causal_forward_host_matches_oracle(oracle):
+    B, N, H, d, L = 2, 1300, 3, 32, 256
+    hQ, hK, hV = _host(B, N, H, d, seed=17, pinned=False)
+    O = ops.block_causal_forward_host(hQ, hK, hV, L, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.block_causal_forward(to_f64(hQ), to_f64(hK), to_f64(hV), L, 1e-15)
+    check_output(O, ref, "block_causal_forward_host")
