@@ -96,10 +96,9 @@ typedef enum {
  * sana_linattn_forward need for these sizes on the current device (a function
  * of the sizes and of the device's SM count; with no device to ask, the
  * B200's 148). The workspace holds the fp32 partial states of the token
- * chunks, and for sana_linattn_forward also the reduced states (staged as
- * bf16 hi + lo parts for the apply), the fp32 state of the three-kernel
- * fallback and four readiness flags per CTA. Returns 0 for invalid or
- * unsupported sizes. Any content is acceptable on entry; it is scratch.
+ * chunks, and for sana_linattn_forward also the reduced state and one
+ * readiness flag per CTA. Returns 0 for invalid or unsupported sizes. Any
+ * content is acceptable on entry; it is scratch.
  */
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d);
 
@@ -139,18 +138,15 @@ sana_la_status sana_linattn_apply(const void* Q, const float* state,
  * The whole forward: sana_linattn_kv_state into the workspace, then
  * sana_linattn_apply. Same arguments and rules as the two calls above; the
  * result is bit-identical to calling them in sequence.
- * It runs as one cooperative kernel launch: the state phase, a reduction of
- * each (b, head group)'s partial states shared by the CTAs that made them (in
- * the order sana_linattn_kv_state sums them), and the apply phase. The head
- * groups are taken in two sets, so the first set's reduction runs while the
- * second set's keys stream in and the second set's while the first set's
- * queries are applied. CTAs signal each other through flags in the workspace
- * tagged with a number unique to the call, so the workspace needs no
- * initialisation. Under stream capture the call also records a memset of
- * those flags before the kernel, because a replayed graph reuses the captured
- * number. Where the device cannot hold the whole grid at once, or B times the
- * head groups exceeds twice the SM count, the call runs the kernels of the
- * two calls above instead.
+ * It runs as one cooperative kernel launch: the state phase; a readiness flag
+ * per CTA; the apply phase, in which each CTA waits for the flags of the CTAs
+ * that made its (b, head group)'s partial states and sums them itself, in the
+ * order sana_linattn_kv_state sums them. The flags are tagged with a number
+ * unique to the call, so the workspace needs no initialisation. Under stream
+ * capture the call also records a memset of those flags before the kernel,
+ * because a replayed graph reuses the captured number. Where the device cannot
+ * hold the whole grid at once, the call falls back to the kernels of the two
+ * calls above.
  */
 sana_la_status sana_linattn_forward(const void* Q, const void* K, const void* V,
                                     int B, int N, int H, int d,

@@ -303,11 +303,12 @@ kvproj_state_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 sched_item(cta, i, tps, p.q, slab, tile, sg);
                 const int h = (slab % p.groups) * G + hh;
                 if (h < p.H) {
+                    // the state kernel's layout: by columns, column j at j * D
                     const long long slot = ((long long)cta * p.q.max_seg + seg) * G + hh;
-                    float* P = partial + slot * DD + (long long)row * (D + 1);
+                    float* P = partial + slot * DD + row;
 #pragma unroll
-                    for (int j = 0; j < D; ++j) P[j] = sv[j];
-                    P[D] = nrm;
+                    for (int j = 0; j < D; ++j) P[j * D] = sv[j];
+                    P[D * D] = nrm;
                 }
             }
         }

@@ -110,14 +110,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
-// 1-D bulk copy (no tensor map) from global memory into this CTA's shared
-// memory, completing on `bar` with the byte count as transaction bytes. Both
-// addresses 16-byte aligned, `bytes` a multiple of 16.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
-
 // 2^x and 1/x on the special-function unit (approximate, subnormals flushed)
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

@@ -97,22 +97,17 @@ struct Plan {
     sana::tc::KsParams ks;
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
-    size_t staged_bytes;    // single launch: one reduced state per slab, staged as bf16 hi + lo
     size_t state_bytes;     // fp32 (B, H, d, d+1); block-causal (B, H, nblk, d, d+1)
-    size_t flag_bytes;      // single launch: four readiness flags per CTA
+    size_t flag_bytes;      // readiness flags of the single-launch forward (one per CTA)
 };
 
-// Lockstep schedule of S slabs of T tiles over at most `sms` CTAs, in one or
-// two sets (see the comment at the top of tc_kernels.cuh).
-sana::tc::Sched make_sched(long long S, long long T, int sms, int nset = 1) {
+// Lockstep schedule of S slabs of T tiles over at most `sms` CTAs (see the
+// comment at the top of tc_kernels.cuh).
+sana::tc::Sched make_sched(long long S, long long T, int sms) {
     sana::tc::Sched q{};
     q.S = (int)S;
     q.T = (int)T;
-    if (nset == 2) {
-        q.P = (int)cdiv(S, 2);
-        q.R = (int)std::max<long long>(1, std::min<long long>(sms / q.P, T));
-        q.max_seg = 2;
-    } else if (S <= sms) {
+    if (S <= sms) {
         q.P = (int)S;
         q.R = (int)std::min<long long>(sms / S, T);
         q.max_seg = 1;
@@ -126,13 +121,6 @@ sana::tc::Sched make_sched(long long S, long long T, int sms, int nset = 1) {
     q.tpb = 0;
     q.rb = 1;
     return q;
-}
-
-// Two sets when every position then holds two slabs (even S), or when the one
-// position with a single slab idles little (S >= 15), and the single launch can
-// still give every CTA at most two segments.
-int plan_sets(long long S, int sms) {
-    return (S >= 2 && S <= 2LL * sms && (S % 2 == 0 || S >= 15)) ? 2 : 1;
 }
 
 // Block-causal schedule: S slabs of nblk blocks of bt tiles; a slab's
@@ -203,24 +191,18 @@ Plan make_plan(int B, int N, int H, int d, int L = 0, int sms = device_sms()) {
         p.ks.q = make_block_sched(S, nblk, L / sana::tc::KS_TILE, sp.rb, sp.rt, sms);
         p.ka.q = make_block_sched(S, nblk, tiles128, sp.rb, sp.rt, sms);
     } else {
-        const int nset = plan_sets(S, sms);
-        p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE), sms, nset);
-        p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE), sms, nset);
+        p.ks.q = make_sched(S, cdiv(N, sana::tc::KS_TILE), sms);
+        p.ka.q = make_sched(S, cdiv(N, sana::tc::KA_TILE), sms);
     }
     p.ka.eps = 0.0f;
     p.ka.state_nblk = (int)nblk;
     p.ka.blk0 = 0;
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
-    const size_t staged = d == 32 ? sana::tc::StateLayout<32>::BYTES : sana::tc::StateLayout<64>::BYTES;
-    p.staged_bytes = L > 0 ? 0 : align256((size_t)S * staged);
     p.state_bytes = align256((size_t)B * H * nblk * dd);
-    p.flag_bytes = align256(4 * sizeof(unsigned long long) * (size_t)p.ks.q.grid);
+    p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
     return p;
 }
-
-// The single launch handles one token block and at most two segments per CTA.
-bool fused_ok(const Plan& p) { return p.ks.q.nblk == 1 && p.ks.q.max_seg <= 2; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -392,7 +374,7 @@ sana_la_status launch_apply(const CUtensorMap& tmQ, const void* O, int B, int N,
     CUtensorMap tmO;
     sana_la_status st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::KaMap<D, OUT_BF16, FM>::BYTES;
+    constexpr int smem = sana::tc::KaMap<D, OUT_BF16>::BYTES;
     if ((st = ensure_smem(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, smem, smem_set)) != SANA_LA_OK) return st;
     return launch(sana::tc::ka_apply_tc<D, OUT_BF16, FM>, dim3(p.ka.q.grid), dim3(sana::tc::kThreads), smem, s,
                   overlap, "ka_apply_tc", tmQ, tmO, p.ka, state);
@@ -447,8 +429,8 @@ int blocks_per_sm(Kernel kernel, int threads, int smem, std::atomic<int> (&cache
 
 template <int D, bool OUT_BF16, int FM>
 sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
-                                    int H, const Plan& p, float* partial, uint8_t* staged,
-                                    unsigned long long* flags, cudaStream_t s) {
+                                    int H, const Plan& p, float* partial, unsigned long long* flags,
+                                    cudaStream_t s) {
     static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     static std::atomic<int> per_sm_cache[kMaxDevicesCached];
     CUtensorMap tmK, tmV, tmQ, tmO;
@@ -457,18 +439,17 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     if ((st = make_tmap(&tmV, V, B, N, H, D, sana::tc::KS_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
-    constexpr int smem = sana::tc::FwdMap<D, OUT_BF16, FM>::BYTES;
+    constexpr int smem = sana::tc::FwdMap<D, OUT_BF16>::BYTES;
     auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16, FM>;
     if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
-    if (!fused_ok(p)) return SANA_LA_ERR_UNSUPPORTED;
-    const int grid = p.ks.q.grid;        // the apply phase's grid is never larger
+    const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
         return SANA_LA_ERR_UNSUPPORTED;
     }
-    const int per_sm = blocks_per_sm(kernel, sana::tc::kFusedThreads, smem, per_sm_cache, dev);
+    const int per_sm = blocks_per_sm(kernel, sana::tc::kThreads, smem, per_sm_cache, dev);
     if (per_sm <= 0 || (long long)sms * per_sm < grid) {
         cudaGetLastError();
         return SANA_LA_ERR_UNSUPPORTED;
@@ -483,7 +464,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
         return SANA_LA_ERR_CUDA;
     }
     if (capture != cudaStreamCaptureStatusNone) {
-        e = cudaMemsetAsync(flags, 0, 4 * sizeof(unsigned long long) * (size_t)grid, s);
+        e = cudaMemsetAsync(flags, 0, sizeof(unsigned long long) * (size_t)grid, s);
         if (e != cudaSuccess) {
             set_last_error("cudaMemsetAsync(grid barrier flags)", e);
             return SANA_LA_ERR_CUDA;
@@ -491,7 +472,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(sana::tc::kFusedThreads);
+    cfg.blockDim = dim3(sana::tc::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -503,8 +484,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     // (same process, A/B): 111.9 vs 119.3 us at 4096px (0.44 GB of inputs),
     // 400.7 vs 404.3 us at N = 262,144 and 1598 vs 1608 us at N = 1,048,576.
     const int evict_first = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, staged, flags, epoch,
-                           evict_first);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch, evict_first);
     if (e != cudaSuccess) {
         set_last_error("fwd_fused_tc", e);
         return SANA_LA_ERR_CUDA;
@@ -549,12 +529,12 @@ sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H
 
 template <int FM>
 sana_la_status forward_fused_dispatch(const void* Q, const void* K, const void* V, void* O, int B, int N,
-                                      int H, int d, bool bf16, const Plan& p, float* partial, uint8_t* staged,
+                                      int H, int d, bool bf16, const Plan& p, float* partial,
                                       unsigned long long* flags, cudaStream_t s) {
-    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s)
-                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s))
-                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s)
-                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, staged, flags, s));
+    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s))
+                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
+                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s));
 }
 
 bool valid_feature(int fm) {
@@ -727,34 +707,28 @@ sana_la_status forward_entry(const void* Q, const void* K, const void* V, int B,
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
     Plan p = make_plan(B, N, H, d);
-    if (workspace_bytes < p.partial_bytes + p.staged_bytes + p.state_bytes + p.flag_bytes)
-        return SANA_LA_ERR_WORKSPACE;
+    if (workspace_bytes < p.partial_bytes + p.state_bytes + p.flag_bytes) return SANA_LA_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     float* partial = reinterpret_cast<float*>(ws);
-    auto* staged = reinterpret_cast<uint8_t*>(ws + p.partial_bytes);
-    float* state = reinterpret_cast<float*>(ws + p.partial_bytes + p.staged_bytes);
-    auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes + p.staged_bytes + p.state_bytes);
+    float* state = reinterpret_cast<float*>(ws + p.partial_bytes);
+    auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes + p.state_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // one cooperative launch: state phase, distributed reduction, apply phase
+    // one cooperative launch: state phase, per-slab readiness flags, apply phase
     p.ka.eps = eps;
     const bool bf16 = out_dtype == SANA_LA_OUT_BF16;
     switch (fm) {
         case sana::kFeatureElu1:
-            st = forward_fused_dispatch<sana::kFeatureElu1>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
-                                                            flags, s);
+            st = forward_fused_dispatch<sana::kFeatureElu1>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
             break;
         case sana::kFeatureCos:
-            st = forward_fused_dispatch<sana::kFeatureCos>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
-                                                           flags, s);
+            st = forward_fused_dispatch<sana::kFeatureCos>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
             break;
         default:
-            st = forward_fused_dispatch<sana::kFeatureRelu>(Q, K, V, O, B, N, H, d, bf16, p, partial, staged,
-                                                            flags, s);
+            st = forward_fused_dispatch<sana::kFeatureRelu>(Q, K, V, O, B, N, H, d, bf16, p, partial, flags, s);
     }
     if (st != SANA_LA_ERR_UNSUPPORTED) return st;
-    // the device cannot hold the whole grid at once, or the CTAs would have
-    // more than two segments: the same kernels as kv_state + apply, overlapped
-    // by programmatic launch
+    // the device cannot hold the whole grid at once: the same kernels as
+    // kv_state + apply, overlapped by programmatic launch
     st = kv_state_impl(K, V, B, N, H, d, 0, state, workspace, p.partial_bytes, s, false, fm);
     if (st != SANA_LA_OK) return st;
     return apply_impl(Q, state, B, N, H, d, 0, O, out_dtype, eps, s, true, fm);
@@ -1002,7 +976,7 @@ extern "C" {
 size_t sana_linattn_workspace_bytes(int B, int N, int H, int d) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK) return 0;
     const Plan p = make_plan(B, N, H, d);
-    return p.partial_bytes + p.staged_bytes + p.state_bytes + p.flag_bytes;
+    return p.partial_bytes + p.state_bytes + p.flag_bytes;
 }
 
 sana_la_status sana_linattn_kv_state(const void* K, const void* V, int B, int N, int H, int d,

@@ -5,8 +5,7 @@
 //     kr_prefix_tc  block-causal: fixed-order prefix sums over token blocks
 // KA  ka_apply_tc   phi(Q) S on UMMA (S split into bf16 hi + lo), then
 //                   O = num / (den + eps) in the epilogue, stored by TMA
-// KF  fwd_fused_tc  KS, a distributed fixed-order reduction and KA in one
-//                   cooperative launch
+// KF  fwd_fused_tc  KS, per-slab readiness flags and KA in one cooperative launch
 //
 // The feature map phi is a template parameter (ReLU, ELU+1, cos; the latter
 // two carried as bf16 hi + lo pairs); the block-causal form is a runtime
@@ -30,35 +29,32 @@
 //              warps w and w+4 share TMEM lanes 32*(w%4).. and split the heads
 //   warp  8    TMA producer (one lane)
 //   warp  9    UMMA issuer (one lane)
-//   warp 10    (single launch only) reductions across CTAs and state copies
 //
-// Schedule ("lockstep", in "positions"). The B*groups (b, group) slabs are
-// dealt out so that the CTAs running at the same time read the same token
-// rows of every group, i.e. whole contiguous rows of Q, K and V, instead of
-// 256-byte pieces of unrelated rows; on B200 that raised the HBM throughput of
-// both phases by 25-50 %. There are P positions; position k holds the slabs
-// k, k + P, k + 2P, ... (one per "set"), and the R CTAs k, k + P, ..., k +
-// (R-1) P share it, CTA r taking tiles r, r + R, r + 2R, ... of each of its
-// slabs, set after set:
-//   one set     S <= 148: P = S, R = min(148 / S, tiles);  S > 148: P = 148, R = 1
-//   two sets    P = ceil(S / 2), R = min(148 / P, tiles): every CTA works on a
-//               slab of the first set, then on one of the second, so in the
-//               single-launch forward the reduction of the first set's states
-//               happens while the second set's K and V stream in, and the
-//               second set's while the first set's queries are applied.
+// Schedule ("lockstep"): the B*groups (b, group) slabs are dealt out so that
+// the CTAs running at the same time read the same token rows of every group,
+// i.e. whole contiguous rows of Q, K and V, instead of 256-byte pieces of
+// unrelated rows; on B200 that raised the HBM throughput of both kernels by
+// 25-50 %. With S slabs and one CTA per SM (`sms` of them) there are P
+// positions; CTA c works on the slabs c % P, c % P + P, ...:
+//   S <= sms: P = S and R = min(sms / S, tiles) CTAs share a slab; CTA c takes
+//             slab c % S and its tiles r, r + R, r + 2R, ... with r = c / S.
+//   S >  sms: P = sms, R = 1: CTA c takes slabs c, c + sms, ... whole.
 // Each (CTA, slab) pair is one "segment"; KS writes one partial state per
-// segment and KR (or the single launch) adds a slab's R partials in ascending
-// CTA order.
+// segment and KR adds a slab's segments in ascending CTA order. (Taking the
+// slabs in two sets, one batch after the other with twice the CTAs per slab,
+// so that one set's reduction could overlap the other's loads, made the state
+// phase's reads 15 % slower on B200: 54 vs 47 us for the 4096px keys and
+// values in a load-only probe, more than the overlap saved.)
 //
-// Block-causal form (blocks of L tokens, L a multiple of 128; one set): the
-// tiles of a slab are padded to whole blocks, and its R = Rb * Rt CTAs split
-// the blocks first: CTA r takes blocks r % Rb, r % Rb + Rb, ... and, of each,
-// the tiles r / Rb, r / Rb + Rt, ... (Rt divides the tiles per block, so every
-// CTA takes tpb of them; tiles past N read as zeros and are not stored). A
-// segment is then one (slab, block) pair: KS writes one partial per (CTA,
-// slab, block), KR turns them into prefix states (ascending blocks, within a
-// block the Rt partials in ascending r), and KA stages the prefix state of a
-// segment's block once for its tpb tiles.
+// Block-causal form (blocks of L tokens, L a multiple of 128): the tiles of a
+// slab are padded to whole blocks, and its R = Rb * Rt CTAs split the blocks
+// first: CTA r takes blocks r % Rb, r % Rb + Rb, ... and, of each, the tiles
+// r / Rb, r / Rb + Rt, ... (Rt divides the tiles per block, so every CTA takes
+// tpb of them; tiles past N read as zeros and are not stored). A segment is
+// then one (slab, block) pair: KS writes one partial per (CTA, slab, block),
+// KR turns them into prefix states (ascending blocks, within a block the Rt
+// partials in ascending r), and KA stages the prefix state of a segment's
+// block once for its tpb tiles.
 // Every mbarrier wait is bounded; a wait that runs out sets an error code and
 // the whole CTA winds down (drains its TMA loads and UMMAs, frees TMEM).
 #pragma once
@@ -76,15 +72,9 @@ constexpr int kWorkerWarps = kWorkerThreads / 32;
 constexpr int kThreads = kWorkerThreads + 64;
 constexpr int kProducerWarp = kWorkerWarps;
 constexpr int kMmaWarp = kWorkerWarps + 1;
-// the single-launch forward adds one warp for the cross-CTA work
-constexpr int kSyncWarp = kWorkerWarps + 2;
-constexpr int kFusedThreads = kThreads + 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytesRow = 128;            // one swizzled row of a box
 constexpr int kSmemLimit = 232448;           // dynamic shared memory per CTA on sm_100
-// Data bytes of a kernel's shared memory: kSmemLimit less the barrier block,
-// the control block and the 1 KB alignment slack of SmemMap below.
-constexpr int kDataMax = kSmemLimit - 2048 - 64 - 1024;
 
 __device__ uint32_t g_device_error;          // first error code seen by any kernel
 
@@ -200,7 +190,7 @@ __host__ __device__ __forceinline__ int sched_block(int c, int seg, const Sched&
     return (c / q.P) % q.rb + (seg % sched_nb(c, q)) * q.rb;
 }
 // i-th tile of CTA c -> (slab, tile, segment index). In round k the R CTAs of
-// a position take tiles kR .. kR + R - 1 of its slab, CTA r always position r.
+// a slab take tiles kR .. kR + R - 1, CTA r always position r.
 // (Rotating the positions from round to round made every CTA finish the state
 // phase together, but all of them at the time the last position finished
 // before: slower overall, measured on B200.) Block-causal: see the comment at
@@ -226,50 +216,38 @@ struct KsParams {
     Sched q;
 };
 
+// A partial state (one per CTA segment and head) is stored by columns: entry
+// (i, j) of phi(K)^T [V | 1] (state row i, column j; j = d the normaliser) at
+// j * d + i. A warp that holds 32 rows of one column in its lanes (the TMEM
+// read-out) then stores 128 contiguous bytes per instruction, where the
+// state's row-major layout made every lane write its own cache line.
+
 constexpr int KS_TILE = 64;                                // tokens per stage
-constexpr int KS_MAX_STAGES = 6;
+constexpr int KS_STAGES = 6;                               // stages with phi = ReLU
 constexpr int KS_BOX_BYTES = KS_TILE * kBoxBytesRow;       // 8 KB
 constexpr int KS_STAGE_BYTES = 4 * KS_BOX_BYTES;           // K0 K1 V0 V1
-constexpr int KS_LO_BYTES = 2 * KS_BOX_BYTES;              // lo parts of phi(K) (feature maps other than ReLU)
-constexpr int KS_NUM_BARS = 3 * KS_MAX_STAGES + 11;
+constexpr int KS_ONES_OFF = KS_STAGES * KS_STAGE_BYTES;
+constexpr int KS_DATA_BYTES = KS_ONES_OFF + 1024;          // stages + the ones tile
+constexpr int KS_NUM_BARS = 3 * KS_STAGES + 5;
+// Other feature maps need phi(K) as bf16 hi + lo: 4 stages, and after them a
+// lo copy of each stage's two K boxes (same swizzled layout), in the same bytes.
+constexpr int KS_STAGES_SPLIT = 4;
+constexpr int KS_LO_OFF = KS_STAGES_SPLIT * KS_STAGE_BYTES;
+constexpr int KS_LO_BYTES = 2 * KS_BOX_BYTES;
+static_assert(KS_LO_OFF + KS_STAGES_SPLIT * KS_LO_BYTES == KS_ONES_OFF, "split layout fits the ReLU one");
 
-// Shared memory of the state phase: NS stages of K and V boxes from STAGE0,
-// NS lo regions from LO_OFF (feature maps other than ReLU carry phi(K) as
-// bf16 hi + lo: the hi part in place, the lo part there, same swizzled
-// layout), and the constant ones tile at ONES_OFF.
-template <int NS_, int STAGE0_, int LO_OFF_, int ONES_OFF_>
-struct KsSmem {
-    static constexpr int NS = NS_;
-    static constexpr int STAGE0 = STAGE0_;
-    static constexpr int LO_OFF = LO_OFF_;
-    static constexpr int ONES_OFF = ONES_OFF_;
-    static_assert(NS >= 2 && NS <= KS_MAX_STAGES, "state-phase stages");
-    static_assert(STAGE0 % 1024 == 0 && LO_OFF % 1024 == 0 && ONES_OFF % 1024 == 0, "swizzle alignment");
-};
-
-// The state kernel's own layout: 6 stages with phi = ReLU; otherwise 4 stages
-// and their lo regions in the same bytes.
 template <int FM>
-struct KsOwnSmem;
-template <>
-struct KsOwnSmem<kFeatureRelu> : KsSmem<6, 0, 6 * KS_STAGE_BYTES, 6 * KS_STAGE_BYTES> {};
-template <int FM>
-struct KsOwnSmem : KsSmem<4, 0, 4 * KS_STAGE_BYTES, 4 * KS_STAGE_BYTES + 4 * KS_LO_BYTES> {};
-constexpr int KS_DATA_BYTES = 6 * KS_STAGE_BYTES + 1024;   // stages + the ones tile
-static_assert(4 * KS_STAGE_BYTES + 4 * KS_LO_BYTES + 1024 <= KS_DATA_BYTES, "split layout fits the ReLU one");
+__host__ __device__ constexpr int ks_stages() { return FM == kFeatureRelu ? KS_STAGES : KS_STAGES_SPLIT; }
 
 struct KsBars {
-    uint64_t* full;        // [KS_MAX_STAGES] K and V tiles landed
-    uint64_t* empty;       // [KS_MAX_STAGES] tiles read by the UMMAs
-    uint64_t* relu_done;   // [KS_MAX_STAGES] phi applied to the K tile
+    uint64_t* full;        // [KS_STAGES] K and V tiles landed
+    uint64_t* empty;       // [KS_STAGES] tiles read by the UMMAs
+    uint64_t* relu_done;   // [KS_STAGES] phi applied to the K tile
     uint64_t* acc_full;    // [2] a segment's accumulator complete
     uint64_t* acc_empty;   // [2] accumulator read by the epilogue warps 0-3
-    uint64_t* mma_done;    // every state-phase UMMA complete
-    uint64_t* seg_written; // [2] (single launch) warps 0-3 wrote a segment's partial states
-    uint64_t* p2_go;       // [2] (single launch) the partials of a set's slab are all in memory
-    uint64_t* p2_done;     // [2] (single launch) this CTA's slice of that slab is reduced
+    uint64_t* mma_done;
     __device__ void init() const {
-        for (int s = 0; s < KS_MAX_STAGES; ++s) {
+        for (int s = 0; s < KS_STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
             ptx::mbar_init(&relu_done[s], kWorkerWarps);
@@ -277,66 +255,47 @@ struct KsBars {
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&acc_full[a], 1);
             ptx::mbar_init(&acc_empty[a], 4);
-            ptx::mbar_init(&seg_written[a], 4);
-            ptx::mbar_init(&p2_go[a], 1);
-            ptx::mbar_init(&p2_done[a], kWorkerWarps);
         }
         ptx::mbar_init(mma_done, 1);
     }
 };
 
 __device__ __forceinline__ KsBars ks_bars(uint64_t* b) {
-    constexpr int S = KS_MAX_STAGES;
-    return KsBars{b, b + S, b + 2 * S, b + 3 * S, b + 3 * S + 2, b + 3 * S + 4, b + 3 * S + 5,
-                  b + 3 * S + 7, b + 3 * S + 9};
+    return KsBars{b, b + KS_STAGES, b + 2 * KS_STAGES, b + 3 * KS_STAGES, b + 3 * KS_STAGES + 2,
+                  b + 3 * KS_STAGES + 4};
 }
 
-__device__ __forceinline__ void ks_fill_ones(uint8_t* ones, int tid) {
+__device__ __forceinline__ void ks_fill_ones(uint8_t* smem, int tid) {
     // constant all-ones bf16 operand (16 tokens x 16 columns) for the normaliser column
     if (tid < 32) {
-        uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-        reinterpret_cast<uint4*>(ones)[tid] = v;
+        uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        reinterpret_cast<uint4*>(smem + KS_ONES_OFF)[tid] = ones;
         ptx::fence_proxy_async_smem();
     }
 }
-
-// Calls a phase makes into the kernel around it (the single-launch forward's
-// readiness flags and reductions); the plain kernels use NoHooks.
-struct NoHooks {
-    // all worker threads, at the top of state-phase iteration i; false = stop
-    __device__ bool ks_worker(int) const { return true; }
-    // the UMMA lane, at the top of state-phase iteration i
-    __device__ void ks_mma(int) const {}
-    // worker warps 0-3 after writing the partial states of segment seg
-    __device__ void ks_segment_written(int, const KsBars&) const {}
-    // all worker threads, at the top of apply-phase iteration i; false = stop
-    __device__ bool ka_worker(int) const { return true; }
-    // the UMMA lane before the UMMAs of apply unit i (tps: units per segment); false = stop
-    __device__ bool ka_mma(int, int) const { return true; }
-};
 
 // The state phase for CTA `cta`: partial states phi(K)^T [V | 1] of its
 // segments into `partial`. Every role returns once its part is done. Stage s
 // of this phase is free again once bar.empty[s] has completed the phase of the
 // last tile that used it (the single-launch kernel's apply phase waits for
 // that before it loads into the same bytes).
-template <int D, int FM, class KL, class Hooks>
+template <int D, int FM>
 __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
                                          int cta, float* __restrict__ partial, uint8_t* smem,
                                          const KsBars& bar, uint32_t tmem, volatile int* abort,
-                                         uint32_t* err, const Hooks& hooks, bool evict_first = false)
+                                         uint32_t* err, bool evict_first = false)
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
-    constexpr int NS = KL::NS;
+    constexpr int NS = ks_stages<FM>();
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     if (cta >= p.q.grid) return;
     const int tps = sched_tps(cta, p.q);
     const int ntiles = tps * sched_nseg(cta, p.q);
-    auto stage_ptr = [&](int s) { return smem + KL::STAGE0 + (size_t)s * KS_STAGE_BYTES; };
-    auto lo_ptr = [&](int s) { return smem + KL::LO_OFF + (size_t)s * KS_LO_BYTES; };
+    auto stage_ptr = [&](int s) { return smem + (size_t)s * KS_STAGE_BYTES; };
+    auto lo_ptr = [&](int s) { return smem + KS_LO_OFF + (size_t)s * KS_LO_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
@@ -376,11 +335,10 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
             constexpr uint32_t idesc_v = ptx::idesc_bf16_f32(128, 128, 1, 1);
             constexpr uint32_t idesc_1 = ptx::idesc_bf16_f32(128, 16, 1, 1);
             const uint64_t ones_desc =
-                ptx::smem_desc(ptx::smem_u32(smem + KL::ONES_OFF), 256, 128, ptx::kLayoutNone);
+                ptx::smem_desc(ptx::smem_u32(smem + KS_ONES_OFF), 256, 128, ptx::kLayoutNone);
             int seg = -1;
             bool first = true;
             for (int i = 0; i < ntiles; ++i) {
-                hooks.ks_mma(i);
                 const bool seg_start = (i % tps) == 0;
                 const bool seg_end = (i % tps) == tps - 1;
                 if (seg_start) {
@@ -420,10 +378,9 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
             ptx::umma_commit(bar.mma_done);
             ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
         }
-    } else if (warp < kWorkerWarps) {
+    } else {
         // --------------------------------------------------------- workers ----
         for (int i = 0; i < ntiles; ++i) {
-            if (!hooks.ks_worker(i)) break;
             const bool seg_end = (i % tps) == tps - 1;
             const int seg = i / tps;
             const int s = i % NS;
@@ -457,12 +414,11 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
                 const int h = (slab % p.groups) * G + hh;
                 if (h < p.H) {
                     const long long slot = ((long long)cta * p.q.max_seg + seg) * G + hh;
-                    float* P = partial + slot * DD + (long long)row * (D + 1);
+                    float* P = partial + slot * DD + row;               // column j at j * D
 #pragma unroll
-                    for (int j = 0; j < D; ++j) P[j] = v[j];
-                    P[D] = nrm;
+                    for (int j = 0; j < D; ++j) P[j * D] = v[j];
+                    P[D * D] = nrm;
                 }
-                hooks.ks_segment_written(seg, bar);
             }
         }
     }
@@ -487,7 +443,8 @@ __device__ __forceinline__ long long ks_block_step(int G, const KsParams& p) {
 
 // ===================================================================== KR ===
 // One thread per state entry (grid: (b, h) x entry blocks), so every load is
-// independent and the kernel costs about one L2 round trip.
+// independent and the kernel costs about one L2 round trip; consecutive
+// threads read consecutive partial entries.
 constexpr int KR_THREADS = 128;
 
 template <int D>
@@ -501,8 +458,9 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     // reading the state.
     ptx::launch_dependents();
     ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
-    const int e = blockIdx.y * KR_THREADS + threadIdx.x;
-    if (e >= DD) return;
+    const int pe = blockIdx.y * KR_THREADS + threadIdx.x;     // entry in the partials' column order
+    if (pe >= DD) return;
+    const int e = (pe % D) * (D + 1) + pe / D;                // the same entry, row-major in the state
     const long long bh = blockIdx.x;
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
@@ -513,7 +471,7 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     // sum over blocks, i.e. the inclusive prefix state of every block
     float s = 0.0f;
     for (int j = 0; j < p.q.nblk; ++j) {
-        const float* src = partial + ks_block_slot(slab, j, h % G, G, p) * DD + e;
+        const float* src = partial + ks_block_slot(slab, j, h % G, G, p) * DD + pe;
         // eight loads in flight, then their additions in ascending order
         for (int r0 = 0; r0 < nr; r0 += 8) {
             float t[8];
@@ -527,8 +485,8 @@ kr_reduce_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     }
 }
 
-// Block-causal prefix states. A CTA takes 32 consecutive state entries (so
-// every load instruction reads 128 contiguous bytes) times 8 block lanes:
+// Block-causal prefix states. A CTA takes 32 consecutive partial-state entries
+// (so every load instruction reads 128 contiguous bytes) times 8 block lanes:
 // lane jl sums the partials (ascending CTA) of blocks jl, jl+8, ... of a
 // 64-block chunk into shared memory, then one thread per entry walks the
 // chunk in block order: prefix_j = prefix_{j-1} + blocksum_j. The same
@@ -548,8 +506,9 @@ kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restr
     ptx::wait_prerequisite_grid();              // the partial states of ks_state_tc
     const int el = threadIdx.x % KP_ENTRIES;
     const int jl = threadIdx.x / KP_ENTRIES;
-    const int e = blockIdx.y * KP_ENTRIES + el;
-    const bool live = e < DD;
+    const int pe = blockIdx.y * KP_ENTRIES + el;              // entry in the partials' column order
+    const bool live = pe < DD;
+    const int e = (pe % D) * (D + 1) + pe / D;                // the same entry, row-major in the state
     const long long bh = blockIdx.x;
     const int b = (int)(bh / p.H);
     const int h = (int)(bh % p.H);
@@ -561,7 +520,7 @@ kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restr
         for (int jj = jl; jj < KP_CHUNK && j0 + jj < p.q.nblk; jj += KP_LANES) {
             float x = 0.0f;
             if (live) {
-                const float* src = partial + ks_block_slot(slab, j0 + jj, h % G, G, p) * DD + e;
+                const float* src = partial + ks_block_slot(slab, j0 + jj, h % G, G, p) * DD + pe;
                 for (int r0 = 0; r0 < nr; r0 += 8) {
                     float t[8];
 #pragma unroll
@@ -599,10 +558,6 @@ kr_prefix_tc(const float* __restrict__ partial, const KsParams p, float* __restr
 //             worker warps stores its own heads' boxes)
 // TMEM: the accumulator at columns [0, 256) (head h at h * 256/G) and two A
 // buffers of 64 columns at 256 and 320.
-// The states of a CTA's segments live in two shared-memory regions, segment
-// j in region j % 2: the apply kernel stages them there from the reduced fp32
-// state; the single launch copies them there with TMA, already reduced and
-// split into bf16 hi and lo parts.
 struct KaParams {
     int N, H, groups;
     Sched q;
@@ -614,62 +569,37 @@ struct KaParams {
 };
 
 constexpr int KA_TILE = 128;                               // tokens = UMMA M
-constexpr int KA_MAX_STAGES = 6;
 constexpr int KA_BOX_BYTES = KA_TILE * kBoxBytesRow;       // 16 KB
 constexpr int KA_STAGE_BYTES = 2 * KA_BOX_BYTES;           // one group row of 128 tokens
 constexpr uint32_t KA_A_COL = 256;                         // first A buffer column
 constexpr uint32_t KA_A_LO_COL = 384;                      // lo parts of phi(Q) (feature maps other than ReLU)
-static_assert(KA_STAGE_BYTES == KS_STAGE_BYTES, "the single launch reuses state-phase stages for Q");
+constexpr int kBarRegion = 4096;                           // barriers + control block + slack
 
-// The staged state of one slab: per head of the group, two bf16 matrices (hi
-// and lo parts) of NA x D, K-major and unswizzled (8 x 8 core matrices): the
-// UMMA's B operand, N = NA columns (d numerators, the normaliser, zeros).
-template <int D>
-struct StateLayout {
+template <int D, bool OUT_BF16>
+struct KaLayout {
     static constexpr int G = 128 / D;
     static constexpr int NA = D + 16;                      // UMMA N: d numerator cols + normaliser + pad
     static constexpr int SBO = (D / 8) * 128;              // 8-row group stride of the K-major state
     static constexpr int MAT_BYTES = (NA / 8) * SBO;       // one bf16 NA x D matrix
-    static constexpr int BYTES = G * 2 * MAT_BYTES;        // hi and lo for every head
-    static_assert(BYTES % 1024 == 0, "regions stay 1 KB aligned");
-};
-
-// Shared memory of the apply kernel and of the single-launch forward:
-//   [0, 2 SB)        two state regions
-//   WORK ..          state phase (single launch): KS_NS stages of K and V,
-//                    their lo regions (feature maps other than ReLU), the ones tile
-//                    apply phase: KA_NS stages of Q, then STG_BUFS output tiles
-// The apply phase's Q stage s is the state phase's stage s.
-template <int D, bool OUT_BF16, int FM>
-struct ApplyLayout {
-    using SL = StateLayout<D>;
-    static constexpr int G = SL::G;
-    static constexpr int STATE_BYTES = SL::BYTES;
-    static constexpr int WORK = 2 * STATE_BYTES;
-    static constexpr int WORK_BYTES = kDataMax - WORK;
-    // apply phase
+    static constexpr int STATE_BYTES = G * 2 * MAT_BYTES;  // hi and lo for every head
     static constexpr int OUT_BYTES = OUT_BF16 ? 2 : 4;
     static constexpr int OUT_BOXES = 128 * OUT_BYTES / kBoxBytesRow;   // boxes per output group row
     static constexpr int OUT_BOX_ELEMS = kBoxBytesRow / OUT_BYTES;
     static constexpr int STG_BYTES = OUT_BOXES * KA_BOX_BYTES;
-    // two staging tiles if that still leaves three Q stages, else one (an
-    // epilogue that has to wait for the previous unit's store to read the
-    // single tile cost the 4096px apply a quarter of its speed on B200)
-    static constexpr int STG_BUFS = (WORK_BYTES - 2 * STG_BYTES) / KA_STAGE_BYTES >= 3 ? 2 : 1;
-    static constexpr int KA_FIT = (WORK_BYTES - STG_BUFS * STG_BYTES) / KA_STAGE_BYTES;
-    static constexpr int KA_NS = KA_FIT > KA_MAX_STAGES ? KA_MAX_STAGES : KA_FIT;
-    static constexpr int STG_OFF = WORK + KA_NS * KA_STAGE_BYTES;
-    // state phase (single launch)
-    static constexpr int KS_LO = FM == kFeatureRelu ? 0 : KS_LO_BYTES;
-    static constexpr int KS_FIT = (WORK_BYTES - 1024) / (KS_STAGE_BYTES + KS_LO);
-    static constexpr int KS_NS = KS_FIT > KS_MAX_STAGES ? KS_MAX_STAGES : KS_FIT;
-    static constexpr int KS_LO_OFF = WORK + KS_NS * KS_STAGE_BYTES;
-    static constexpr int KS_ONES_OFF = KS_LO_OFF + KS_NS * KS_LO;
-    using Ks = KsSmem<KS_NS, WORK, KS_LO_OFF, KS_ONES_OFF>;
-    static constexpr int APPLY_END = STG_OFF + STG_BUFS * STG_BYTES;
-    static constexpr int FUSED_END = KS_ONES_OFF + 1024 > APPLY_END ? KS_ONES_OFF + 1024 : APPLY_END;
-    static_assert(KA_NS >= 2, "the apply phase needs two Q stages");
-    static_assert(FUSED_END <= kDataMax, "shared memory");
+    static constexpr int AVAIL = kSmemLimit - 1024 - kBarRegion - STATE_BYTES;
+    // two staging tiles if that still leaves four Q stages, else one (an
+    // epilogue that waits for the previous unit's store to read a single tile
+    // made the 4096px apply a quarter slower on B200, and three Q stages
+    // instead of four 6 % slower)
+    static constexpr int STG_BUFS = (AVAIL - 2 * STG_BYTES) / KA_STAGE_BYTES >= 4 ? 2 : 1;
+    static constexpr int STAGES_FIT = (AVAIL - STG_BUFS * STG_BYTES) / KA_STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+    static constexpr int STATE_OFF = STAGES * KA_STAGE_BYTES;
+    static constexpr int STG_OFF = STATE_OFF + STATE_BYTES;
+    static constexpr int DATA_BYTES = STG_OFF + STG_BUFS * STG_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 14;
+    static constexpr int ACC_COLS = 256 / G;               // TMEM columns per head
+    static_assert(STAGES >= 3, "KA needs at least three Q stages");
 };
 
 // element (n, k) of a K-major, unswizzled bf16 matrix made of 8x8 core matrices
@@ -678,19 +608,21 @@ __host__ __device__ __forceinline__ int state_off(int n, int k) {
     return (n >> 3) * SBO + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
 }
 
+template <int D, bool OUT_BF16>
 struct KaBars {
-    uint64_t* full;        // [KA_MAX_STAGES] Q tile landed
-    uint64_t* empty;       // [KA_MAX_STAGES] Q tile read by every worker warp
+    using L = KaLayout<D, OUT_BF16>;
+    uint64_t* full;        // [STAGES] Q tile landed
+    uint64_t* empty;       // [STAGES] Q tile read by every worker warp
     uint64_t* a_full;      // [2] A operand in TMEM (and the state staged)
     uint64_t* acc_full;    // UMMAs of a unit done
     uint64_t* acc_empty;   // accumulator read by every worker warp
     uint64_t* stg_free;    // [2 halves] this half's staging boxes may be written
     uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
     uint64_t* mma_done;
-    uint64_t* state_full;  // [2] (single launch) a state region's TMA copy landed
+    uint64_t* grid_ready;  // (single launch) the staged slab's partial states are in memory
     uint64_t* p1_written;  // (single launch) this CTA's partial states are written
     __device__ void init() const {
-        for (int s = 0; s < KA_MAX_STAGES; ++s) {
+        for (int s = 0; s < L::STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], kWorkerWarps);
         }
@@ -704,83 +636,125 @@ struct KaBars {
             ptx::mbar_init(&stg_full[2 * h + 1], kWorkerWarps / 2);
         }
         ptx::mbar_init(mma_done, 1);
-        ptx::mbar_init(&state_full[0], 1);
-        ptx::mbar_init(&state_full[1], 1);
+        ptx::mbar_init(grid_ready, 1);
         ptx::mbar_init(p1_written, 4);
     }
 };
-constexpr int KA_NUM_BARS = 2 * KA_MAX_STAGES + 15;
 
-__device__ __forceinline__ KaBars ka_bars(uint64_t* b) {
-    constexpr int S = KA_MAX_STAGES;
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ KaBars<D, OUT_BF16> ka_bars(uint64_t* b) {
+    constexpr int S = KaLayout<D, OUT_BF16>::STAGES;
     uint64_t* a = b + 2 * S;
-    return KaBars{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 13};
+    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 12};
 }
 
-// zero the padding columns n in (d, NA) of both staged-state regions
-template <int D>
+// zero the padding columns n in (d, NA) of the staged state
+template <int D, bool OUT_BF16>
 __device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid) {
-    using SL = StateLayout<D>;
+    using L = KaLayout<D, OUT_BF16>;
     if (tid < kWorkerThreads) {
-        constexpr int PAD = SL::NA - D - 1;
-        for (int e = tid; e < 2 * SL::G * 2 * PAD * D; e += kWorkerThreads) {
+        constexpr int PAD = L::NA - D - 1;
+        for (int e = tid; e < L::G * 2 * PAD * D; e += kWorkerThreads) {
             const int k = e % D;
             const int n = D + 1 + (e / D) % PAD;
             const int mat = e / (D * PAD);
-            *reinterpret_cast<__nv_bfloat16*>(smem + mat * SL::MAT_BYTES + state_off<SL::SBO>(n, k)) =
-                __float2bfloat16_rn(0.0f);
+            *reinterpret_cast<__nv_bfloat16*>(smem + L::STATE_OFF + mat * L::MAT_BYTES +
+                                              state_off<L::SBO>(n, k)) = __float2bfloat16_rn(0.0f);
         }
     }
 }
 
+// Where the apply phase gets the state of a slab from:
+//   state != nullptr   the reduced fp32 state (B, H, d, d+1) of the reduction kernel
+//   otherwise          the partial states of the state phase (same launch), summed
+//                      here in the reduction kernel's order, once the arrival
+//                      flags of the CTAs that wrote them hold this launch's epoch
+struct KaStateSrc {
+    const float* state;
+    const float* partial;
+    KsParams ks;
+    const unsigned long long* flags;   // one arrival flag per CTA of the grid
+    unsigned long long epoch;          // unique to this launch (set by the host)
+};
+
+// Readiness flags of the single-launch forward. CTA c announces that all its
+// partial states are in memory by storing the launch's epoch into flags[c]
+// (after a fence). Before staging a slab's state, a CTA waits only for the
+// flags of the CTAs that wrote that slab's partials (its R siblings), not for
+// the whole grid. The host draws a new 64-bit epoch for every launch, so flags
+// left by earlier launches (or any other bytes) never pass for this one and
+// the flag array needs no reset between launches.
+__device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned long long epoch) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
+}
+
+// Bounded spin of one whole warp until flags[first + r * stride] hold `epoch`
+// for r < count (warp-uniform result). On a timeout it records the error code
+// and sets *abort.
+__device__ __forceinline__ bool flags_wait(const unsigned long long* flags, int first, int stride, int count,
+                                           unsigned long long epoch, volatile int* abort, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (;;) {
+        bool mine = true;
+        for (int r = lane; r < count; r += 32) {
+            unsigned long long v;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + first + r * stride) : "memory");
+            mine = mine && v == epoch;
+        }
+        if (__all_sync(0xffffffffu, mine)) return true;
+        bool give_up = *abort != 0;
+        if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
+            if (lane == 0) {
+                atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
+                *abort = 1;
+            }
+            give_up = true;
+        }
+        if (__any_sync(0xffffffffu, give_up)) return false;
+        __nanosleep(200);
+    }
+}
+
 // The apply phase for CTA `cta`.
-// FUSED = false: the state of every segment is staged from `state`, the
-// reduced fp32 states (B, H, nblk, d, d+1) of the reduction kernel, by the
-// worker warps (the first two segments before the first unit, later ones into
-// the region of the segment two back, once its UMMAs are done).
-// FUSED = true (single launch): the UMMA lane waits for a region's TMA copy
-// (hooks.ka_mma) before the first unit of a segment; the workers stage nothing.
-// `prev`/`prev_tiles` (single launch): the state phase's barriers and how many
-// tiles it loaded; Q stage s reuses the state phase's stage s, so the first
-// load into each waits until the state phase released that stage (or, for a
-// stage past the state phase's, until all its UMMAs are done).
-template <int D, bool OUT_BF16, int FM, bool FUSED, class Hooks>
+// `prev_empty`/`prev_tiles` (single launch): the state phase's stage barriers
+// and how many tiles it loaded; Q stage s (< 6) reuses its stage s, so the
+// first load into each waits until the state phase released that stage.
+template <int D, bool OUT_BF16, int FM>
 __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorMap* tmO, const KaParams& p,
-                                         int cta, const float* __restrict__ state, uint8_t* smem,
-                                         const KaBars& bar, uint32_t tmem, volatile int* abort, uint32_t* err,
-                                         const Hooks& hooks, const KsBars* prev = nullptr, int prev_tiles = 0,
+                                         int cta, const KaStateSrc& src, uint8_t* smem,
+                                         const KaBars<D, OUT_BF16>& bar, uint32_t tmem,
+                                         volatile int* abort, uint32_t* err,
+                                         uint64_t* prev_empty = nullptr, int prev_tiles = 0,
                                          bool evict_first = false)
 {
-    using L = ApplyLayout<D, OUT_BF16, FM>;
-    using SL = StateLayout<D>;
+    using L = KaLayout<D, OUT_BF16>;
     constexpr int G = L::G;
     constexpr int DD = D * (D + 1);
-    constexpr int S = L::KA_NS;
+    constexpr int S = L::STAGES;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     if (cta >= p.q.grid) return;
+    uint8_t* sstate = smem + L::STATE_OFF;
     const int tps = sched_tps(cta, p.q);
-    const int nseg = sched_nseg(cta, p.q);
-    const int nunits = tps * nseg;
-    auto stage_ptr = [&](int s) { return smem + L::WORK + (size_t)s * KA_STAGE_BYTES; };
+    const int nunits = tps * sched_nseg(cta, p.q);
+    auto stage_ptr = [&](int s) { return smem + (size_t)s * KA_STAGE_BYTES; };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
             int issued = 0;
-            constexpr int PS = L::KS_NS;      // the state phase's stages (single launch)
+            constexpr int PS = ks_stages<FM>();       // the state phase's stages (single launch)
+            static_assert(L::STAGES <= PS && KA_STAGE_BYTES == KS_STAGE_BYTES, "stage reuse");
             for (int i = 0; i < nunits; ++i) {
                 const int s = i % S;
                 if (!ptx::mbar_wait(&bar.empty[s], ((i / S) & 1) ^ 1, abort, err)) break;
-                if (prev != nullptr && i < S) {
-                    if (s < PS) {
-                        // the state phase's next (never issued) use of stage s
-                        const int j = prev_tiles + ((s - prev_tiles) % PS + PS) % PS;
-                        if (!ptx::mbar_wait(&prev->empty[s], ((j / PS) & 1) ^ 1, abort, err)) break;
-                    } else if (!ptx::mbar_wait(prev->mma_done, 0, abort, err)) {
-                        break;
-                    }
+                if (prev_empty != nullptr && i < S) {
+                    // the state phase's next (never issued) use of stage s
+                    const int j = prev_tiles + ((s - prev_tiles) % PS + PS) % PS;
+                    if (!ptx::mbar_wait(&prev_empty[s], ((j / PS) & 1) ^ 1, abort, err)) break;
                 }
                 int slab, tile, seg;
                 sched_item(cta, i, tps, p.q, slab, tile, seg);
@@ -804,32 +778,30 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- UMMA issuer ----
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, SL::NA, 0, 0);
-            const uint32_t s_base0 = ptx::smem_u32(smem);
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, L::NA, 0, 0);
+            const uint32_t s_base = ptx::smem_u32(sstate);
             for (int i = 0; i < nunits; ++i) {
-                if (!hooks.ka_mma(i, tps)) break;
                 if (!ptx::mbar_wait(&bar.a_full[i & 1], (i >> 1) & 1, abort, err)) break;
                 if (!ptx::mbar_wait(bar.acc_empty, (i & 1) ^ 1, abort, err)) break;
                 ptx::tc_fence_after_sync();
-                const uint32_t s_base = s_base0 + (uint32_t)((i / tps) & 1) * (uint32_t)L::STATE_BYTES;
                 const uint32_t a_base = tmem + KA_A_COL + (uint32_t)(i & 1) * 64u;
                 const uint32_t a_lo_base = tmem + KA_A_LO_COL + (uint32_t)(i & 1) * 64u;
 #pragma unroll
                 for (int hh = 0; hh < G; ++hh) {
-                    const uint32_t d_tmem = tmem + (uint32_t)(hh * (256 / G));
+                    const uint32_t d_tmem = tmem + (uint32_t)(hh * L::ACC_COLS);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t a = a_base + (uint32_t)(hh * D / 2 + ks * 8);
-                        const uint32_t hi = s_base + (hh * 2 + 0) * SL::MAT_BYTES + ks * 256;
-                        const uint32_t lo = s_base + (hh * 2 + 1) * SL::MAT_BYTES + ks * 256;
-                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(hi, 128, SL::SBO, ptx::kLayoutNone),
+                        const uint32_t hi = s_base + (hh * 2 + 0) * L::MAT_BYTES + ks * 256;
+                        const uint32_t lo = s_base + (hh * 2 + 1) * L::MAT_BYTES + ks * 256;
+                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(hi, 128, L::SBO, ptx::kLayoutNone),
                                          idesc, ks > 0);
-                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(lo, 128, SL::SBO, ptx::kLayoutNone),
+                        ptx::umma_f16_ts(d_tmem, a, ptx::smem_desc(lo, 128, L::SBO, ptx::kLayoutNone),
                                          idesc, true);
                         if constexpr (FM != kFeatureRelu) {
                             // phi(Q) lo x S hi (lo x lo is below fp32 rounding)
                             const uint32_t al = a_lo_base + (uint32_t)(hh * D / 2 + ks * 8);
-                            ptx::umma_f16_ts(d_tmem, al, ptx::smem_desc(hi, 128, SL::SBO, ptx::kLayoutNone),
+                            ptx::umma_f16_ts(d_tmem, al, ptx::smem_desc(hi, 128, L::SBO, ptx::kLayoutNone),
                                              idesc, true);
                         }
                     }
@@ -839,7 +811,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
             ptx::umma_commit(bar.mma_done);
             ptx::mbar_wait(bar.mma_done, 0, nullptr, err);
         }
-    } else if (warp < kWorkerWarps) {
+    } else {
         // --------------------------------------------------------- workers ----
         // Warps w and w+4 own token rows m = 32*(w%4) + lane (their TMEM lanes);
         // warp w < 4 takes box 0 of the group row and heads [0, G/2), warp w >= 4
@@ -856,59 +828,124 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         // With the reduced state from a preceding kernel: this kernel may have
         // started before that kernel finished (programmatic launch); the Q loads
         // do not depend on it, the state does.
-        if (!FUSED) ptx::wait_prerequisite_grid();
+        if (src.state != nullptr) ptx::wait_prerequisite_grid();
 
-        // stage the state of segment `seg` (its slab and token block) in region
-        // seg % 2 as bf16 hi + lo parts
-        auto stage_state = [&](int seg) {
-            int slab, tile, sg;
-            sched_item(cta, seg * tps, tps, p.q, slab, tile, sg);
-            const int blk = sched_block(cta, seg, p.q);
+        // stage the state of `slab` in shared memory as bf16 hi + lo parts
+        int nsync = 0;      // slabs staged from partial states so far
+        auto stage_state = [&](int slab, int blk) -> bool {
+            if (src.state == nullptr) {
+                // the CTAs that wrote this slab's partials (slab % grid + r S,
+                // r < R) must be done; warp 0 waits and tells the others
+                if (warp == 0) {
+                    if (flags_wait(src.flags, slab % src.ks.q.P, src.ks.q.P, src.ks.q.R, src.epoch, abort, err)
+                        && lane == 0)
+                        ptx::mbar_arrive(bar.grid_ready);
+                }
+                if (!warp_wait(bar.grid_ready, nsync & 1, abort, err)) return false;
+                ++nsync;
+            }
             const int b = slab / p.groups;
             const int g = slab % p.groups;
-            uint8_t* sstate = smem + (seg & 1) * L::STATE_BYTES;
-            // entry x = hh * DD + e of the group; this thread takes x = tid + 256 j
-            constexpr int NE = (G * DD + kWorkerThreads - 1) / kWorkerThreads;
-            float v[NE];
+            // Chunks of four entries of one column (rows k0 .. k0 + 3 of column
+            // n of head hh): chunk c of the group is the c-th float4 of the
+            // heads' partial states (stored by columns); this thread takes
+            // chunks tid, tid + 256, ...
+            constexpr int NC = G * DD / 4;
+            constexpr int NCT = (NC + kWorkerThreads - 1) / kWorkerThreads;
+            float4 v[NCT];
 #pragma unroll
-            for (int j = 0; j < NE; ++j) {
-                const int x = tid + j * kWorkerThreads;
-                const int h = g * G + x / DD;
-                v[j] = (x < G * DD && h < p.H)
-                           ? state[(((long long)b * p.H + h) * p.state_nblk + p.blk0 + blk) * DD + x % DD] : 0.0f;
+            for (int j = 0; j < NCT; ++j) v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (src.state != nullptr) {
+                // the reduced state (row-major per head): four loads per chunk
+#pragma unroll
+                for (int j = 0; j < NCT; ++j) {
+                    const int c = tid + j * kWorkerThreads;
+                    const int hh = c / (DD / 4);
+                    const int w = c % (DD / 4);
+                    const int n = w / (D / 4);
+                    const int k0 = (w % (D / 4)) * 4;
+                    if (c < NC && g * G + hh < p.H) {
+                        const float* st = src.state +
+                            (((long long)b * p.H + g * G + hh) * p.state_nblk + p.blk0 + blk) * DD + n;
+                        v[j] = make_float4(st[(k0 + 0) * (D + 1)], st[(k0 + 1) * (D + 1)],
+                                           st[(k0 + 2) * (D + 1)], st[(k0 + 3) * (D + 1)]);
+                    }
+                }
+            } else {
+                // the same additions, in the same order, as kr_reduce_tc: the R
+                // partials of the slab in ascending r; RB partials' loads in
+                // flight together, one float4 per chunk
+                const long long kstep = ks_block_step(G, src.ks) * DD;
+                const float* base = src.partial + ks_slot(slab % src.ks.q.P, slab / src.ks.q.P, 0, G, src.ks) * DD;
+                constexpr int RB = D == 32 ? 4 : 2;
+                for (int r0 = 0; r0 < src.ks.q.R; r0 += RB) {
+                    float4 t[RB][NCT];
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+#pragma unroll
+                        for (int j = 0; j < NCT; ++j) {
+                            const int c = tid + j * kWorkerThreads;
+                            t[rb][j] = (c < NC && r0 + rb < src.ks.q.R)
+                                ? __ldcg(reinterpret_cast<const float4*>(base + (r0 + rb) * kstep) + c)
+                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        }
+                    }
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        if (r0 + rb < src.ks.q.R) {
+#pragma unroll
+                            for (int j = 0; j < NCT; ++j) {
+                                v[j].x += t[rb][j].x;
+                                v[j].y += t[rb][j].y;
+                                v[j].z += t[rb][j].z;
+                                v[j].w += t[rb][j].w;
+                            }
+                        }
+                    }
+                }
             }
 #pragma unroll
-            for (int j = 0; j < NE; ++j) {
-                const int x = tid + j * kWorkerThreads;
-                if (x < G * DD) {
-                    const int hh = x / DD;
-                    const int e = x % DD;
-                    const int k = e / (D + 1);       // state row i = UMMA K index
-                    const int n = e % (D + 1);       // state column j = UMMA N index
-                    const __nv_bfloat16 vh = __float2bfloat16_rn(v[j]);
-                    const __nv_bfloat16 vl = __float2bfloat16_rn(v[j] - __bfloat162float(vh));
-                    *reinterpret_cast<__nv_bfloat16*>(sstate + (hh * 2 + 0) * SL::MAT_BYTES +
-                                                      state_off<SL::SBO>(n, k)) = vh;
-                    *reinterpret_cast<__nv_bfloat16*>(sstate + (hh * 2 + 1) * SL::MAT_BYTES +
-                                                      state_off<SL::SBO>(n, k)) = vl;
+            for (int j = 0; j < NCT; ++j) {
+                const int c = tid + j * kWorkerThreads;
+                if (c < NC) {
+                    const int hh = c / (DD / 4);
+                    const int w = c % (DD / 4);
+                    const int n = w / (D / 4);               // state column j = UMMA N index
+                    const int k0 = (w % (D / 4)) * 4;        // state rows k0.. = UMMA K indices
+                    const bool live = g * G + hh < p.H;
+                    const float x[4] = {live ? v[j].x : 0.0f, live ? v[j].y : 0.0f,
+                                        live ? v[j].z : 0.0f, live ? v[j].w : 0.0f};
+                    uint32_t hw[2], lw[2];
+#pragma unroll
+                    for (int u = 0; u < 4; u += 2) {
+                        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[u]);
+                        const __nv_bfloat16 h1 = __float2bfloat16_rn(x[u + 1]);
+                        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[u] - __bfloat162float(h0));
+                        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[u + 1] - __bfloat162float(h1));
+                        hw[u / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                        lw[u / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+                    }
+                    // four consecutive K of one column: 8 contiguous bytes of a core matrix
+                    const int off = state_off<L::SBO>(n, k0);
+                    *reinterpret_cast<uint2*>(sstate + (hh * 2 + 0) * L::MAT_BYTES + off) = make_uint2(hw[0], hw[1]);
+                    *reinterpret_cast<uint2*>(sstate + (hh * 2 + 1) * L::MAT_BYTES + off) = make_uint2(lw[0], lw[1]);
                 }
             }
             ptx::fence_proxy_async_smem();
+            return true;
         };
 
         // A operand of unit i: phi(Q) row m, this warp's half, into A buffer
-        // i & 1; before the first unit the states of the first two segments,
-        // at the first unit of a later segment its state.
+        // i & 1; at the first unit of a segment also the state of its slab.
         auto prep = [&](int i) -> bool {
-            if constexpr (!FUSED) {
-                if (i == 0) {
-                    stage_state(0);
-                    if (nseg > 1) stage_state(1);
-                } else if (i % tps == 0 && i / tps >= 2) {
-                    // the UMMAs of the segment two back must be done reading its region
+            if (i % tps == 0) {
+                if (i > 0) {
+                    // the previous unit's UMMAs must be done reading the state
                     if (!warp_wait(bar.acc_full, (i - 1) & 1, abort, err)) return false;
-                    stage_state(i / tps);
                 }
+                int slab, tile, seg;
+                sched_item(cta, i, tps, p.q, slab, tile, seg);
+                if (!stage_state(slab, sched_block(cta, seg, p.q))) return false;
             }
             const int s = i % S;
             if (!warp_wait(&bar.full[s], (i / S) & 1, abort, err)) return false;
@@ -948,7 +985,6 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
 
         bool ok = nunits > 0 ? prep(0) : true;
         for (int i = 0; i < nunits && ok; ++i) {
-            if (!hooks.ka_worker(i)) break;
             if (i + 1 < nunits && !prep(i + 1)) break;
             // ---- epilogue of unit i
             if (!warp_wait(bar.acc_full, i & 1, abort, err)) break;
@@ -957,7 +993,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < HPW; ++j) {
-                const uint32_t col = (uint32_t)((half * HPW + j) * (256 / G));
+                const uint32_t col = (uint32_t)((half * HPW + j) * L::ACC_COLS);
                 ptx::tmem_ld_row<D>(lane_base + col, lane_base + col + D, num[j], &den[j]);
             }
             ptx::tc_fence_before_sync();
@@ -1023,216 +1059,6 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
     }
 }
 
-// ===================================================== single-launch forward ===
-// Readiness flags of the single-launch forward, one 64-bit word per (CTA,
-// set) for "partial states written" and one for "slice reduced". A CTA
-// publishes an event by storing the launch's epoch (after a fence); a waiter
-// compares with the epoch. The host draws a new 64-bit epoch for every launch,
-// so words left by earlier launches (or any other bytes) never pass for this
-// one and the flag array needs no reset between launches.
-__device__ __forceinline__ void publish(unsigned long long* flag, unsigned long long epoch) {
-    __threadfence();
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
-}
-
-// Bounded spin of one whole warp until flags[first + r * stride] hold `epoch`
-// for r < count (warp-uniform result). On a timeout it records the error code
-// and sets *abort.
-__device__ __forceinline__ bool flags_wait(const unsigned long long* flags, int first, int stride, int count,
-                                           unsigned long long epoch, volatile int* abort, uint32_t* err) {
-    const int lane = threadIdx.x & 31;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    for (;;) {
-        bool mine = true;
-        for (int r = lane; r < count; r += 32) {
-            unsigned long long v;
-            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + first + r * stride) : "memory");
-            mine = mine && v == epoch;
-        }
-        if (__all_sync(0xffffffffu, mine)) {
-            __threadfence();      // acquire: what the publishers wrote before their flags
-            return true;
-        }
-        bool give_up = *abort != 0;
-        if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
-            if (lane == 0) {
-                atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
-                *abort = 1;
-            }
-            give_up = true;
-        }
-        if (__any_sync(0xffffffffu, give_up)) return false;
-        __nanosleep(100);
-    }
-}
-
-// One slice of a slab's reduction: the sum of the R partial states of the
-// slab (ascending CTA, the reduction kernel's order), split into bf16 hi and
-// lo parts and written in the staged layout (StateLayout, zeros in the padding
-// columns and for heads past H) to `dst`. The slab's staged bytes are cut into
-// 16-byte chunks, one column n and eight rows k of one matrix; CTA r of the R
-// writes chunk pairs (hi and lo of the same entries) [q0, q1) of its share.
-template <int D>
-__device__ __forceinline__ void reduce_slice(const float* __restrict__ partial, const KsParams& ks, int slab,
-                                             int r, uint8_t* __restrict__ dst, int tid, int nthreads) {
-    using SL = StateLayout<D>;
-    constexpr int G = SL::G;
-    constexpr int DD = D * (D + 1);
-    constexpr int KB = D / 8;
-    constexpr int NQ = G * SL::NA * KB;
-    constexpr int RB = 8;                       // partials per batch of loads in flight
-    const int R = ks.q.R;
-    const int pos = slab % ks.q.P;
-    const int g = slab % ks.groups;
-    const float* base = partial + ks_slot(pos, slab / ks.q.P, 0, G, ks) * DD;
-    const long long rstep = (long long)ks.q.P * ks.q.max_seg * G * DD;    // CTA c -> c + P
-    const int q0 = (int)((long long)NQ * r / R);
-    const int q1 = (int)((long long)NQ * (r + 1) / R);
-    for (int q = q0 + tid; q < q1; q += nthreads) {
-        const int kb = q % KB;
-        const int n = (q / KB) % SL::NA;
-        const int hh = q / (KB * SL::NA);
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-        if (n <= D && g * G + hh < ks.H) {
-            const float* src = base + (long long)hh * DD + (long long)(kb * 8) * (D + 1) + n;
-            for (int r0 = 0; r0 < R; r0 += RB) {
-                float t[RB][8];
-#pragma unroll
-                for (int u = 0; u < RB; ++u) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        t[u][e] = r0 + u < R ? __ldcg(src + (r0 + u) * rstep + e * (D + 1)) : 0.0f;
-                }
-#pragma unroll
-                for (int u = 0; u < RB; ++u) {
-                    if (r0 + u < R) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] += t[u][e];
-                    }
-                }
-            }
-        }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(v[e]), h1 = __float2bfloat16_rn(v[e + 1]);
-            const __nv_bfloat16 l0 = __float2bfloat16_rn(v[e] - __bfloat162float(h0));
-            const __nv_bfloat16 l1 = __float2bfloat16_rn(v[e + 1] - __bfloat162float(h1));
-            hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-        }
-        const int off = state_off<SL::SBO>(n, kb * 8);
-        *reinterpret_cast<uint4*>(dst + (hh * 2 + 0) * SL::MAT_BYTES + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(dst + (hh * 2 + 1) * SL::MAT_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-}
-
-// What the single launch adds to the two phases, per CTA with at most two
-// segments (sets j = 0, 1; slab k + j P for position k = cta % P):
-//   P1  worker warps 0-3, after writing a segment's partial states: publish
-//       "partial written" (flag j of this CTA)
-//   P2  wait for the partial flags of the R CTAs of the slab, reduce this
-//       CTA's slice (reduce_slice) into `staged`, publish "slice reduced"
-//   P3  wait for the slice flags of the R CTAs of the slab, then one TMA bulk
-//       copy of the slab's staged state into region j (state_full[j])
-// The sync warp runs P2 and P3 of both sets in the background, one after the
-// other, while the other warps stream the second set's keys and the first
-// set's queries; the UMMA lane only waits for state_full[j] before the first
-// unit of segment j. A CTA with a single segment has its eight worker warps run
-// P2 right after its state phase (they would wait anyway; one warp reduces a
-// slice several times slower). Each wait is on events that every CTA reaches
-// without waiting for a later event of another CTA (partials need nothing,
-// slices need partials, copies need slices), so no cycle of waits can form.
-template <int D>
-struct FusedHooks {
-    const float* partial;
-    uint8_t* staged;                  // S x StateLayout<D>::BYTES
-    unsigned long long* flags;        // [grid][2] partial written, then [grid][2] slice reduced
-    unsigned long long epoch;
-    const KsParams* ks;
-    uint8_t* smem;                    // the two state regions
-    const KsBars* kbar;
-    const KaBars* abar;
-    volatile int* abort;
-    uint32_t* err;
-    int cta;
-
-    __device__ unsigned long long* flag_partial(int c, int j) const { return flags + 2 * c + j; }
-    __device__ unsigned long long* flag_slice(int c, int j) const { return flags + 2 * ks->q.grid + 2 * c + j; }
-    __device__ int slab(int j) const { return cta % ks->q.P + j * ks->q.P; }
-
-    // P2 by the eight worker warps (a CTA with one segment, after its state phase)
-    __device__ bool p2_workers(int j) const {
-        const int warp = threadIdx.x >> 5;
-        const int lane = threadIdx.x & 31;
-        const int P = ks->q.P;
-        if (warp == 0) {
-            const bool ok = flags_wait(flags, 2 * (cta % P) + j, 2 * P, ks->q.R, epoch, abort, err);
-            if (ok && lane == 0) ptx::mbar_arrive(&kbar->p2_go[j]);
-        }
-        if (!warp_wait(&kbar->p2_go[j], 0, abort, err)) return false;
-        reduce_slice<D>(partial, *ks, slab(j), cta / P, staged + (size_t)slab(j) * StateLayout<D>::BYTES,
-                        threadIdx.x, kWorkerThreads);
-        __threadfence();
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        warp_arrive(&kbar->p2_done[j]);
-        if (warp == 0) {
-            if (!warp_wait(&kbar->p2_done[j], 0, abort, err)) return false;
-            if (lane == 0) publish(flag_slice(cta, j), epoch);
-        }
-        return true;
-    }
-
-    // P2 by the sync warp
-    __device__ bool p2_sync(int j) const {
-        const int lane = threadIdx.x & 31;
-        const int P = ks->q.P;
-        if (!flags_wait(flags, 2 * (cta % P) + j, 2 * P, ks->q.R, epoch, abort, err)) return false;
-        reduce_slice<D>(partial, *ks, slab(j), cta / P, staged + (size_t)slab(j) * StateLayout<D>::BYTES,
-                        lane, 32);
-        __threadfence();
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) publish(flag_slice(cta, j), epoch);
-        return true;
-    }
-
-    // P3 by the sync warp
-    __device__ bool p3_sync(int j) const {
-        const int P = ks->q.P;
-        if (!flags_wait(flags + 2 * ks->q.grid, 2 * (cta % P) + j, 2 * P, ks->q.R, epoch, abort, err))
-            return false;
-        asm volatile("fence.proxy.async.global;" ::: "memory");   // the slices, for the async proxy
-        if ((threadIdx.x & 31) == 0) {
-            constexpr uint32_t bytes = StateLayout<D>::BYTES;
-            ptx::mbar_arrive_expect_tx(&abar->state_full[j], bytes);
-            ptx::bulk_load(smem + j * bytes, staged + (size_t)slab(j) * bytes, bytes, &abar->state_full[j]);
-        }
-        __syncwarp();
-        return true;
-    }
-
-    __device__ bool ks_worker(int) const { return true; }
-    __device__ void ks_mma(int) const {}
-    __device__ void ks_segment_written(int seg, const KsBars& bar) const {
-        const int warp = threadIdx.x >> 5;
-        __threadfence();
-        warp_arrive(&bar.seg_written[seg & 1]);
-        if (warp == 0 && warp_wait(&bar.seg_written[seg & 1], 0, abort, err) && (threadIdx.x & 31) == 0)
-            publish(flag_partial(cta, seg), epoch);
-    }
-    __device__ bool ka_worker(int) const { return true; }
-    __device__ bool ka_mma(int i, int tps) const {
-        if (i % tps == 0) {
-            if (!ptx::mbar_wait(&abar->state_full[i / tps], 0, abort, err)) return false;
-            ptx::tc_fence_after_sync();
-        }
-        return true;
-    }
-};
-
 // ============================================================ the kernels ===
 // Shared memory of every kernel: a data region (the largest phase it runs;
 // the phases of the single-launch kernel reuse it one after the other), then
@@ -1264,17 +1090,17 @@ __device__ __forceinline__ void kernel_epilogue(SharedCtl* ctl, int tid) {
 }
 
 using KsMap = SmemMap<KS_DATA_BYTES>;
-template <int D, bool OUT_BF16, int FM>
-using KaMap = SmemMap<ApplyLayout<D, OUT_BF16, FM>::APPLY_END>;
-template <int D, bool OUT_BF16, int FM>
-using FwdMap = SmemMap<ApplyLayout<D, OUT_BF16, FM>::FUSED_END>;
+template <int D, bool OUT_BF16>
+using KaMap = SmemMap<KaLayout<D, OUT_BF16>::DATA_BYTES>;
+template <int D, bool OUT_BF16>
+using FwdMap = SmemMap<(KaLayout<D, OUT_BF16>::DATA_BYTES > KS_DATA_BYTES ? KaLayout<D, OUT_BF16>::DATA_BYTES
+                                                                          : KS_DATA_BYTES)>;
 
 template <int D, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
 ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
             const KsParams p, float* __restrict__ partial)
 {
-    using KL = KsOwnSmem<FM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     const KsBars bar = ks_bars(reinterpret_cast<uint64_t*>(smem + KsMap::BAR_OFF));
@@ -1289,14 +1115,13 @@ ks_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         ptx::prefetch_tmap(&tmK);
         ptx::prefetch_tmap(&tmV);
     }
-    ks_fill_ones(smem + KL::ONES_OFF, tid);
+    ks_fill_ones(smem, tid);
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
     // the reduction kernel may be scheduled now; it waits for this grid's results
     if (tid == 0) ptx::launch_dependents();
-    ks_phase<D, FM, KL>(&tmK, &tmV, p, blockIdx.x, partial, smem, bar, ctl->tmem_base, &ctl->abort,
-                        &g_device_error, NoHooks{});
+    ks_phase<D, FM>(&tmK, &tmV, p, blockIdx.x, partial, smem, bar, ctl->tmem_base, &ctl->abort, &g_device_error);
     kernel_epilogue(ctl, tid);
 }
 
@@ -1305,10 +1130,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
             const KaParams p, const float* __restrict__ state)
 {
-    using Map = KaMap<D, OUT_BF16, FM>;
+    using Map = KaMap<D, OUT_BF16>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    const KaBars bar = ka_bars(reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF));
+    const auto bar = ka_bars<D, OUT_BF16>(reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF));
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Map::CTL_OFF);
     const int tid = threadIdx.x;
     if (tid == 0) {
@@ -1320,33 +1145,34 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         ptx::prefetch_tmap(&tmQ);
         ptx::prefetch_tmap(&tmO);
     }
-    ka_zero_state_padding<D>(smem, tid);
+    ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    ka_phase<D, OUT_BF16, FM, false>(&tmQ, &tmO, p, blockIdx.x, state, smem, bar, ctl->tmem_base, &ctl->abort,
-                                     &g_device_error, NoHooks{});
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull};
+    ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
+                          &g_device_error);
     kernel_epilogue(ctl, tid);
 }
 
 // The whole forward in one cooperative launch (all CTAs resident, so a CTA
-// may wait for another), on the two-set schedule: the state phase, whose
-// partial states each slab's CTAs reduce together in the reduction kernel's
-// order (P1-P3 above, overlapped with the phases), then the apply phase.
-// `staged` holds one staged state per slab; `flags` four words per CTA;
+// may wait for another): the state phase; a readiness flag per CTA; then the
+// apply phase, which waits (bounded) for the flags of the CTAs that wrote its
+// slab's partial states and sums them itself in the reduction kernel's order.
+// The apply phase's Q loads start as soon as the state phase has released its
+// shared memory, so they overlap that wait. `flags` has one slot per CTA;
 // `epoch` is unique to the launch.
 template <int D, bool OUT_BF16, int FM>
-__global__ void __launch_bounds__(kFusedThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-             const KsParams ks, const KaParams ka, float* __restrict__ partial, uint8_t* __restrict__ staged,
+             const KsParams ks, const KaParams ka, float* __restrict__ partial,
              unsigned long long* flags, const unsigned long long epoch, const int evict_first)
 {
-    using AL = ApplyLayout<D, OUT_BF16, FM>;
-    using Map = FwdMap<D, OUT_BF16, FM>;
-    // one token block, at most two segments per CTA; the three-kernel path
-    // takes everything else
-    if (ks.q.nblk != 1 || ks.q.max_seg > 2 || ka.q.P != ks.q.P || ka.q.grid > ks.q.grid) {
+    using Map = FwdMap<D, OUT_BF16>;
+    // the apply phase here sums one block's partials; prefix states over token
+    // blocks take the three-kernel path
+    if (ks.q.nblk != 1 || ka.q.nblk != 1) {
         if (threadIdx.x == 0) atomicCAS(&g_device_error, ptx::kErrNone, ptx::kErrUnsupported);
         return;
     }
@@ -1354,11 +1180,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Map::BAR_OFF);
     const KsBars kbar = ks_bars(bars);
-    const KaBars abar = ka_bars(bars + KS_NUM_BARS);
+    const auto abar = ka_bars<D, OUT_BF16>(bars + KS_NUM_BARS);
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Map::CTL_OFF);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int cta = blockIdx.x;
     if (tid == 0) {
         kbar.init();
         abar.init();
@@ -1371,50 +1196,36 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         ptx::prefetch_tmap(&tmQ);
         ptx::prefetch_tmap(&tmO);
     }
-    ks_fill_ones(smem + AL::KS_ONES_OFF, tid);
+    ks_fill_ones(smem, tid);
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
-    const int nseg = sched_nseg(cta, ks.q);                    // 1 or 2
-    const int tps_s = sched_tps(cta, ks.q);
-    const bool apply = cta < ka.q.grid;
-    const FusedHooks<D> hk{partial, staged, flags, epoch, &ks, smem, &kbar, &abar, &ctl->abort, &g_device_error,
-                           cta};
+    // with evict_first, K, V and Q (read once) are marked first to go when L2
+    // needs room
+    ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error,
+                    evict_first != 0);
 
-    if (warp == kSyncWarp) {
-        // P2 (two segments) and P3 of each set, in order; then the copies must
-        // land before the CTA may exit
-        int issued = 0;
-        for (int j = 0; j < nseg; ++j) {
-            if (nseg == 2 && !hk.p2_sync(j)) break;
-            if (apply) {
-                if (!hk.p3_sync(j)) break;
-                issued = j + 1;
-            }
-        }
-        if ((tid & 31) == 0)
-            for (int j = 0; j < issued; ++j) ptx::mbar_wait(&abar.state_full[j], 0, nullptr, &g_device_error);
-        __syncwarp();
-    } else {
-        // with evict_first, K, V and Q (read once) are marked first to go when
-        // L2 needs room
-        ks_phase<D, FM, typename AL::Ks>(&tmK, &tmV, ks, cta, partial, smem, kbar, tmem, &ctl->abort,
-                                         &g_device_error, hk, evict_first != 0);
-
-        // Warps 0-3 have written this CTA's partial states (after the last
-        // accumulator was complete, i.e. after every state-phase UMMA): every
-        // worker waits for that before it touches the apply phase's shared
-        // memory or TMEM, which reuse the state phase's.
-        if (warp < 4) warp_arrive(abar.p1_written);
-        if (warp < kWorkerWarps) {
-            const bool ok = warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
-            if (ok && nseg == 1) hk.p2_workers(0);
-        }
-        ka_phase<D, OUT_BF16, FM, true>(&tmQ, &tmO, ka, cta, nullptr, smem, abar, tmem, &ctl->abort,
-                                        &g_device_error, hk, &kbar, tps_s * nseg, evict_first != 0);
+    // Warps 0-3 have written this CTA's partial states (after the last
+    // accumulator was complete, i.e. after every state-phase UMMA): make them
+    // visible and arrive. Every worker waits for that before it touches the
+    // apply phase's shared memory or TMEM, which reuse the state phase's.
+    if (warp < 4) {
+        __threadfence();
+        warp_arrive(abar.p1_written);
     }
+    if (warp < kWorkerWarps) {
+        warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
+        // every CTA raises its readiness flag, with or without apply work
+        if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
+        ka_zero_state_padding<D, OUT_BF16>(smem, tid);
+    }
+    KaStateSrc src{nullptr, partial, ks, flags, epoch};
+    const int ks_tiles = (int)blockIdx.x < ks.q.grid
+        ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
+    ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
+                          kbar.empty, ks_tiles, evict_first != 0);
     kernel_epilogue(ctl, tid);
 }
 
