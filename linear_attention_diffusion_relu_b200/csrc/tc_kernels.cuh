@@ -619,7 +619,6 @@ struct KaBars {
     uint64_t* stg_free;    // [2 halves] this half's staging boxes may be written
     uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
     uint64_t* mma_done;
-    uint64_t* grid_ready;  // (single launch) the staged slab's partial states are in memory
     uint64_t* p1_written;  // (single launch) this CTA's partial states are written
     __device__ void init() const {
         for (int s = 0; s < L::STAGES; ++s) {
@@ -636,7 +635,6 @@ struct KaBars {
             ptx::mbar_init(&stg_full[2 * h + 1], kWorkerWarps / 2);
         }
         ptx::mbar_init(mma_done, 1);
-        ptx::mbar_init(grid_ready, 1);
         ptx::mbar_init(p1_written, 4);
     }
 };
@@ -645,7 +643,7 @@ template <int D, bool OUT_BF16>
 __device__ __forceinline__ KaBars<D, OUT_BF16> ka_bars(uint64_t* b) {
     constexpr int S = KaLayout<D, OUT_BF16>::STAGES;
     uint64_t* a = b + 2 * S;
-    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 12};
+    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11};
 }
 
 // zero the padding columns n in (d, NA) of the staged state
@@ -679,42 +677,15 @@ struct KaStateSrc {
 
 // Readiness flags of the single-launch forward. CTA c announces that all its
 // partial states are in memory by storing the launch's epoch into flags[c]
-// (after a fence). Before staging a slab's state, a CTA waits only for the
-// flags of the CTAs that wrote that slab's partials (its R siblings), not for
-// the whole grid. The host draws a new 64-bit epoch for every launch, so flags
-// left by earlier launches (or any other bytes) never pass for this one and
-// the flag array needs no reset between launches.
+// (after a fence). Before staging a slab's state, a CTA reads only the flags
+// of the CTAs that wrote that slab's partials (its R siblings), not those of
+// the whole grid, and adds each partial as soon as it and the ones before it
+// are in. The host draws a new 64-bit epoch for every launch, so flags left by
+// earlier launches (or any other bytes) never pass for this one and the flag
+// array needs no reset between launches.
 __device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned long long epoch) {
     __threadfence();
     asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
-}
-
-// Bounded spin of one whole warp until flags[first + r * stride] hold `epoch`
-// for r < count (warp-uniform result). On a timeout it records the error code
-// and sets *abort.
-__device__ __forceinline__ bool flags_wait(const unsigned long long* flags, int first, int stride, int count,
-                                           unsigned long long epoch, volatile int* abort, uint32_t* err) {
-    const int lane = threadIdx.x & 31;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    for (;;) {
-        bool mine = true;
-        for (int r = lane; r < count; r += 32) {
-            unsigned long long v;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flags + first + r * stride) : "memory");
-            mine = mine && v == epoch;
-        }
-        if (__all_sync(0xffffffffu, mine)) return true;
-        bool give_up = *abort != 0;
-        if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
-            if (lane == 0) {
-                atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
-                *abort = 1;
-            }
-            give_up = true;
-        }
-        if (__any_sync(0xffffffffu, give_up)) return false;
-        __nanosleep(200);
-    }
 }
 
 // The apply phase for CTA `cta`.
@@ -831,19 +802,7 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         if (src.state != nullptr) ptx::wait_prerequisite_grid();
 
         // stage the state of `slab` in shared memory as bf16 hi + lo parts
-        int nsync = 0;      // slabs staged from partial states so far
         auto stage_state = [&](int slab, int blk) -> bool {
-            if (src.state == nullptr) {
-                // the CTAs that wrote this slab's partials (slab % grid + r S,
-                // r < R) must be done; warp 0 waits and tells the others
-                if (warp == 0) {
-                    if (flags_wait(src.flags, slab % src.ks.q.P, src.ks.q.P, src.ks.q.R, src.epoch, abort, err)
-                        && lane == 0)
-                        ptx::mbar_arrive(bar.grid_ready);
-                }
-                if (!warp_wait(bar.grid_ready, nsync & 1, abort, err)) return false;
-                ++nsync;
-            }
             const int b = slab / p.groups;
             const int g = slab % p.groups;
             // Chunks of four entries of one column (rows k0 .. k0 + 3 of column
@@ -872,36 +831,70 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                     }
                 }
             } else {
-                // the same additions, in the same order, as kr_reduce_tc: the R
-                // partials of the slab in ascending r; RB partials' loads in
-                // flight together, one float4 per chunk
+                // The same additions, in the same order, as kr_reduce_tc: the R
+                // partials of the slab in ascending r. Partial r is in memory
+                // once flags[slab % P + r P] holds this launch's epoch (its CTA
+                // stored it after its partials). Each warp polls the flags itself
+                // and adds the partials of the ready prefix while it waits for
+                // the rest, RB partials' loads in flight together, one float4
+                // per chunk; only the last ones are loaded after the slowest CTA
+                // of the slab is done.
                 const long long kstep = ks_block_step(G, src.ks) * DD;
                 const float* base = src.partial + ks_slot(slab % src.ks.q.P, slab / src.ks.q.P, 0, G, src.ks) * DD;
+                const unsigned long long* fl = src.flags + slab % src.ks.q.P;
+                const int R = src.ks.q.R;
                 constexpr int RB = D == 32 ? 4 : 2;
-                for (int r0 = 0; r0 < src.ks.q.R; r0 += RB) {
-                    float4 t[RB][NCT];
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-#pragma unroll
-                        for (int j = 0; j < NCT; ++j) {
-                            const int c = tid + j * kWorkerThreads;
-                            t[rb][j] = (c < NC && r0 + rb < src.ks.q.R)
-                                ? __ldcg(reinterpret_cast<const float4*>(base + (r0 + rb) * kstep) + c)
-                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                        }
+                const uint64_t t0 = ptx::globaltimer_ns();
+                for (int r = 0; r < R;) {
+                    bool ready = true;
+                    if (r + lane < R) {
+                        unsigned long long f;
+                        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
+                                     : "=l"(f) : "l"(fl + (long long)(r + lane) * src.ks.q.P) : "memory");
+                        ready = f == src.epoch;
                     }
+                    const unsigned waiting = __ballot_sync(0xffffffffu, !ready);
+                    const int k = min(waiting ? __ffs(waiting) - 1 : 32, R - r);   // ready prefix from r
+                    if (k == 0) {
+                        bool give_up = *abort != 0;
+                        if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
+                            if (lane == 0) {
+                                atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
+                                *abort = 1;
+                            }
+                            give_up = true;
+                        }
+                        if (__any_sync(0xffffffffu, give_up)) return false;
+                        __nanosleep(64);
+                        continue;
+                    }
+                    __syncwarp();          // every lane's reads after every lane's flag
+                    for (int r0 = r; r0 < r + k; r0 += RB) {
+                        float4 t[RB][NCT];
 #pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        if (r0 + rb < src.ks.q.R) {
+                        for (int rb = 0; rb < RB; ++rb) {
 #pragma unroll
                             for (int j = 0; j < NCT; ++j) {
-                                v[j].x += t[rb][j].x;
-                                v[j].y += t[rb][j].y;
-                                v[j].z += t[rb][j].z;
-                                v[j].w += t[rb][j].w;
+                                const int c = tid + j * kWorkerThreads;
+                                t[rb][j] = (c < NC && r0 + rb < r + k)
+                                    ? __ldcg(reinterpret_cast<const float4*>(base + (r0 + rb) * kstep) + c)
+                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                            }
+                        }
+#pragma unroll
+                        for (int rb = 0; rb < RB; ++rb) {
+                            if (r0 + rb < r + k) {
+#pragma unroll
+                                for (int j = 0; j < NCT; ++j) {
+                                    v[j].x += t[rb][j].x;
+                                    v[j].y += t[rb][j].y;
+                                    v[j].z += t[rb][j].z;
+                                    v[j].w += t[rb][j].w;
+                                }
                             }
                         }
                     }
+                    r += k;
                 }
             }
 #pragma unroll
