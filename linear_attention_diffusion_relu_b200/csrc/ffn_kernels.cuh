@@ -392,57 +392,79 @@ gemm_bf16_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 }
 
 // ====================================================== depthwise + GLU ===
-// A CTA takes one batch image's tile of DW_TY grid rows x DW_TX columns and 64
+// A CTA takes one batch image's tile of TY grid rows x TX columns and 64
 // channels of each half (value a: c0 .. c0+63, gate g: Ch+c0 .. Ch+c0+63). Two
 // TMA loads bring the tile plus a one-token halo of each half into shared
 // memory ([row][column][64 channels], zeros outside the grid: the load starts
 // at column x0-1 and row y0-1). Lane l owns channels 2l and 2l+1 of both
-// halves, with their 2 x 2 x 9 fp32 taps in registers; warp w owns one output
-// row and a strip of DW_SX columns, along which it slides a 3 x 3 window of
-// unpacked values: each output column loads only the window's new column
-// (3 rows x 2 halves, 4 bytes per lane, one 128-byte line per warp) and
-// accumulates the 9 taps of both channels with packed fp32x2 FMAs. Then
-// Z = a * sigmoid(g) as bf16x2, kept in registers until every warp is done
-// with the input tile, written over it ([row][column][64 channels]) and
-// stored with one TMA store, which leaves out what lies outside the grid or
-// past the last channel.
+// halves, with their 2 x 2 x 9 fp32 taps in registers; warp w owns RPW output
+// rows and a strip of SX columns. It walks the strip's SX + 2 halo columns
+// once: each step loads one column (RPW + 2 rows x 2 halves, 4 bytes per
+// lane, one 128-byte line per warp), unpacks it to fp32 and adds its products
+// with the taps (packed fp32x2 FMAs) into the accumulators of the three
+// outputs of each row that use it (tap column dx for the output dx columns to
+// its left). An accumulator thus receives its nine products one column at a
+// time, a whole step apart, instead of in one dependent chain, and an output
+// is done once its last column has been added: Z = a * sigmoid(g) as bf16x2,
+// kept in registers until every warp is done with the input tile, written
+// over it ([row][column][64 channels]) and stored with one TMA store, which
+// leaves out what lies outside the grid or past the last channel.
 // U (tensor map): (B, Hg, Wg, 2*Ch) bf16; Kdw: (2*Ch, 3, 3) fp32; Z (tensor
 // map): (B, Hg, Wg, Ch) bf16.
-constexpr int DW_TY = 4;                        // grid rows per CTA
-constexpr int DW_TX = 64;                       // grid columns per CTA
-constexpr int DW_SX = 32;                       // columns per warp strip
 constexpr int DW_CH = 64;                       // channels of each half per CTA
-constexpr int DW_THREADS = 256;
-constexpr int DW_ROW_BYTES = (DW_TX + 2) * DW_CH * 2;                  // one halo row of one half
-constexpr int DW_HALF_BYTES = (DW_TY + 2) * DW_ROW_BYTES;              // one half's box: 50,688 B
-constexpr int DW_TAPS_OFF = 2 * DW_HALF_BYTES;                        // fp32 [half][tap][64 channels]
-constexpr int DW_BAR_OFF = DW_TAPS_OFF + 2 * 9 * DW_CH * 4;
-constexpr int DW_SMEM = DW_BAR_OFF + 16 + 128;  // barrier, flag, alignment slack
-static_assert(DW_TY * (DW_TX / DW_SX) == DW_THREADS / 32, "one strip per warp");
-static_assert(DW_TY * DW_TX * DW_CH * 2 <= DW_HALF_BYTES, "the output tile fits over the value half");
+
+template <int TY_, int TX_, int SX_, int RPW_, int MINB_>
+struct DwCfg {
+    static constexpr int TY = TY_;              // grid rows per CTA
+    static constexpr int TX = TX_;              // grid columns per CTA
+    static constexpr int SX = SX_;              // columns per warp strip
+    static constexpr int RPW = RPW_;            // output rows per warp
+    static constexpr int MINB = MINB_;          // CTAs per SM the registers are sized for
+    static constexpr int WARPS = (TY / RPW) * (TX / SX);
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int ROW_BYTES = (TX + 2) * DW_CH * 2;          // one halo row of one half
+    static constexpr int HALF_BYTES = (TY + 2) * ROW_BYTES;         // one half's box
+    static constexpr int TAPS_OFF = 2 * HALF_BYTES;                 // fp32 [half][tap][64 channels]
+    static constexpr int BAR_OFF = TAPS_OFF + 2 * 9 * DW_CH * 4;
+    static constexpr int SMEM = BAR_OFF + 16 + 128;                 // barrier, flag, alignment slack
+    static_assert(TY % RPW == 0 && TX % SX == 0, "whole strips");
+    static_assert(TY * TX * DW_CH * 2 <= HALF_BYTES, "the output tile fits over the value half");
+};
+// 4 x 32 tiles, 4 warps of 2 rows x 16 columns, 4 CTAs per SM (measured on
+// B200 at the 4096px shape: 268 us, against 283 for 8 x 32 tiles with 8 warps
+// and 2 CTAs per SM, 299 for 4 x 64 tiles of 1-row warps; summing each output's
+// nine products in one dependent chain per half instead: 290-305 us)
+using DwConfig = DwCfg<4, 32, 16, 2, 4>;
 
 __device__ __forceinline__ float2 bf16x2_unpack(uint32_t v) {
     return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
-__global__ void __launch_bounds__(DW_THREADS, 2)
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, Cfg::MINB)
 dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmZ,
            const float* __restrict__ Kdw, int Hg, int Wg, int Ch)
 {
+    constexpr int TY = Cfg::TY, TX = Cfg::TX, SX = Cfg::SX, RPW = Cfg::RPW;
+    constexpr int ROW_BYTES = Cfg::ROW_BYTES, HALF_BYTES = Cfg::HALF_BYTES;
     extern __shared__ uint8_t dsm_raw[];
     uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
-    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + DW_BAR_OFF);
-    int* loaded = reinterpret_cast<int*>(dsm + DW_BAR_OFF + 8);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + Cfg::BAR_OFF);
+    int* loaded = reinterpret_cast<int*>(dsm + Cfg::BAR_OFF + 8);
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int tiles_x = (Wg + DW_TX - 1) / DW_TX;
-    const int tiles_y = (Hg + DW_TY - 1) / DW_TY;
-    const int c0 = blockIdx.x * DW_CH;                       // first channel of the group (each half)
-    const int b = blockIdx.y / (tiles_y * tiles_x);
-    const int ty = (blockIdx.y / tiles_x) % tiles_y;
-    const int tx = blockIdx.y % tiles_x;
-    const int y0 = ty * DW_TY, x0 = tx * DW_TX;
+    const int tiles_x = (Wg + TX - 1) / TX;
+    const int tiles_y = (Hg + TY - 1) / TY;
+    // CTA = tile * groups + group: the CTAs running at the same time take every
+    // group of a few tiles, i.e. whole token rows of U
+    const int ngroups = (Ch + DW_CH - 1) / DW_CH;
+    const int c0 = (int)(blockIdx.x % ngroups) * DW_CH;      // first channel of the group (each half)
+    const int tile = (int)(blockIdx.x / ngroups);
+    const int b = tile / (tiles_y * tiles_x);
+    const int ty = (tile / tiles_x) % tiles_y;
+    const int tx = tile % tiles_x;
+    const int y0 = ty * TY, x0 = tx * TX;
     const int nch = min(DW_CH, Ch - c0);                     // channels of this group (multiple of 8)
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
@@ -450,14 +472,14 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUte
     }
     __syncthreads();
     if (tid == 0) {
-        ptx::mbar_arrive_expect_tx(bar, 2 * DW_HALF_BYTES);
+        ptx::mbar_arrive_expect_tx(bar, 2 * HALF_BYTES);
         ptx::tma_load_4d(dsm, &tmU, bar, c0, x0 - 1, y0 - 1, b);
-        ptx::tma_load_4d(dsm + DW_HALF_BYTES, &tmU, bar, Ch + c0, x0 - 1, y0 - 1, b);
+        ptx::tma_load_4d(dsm + HALF_BYTES, &tmU, bar, Ch + c0, x0 - 1, y0 - 1, b);
     }
     // the group's taps, read in address order (each half's 64 x 9 block is
     // contiguous) into [half][tap][channel]; zeros past the group's channels
-    float* taps = reinterpret_cast<float*>(dsm + DW_TAPS_OFF);
-    for (int e = tid; e < 2 * DW_CH * 9; e += DW_THREADS) {
+    float* taps = reinterpret_cast<float*>(dsm + Cfg::TAPS_OFF);
+    for (int e = tid; e < 2 * DW_CH * 9; e += Cfg::THREADS) {
         const int half = e / (DW_CH * 9), j = e % (DW_CH * 9);
         const int ch = j / 9, t = j % 9;
         taps[(half * 9 + t) * DW_CH + ch] =
@@ -481,47 +503,66 @@ dwconv_glu(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUte
         wa[t] = *reinterpret_cast<const float2*>(taps + t * DW_CH + cp);
         wg[t] = *reinterpret_cast<const float2*>(taps + (9 + t) * DW_CH + cp);
     }
-    constexpr int STRIPS = DW_TX / DW_SX;
-    const int ly = warp / STRIPS;                           // output row y0 + ly = halo row ly + 1
-    const int sx = (warp % STRIPS) * DW_SX;                 // first output column of the strip
-    // halo row ly + r, halo column sx + j holds grid (y0 + ly - 1 + r, x0 + sx - 1 + j)
-    const uint8_t* base = dsm + (size_t)ly * DW_ROW_BYTES + (size_t)sx * (DW_CH * 2) + lane * 4;
-    float2 win[2][3][3];                                    // [half][row][column slot]
-    auto load_col = [&](int j, int slot) {
-#pragma unroll
-        for (int r = 0; r < 3; ++r) {
-            const uint8_t* q = base + r * DW_ROW_BYTES + j * (DW_CH * 2);
-            win[0][r][slot] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q));
-            win[1][r][slot] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q + DW_HALF_BYTES));
-        }
-    };
+    constexpr int STRIPS = TX / SX;
+    const int ly = (warp / STRIPS) * RPW;                   // output rows y0 + ly .. = halo rows ly + 1 ..
+    const int sx = (warp % STRIPS) * SX;                    // first output column of the strip
+    // halo row ly + r, halo column sx + j holds grid (y0 + ly - 1 + r, x0 + sx - 1 + j);
+    // output x of the strip (halo column sx + x + 1) takes halo columns
+    // sx + x .. sx + x + 2 with tap columns dx = 0, 1, 2
+    const uint8_t* base = dsm + (size_t)ly * ROW_BYTES + (size_t)sx * (DW_CH * 2) + lane * 4;
     constexpr float kLog2e = 1.4426950408889634f;
-    uint32_t zo[DW_SX];
-    load_col(0, 0);
-    load_col(1, 1);
+    float2 acc[2][RPW][3];                                  // [half][row][output x % 3]
+    uint32_t zo[RPW][SX];
 #pragma unroll
-    for (int k = 0; k < DW_SX; ++k) {
-        load_col(k + 2, (k + 2) % 3);
-        float2 a = make_float2(0.0f, 0.0f), g = make_float2(0.0f, 0.0f);
+    for (int j = 0; j < SX + 2; ++j) {
+        float2 v[2][RPW + 2];
 #pragma unroll
-        for (int dy = 0; dy < 3; ++dy) {
+        for (int r = 0; r < RPW + 2; ++r) {
+            const uint8_t* q = base + r * ROW_BYTES + j * (DW_CH * 2);
+            v[0][r] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q));
+            v[1][r] = bf16x2_unpack(*reinterpret_cast<const uint32_t*>(q + HALF_BYTES));
+        }
 #pragma unroll
-            for (int dx = 0; dx < 3; ++dx) {
-                a = __ffma2_rn(win[0][dy][(k + dx) % 3], wa[dy * 3 + dx], a);
-                g = __ffma2_rn(win[1][dy][(k + dx) % 3], wg[dy * 3 + dx], g);
+        for (int dx = 0; dx < 3; ++dx) {
+            const int x = j - dx;                           // the output this column feeds with tap column dx
+            if (x < 0 || x >= SX) continue;
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+#pragma unroll
+                for (int dy = 0; dy < 3; ++dy) {
+                    const int t = dy * 3 + dx;
+                    if (dx == 0 && dy == 0) {
+                        acc[0][r][x % 3] = __fmul2_rn(v[0][r], wa[t]);
+                        acc[1][r][x % 3] = __fmul2_rn(v[1][r], wg[t]);
+                    } else {
+                        acc[0][r][x % 3] = __ffma2_rn(v[0][r + dy], wa[t], acc[0][r][x % 3]);
+                        acc[1][r][x % 3] = __ffma2_rn(v[1][r + dy], wg[t], acc[1][r][x % 3]);
+                    }
+                }
             }
         }
-        // sigmoid(g) = 1 / (1 + 2^(-g log2 e))
-        const float2 t = __fmul2_rn(g, make_float2(-kLog2e, -kLog2e));
-        const float2 d = __fadd2_rn(make_float2(ptx::ex2_approx(t.x), ptx::ex2_approx(t.y)), make_float2(1.0f, 1.0f));
-        const float2 z = __fmul2_rn(a, make_float2(ptx::rcp_approx(d.x), ptx::rcp_approx(d.y)));
-        zo[k] = float2_to_bf16x2(z.x, z.y);
+        const int xd = j - 2;                               // the output completed by this column
+        if (xd >= 0) {
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+                const float2 a = acc[0][r][xd % 3], g = acc[1][r][xd % 3];
+                // sigmoid(g) = 1 / (1 + 2^(-g log2 e))
+                const float2 t = __fmul2_rn(g, make_float2(-kLog2e, -kLog2e));
+                const float2 d = __fadd2_rn(make_float2(ptx::ex2_approx(t.x), ptx::ex2_approx(t.y)),
+                                            make_float2(1.0f, 1.0f));
+                const float2 z = __fmul2_rn(a, make_float2(ptx::rcp_approx(d.x), ptx::rcp_approx(d.y)));
+                zo[r][xd] = float2_to_bf16x2(z.x, z.y);
+            }
+        }
     }
     __syncthreads();                                        // every warp is done with the input tile
     // output tile [row][column][64 channels] over the value half
-    uint8_t* zt = dsm + ((size_t)ly * DW_TX + sx) * (DW_CH * 2) + lane * 4;
 #pragma unroll
-    for (int k = 0; k < DW_SX; ++k) *reinterpret_cast<uint32_t*>(zt + k * (DW_CH * 2)) = zo[k];
+    for (int r = 0; r < RPW; ++r) {
+        uint8_t* zt = dsm + ((size_t)(ly + r) * TX + sx) * (DW_CH * 2) + lane * 4;
+#pragma unroll
+        for (int x = 0; x < SX; ++x) *reinterpret_cast<uint32_t*>(zt + x * (DW_CH * 2)) = zo[r][x];
+    }
     ptx::fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {

@@ -1077,10 +1077,11 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
     // 1x1 expand: U = X W1^T (2 Ch channels)
     if ((st = launch_gemm(X, W1, U, M, 2 * Ch, C, 2 * Ch, s)) != SANA_LA_OK) return st;
     // 3x3 depthwise over the grid and the GLU, fused
+    using DwC = sana::tc::DwConfig;
     static std::atomic<unsigned long long> dw_smem_set[kMaxDevicesCached];
-    if ((st = ensure_smem(sana::tc::dwconv_glu, sana::tc::DW_SMEM, dw_smem_set)) != SANA_LA_OK) return st;
-    // U as {2 Ch, Wg, Hg, B}: a load box is 64 channels x (DW_TX + 2) columns x
-    // (DW_TY + 2) rows; Z as {Ch, Wg, Hg, B}: a store box is 64 x DW_TX x DW_TY
+    if ((st = ensure_smem(sana::tc::dwconv_glu<DwC>, DwC::SMEM, dw_smem_set)) != SANA_LA_OK) return st;
+    // U as {2 Ch, Wg, Hg, B}: a load box is 64 channels x (TX + 2) columns x
+    // (TY + 2) rows; Z as {Ch, Wg, Hg, B}: a store box is 64 x TX x TY
     CUtensorMap tmU, tmZ;
     {
         auto encode = tensor_map_encoder();
@@ -1091,8 +1092,8 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
             cuuint64_t dims[4] = {ch, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
             cuuint64_t strides[3] = {ch * 2, ch * 2 * Wg, ch * 2 * Wg * Hg};
             const int halo = which == 0 ? 2 : 0;
-            cuuint32_t box[4] = {(cuuint32_t)sana::tc::DW_CH, (cuuint32_t)(sana::tc::DW_TX + halo),
-                                 (cuuint32_t)(sana::tc::DW_TY + halo), 1};
+            cuuint32_t box[4] = {(cuuint32_t)sana::tc::DW_CH, (cuuint32_t)(DwC::TX + halo),
+                                 (cuuint32_t)(DwC::TY + halo), 1};
             CUresult r = encode(which == 0 ? &tmU : &tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                                 which == 0 ? U : Z, dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1103,10 +1104,10 @@ sana_la_status sana_linattn_mix_ffn(const void* X, const void* W1, const float* 
             }
         }
     }
-    const long long dw_tiles = (long long)B * cdiv(Hg, sana::tc::DW_TY) * cdiv(Wg, sana::tc::DW_TX);
-    if (dw_tiles > 65535) return SANA_LA_ERR_UNSUPPORTED;
-    const dim3 dw_grid((unsigned)cdiv(Ch, sana::tc::DW_CH), (unsigned)dw_tiles);
-    if ((st = launch(sana::tc::dwconv_glu, dw_grid, dim3(sana::tc::DW_THREADS), sana::tc::DW_SMEM, s,
+    const long long dw_ctas = (long long)B * cdiv(Hg, DwC::TY) * cdiv(Wg, DwC::TX) * cdiv(Ch, sana::tc::DW_CH);
+    if (dw_ctas > 0x7fffffffLL) return SANA_LA_ERR_UNSUPPORTED;
+    const dim3 dw_grid((unsigned)dw_ctas);
+    if ((st = launch(sana::tc::dwconv_glu<DwC>, dw_grid, dim3(DwC::THREADS), DwC::SMEM, s,
                      false, "dwconv_glu", tmU, tmZ, Kdw, Hg, Wg, Ch)) != SANA_LA_OK)
         return st;
     // 1x1 project: Y = Z W2^T
