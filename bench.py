@@ -389,6 +389,31 @@ def run_ours(args):
 
     fp32 = None if L else run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl)
 
+    # block-causal: the one-launch form (bit-identical), timed the same way
+    single = None
+    if L:
+        def single_step():
+            ops.block_causal_forward(Q, K, V, L, out_dtype=torch.bfloat16, eps=w.eps, out=out, workspace=ws,
+                                     single_launch=True)
+        n_single = min(args.steps, 200)
+        for _ in range(args.warmup):
+            single_step()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_single + 1)]
+        torch.cuda.synchronize(dev)
+        ev[0].record(stream)
+        for k in range(n_single):
+            single_step()
+            ev[k + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        per = [ev[k].elapsed_time(ev[k + 1]) for k in range(n_single)]
+        s_ms = ev[0].elapsed_time(ev[-1]) / n_single
+        s_gbs = bytes_per_step / (s_ms / 1e3) / 1e9
+        single = {"ms_per_step": s_ms, "ms_per_step_median": statistics.median(per), "ms_per_step_min": min(per),
+                  "value": s_gbs, "unit": UNIT, "frac": s_gbs / hbm_peak, "steps": n_single,
+                  "kernel": "fwd_fused_tc (block-causal instance)",
+                  "gpu_launches": ops.block_causal_forward_launches(B, N, H, d, L, single_launch=True) * n_single,
+                  "call": "block_causal_forward_single"}
+
     e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, world)
 
     cpu = None
@@ -417,6 +442,8 @@ def run_ours(args):
             "roofline": roof, "fp32_out": fp32, "e2e": e2e, "clocks": clk,
             "gpu_launches": launches * args.steps,
         }
+        if single is not None:
+            line["single_launch"] = single
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

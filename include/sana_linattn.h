@@ -301,6 +301,28 @@ sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, c
 int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L);
 
 /*
+ * The same forward in one cooperative launch: the state phase writes the
+ * per-block partial states; each CTA of the apply phase, once the CTAs of its
+ * slab have raised their readiness flags, adds the partials of every block up
+ * to the one it applies onto a running prefix (kept between its segments in
+ * the workspace), with the prefix reduction's additions in its order. Same
+ * arguments, workspace and errors as sana_linattn_block_causal_forward, and
+ * bit-identical to it. If the device cannot hold the whole grid at once, the
+ * three kernels run instead. (Measured on B200 it is not faster: 145 against
+ * 141 us for 16 frames of 4,096 tokens, 1.73 against 1.59 ms for 16 frames of
+ * 65,536, 36 heads of 32; its CTAs re-add every earlier block's partials where
+ * the prefix reduction does that once.)
+ */
+sana_la_status sana_linattn_block_causal_forward_single(const void* Q, const void* K, const void* V,
+                                                        int B, int N, int H, int d, int L,
+                                                        void* O, sana_la_out_dtype out_dtype, float eps,
+                                                        void* workspace, size_t workspace_bytes,
+                                                        sana_la_stream_t stream);
+
+/* Kernel launches one sana_linattn_block_causal_forward_single call enqueues (0 if invalid). */
+int sana_linattn_block_causal_forward_single_launches(int B, int N, int H, int d, int L);
+
+/*
  * sana_linattn_block_causal_forward from and to HOST memory, with the copies
  * overlapped by the library as in sana_linattn_forward_host (below): K and V
  * are copied in and the prefix states computed over all blocks; then Q is

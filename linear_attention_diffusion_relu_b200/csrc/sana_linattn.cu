@@ -98,6 +98,7 @@ struct Plan {
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
     size_t state_bytes;     // fp32 (B, H, d, d+1); block-causal (B, H, nblk, d, d+1)
+    size_t carry_bytes;     // block-causal single launch: one group's state per CTA
     size_t flag_bytes;      // readiness flags of the single-launch forward (one per CTA)
 };
 
@@ -201,6 +202,7 @@ Plan make_plan(int B, int N, int H, int d, int L = 0, int sms = device_sms()) {
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * nblk * dd);
     p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
+    p.carry_bytes = L > 0 ? align256((size_t)std::max(p.ks.q.grid, p.ka.q.grid) * G * dd) : 0;
     return p;
 }
 
@@ -427,10 +429,10 @@ int blocks_per_sm(Kernel kernel, int threads, int smem, std::atomic<int> (&cache
     return v;
 }
 
-template <int D, bool OUT_BF16, int FM>
+template <int D, bool OUT_BF16, int FM, bool BC>
 sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V, void* O, int B, int N,
                                     int H, const Plan& p, float* partial, unsigned long long* flags,
-                                    cudaStream_t s) {
+                                    float* carry, cudaStream_t s) {
     static std::atomic<unsigned long long> smem_set[kMaxDevicesCached];
     static std::atomic<int> per_sm_cache[kMaxDevicesCached];
     CUtensorMap tmK, tmV, tmQ, tmO;
@@ -440,7 +442,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     if ((st = make_tmap(&tmQ, Q, B, N, H, D, sana::tc::KA_TILE)) != SANA_LA_OK) return st;
     if ((st = make_tmap(&tmO, O, B, N, H, D, sana::tc::KA_TILE, !OUT_BF16)) != SANA_LA_OK) return st;
     constexpr int smem = sana::tc::FwdMap<D, OUT_BF16>::BYTES;
-    auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16, FM>;
+    auto kernel = sana::tc::fwd_fused_tc<D, OUT_BF16, FM, BC>;
     if ((st = ensure_smem(kernel, smem, smem_set)) != SANA_LA_OK) return st;
     const int grid = std::max(p.ks.q.grid, p.ka.q.grid);
     int dev = 0, sms = 0;
@@ -484,7 +486,8 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
     // (same process, A/B): 111.9 vs 119.3 us at 4096px (0.44 GB of inputs),
     // 400.7 vs 404.3 us at N = 262,144 and 1598 vs 1608 us at N = 1,048,576.
     const int evict_first = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch, evict_first);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, tmQ, tmO, p.ks, p.ka, partial, flags, epoch, evict_first,
+                           carry);
     if (e != cudaSuccess) {
         set_last_error("fwd_fused_tc", e);
         return SANA_LA_ERR_CUDA;
@@ -527,14 +530,16 @@ sana_la_status apply_impl(const void* Q, const float* state, int B, int N, int H
     return SANA_LA_ERR_INVALID_ARG;
 }
 
-template <int FM>
+// BC: the block-causal instance (running prefix states in `carry`)
+template <int FM, bool BC = false>
 sana_la_status forward_fused_dispatch(const void* Q, const void* K, const void* V, void* O, int B, int N,
                                       int H, int d, bool bf16, const Plan& p, float* partial,
-                                      unsigned long long* flags, cudaStream_t s) {
-    return d == 32 ? (bf16 ? launch_forward_fused<32, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                           : launch_forward_fused<32, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s))
-                   : (bf16 ? launch_forward_fused<64, true, FM>(Q, K, V, O, B, N, H, p, partial, flags, s)
-                           : launch_forward_fused<64, false, FM>(Q, K, V, O, B, N, H, p, partial, flags, s));
+                                      unsigned long long* flags, cudaStream_t s, float* carry = nullptr) {
+    return d == 32
+        ? (bf16 ? launch_forward_fused<32, true, FM, BC>(Q, K, V, O, B, N, H, p, partial, flags, carry, s)
+                : launch_forward_fused<32, false, FM, BC>(Q, K, V, O, B, N, H, p, partial, flags, carry, s))
+        : (bf16 ? launch_forward_fused<64, true, FM, BC>(Q, K, V, O, B, N, H, p, partial, flags, carry, s)
+                : launch_forward_fused<64, false, FM, BC>(Q, K, V, O, B, N, H, p, partial, flags, carry, s));
 }
 
 bool valid_feature(int fm) {
@@ -1119,10 +1124,15 @@ int sana_linattn_mix_ffn_launches(int B, int Hg, int Wg, int C, int Ch) {
 }
 
 // ------------------------------------------------------- block-causal ----
+// Block-causal workspace: the partial states, then either the prefix states
+// (three-kernel form) or the single launch's flags and per-CTA running prefixes.
+size_t block_causal_ws_bytes(const Plan& p) {
+    return p.partial_bytes + std::max(p.state_bytes, p.flag_bytes + p.carry_bytes);
+}
+
 size_t sana_linattn_block_causal_workspace_bytes(int B, int N, int H, int d, int L) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
-    const Plan p = make_plan(B, N, H, d, L);
-    return p.partial_bytes + p.state_bytes;
+    return block_causal_ws_bytes(make_plan(B, N, H, d, L));
 }
 
 sana_la_status sana_linattn_block_causal_kv_state(const void* K, const void* V, int B, int N, int H,
@@ -1155,11 +1165,14 @@ sana_la_status sana_linattn_block_causal_apply(const void* Q, const float* state
                       reinterpret_cast<cudaStream_t>(stream), false);
 }
 
-sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, const void* V,
-                                                 int B, int N, int H, int d, int L,
-                                                 void* O, sana_la_out_dtype out_dtype, float eps,
-                                                 void* workspace, size_t workspace_bytes,
-                                                 sana_la_stream_t stream) {
+// single: one cooperative launch with running prefix states (fwd_fused_tc,
+// block-causal instance); otherwise, and whenever the device cannot hold that
+// grid at once, the state kernel and the prefix reduction, then the apply
+// kernel (programmatic launch). Bit-identical either way.
+static sana_la_status block_causal_forward_entry(const void* Q, const void* K, const void* V, int B, int N,
+                                                 int H, int d, int L, void* O, sana_la_out_dtype out_dtype,
+                                                 float eps, void* workspace, size_t workspace_bytes,
+                                                 sana_la_stream_t stream, bool single) {
     g_last_error[0] = '\0';
     if (!Q || !K || !V || !O || !workspace) return SANA_LA_ERR_INVALID_ARG;
     sana_la_status st = check_sizes(B, N, H, d);
@@ -1169,19 +1182,54 @@ sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, c
     if ((st = check_eps(eps)) != SANA_LA_OK) return st;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return SANA_LA_ERR_INVALID_ARG;
-    const Plan p = make_plan(B, N, H, d, L);
-    if (workspace_bytes < p.partial_bytes + p.state_bytes) return SANA_LA_ERR_WORKSPACE;
-    float* states = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.partial_bytes);
+    Plan p = make_plan(B, N, H, d, L);
+    if (workspace_bytes < block_causal_ws_bytes(p)) return SANA_LA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    float* partial = reinterpret_cast<float*>(ws);
+    float* states = reinterpret_cast<float*>(ws + p.partial_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // state kernel + prefix reduction, then the apply kernel (programmatic launch)
+    if (single) {
+        // flags and per-CTA prefixes where the three-kernel form keeps the
+        // prefix states
+        p.ka.eps = eps;
+        auto* flags = reinterpret_cast<unsigned long long*>(ws + p.partial_bytes);
+        float* carry = reinterpret_cast<float*>(ws + p.partial_bytes + p.flag_bytes);
+        st = forward_fused_dispatch<sana::kFeatureRelu, true>(Q, K, V, O, B, N, H, d,
+                                                              out_dtype == SANA_LA_OUT_BF16, p, partial, flags, s,
+                                                              carry);
+        if (st != SANA_LA_ERR_UNSUPPORTED) return st;
+    }
     st = kv_state_impl(K, V, B, N, H, d, L, states, workspace, workspace_bytes, s, true);
     if (st != SANA_LA_OK) return st;
     return apply_impl(Q, states, B, N, H, d, L, O, out_dtype, eps, s, true);
 }
 
+sana_la_status sana_linattn_block_causal_forward(const void* Q, const void* K, const void* V,
+                                                 int B, int N, int H, int d, int L,
+                                                 void* O, sana_la_out_dtype out_dtype, float eps,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 sana_la_stream_t stream) {
+    return block_causal_forward_entry(Q, K, V, B, N, H, d, L, O, out_dtype, eps, workspace, workspace_bytes,
+                                      stream, false);
+}
+
 int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L) {
     if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
-    return 3;   // ks_state_tc, kr_reduce_tc (prefix states), ka_apply_tc
+    return 3;   // ks_state_tc, kr_prefix_tc (prefix states), ka_apply_tc
+}
+
+sana_la_status sana_linattn_block_causal_forward_single(const void* Q, const void* K, const void* V,
+                                                        int B, int N, int H, int d, int L,
+                                                        void* O, sana_la_out_dtype out_dtype, float eps,
+                                                        void* workspace, size_t workspace_bytes,
+                                                        sana_la_stream_t stream) {
+    return block_causal_forward_entry(Q, K, V, B, N, H, d, L, O, out_dtype, eps, workspace, workspace_bytes,
+                                      stream, true);
+}
+
+int sana_linattn_block_causal_forward_single_launches(int B, int N, int H, int d, int L) {
+    if (check_sizes(B, N, H, d) != SANA_LA_OK || check_block(B, N, H, d, L) != SANA_LA_OK) return 0;
+    return 1;   // fwd_fused_tc (plus a memset of its barrier flags when captured in a graph)
 }
 
 size_t sana_linattn_block_causal_forward_host_workspace_bytes(int B, int N, int H, int d, int L,

@@ -673,6 +673,7 @@ struct KaStateSrc {
     KsParams ks;
     const unsigned long long* flags;   // one arrival flag per CTA of the grid
     unsigned long long epoch;          // unique to this launch (set by the host)
+    float* carry;                      // block-causal: one state-sized scratch per CTA
 };
 
 // Readiness flags of the single-launch forward. CTA c announces that all its
@@ -692,7 +693,7 @@ __device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned l
 // `prev_empty`/`prev_tiles` (single launch): the state phase's stage barriers
 // and how many tiles it loaded; Q stage s (< 6) reuses its stage s, so the
 // first load into each waits until the state phase released that stage.
-template <int D, bool OUT_BF16, int FM>
+template <int D, bool OUT_BF16, int FM, bool BC = false>
 __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorMap* tmO, const KaParams& p,
                                          int cta, const KaStateSrc& src, uint8_t* smem,
                                          const KaBars<D, OUT_BF16>& bar, uint32_t tmem,
@@ -801,16 +802,55 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         // do not depend on it, the state does.
         if (src.state != nullptr) ptx::wait_prerequisite_grid();
 
+        // Chunks of four entries of one column (rows k0 .. k0 + 3 of column n
+        // of head hh): chunk c of the group is the c-th float4 of the heads'
+        // partial states (stored by columns); this thread takes chunks tid,
+        // tid + 256, ...
+        constexpr int NC = G * DD / 4;
+        constexpr int NCT = (NC + kWorkerThreads - 1) / kWorkerThreads;
+        // single launch, block-causal: the slab this CTA staged last and its
+        // last block; the running prefix itself waits in src.carry between
+        // segments (registers would have to hold it through the apply loop)
+        int carry_slab = -1, carry_blk = -1;
+        // single launch: wait (bounded) until the flags of CTAs slab % P + r P,
+        // r in [r0, r0 + k), hold this launch's epoch; k = 0: wait for none.
+        // Returns the length of the ready prefix (at least 1 if any remain),
+        // or -1 if the wait gave up.
+        auto ready_prefix = [&](int slab, int r, bool all) -> int {
+            const unsigned long long* fl = src.flags + slab % src.ks.q.P;
+            const int R = src.ks.q.R;
+            const uint64_t t0 = ptx::globaltimer_ns();
+            for (;;) {
+                bool ready = true;
+                if (r + lane < R) {
+                    unsigned long long f;
+                    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
+                                 : "=l"(f) : "l"(fl + (long long)(r + lane) * src.ks.q.P) : "memory");
+                    ready = f == src.epoch;
+                }
+                const unsigned waiting = __ballot_sync(0xffffffffu, !ready);
+                const int k = min(waiting ? __ffs(waiting) - 1 : 32, R - r);   // ready prefix from r
+                if (k > 0 && (!all || k == min(32, R - r))) {
+                    __syncwarp();          // every lane's reads after every lane's flag
+                    return k;
+                }
+                bool give_up = *abort != 0;
+                if (!give_up && ptx::globaltimer_ns() - t0 > 2000000000ull) {
+                    if (lane == 0) {
+                        atomicCAS(err, ptx::kErrNone, ptx::kErrWaitTimeout);
+                        *abort = 1;
+                    }
+                    give_up = true;
+                }
+                if (__any_sync(0xffffffffu, give_up)) return -1;
+                __nanosleep(64);
+            }
+        };
+
         // stage the state of `slab` in shared memory as bf16 hi + lo parts
         auto stage_state = [&](int slab, int blk) -> bool {
             const int b = slab / p.groups;
             const int g = slab % p.groups;
-            // Chunks of four entries of one column (rows k0 .. k0 + 3 of column
-            // n of head hh): chunk c of the group is the c-th float4 of the
-            // heads' partial states (stored by columns); this thread takes
-            // chunks tid, tid + 256, ...
-            constexpr int NC = G * DD / 4;
-            constexpr int NCT = (NC + kWorkerThreads - 1) / kWorkerThreads;
             float4 v[NCT];
 #pragma unroll
             for (int j = 0; j < NCT; ++j) v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -829,6 +869,106 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                         v[j] = make_float4(st[(k0 + 0) * (D + 1)], st[(k0 + 1) * (D + 1)],
                                            st[(k0 + 2) * (D + 1)], st[(k0 + 3) * (D + 1)]);
                     }
+                }
+            } else if constexpr (BC) {
+                // Block-causal: the inclusive prefix over the slab's blocks
+                // 0 .. blk, carried on from this CTA's previous segment of the
+                // slab, with the additions of kr_prefix_tc in its order: each
+                // block's partials summed in ascending order, then that sum
+                // added to the running prefix. The partials of every block
+                // come from the slab's R CTAs, so all their flags are waited for.
+                float4* cs = reinterpret_cast<float4*>(src.carry) + (long long)cta * NC;   // this CTA's prefix
+                if (slab != carry_slab) {
+                    for (int r = 0; r < src.ks.q.R; r += 32)
+                        if (ready_prefix(slab, r, true) < 0) return false;
+                    carry_slab = slab;
+                    carry_blk = -1;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NCT; ++j) {
+                        const int c = tid + j * kWorkerThreads;
+                        if (c < NC) v[j] = __ldcg(cs + c);      // written by this thread
+                    }
+                }
+                // the partials of blocks carry_blk + 1 .. blk, nr per block, in
+                // that order; d = 32: four loads in flight at a time (d = 64
+                // one block's at a time: registers)
+                const long long kstep = ks_block_step(G, src.ks) * DD;
+                const int nr = src.ks.q.R / src.ks.q.rb;
+                float4 bs[NCT];
+                if constexpr (D == 32) {
+                    constexpr int RB = 4;
+                    const int total = (blk - carry_blk) * nr;
+                    for (int q0 = 0; q0 < total; q0 += RB) {
+                        float4 t[RB][NCT];
+#pragma unroll
+                        for (int u = 0; u < RB; ++u) {
+                            const int q = q0 + u;
+                            const float* base = q < total
+                                ? src.partial + ks_block_slot(slab, carry_blk + 1 + q / nr, 0, G, src.ks) * DD
+                                              + (q % nr) * kstep
+                                : nullptr;
+#pragma unroll
+                            for (int j = 0; j < NCT; ++j) {
+                                const int c = tid + j * kWorkerThreads;
+                                t[u][j] = (c < NC && q < total) ? __ldcg(reinterpret_cast<const float4*>(base) + c)
+                                                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < RB; ++u) {
+                            const int q = q0 + u;
+                            if (q < total) {
+                                const int tt = q % nr;
+#pragma unroll
+                                for (int j = 0; j < NCT; ++j) {
+                                    if (tt == 0) bs[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                                    bs[j].x += t[u][j].x;
+                                    bs[j].y += t[u][j].y;
+                                    bs[j].z += t[u][j].z;
+                                    bs[j].w += t[u][j].w;
+                                    if (tt == nr - 1) {
+                                        v[j].x += bs[j].x;
+                                        v[j].y += bs[j].y;
+                                        v[j].z += bs[j].z;
+                                        v[j].w += bs[j].w;
+                                    }
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    for (int jb = carry_blk + 1; jb <= blk; ++jb) {
+                        const float* base = src.partial + ks_block_slot(slab, jb, 0, G, src.ks) * DD;
+#pragma unroll
+                        for (int j = 0; j < NCT; ++j) bs[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        for (int t = 0; t < nr; ++t) {
+#pragma unroll
+                            for (int j = 0; j < NCT; ++j) {
+                                const int c = tid + j * kWorkerThreads;
+                                if (c < NC) {
+                                    const float4 x = __ldcg(reinterpret_cast<const float4*>(base + t * kstep) + c);
+                                    bs[j].x += x.x;
+                                    bs[j].y += x.y;
+                                    bs[j].z += x.z;
+                                    bs[j].w += x.w;
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < NCT; ++j) {
+                            v[j].x += bs[j].x;
+                            v[j].y += bs[j].y;
+                            v[j].z += bs[j].z;
+                            v[j].w += bs[j].w;
+                        }
+                    }
+                }
+                carry_blk = blk;
+#pragma unroll
+                for (int j = 0; j < NCT; ++j) {
+                    const int c = tid + j * kWorkerThreads;
+                    if (c < NC) __stcg(cs + c, v[j]);
                 }
             } else {
                 // The same additions, in the same order, as kr_reduce_tc: the R
@@ -1142,7 +1282,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull};
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, nullptr};
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
                           &g_device_error);
     kernel_epilogue(ctl, tid);
@@ -1151,23 +1291,28 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 // The whole forward in one cooperative launch (all CTAs resident, so a CTA
 // may wait for another): the state phase; a readiness flag per CTA; then the
 // apply phase, which waits (bounded) for the flags of the CTAs that wrote its
-// slab's partial states and sums them itself in the reduction kernel's order.
+// slab's partial states and sums them itself in the reduction kernel's order
+// (BC, block-causal: the prefix kernel's, carried from block to block in
+// `carry`, one state-sized scratch per CTA; a separate instance, so that the
+// plain forward's code is not touched by it).
 // The apply phase's Q loads start as soon as the state phase has released its
 // shared memory, so they overlap that wait. `flags` has one slot per CTA;
 // `epoch` is unique to the launch.
-template <int D, bool OUT_BF16, int FM>
+template <int D, bool OUT_BF16, int FM, bool BC>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
              const KsParams ks, const KaParams ka, float* __restrict__ partial,
-             unsigned long long* flags, const unsigned long long epoch, const int evict_first)
+             unsigned long long* flags, const unsigned long long epoch, const int evict_first,
+             float* __restrict__ carry)
 {
     using Map = FwdMap<D, OUT_BF16>;
-    // the apply phase here sums one block's partials; prefix states over token
-    // blocks take the three-kernel path
-    if (ks.q.nblk != 1 || ka.q.nblk != 1) {
-        if (threadIdx.x == 0) atomicCAS(&g_device_error, ptx::kErrNone, ptx::kErrUnsupported);
-        return;
+    if constexpr (!BC) {
+        // prefix states over token blocks take the BC instance
+        if (ks.q.nblk != 1 || ka.q.nblk != 1) {
+            if (threadIdx.x == 0) atomicCAS(&g_device_error, ptx::kErrNone, ptx::kErrUnsupported);
+            return;
+        }
     }
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -1214,10 +1359,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
         ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     }
-    KaStateSrc src{nullptr, partial, ks, flags, epoch};
+    KaStateSrc src{nullptr, partial, ks, flags, epoch, carry};
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
-    ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
+    ka_phase<D, OUT_BF16, FM, BC>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
                           kbar.empty, ks_tiles, evict_first != 0);
     kernel_epilogue(ctl, tid);
 }

@@ -32,7 +32,8 @@ and the block-causal form (blocks of L tokens, L a multiple of 128):
     block_causal_workspace_bytes(B, N, H, d, L)
     block_causal_kv_state(K, V, L, states=None, workspace=None) -> (B, H, nblk, d, d+1) fp32
     block_causal_apply(Q, states, L, out_dtype=..., eps=..., out=None) -> O
-    block_causal_forward(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None) -> O
+    block_causal_forward(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None,
+                         single_launch=False) -> O
     block_causal_forward_host(Q, K, V, L, out_dtype=..., eps=..., out=None, workspace=None) -> O (CPU)
 """
 from __future__ import annotations
@@ -70,6 +71,8 @@ SYMBOLS = (
     "sana_linattn_block_causal_apply",
     "sana_linattn_block_causal_forward",
     "sana_linattn_block_causal_forward_launches",
+    "sana_linattn_block_causal_forward_single",
+    "sana_linattn_block_causal_forward_single_launches",
     "sana_linattn_block_causal_forward_host_workspace_bytes",
     "sana_linattn_block_causal_forward_host",
     "sana_linattn_block_causal_forward_host_launches",
@@ -157,6 +160,10 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
         lib.sana_linattn_block_causal_forward.restype = st
         lib.sana_linattn_block_causal_forward_launches.argtypes = [i, i, i, i, i]
         lib.sana_linattn_block_causal_forward_launches.restype = ctypes.c_int
+        lib.sana_linattn_block_causal_forward_single.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
+        lib.sana_linattn_block_causal_forward_single.restype = st
+        lib.sana_linattn_block_causal_forward_single_launches.argtypes = [i, i, i, i, i]
+        lib.sana_linattn_block_causal_forward_single_launches.restype = ctypes.c_int
         lib.sana_linattn_block_causal_forward_host_workspace_bytes.argtypes = [i, i, i, i, i, i]
         lib.sana_linattn_block_causal_forward_host_workspace_bytes.restype = sz
         lib.sana_linattn_block_causal_forward_host.argtypes = [vp, vp, vp, i, i, i, i, i, vp, i, f, vp, sz, vp]
@@ -394,8 +401,11 @@ def block_causal_workspace_bytes(B: int, N: int, H: int, d: int, L: int) -> int:
     return int(load_library().sana_linattn_block_causal_workspace_bytes(B, N, H, d, L))
 
 
-def block_causal_forward_launches(B: int, N: int, H: int, d: int, L: int) -> int:
-    return int(load_library().sana_linattn_block_causal_forward_launches(B, N, H, d, L))
+def block_causal_forward_launches(B: int, N: int, H: int, d: int, L: int, single_launch: bool = False) -> int:
+    lib = load_library()
+    if single_launch:
+        return int(lib.sana_linattn_block_causal_forward_single_launches(B, N, H, d, L))
+    return int(lib.sana_linattn_block_causal_forward_launches(B, N, H, d, L))
 
 
 def make_block_causal_workspace(B: int, N: int, H: int, d: int, L: int, device="cuda") -> torch.Tensor:
@@ -449,8 +459,9 @@ def block_causal_apply(Q: torch.Tensor, states: torch.Tensor, L: int, out_dtype=
 
 def block_causal_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: int,
                          out_dtype=torch.bfloat16, eps: float = 1e-15, out: torch.Tensor | None = None,
-                         workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Whole block-causal forward; bit-identical to block_causal_kv_state + block_causal_apply."""
+                         workspace: torch.Tensor | None = None, single_launch: bool = False) -> torch.Tensor:
+    """Whole block-causal forward; bit-identical to block_causal_kv_state + block_causal_apply.
+    single_launch: the one-launch form (sana_linattn_block_causal_forward_single)."""
     _check_bnhd("Q", Q)
     _check_bnhd("K", K, Q.shape)
     _check_bnhd("V", V, Q.shape)
@@ -460,12 +471,11 @@ def block_causal_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L: i
     if workspace is None:
         workspace = make_block_causal_workspace(B, N, H, d, L, Q.device)
     lib = load_library()
-    st = lib.sana_linattn_block_causal_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d,
-                                               int(L), out.data_ptr(), code, float(eps),
-                                               workspace.data_ptr(),
-                                               workspace.numel() * workspace.element_size(),
-                                               _stream(Q.device))
-    _check(lib, st, "sana_linattn_block_causal_forward")
+    name = "sana_linattn_block_causal_forward" + ("_single" if single_launch else "")
+    st = getattr(lib, name)(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, N, H, d, int(L), out.data_ptr(), code,
+                            float(eps), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            _stream(Q.device))
+    _check(lib, st, name)
     return out
 
 

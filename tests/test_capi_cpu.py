@@ -129,6 +129,8 @@ def test_block_causal_host_checks(lib):
     assert wsb(1, 1 << 24, 36, 32, 65536) > 0
     n = lib.sana_linattn_block_causal_forward_launches
     assert n(2, 3572, 6, 32, 1024) == 3 and n(2, 3572, 6, 32, 96) == 0
+    n1 = lib.sana_linattn_block_causal_forward_single_launches
+    assert n1(2, 3572, 6, 32, 1024) == 1 and n1(2, 3572, 6, 32, 96) == 0
     f = lib.sana_linattn_block_causal_forward
     ws = wsb(1, 1024, 2, 32, 256)
     assert f(FAKE, FAKE, FAKE, 1, 1024, 2, 32, 100, FAKE, 1, 1e-15, FAKE, ws, None) == ops.ERR_UNSUPPORTED

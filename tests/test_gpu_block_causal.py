@@ -6,9 +6,11 @@ Blocks of L tokens; a query of block j uses the prefix state of blocks 0 .. j.
 Small and mid-size shapes compare every output element (ragged last blocks,
 L >= N, more slabs than SMs, head size 64, block lengths whose tile counts
 force few CTAs per slab); the 16-frame video shape compares sampled heads and
-rows, including the first and last token of every block. Also: the prefix
-states themselves, forward == kv_state + apply bit for bit, determinism, and
-that later blocks never reach earlier outputs."""
+rows, including the first and last token of every block. The one-launch form
+(running prefix states in the apply phase) is checked bit for bit against the
+three-kernel forward at every shape. Also: the prefix states themselves,
+forward == kv_state + apply bit for bit, determinism, and that later blocks
+never reach earlier outputs."""
 import numpy as np
 import pytest
 import torch
@@ -60,9 +62,12 @@ def test_block_causal_every_element(oracle, shape, dtype):
     B, N, H, d, L = shape
     Q, K, V = make_inputs(Workload("bc", B, N, H, d, seed=200 + N + L), device="cuda")
     O = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype)
+    O1 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype, single_launch=True)
     torch.cuda.synchronize()
     ref = oracle.block_causal_forward(to_f64(Q), to_f64(K), to_f64(V), L, 1e-15)
     check_output(O, ref, f"block-causal {shape}")
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(O1.view(bits), O.view(bits)), "single launch differs from the three kernels"
     assert ops.device_error() == 0
 
 
@@ -88,9 +93,13 @@ def test_block_causal_forward_equals_two_calls_and_is_deterministic(shape):
         O1 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype)
         O2 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype)
         O3 = ops.block_causal_apply(Q, ops.block_causal_kv_state(K, V, L), L, out_dtype=dtype)
+        O4 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype, single_launch=True)
+        O5 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype, single_launch=True)
         torch.cuda.synchronize()
         assert torch.equal(O1.view(bits), O2.view(bits))
         assert torch.equal(O1.view(bits), O3.view(bits))
+        assert torch.equal(O1.view(bits), O4.view(bits))
+        assert torch.equal(O4.view(bits), O5.view(bits))
 
 
 def test_block_causal_later_blocks_never_reach_earlier_outputs():
@@ -121,9 +130,10 @@ def test_video16f_1024px_every_element(oracle):
     Q, K, V = make_inputs(w, device="cuda")
     ref = oracle.block_causal_forward(to_f64(Q), to_f64(K), to_f64(V), w.block, w.eps)
     for dtype in OUT_DTYPES:
-        O = ops.block_causal_forward(Q, K, V, w.block, out_dtype=dtype, eps=w.eps)
-        torch.cuda.synchronize()
-        check_output(O, ref, f"{w.name} {_dt(dtype)}")
+        for single in (False, True):
+            O = ops.block_causal_forward(Q, K, V, w.block, out_dtype=dtype, eps=w.eps, single_launch=single)
+            torch.cuda.synchronize()
+            check_output(O, ref, f"{w.name} {_dt(dtype)}" + (" single launch" if single else ""))
 
 
 def test_video16f_4096px_sampled_heads_and_rows(oracle):
@@ -142,7 +152,11 @@ def test_video16f_4096px_sampled_heads_and_rows(oracle):
     Qh = head_slice(Q, heads)
     for dtype in OUT_DTYPES:
         O = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype, eps=w.eps)
+        O1 = ops.block_causal_forward(Q, K, V, L, out_dtype=dtype, eps=w.eps, single_launch=True)
         torch.cuda.synchronize()
+        bits = torch.int32 if dtype == torch.float32 else torch.int16
+        assert torch.equal(O1.view(bits), O.view(bits)), "single launch differs from the three kernels"
+        del O1
         got = O[:, :, heads, :]
         for j in range(w.N // L):
             sel = rows[(rows >= j * L) & (rows < (j + 1) * L)]
