@@ -321,22 +321,20 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
     start.record(stream)
     for k in range(args.steps):
         step()
-        if k < args.steps - 1:
-            marks[k].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-
     ms = start.elapsed_time(end) / args.steps
-    bounds = [start, *marks, end]
-    per_step = [bounds[k].elapsed_time(bounds[k + 1]) for k in range(args.steps)]
     ms_max = max_over_ranks(ms, dev)
+    # the per-step distribution from a second loop with an event between
+    # steps (an event record between two launches adds ~2 us at the small
+    # shapes, so the timed region above has none)
+    per_step = per_step_times(step, stream, min(args.steps, 1000))
     bytes_per_step = w.algorithmic_bytes(2)
     value = aggregate_gbs(bytes_per_step, world, ms_max / 1e3)
     mtok = B * N * world / (ms_max / 1e3) / 1e6
@@ -384,7 +382,8 @@ def run_ours(args):
         roof["ms_per_launch_min"] = min(per_step)
     roof["split_api_ms"] = {"kv_state(KS+KR)": ks_ms, "apply(KA)": ka_ms}
     roof["timing"] = ("launch duration: CUDA events over the timed region / steps (one launch per "
-                      "step); split_api_ms: events around kv_state and apply in a "
+                      "step); median and min: per-step events in a second loop of "
+                      f"{min(args.steps, 1000)} steps; split_api_ms: events around kv_state and apply in a "
                       f"{n_split}-step loop of the two-call API after the timed region")
 
     fp32 = None if L else run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl)
@@ -453,10 +452,23 @@ def run_ours(args):
     return 0
 
 
+def per_step_times(step, stream, n):
+    """Milliseconds of each of n consecutive calls of step(), from an event
+    recorded between every two steps on `stream`."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    ev[0].record(stream)
+    for k in range(n):
+        step()
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize()
+    return [ev[k].elapsed_time(ev[k + 1]) for k in range(n)]
+
+
 def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl):
     """The same forward with O in fp32 (the output type the 1e-4 per-row
     tolerance is stated for): its own timed loop after the main one, the same
-    step count and per-step events, algorithmic bytes with 4-byte outputs."""
+    step count, algorithmic bytes with 4-byte outputs."""
     import torch
     from linear_attention_diffusion_relu_b200 import ops
     out32 = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.float32, device=dev)
@@ -467,15 +479,15 @@ def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, i
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    ev[0].record(stream)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
     for k in range(args.steps):
         step()
-        ev[k + 1].record(stream)
+    b.record(stream)
     torch.cuda.synchronize(dev)
-    per_step = [ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)]
-    ms = ev[0].elapsed_time(ev[-1]) / args.steps
+    ms = a.elapsed_time(b) / args.steps
     ms_max = max_over_ranks(ms, dev)
+    per_step = per_step_times(step, stream, min(args.steps, 1000))
     nbytes = w.algorithmic_bytes(4)
     achieved = nbytes / (ms / 1e3) / 1e9
     return {
