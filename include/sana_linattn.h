@@ -308,10 +308,10 @@ int sana_linattn_block_causal_forward_launches(int B, int N, int H, int d, int L
  * the workspace), with the prefix reduction's additions in its order. Same
  * arguments, workspace and errors as sana_linattn_block_causal_forward, and
  * bit-identical to it. If the device cannot hold the whole grid at once, the
- * three kernels run instead. (Measured on B200 it is not faster: 145 against
- * 141 us for 16 frames of 4,096 tokens, 1.73 against 1.59 ms for 16 frames of
- * 65,536, 36 heads of 32; its CTAs re-add every earlier block's partials where
- * the prefix reduction does that once.)
+ * three kernels run instead. (Measured on B200 it is not faster: 143 against
+ * 133 us for 16 frames of 4,096 tokens, 1.79 against 1.67 ms for 16 frames of
+ * 65,536, 36 heads of 32: each CTA adds every earlier block's (shared) block
+ * sum itself, where the prefix reduction forms each prefix once.)
  */
 sana_la_status sana_linattn_block_causal_forward_single(const void* Q, const void* K, const void* V,
                                                         int B, int N, int H, int d, int L,

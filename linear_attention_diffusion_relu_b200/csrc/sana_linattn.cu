@@ -98,7 +98,7 @@ struct Plan {
     sana::tc::KaParams ka;
     size_t partial_bytes;   // fp32 partial states, one per (CTA segment, head)
     size_t state_bytes;     // fp32 (B, H, d, d+1); block-causal (B, H, nblk, d, d+1)
-    size_t carry_bytes;     // block-causal single launch: one group's state per CTA
+    size_t carry_bytes;     // block-causal single launch: one group's state per CTA and per slab block
     size_t flag_bytes;      // readiness flags of the single-launch forward (one per CTA)
 };
 
@@ -201,8 +201,12 @@ Plan make_plan(int B, int N, int H, int d, int L = 0, int sms = device_sms()) {
     const size_t dd = (size_t)d * (d + 1) * sizeof(float);
     p.partial_bytes = align256((size_t)p.ks.q.grid * p.ks.q.max_seg * G * dd);
     p.state_bytes = align256((size_t)B * H * nblk * dd);
-    p.flag_bytes = align256(sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
-    p.carry_bytes = L > 0 ? align256((size_t)std::max(p.ks.q.grid, p.ka.q.grid) * G * dd) : 0;
+    // two flags per CTA (partial states written; block-causal one-launch form:
+    // its block sums written)
+    p.flag_bytes = align256(2 * sizeof(unsigned long long) * (size_t)std::max(p.ks.q.grid, p.ka.q.grid));
+    // block-causal one-launch form: one running prefix per CTA, then one block
+    // sum per slab and block
+    p.carry_bytes = L > 0 ? align256(((size_t)std::max(p.ks.q.grid, p.ka.q.grid) + (size_t)S * nblk) * G * dd) : 0;
     return p;
 }
 
@@ -466,7 +470,7 @@ sana_la_status launch_forward_fused(const void* Q, const void* K, const void* V,
         return SANA_LA_ERR_CUDA;
     }
     if (capture != cudaStreamCaptureStatusNone) {
-        e = cudaMemsetAsync(flags, 0, sizeof(unsigned long long) * (size_t)grid, s);
+        e = cudaMemsetAsync(flags, 0, 2 * sizeof(unsigned long long) * (size_t)grid, s);
         if (e != cudaSuccess) {
             set_last_error("cudaMemsetAsync(grid barrier flags)", e);
             return SANA_LA_ERR_CUDA;

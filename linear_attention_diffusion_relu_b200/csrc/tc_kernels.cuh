@@ -620,6 +620,7 @@ struct KaBars {
     uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
     uint64_t* mma_done;
     uint64_t* p1_written;  // (single launch) this CTA's partial states are written
+    uint64_t* bs_done;     // (block-causal single launch) this CTA's block sums are written
     __device__ void init() const {
         for (int s = 0; s < L::STAGES; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -636,6 +637,7 @@ struct KaBars {
         }
         ptx::mbar_init(mma_done, 1);
         ptx::mbar_init(p1_written, 4);
+        ptx::mbar_init(bs_done, kWorkerWarps);
     }
 };
 
@@ -643,7 +645,7 @@ template <int D, bool OUT_BF16>
 __device__ __forceinline__ KaBars<D, OUT_BF16> ka_bars(uint64_t* b) {
     constexpr int S = KaLayout<D, OUT_BF16>::STAGES;
     uint64_t* a = b + 2 * S;
-    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11};
+    return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 12};
 }
 
 // zero the padding columns n in (d, NA) of the staged state
@@ -674,6 +676,8 @@ struct KaStateSrc {
     const unsigned long long* flags;   // one arrival flag per CTA of the grid
     unsigned long long epoch;          // unique to this launch (set by the host)
     float* carry;                      // block-causal: one state-sized scratch per CTA
+    float* bsums;                      // block-causal, R > 1: the slabs' block sums (one state each)
+    unsigned long long* flags2;        // block-causal, R > 1: a CTA's block sums are stored
 };
 
 // Readiness flags of the single-launch forward. CTA c announces that all its
@@ -816,8 +820,8 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
         // r in [r0, r0 + k), hold this launch's epoch; k = 0: wait for none.
         // Returns the length of the ready prefix (at least 1 if any remain),
         // or -1 if the wait gave up.
-        auto ready_prefix = [&](int slab, int r, bool all) -> int {
-            const unsigned long long* fl = src.flags + slab % src.ks.q.P;
+        auto ready_prefix = [&](const unsigned long long* flags, int slab, int r, bool all) -> int {
+            const unsigned long long* fl = flags + slab % src.ks.q.P;
             const int R = src.ks.q.R;
             const uint64_t t0 = ptx::globaltimer_ns();
             for (;;) {
@@ -877,10 +881,57 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                 // block's partials summed in ascending order, then that sum
                 // added to the running prefix. The partials of every block
                 // come from the slab's R CTAs, so all their flags are waited for.
+                // With several partials per block (nr > 1), the slab's R CTAs
+                // share the block sums: CTA r of the slab sums the partials of
+                // blocks r, r + R, ... once (ascending, from zero) into
+                // src.bsums and raises its second flag; each CTA then adds
+                // block sums instead of partials.
                 float4* cs = reinterpret_cast<float4*>(src.carry) + (long long)cta * NC;   // this CTA's prefix
+                const long long kstep = ks_block_step(G, src.ks) * DD;
+                const int R = src.ks.q.R;
+                const int P = src.ks.q.P;
+                const int nr = R / src.ks.q.rb;
+                const bool shared = nr > 1;                 // (then R > 1: one slab per CTA)
+                float4* bsum = shared ? reinterpret_cast<float4*>(src.bsums) + (long long)slab * src.ks.q.nblk * NC
+                                      : nullptr;
                 if (slab != carry_slab) {
-                    for (int r = 0; r < src.ks.q.R; r += 32)
-                        if (ready_prefix(slab, r, true) < 0) return false;
+                    for (int r = 0; r < R; r += 32)
+                        if (ready_prefix(src.flags, slab, r, true) < 0) return false;
+                    if (shared) {
+                        for (int jb = cta / P; jb < src.ks.q.nblk; jb += R) {
+                            const float* base = src.partial + ks_block_slot(slab, jb, 0, G, src.ks) * DD;
+                            for (int c = tid; c < NC; c += kWorkerThreads) {
+                                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                                for (int t0 = 0; t0 < nr; t0 += 8) {
+                                    float4 x[8];
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u)
+                                        x[u] = t0 + u < nr
+                                            ? __ldcg(reinterpret_cast<const float4*>(base + (t0 + u) * kstep) + c)
+                                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u) {
+                                        if (t0 + u < nr) {
+                                            acc.x += x[u].x;
+                                            acc.y += x[u].y;
+                                            acc.z += x[u].z;
+                                            acc.w += x[u].w;
+                                        }
+                                    }
+                                }
+                                __stcg(bsum + (long long)jb * NC + c, acc);
+                            }
+                        }
+                        __threadfence();
+                        warp_arrive(bar.bs_done);
+                        if (warp == 0) {
+                            if (!warp_wait(bar.bs_done, 0, abort, err)) return false;
+                            if (lane == 0) grid_arrive(src.flags2 + cta, src.epoch);
+                        }
+                        // every block sum of the slab, so later segments need no flags
+                        for (int r = 0; r < R; r += 32)
+                            if (ready_prefix(src.flags2, slab, r, true) < 0) return false;
+                    }
                     carry_slab = slab;
                     carry_blk = -1;
                 } else {
@@ -890,13 +941,25 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                         if (c < NC) v[j] = __ldcg(cs + c);      // written by this thread
                     }
                 }
-                // the partials of blocks carry_blk + 1 .. blk, nr per block, in
-                // that order; d = 32: four loads in flight at a time (d = 64
-                // one block's at a time: registers)
-                const long long kstep = ks_block_step(G, src.ks) * DD;
-                const int nr = src.ks.q.R / src.ks.q.rb;
                 float4 bs[NCT];
-                if constexpr (D == 32) {
+                if (shared) {
+                    // block sums of blocks carry_blk + 1 .. blk, in that order
+                    // (all in memory: their flags were seen at the slab's first segment)
+                    for (int jb = carry_blk + 1; jb <= blk; ++jb) {
+#pragma unroll
+                        for (int j = 0; j < NCT; ++j) {
+                            const int c = tid + j * kWorkerThreads;
+                            bs[j] = c < NC ? __ldcg(bsum + (long long)jb * NC + c) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        }
+#pragma unroll
+                        for (int j = 0; j < NCT; ++j) {
+                            v[j].x += bs[j].x;
+                            v[j].y += bs[j].y;
+                            v[j].z += bs[j].z;
+                            v[j].w += bs[j].w;
+                        }
+                    }
+                } else if constexpr (D == 32) {
                     constexpr int RB = 4;
                     const int total = (blk - carry_blk) * nr;
                     for (int q0 = 0; q0 < total; q0 += RB) {
@@ -1282,7 +1345,7 @@ ka_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, nullptr};
+    KaStateSrc src{state, nullptr, KsParams{}, nullptr, 0ull, nullptr, nullptr, nullptr};
     ka_phase<D, OUT_BF16, FM>(&tmQ, &tmO, p, blockIdx.x, src, smem, bar, ctl->tmem_base, &ctl->abort,
                           &g_device_error);
     kernel_epilogue(ctl, tid);
@@ -1359,7 +1422,10 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
         ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     }
-    KaStateSrc src{nullptr, partial, ks, flags, epoch, carry};
+    // block-causal: after the per-CTA prefixes, the slabs' block sums
+    float* bsums = carry == nullptr ? nullptr
+        : carry + (size_t)gridDim.x * (128 / D) * (D * (D + 1));
+    KaStateSrc src{nullptr, partial, ks, flags, epoch, carry, bsums, flags + gridDim.x};
     const int ks_tiles = (int)blockIdx.x < ks.q.grid
         ? sched_tps(blockIdx.x, ks.q) * sched_nseg(blockIdx.x, ks.q) : 0;
     ka_phase<D, OUT_BF16, FM, BC>(&tmQ, &tmO, ka, blockIdx.x, src, smem, abar, tmem, &ctl->abort, &g_device_error,
