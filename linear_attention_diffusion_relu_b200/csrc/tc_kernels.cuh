@@ -682,14 +682,16 @@ struct KaStateSrc {
 
 // Readiness flags of the single-launch forward. CTA c announces that all its
 // partial states are in memory by storing the launch's epoch into flags[c]
-// (after a fence). Before staging a slab's state, a CTA reads only the flags
-// of the CTAs that wrote that slab's partials (its R siblings), not those of
-// the whole grid, and adds each partial as soon as it and the ones before it
-// are in. The host draws a new 64-bit epoch for every launch, so flags left by
+// with release semantics. The writers fenced their own stores and arrived on a
+// CTA barrier that this thread waited on, so the release store orders them
+// too (release is cumulative); a second fence here only added latency (0-1 us
+// per forward at the mid-size shapes, measured on B200). Before staging a
+// slab's state, a CTA reads only the flags of the CTAs that wrote that slab's
+// partials (its R siblings), not those of the whole grid, and adds each
+// partial as soon as it and the ones before it are in. The host draws a new 64-bit epoch for every launch, so flags left by
 // earlier launches (or any other bytes) never pass for this one and the flag
 // array needs no reset between launches.
 __device__ __forceinline__ void grid_arrive(unsigned long long* flag, unsigned long long epoch) {
-    __threadfence();
     asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(flag), "l"(epoch) : "memory");
 }
 
