@@ -736,11 +736,14 @@ __device__ __forceinline__ void ka_phase(const CUtensorMap* tmQ, const CUtensorM
                     // the state phase's next (never issued) use of stage s
                     const int j = prev_tiles + ((s - prev_tiles) % PS + PS) % PS;
                     if (!ptx::mbar_wait(&prev_empty[s], ((j / PS) & 1) ^ 1, abort, err)) break;
-                    // Only kQAhead Q tiles are loaded before the first unit's tile
-                    // has been read (the state is staged by then): the partial
-                    // states and flags the workers read meanwhile are not queued
-                    // behind the rest. Four ahead instead of two: 2 us slower at
-                    // d = 64 and N = 16,384, the same at 4096 px (B200).
+                    // The first Q load waits until this CTA's partial states are
+                    // written and fenced, and only kQAhead Q tiles are loaded before
+                    // the first unit's tile has been read (the state is staged by
+                    // then): the fence and the partial states the workers read
+                    // meanwhile are not queued behind Q loads. Measured on B200
+                    // against four tiles ahead from the state phase's end: 2 us
+                    // faster at 2048px, d = 64 and N = 16,384, the same at 4096 px.
+                    if (i == 0 && !ptx::mbar_wait(bar.p1_written, 0, abort, err)) break;
                     if (i >= kQAhead && !ptx::mbar_wait(&bar.empty[0], 0, abort, err)) break;
                 }
                 int slab, tile, seg;
