@@ -619,7 +619,7 @@ struct KaBars {
     uint64_t* stg_free;    // [2 halves] this half's staging boxes may be written
     uint64_t* stg_full;    // [2 halves][2] this half's staging boxes written
     uint64_t* mma_done;
-    uint64_t* p1_written;  // (single launch) this CTA's partial states are written
+    uint64_t* p1_written;  // (single launch) partial states written (warps 0-3), state padding zeroed (4-7)
     uint64_t* bs_done;     // (block-causal single launch) this CTA's block sums are written
     __device__ void init() const {
         for (int s = 0; s < L::STAGES; ++s) {
@@ -636,7 +636,7 @@ struct KaBars {
             ptx::mbar_init(&stg_full[2 * h + 1], kWorkerWarps / 2);
         }
         ptx::mbar_init(mma_done, 1);
-        ptx::mbar_init(p1_written, 4);
+        ptx::mbar_init(p1_written, kWorkerWarps);
         ptx::mbar_init(bs_done, kWorkerWarps);
     }
 };
@@ -648,13 +648,13 @@ __device__ __forceinline__ KaBars<D, OUT_BF16> ka_bars(uint64_t* b) {
     return KaBars<D, OUT_BF16>{b, b + S, a, a + 2, a + 3, a + 4, a + 6, a + 10, a + 11, a + 12};
 }
 
-// zero the padding columns n in (d, NA) of the staged state
+// zero the padding columns n in (d, NA) of the staged state (threads [0, nthreads))
 template <int D, bool OUT_BF16>
-__device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid) {
+__device__ __forceinline__ void ka_zero_state_padding(uint8_t* smem, int tid, int nthreads = kWorkerThreads) {
     using L = KaLayout<D, OUT_BF16>;
-    if (tid < kWorkerThreads) {
+    if (tid < nthreads) {
         constexpr int PAD = L::NA - D - 1;
-        for (int e = tid; e < L::G * 2 * PAD * D; e += kWorkerThreads) {
+        for (int e = tid; e < L::G * 2 * PAD * D; e += nthreads) {
             const int k = e % D;
             const int n = D + 1 + (e / D) % PAD;
             const int mat = e / (D * PAD);
@@ -1424,17 +1424,26 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 
     // Warps 0-3 have written this CTA's partial states (after the last
     // accumulator was complete, i.e. after every state-phase UMMA): make them
-    // visible and arrive. Every worker waits for that before it touches the
-    // apply phase's shared memory or TMEM, which reuse the state phase's.
+    // visible and arrive. Warps 4-7 meanwhile zero the staged state's padding
+    // columns, once every state-phase UMMA is done with those bytes (they were
+    // a K/V stage); off the path from the last partial to the flag and the
+    // first poll, where it cost ~0.8 us. Every worker waits for both before
+    // it touches the apply phase's shared memory or TMEM, which reuse the
+    // state phase's.
     if (warp < 4) {
         __threadfence();
+        warp_arrive(abar.p1_written);
+    } else if (warp < kWorkerWarps) {
+        // (a CTA without state-phase tiles issued no UMMAs and commits none)
+        if ((int)blockIdx.x < ks.q.grid) warp_wait(kbar.mma_done, 0, &ctl->abort, &g_device_error);
+        ka_zero_state_padding<D, OUT_BF16>(smem, tid - 4 * 32, kWorkerThreads / 2);
+        ptx::fence_proxy_async_smem();
         warp_arrive(abar.p1_written);
     }
     if (warp < kWorkerWarps) {
         warp_wait(abar.p1_written, 0, &ctl->abort, &g_device_error);
         // every CTA raises its readiness flag, with or without apply work
         if (tid == 0) grid_arrive(flags + blockIdx.x, epoch);
-        ka_zero_state_padding<D, OUT_BF16>(smem, tid);
     }
     // block-causal: after the per-CTA prefixes, the slabs' block sums
     float* bsums = carry == nullptr ? nullptr
