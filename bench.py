@@ -12,7 +12,11 @@ than the 126 MB L2, so no explicit L2 flush is done between steps.
 Prints one JSON line (rank 0). `value` is GB/s of algorithmic traffic (Q, K, V
 read once, O written once) over the device-timed steps, summed over ranks and
 divided by the slowest rank's time. Multi-GPU runs give every rank its own
-4096px problem (independent batches: weak scaling, no data-path collective).
+4096px problem (independent batches: weak scaling, no data-path collective);
+`--scaling strong` splits one problem over the ranks instead, by batches and
+then by ranges of whole head groups (still no collective: the (b, h) problems
+are independent), and `value` is that one problem's bytes over the slowest
+rank's time.
 
 `--impl reference` times the fp64 CPU oracle (the only reference there is) on
 bounded samples of the same workload, on the host cores, rank 0 only.
@@ -25,6 +29,7 @@ next to the unfused pipeline it replaces (one GPU, TFLOP/s).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -71,6 +76,9 @@ def parse_args(argv=None):
                    help="named workload (profiling runs use smaller ones; the bench line is 4096px)")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
+    p.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                   help="weak: every rank its own batch of the workload; strong: one workload split "
+                        "over the ranks by batches and head groups (no data-path collective)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -107,6 +115,38 @@ def max_over_ranks(x: float, device=None) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard(world: int, rank: int, B: int, H: int, G: int):
+    """Strong scaling: the batches [b0, b1) and heads [h0, h1) of rank `rank`
+    when one job of B batches of H heads is split over `world` GPUs. Whole
+    batches when world divides B; when world = k B, each batch is split into k
+    ranges of whole head groups (G heads each, one slab of the kernels). The
+    (b, h) problems are independent, so the ranks exchange nothing."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    if B % world == 0:
+        per = B // world
+        return rank * per, (rank + 1) * per, 0, H
+    if world % B == 0:
+        k = world // B
+        groups = -(-H // G)
+        if groups < k:
+            raise ValueError(f"{H} heads ({groups} groups of {G}) cannot be split {k} ways")
+        b, j = divmod(rank, k)
+        g0, g1 = j * groups // k, (j + 1) * groups // k
+        return b, b + 1, g0 * G, min(g1 * G, H)
+    raise ValueError(f"{world} GPUs neither divide {B} batches nor are a multiple of them")
+
+
+def rank_workload(w, world: int, rank: int, scaling: str):
+    """This rank's workload and its (b0, b1, h0, h1) part of the job (None for
+    weak scaling, where every rank runs the whole workload `w`)."""
+    if scaling != "strong" or world == 1:
+        return w, None
+    part = shard(world, rank, w.B, w.H, 128 // w.d)
+    b0, b1, h0, h1 = part
+    return dataclasses.replace(w, name=f"{w.name}[b{b0}:{b1},h{h0}:{h1}]", B=b1 - b0, H=h1 - h0), part
 
 
 def aggregate_gbs(bytes_per_rank: int, world: int, max_seconds: float) -> float:
@@ -272,9 +312,15 @@ def run_ours(args):
     ops.load_library()
 
     w = WORKLOADS[args.workload]
+    # the whole job: weak scaling, one workload per rank; strong, one workload
+    # split over the ranks (this rank's part becomes `w`)
+    strong = args.scaling == "strong"
+    job = w
+    job_copies = 1 if strong else world
+    w, part = rank_workload(job, world, rank, args.scaling)
     B, N, H, d, L = w.B, w.N, w.H, w.d, w.block
     Q, K, V = make_inputs(w, device=dev, generator_device=input_generator(w))
-    if rank > 0:   # every rank its own independent batch of the same shape
+    if rank > 0 and not strong:   # every rank its own independent batch of the same shape
         Q, K, V = (t.roll(shifts=rank, dims=1).contiguous() for t in (Q, K, V))
     out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -336,8 +382,9 @@ def run_ours(args):
     # shapes, so the timed region above has none)
     per_step = per_step_times(step, stream, min(args.steps, 1000))
     bytes_per_step = w.algorithmic_bytes(2)
-    value = aggregate_gbs(bytes_per_step, world, ms_max / 1e3)
-    mtok = B * N * world / (ms_max / 1e3) / 1e6
+    # whole-job bytes and tokens over the slowest rank's time
+    value = aggregate_gbs(job.algorithmic_bytes(2), job_copies, ms_max / 1e3)
+    mtok = job.B * job.N * job_copies / (ms_max / 1e3) / 1e6
 
     # ---- breakdown: the same phases as separate kernels through the two-call
     # API, with events between the state half and the apply half
@@ -386,7 +433,8 @@ def run_ours(args):
                       f"{min(args.steps, 1000)} steps; split_api_ms: events around kv_state and apply in a "
                       f"{n_split}-step loop of the two-call API after the timed region")
 
-    fp32 = None if L else run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl)
+    fp32 = None if L else run_fp32_out(args, w, Q, K, V, ws, dev, stream, job, job_copies, hbm_peak, peak_src,
+                                       impl)
 
     # block-causal: the one-launch form (bit-identical), timed the same way
     single = None
@@ -413,7 +461,7 @@ def run_ours(args):
                   "gpu_launches": ops.block_causal_forward_launches(B, N, H, d, L, single_launch=True) * n_single,
                   "call": "block_causal_forward_single"}
 
-    e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, world)
+    e2e = None if args.no_e2e else run_e2e(args, w, dev, stream, job, job_copies)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -425,15 +473,17 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "mtokens_per_s": mtok, "pct_of_hbm_peak": 100.0 * value / (hbm_peak * world),
-            "config": {"workload": w.name, "B": B, "N": N, "H": H, "d": d,
+            "config": {"workload": job.name, "B": job.B, "N": N, "H": job.H, "d": d,
                        **({"form": "block-causal", "block": L} if L else {}),
                        **({"feature_map": fm} if fm != "relu" else {}),
                        "io": "bf16 Q/K/V in, bf16 O out, fp32 state and accumulation",
-                       "eps": w.eps, "per_rank": f"one independent {w.name} batch",
-                       "parallelism": f"dp{world}",
+                       "eps": w.eps,
+                       "per_rank": (f"one independent {w.name} batch" if part is None else
+                                    f"rank 0: batches {part[0]}-{part[1] - 1}, heads {part[2]}-{part[3] - 1}"),
+                       "parallelism": f"dp{world}" if part is None else f"batch/head-group split over {world}",
                        "l2": (f"inputs {w.token_heads * d * 6 / 1e6:.0f} MB + output "
                               f"{w.token_heads * d * 2 / 1e6:.0f} MB per step vs the 126 MB L2; no flush"),
                        "kernel_impl": impl["name"]},
@@ -465,7 +515,7 @@ def per_step_times(step, stream, n):
     return [ev[k].elapsed_time(ev[k + 1]) for k in range(n)]
 
 
-def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, impl):
+def run_fp32_out(args, w, Q, K, V, ws, dev, stream, job, job_copies, hbm_peak, peak_src, impl):
     """The same forward with O in fp32 (the output type the 1e-4 per-row
     tolerance is stated for): its own timed loop after the main one, the same
     step count, algorithmic bytes with 4-byte outputs."""
@@ -491,9 +541,10 @@ def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, i
     nbytes = w.algorithmic_bytes(4)
     achieved = nbytes / (ms / 1e3) / 1e9
     return {
-        "value": aggregate_gbs(nbytes, world, ms_max / 1e3), "unit": UNIT, "ms_per_step": ms_max,
+        "value": aggregate_gbs(job.algorithmic_bytes(4), job_copies, ms_max / 1e3), "unit": UNIT,
+        "ms_per_step": ms_max,
         "ms_per_step_median": statistics.median(per_step), "ms_per_step_min": min(per_step),
-        "mtokens_per_s": w.B * w.N * world / (ms_max / 1e3) / 1e6,
+        "mtokens_per_s": job.B * job.N * job_copies / (ms_max / 1e3) / 1e6,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "kernel": "fwd_fused_tc",
                      "traffic": TRAFFIC_PER_LAUNCH.get((impl["name"], w.name, "fwd_fused_tc", 4)),
@@ -503,7 +554,7 @@ def run_fp32_out(args, w, Q, K, V, ws, dev, stream, world, hbm_peak, peak_src, i
     }
 
 
-def run_e2e(args, w, dev, stream, world):
+def run_e2e(args, w, dev, stream, job, job_copies):
     """Same metric through the public call with host buffers: every step copies
     Q, K, V from pinned host memory to the device and O back, the copies made
     by the library (ops.forward_host, or ops.block_causal_forward_host): K and
@@ -542,7 +593,7 @@ def run_e2e(args, w, dev, stream, world):
     ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, dev)
     h2d = 3 * hQ.numel() * hQ.element_size()
     d2h = hO.numel() * hO.element_size()
-    return {"value": aggregate_gbs(w.algorithmic_bytes(2), world, ms / 1e3), "unit": UNIT,
+    return {"value": aggregate_gbs(job.algorithmic_bytes(2), job_copies, ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "call": ("block_causal_forward_host" if L else "forward_host") + " (copies by the library)"}
 

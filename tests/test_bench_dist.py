@@ -81,3 +81,51 @@ def test_reference_arm_json_line(capsys):
     e2e = j["e2e"]
     assert e2e["value"] == j["value"] and e2e["unit"] == j["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_strong_scaling_shards_partition_the_job():
+    """--scaling strong: the ranks' (batch, head) ranges cover every (b, h) of
+    the job exactly once, on whole head groups, for every supported GPU count."""
+    import bench
+    for B, H, G in [(2, 70, 4), (2, 36, 4), (1, 18, 2), (4, 9, 4), (1, 70, 4)]:
+        groups = -(-H // G)
+        for world in (1, 2, 4, 8):
+            if not (B % world == 0 or (world % B == 0 and groups >= world // B)):
+                with pytest.raises(ValueError):
+                    bench.shard(world, 0, B, H, G)
+                continue
+            seen = {}
+            for r in range(world):
+                b0, b1, h0, h1 = bench.shard(world, r, B, H, G)
+                assert 0 <= b0 < b1 <= B and 0 <= h0 < h1 <= H
+                assert h0 % G == 0 and (h1 % G == 0 or h1 == H)
+                for b in range(b0, b1):
+                    for h in range(h0, h1):
+                        assert (b, h) not in seen
+                        seen[(b, h)] = r
+            assert len(seen) == B * H
+    # the 4096px job over 8 GPUs: a batch per four ranks, head groups 4 / 5 / 4 / 5
+    assert [bench.shard(8, r, 2, 70, 4) for r in range(4)] == [
+        (0, 1, 0, 16), (0, 1, 16, 36), (0, 1, 36, 52), (0, 1, 52, 70)]
+    with pytest.raises(ValueError):
+        bench.shard(3, 0, 2, 70, 4)
+
+
+def test_strong_scaling_flag_parses():
+    import bench
+    assert bench.parse_args(["--scaling", "strong", "--gpus", "4"]).scaling == "strong"
+    assert bench.parse_args([]).scaling == "weak"
+
+
+def test_strong_scaling_rank_workloads_sum_to_the_job():
+    import bench
+    from linear_attention_diffusion_relu_b200.workloads import WORKLOADS
+    job = WORKLOADS["4096px"]
+    for world in (2, 4, 8):
+        parts = [bench.rank_workload(job, world, r, "strong") for r in range(world)]
+        assert sum(w.algorithmic_bytes(2) for w, _ in parts) == job.algorithmic_bytes(2)
+        assert all(w.N == job.N and w.d == job.d and w.name != job.name for w, _ in parts)
+    w, part = bench.rank_workload(job, 8, 1, "strong")
+    assert (w.B, w.H, part) == (1, 20, (0, 1, 16, 36))
+    assert bench.rank_workload(job, 8, 1, "weak") == (job, None)
+    assert bench.rank_workload(job, 1, 0, "strong") == (job, None)
