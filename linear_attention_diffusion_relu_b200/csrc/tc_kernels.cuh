@@ -274,6 +274,31 @@ __device__ __forceinline__ void ks_fill_ones(uint8_t* smem, int tid) {
     }
 }
 
+// TMA loads of the state phase's tile i of CTA `cta` (K and V boxes of its
+// group row) into stage `s`, completing on full[s].
+__device__ __forceinline__ void ks_load_tile(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
+                                             int cta, int i, int tps, uint8_t* st, uint64_t* full,
+                                             bool evict_first) {
+    int slab, tile, seg;
+    sched_item(cta, i, tps, p.q, slab, tile, seg);
+    const int b = slab / p.groups;
+    const int x0 = (slab % p.groups) * 128;
+    const int y = tile * KS_TILE;
+    ptx::mbar_arrive_expect_tx(full, KS_STAGE_BYTES);
+    if (evict_first) {
+        const uint64_t pol = ptx::l2_policy_evict_first();
+        ptx::tma_load_3d_hint(st + 0 * KS_BOX_BYTES, tmK, full, x0, y, b, pol);
+        ptx::tma_load_3d_hint(st + 1 * KS_BOX_BYTES, tmK, full, x0 + 64, y, b, pol);
+        ptx::tma_load_3d_hint(st + 2 * KS_BOX_BYTES, tmV, full, x0, y, b, pol);
+        ptx::tma_load_3d_hint(st + 3 * KS_BOX_BYTES, tmV, full, x0 + 64, y, b, pol);
+    } else {
+        ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, tmK, full, x0, y, b);
+        ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, tmK, full, x0 + 64, y, b);
+        ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, tmV, full, x0, y, b);
+        ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, tmV, full, x0 + 64, y, b);
+    }
+}
+
 // The state phase for CTA `cta`: partial states phi(K)^T [V | 1] of its
 // segments into `partial`. Every role returns once its part is done. Stage s
 // of this phase is free again once bar.empty[s] has completed the phase of the
@@ -283,7 +308,7 @@ template <int D, int FM>
 __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const KsParams& p,
                                          int cta, float* __restrict__ partial, uint8_t* smem,
                                          const KsBars& bar, uint32_t tmem, volatile int* abort,
-                                         uint32_t* err, bool evict_first = false)
+                                         uint32_t* err, bool evict_first = false, int pre_issued = 0)
 {
     constexpr int G = 128 / D;
     constexpr int DD = D * (D + 1);
@@ -300,29 +325,13 @@ __device__ __forceinline__ void ks_phase(const CUtensorMap* tmK, const CUtensorM
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ----
         if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
+            // (tiles [0, pre_issued) were loaded by the caller, before its
+            // CTA-wide sync, into their stages; pre_issued <= NS)
+            int issued = min(pre_issued, ntiles);
+            for (int i = issued; i < ntiles; ++i) {
                 const int s = i % NS;
                 if (!ptx::mbar_wait(&bar.empty[s], ((i / NS) & 1) ^ 1, abort, err)) break;
-                int slab, tile, seg;
-                sched_item(cta, i, tps, p.q, slab, tile, seg);
-                const int b = slab / p.groups;
-                const int x0 = (slab % p.groups) * 128;
-                const int y = tile * KS_TILE;
-                uint8_t* st = stage_ptr(s);
-                ptx::mbar_arrive_expect_tx(&bar.full[s], KS_STAGE_BYTES);
-                if (evict_first) {
-                    const uint64_t pol = ptx::l2_policy_evict_first();
-                    ptx::tma_load_3d_hint(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b, pol);
-                    ptx::tma_load_3d_hint(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b, pol);
-                    ptx::tma_load_3d_hint(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b, pol);
-                    ptx::tma_load_3d_hint(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b, pol);
-                } else {
-                    ptx::tma_load_3d(st + 0 * KS_BOX_BYTES, tmK, &bar.full[s], x0, y, b);
-                    ptx::tma_load_3d(st + 1 * KS_BOX_BYTES, tmK, &bar.full[s], x0 + 64, y, b);
-                    ptx::tma_load_3d(st + 2 * KS_BOX_BYTES, tmV, &bar.full[s], x0, y, b);
-                    ptx::tma_load_3d(st + 3 * KS_BOX_BYTES, tmV, &bar.full[s], x0 + 64, y, b);
-                }
+                ks_load_tile(tmK, tmV, p, cta, i, tps, stage_ptr(s), &bar.full[s], evict_first);
                 issued = i + 1;
             }
             // drain: every issued load must land before the CTA may exit
@@ -1399,18 +1408,31 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + Map::CTL_OFF);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    if (tid == 0) {
+    // The producer thread initialises the state phase's barriers and issues
+    // its first tiles' loads at once, ahead of the TMEM allocation and the
+    // CTA-wide sync below (the other threads touch those barriers only after
+    // that sync, and the loads' stages are not written before it).
+    int pre_issued = 0;
+    if (tid == kProducerWarp * 32) {
         kbar.init();
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmK);
+        ptx::prefetch_tmap(&tmV);
+        if ((int)blockIdx.x < ks.q.grid) {
+            const int tps = sched_tps(blockIdx.x, ks.q);
+            pre_issued = min(ks_stages<FM>(), tps * sched_nseg(blockIdx.x, ks.q));
+            for (int i = 0; i < pre_issued; ++i)
+                ks_load_tile(&tmK, &tmV, ks, blockIdx.x, i, tps, smem + (size_t)i * KS_STAGE_BYTES, &kbar.full[i],
+                             evict_first != 0);
+        }
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmO);
+    }
+    if (tid == 0) {
         abar.init();
         ptx::fence_mbar_init();
     }
     kernel_prologue(ctl, tid);
-    if (tid == kProducerWarp * 32) {
-        ptx::prefetch_tmap(&tmK);
-        ptx::prefetch_tmap(&tmV);
-        ptx::prefetch_tmap(&tmQ);
-        ptx::prefetch_tmap(&tmO);
-    }
     ks_fill_ones(smem, tid);
     ptx::tc_fence_before_sync();
     __syncthreads();
@@ -1420,7 +1442,7 @@ fwd_fused_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     // with evict_first, K, V and Q (read once) are marked first to go when L2
     // needs room
     ks_phase<D, FM>(&tmK, &tmV, ks, blockIdx.x, partial, smem, kbar, tmem, &ctl->abort, &g_device_error,
-                    evict_first != 0);
+                    evict_first != 0, pre_issued);
 
     // Warps 0-3 have written this CTA's partial states (after the last
     // accumulator was complete, i.e. after every state-phase UMMA): make them
